@@ -1,0 +1,157 @@
+"""Seeded synthetic inputs for the GSPN line-scan operator.
+
+This module only draws random numbers and lays them out. It holds none of the
+operator's arithmetic; both the CPU oracle (``oracle/``) and the CUDA library
+(``linear_spatial_propagation_b200``) receive the very same bytes from here.
+
+Tensor layouts (dense, row-major), as the C ABI in ``include/gspn.h`` states:
+
+* ``x``, ``dout``:        ``[B, C, H, W]``
+* ``lam`` (lambda):       ``[D, B, C, H, W]``     D = number of directions
+* ``logits``:             ``[D, B, Cw, 3, H, W]``  Cw = 1 when taps are shared
+
+Draws (each tensor from its own child stream of ``SeedSequence(seed)``, spawned
+in the order x, lambda, logits, dout):
+
+* x ~ N(0, 1), lambda ~ U(0, 1), logits ~ N(0, logit_std), dout ~ N(0, 1),
+  all drawn in float32 by numpy's PCG64 generator;
+* bf16 tensors are the float32 draws rounded to nearest-even bf16 and are
+  stored as ``uint16`` bit patterns (numpy has no bf16 dtype).
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Dict, Optional
+
+import numpy as np
+
+DIR_T2B, DIR_B2T, DIR_L2R, DIR_R2L = 1, 2, 4, 8
+ALL_DIRS = DIR_T2B | DIR_B2T | DIR_L2R | DIR_R2L
+DTYPES = ("f32", "bf16")
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """Shape, mode and input distribution of one GSPN invocation."""
+
+    name: str
+    B: int
+    C: int
+    H: int
+    W: int
+    dir_mask: int
+    groups: int
+    shared: bool
+    dtype: str
+    logit_std: float
+    seed: int
+    backward: bool = False
+
+    @property
+    def D(self) -> int:
+        return bin(self.dir_mask).count("1")
+
+    @property
+    def Cw(self) -> int:
+        return 1 if self.shared else self.C
+
+    @property
+    def elt_bytes(self) -> int:
+        return 4 if self.dtype == "f32" else 2
+
+    def shapes(self) -> Dict[str, tuple]:
+        return {
+            "x": (self.B, self.C, self.H, self.W),
+            "lam": (self.D, self.B, self.C, self.H, self.W),
+            "logits": (self.D, self.B, self.Cw, 3, self.H, self.W),
+            "dout": (self.B, self.C, self.H, self.W),
+        }
+
+    def replace(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads the operator is specified and measured on.  Names say
+# what they are; sizes follow the GSPN / GSPN-2 / C-GSPN pages (tiny-backbone
+# stage-1 shape 56x56, 28x28 local stage, the 1K foundation shape B=32 C=1152
+# 64x64, and the 2K shape 128x128).
+WORKLOADS: Dict[str, Workload] = {
+    w.name: w
+    for w in (
+        Workload("t2b_f32_b1c4_16x16", 1, 4, 16, 16, DIR_T2B, 1, False, "f32", 1.0, 0),
+        Workload("4dir_f32_b8c96_56x56", 8, 96, 56, 56, ALL_DIRS, 1, False, "f32", 1.0, 1),
+        Workload("4dir_local4_bf16_b32c192_28x28", 32, 192, 28, 28, ALL_DIRS, 4, False, "bf16", 2.0, 2),
+        Workload("compact_4dir_bf16_b32c1152_64x64", 32, 1152, 64, 64, ALL_DIRS, 1, True, "bf16", 1.0, 3),
+        Workload("compact_4dir_bf16_b2c1152_128x128_fwdbwd", 2, 1152, 128, 128, ALL_DIRS, 1, True, "bf16", 1.0, 4,
+                 backward=True),
+    )
+}
+
+HEADLINE = "compact_4dir_bf16_b32c1152_64x64"
+
+
+def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round float32 values to the nearest-even bf16; return the uint16 bits."""
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    u = a.view(np.uint32)
+    rounding = np.uint32(0x7FFF) + ((u >> np.uint32(16)) & np.uint32(1))
+    return ((u + rounding) >> np.uint32(16)).astype(np.uint16)
+
+
+def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
+    """Widen bf16 bit patterns (uint16) to float32 exactly."""
+    return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
+
+
+def _draw(rng: np.random.Generator, kind: str, shape: tuple, scale: float = 1.0,
+          chunk: int = 1 << 26) -> np.ndarray:
+    n = int(np.prod(shape))
+    out = np.empty(n, dtype=np.float32)
+    for s in range(0, n, chunk):
+        e = min(n, s + chunk)
+        if kind == "normal":
+            rng.standard_normal(e - s, dtype=np.float32, out=out[s:e])
+            if scale != 1.0:
+                out[s:e] *= np.float32(scale)
+        else:
+            rng.random(e - s, dtype=np.float32, out=out[s:e])
+    return out.reshape(shape)
+
+
+def make_inputs(w: Workload, with_dout: Optional[bool] = None) -> Dict[str, np.ndarray]:
+    """Draw the seeded inputs of workload ``w``.
+
+    Returns float32 arrays for ``dtype == 'f32'`` and uint16 bf16 bit patterns
+    for ``dtype == 'bf16'``.  ``dout`` is drawn when ``with_dout`` (default:
+    ``w.backward``).
+    """
+    if with_dout is None:
+        with_dout = w.backward
+    kids = np.random.SeedSequence(w.seed).spawn(4)
+    shp = w.shapes()
+    out = {
+        "x": _draw(np.random.Generator(np.random.PCG64(kids[0])), "normal", shp["x"]),
+        "lam": _draw(np.random.Generator(np.random.PCG64(kids[1])), "uniform", shp["lam"]),
+        "logits": _draw(np.random.Generator(np.random.PCG64(kids[2])), "normal", shp["logits"], w.logit_std),
+    }
+    if with_dout:
+        out["dout"] = _draw(np.random.Generator(np.random.PCG64(kids[3])), "normal", shp["dout"])
+    if w.dtype == "bf16":
+        out = {k: f32_to_bf16_bits(v) for k, v in out.items()}
+    return out
+
+
+def plane_slice(w: Workload, inp: Dict[str, np.ndarray], b: int, c: int) -> Dict[str, np.ndarray]:
+    """Inputs of the single (b, c) plane, as a B=1, C=1 workload's arrays.
+
+    Pure indexing: with shared taps the plane keeps logits channel 0 of batch b.
+    """
+    cw = 0 if w.shared else c
+    sl = {
+        "x": inp["x"][b:b + 1, c:c + 1],
+        "lam": inp["lam"][:, b:b + 1, c:c + 1],
+        "logits": inp["logits"][:, b:b + 1, cw:cw + 1],
+    }
+    if "dout" in inp:
+        sl["dout"] = inp["dout"][b:b + 1, c:c + 1]
+    return {k: np.ascontiguousarray(v) for k, v in sl.items()}
