@@ -1,0 +1,399 @@
+#!/usr/bin/env python
+"""Benchmark of the GSPN line scan (libgspn) on B200.
+
+One step = one pass of the whole hot path over one batch: the forward
+(gate normalisation, four-direction line scan, summed merge) followed by the
+backward (reverse adjoint scans, dx / dlambda / dlogits), through the C ABI.
+Default workload: compact (channel-shared taps) 4-direction global scan, bf16
+storage, fp32 arithmetic, B=32, C=1152, H=W=64 -- the 1K foundation shape.
+
+Metric: achieved HBM GB/s = compulsory bytes / time, where the compulsory
+bytes are every input read once and every output written once
+(forward: x, lambda, logits, out; backward: x, lambda, logits, dout, dx,
+dlambda, dlogits).  Also reported: % of the measured HBM copy peak and
+Gpixel*channel/s.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl libgspn|reference]
+
+For N > 1 it runs under torch.distributed.run, one rank per GPU; each rank
+processes its own batch (weak scaling, no collective on the data path) and
+rank 0 prints one JSON line with the max-over-ranks time.
+--impl reference times the CPU oracle (plain double-precision C) on the host
+cores on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "GSPN scan achieved HBM GB/s (% of B200 peak) and Gpixel·ch/s, fwd and fwd+bwd"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="libgspn", choices=["libgspn", "reference"])
+    ap.add_argument("--workload", default=synth.HEADLINE, choices=list(synth.WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the oracle sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def pass_bytes(w: synth.Workload):
+    """Compulsory bytes of one forward and one backward pass."""
+    e = w.elt_bytes
+    n = w.B * w.C * w.H * w.W
+    lam = w.D * n
+    lg = w.D * w.B * w.Cw * 3 * w.H * w.W
+    fwd = e * (n + lam + lg + n)
+    bwd = e * (n + lam + lg + n + n + lam + lg)
+    return fwd, bwd
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def csrc_hash() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "linear_spatial_propagation_b200", "csrc")
+    for f in sorted(os.listdir(d)):
+        h.update(f.encode())
+        h.update(open(os.path.join(d, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_pass: str, w: synth.Workload):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel sources."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    ent = d.get(w.name, {}).get(kernel_pass)
+    if not ent or ent.get("csrc_hash") != csrc_hash():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9:
+                    rows.append(f)
+        except Exception:
+            return None
+        finally:
+            try:
+                os.unlink(self.path)
+            except OSError:
+                pass
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[5:9]) if v.lower() == "active"})
+        load = [s for s in sm if mx and s > 0.3 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(load) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ------------------------------------------------------------------------------
+def oracle_sample(w: synth.Workload, target_s: float, nthreads: int):
+    """Time the oracle's forward + backward on a sample of w's planes: B=1 and
+    as many channels as fit in about target_s seconds."""
+    import oracle
+
+    def run(cs):
+        sw = w.replace(B=1, C=cs, seed=w.seed + 7)
+        inp = synth.make_inputs(sw, with_dout=True)
+        t0 = time.perf_counter()
+        oracle.fwd_workload(sw, inp, nthreads=nthreads)
+        oracle.bwd_workload(sw, inp, nthreads=nthreads)
+        return time.perf_counter() - t0, sw
+
+    probe_c = min(w.C, max(1, nthreads))
+    t, sw = run(probe_c)
+    cs = int(min(w.C, max(1, probe_c * target_s / max(t, 1e-6))))
+    if cs > probe_c:
+        t, sw = run(cs)
+    f, b = pass_bytes(sw)
+    return {"seconds": t, "bytes": f + b, "pixch": sw.B * sw.C * sw.H * sw.W, "channels": sw.C, "sw": sw}
+
+
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    nthreads = os.cpu_count() or 1
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    per_step = max(0.5, min(args.cpu_seconds, 150.0 / (steps + warm)))
+    cal = oracle_sample(w, per_step, nthreads)
+    import oracle
+    sw = cal["sw"]
+    inp = synth.make_inputs(sw, with_dout=True)
+    for _ in range(warm):
+        oracle.fwd_workload(sw, inp, nthreads=nthreads)
+        oracle.bwd_workload(sw, inp, nthreads=nthreads)
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.fwd_workload(sw, inp, nthreads=nthreads)
+        oracle.bwd_workload(sw, inp, nthreads=nthreads)
+    dt = (time.perf_counter() - t0) / steps
+    f, b = pass_bytes(sw)
+    val = (f + b) / dt / 1e9
+    sample = f"B=1, C={sw.C} of {w.name} (fwd+bwd), {nthreads} threads"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": warm, "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
+        "config": config_of(w, args.gpus),
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": nthreads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def config_of(w, n):
+    return {"workload": w.name, "B": w.B, "C": w.C, "H": w.H, "W": w.W,
+            "directions": "+".join(n_ for b, n_ in ((1, "T2B"), (2, "B2T"), (4, "L2R"), (8, "R2L")) if w.dir_mask & b),
+            "groups": w.groups, "shared_taps": w.shared, "io_dtype": w.dtype, "pass": "fwd+bwd",
+            "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"}
+
+
+# ------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------
+def run_gpu(args, w):
+    import torch
+
+    import linear_spatial_propagation_b200 as lsp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    lsp.load(build_if_missing=False)
+
+    wr = w.replace(seed=w.seed + 1000 * rank)
+    inp = synth.make_inputs(wr, with_dout=True)
+    tdt = torch.bfloat16 if w.dtype == "bf16" else torch.float32
+
+    def pinned(a):
+        t = torch.from_numpy(a)
+        if w.dtype == "bf16":
+            t = t.view(torch.bfloat16)
+        return t.pin_memory()
+
+    h = {k: pinned(v) for k, v in inp.items()}
+    del inp
+    d = {k: v.to(dev) for k, v in h.items()}
+    out = torch.empty_like(d["x"])
+    grads = (torch.empty_like(d["x"]), torch.empty_like(d["logits"]), torch.empty_like(d["lam"]))
+    desc = lsp.make_desc(w.B, w.C, w.H, w.W, w.dir_mask, w.groups, w.shared, w.dtype)
+    wsf = lsp.workspace(desc, 0, dev)
+    wsb = lsp.workspace(desc, 1, dev)
+    stream = torch.cuda.current_stream(dev)
+    sp = stream.cuda_stream
+
+    def fwd():
+        st = lsp.gspn_fwd(desc, d["x"].data_ptr(), d["logits"].data_ptr(), d["lam"].data_ptr(), out.data_ptr(),
+                          wsf.data_ptr() if wsf is not None else 0, wsf.numel() if wsf is not None else 0, sp)
+        if st:
+            raise lsp.GspnError(st, "gspn_fwd")
+
+    def bwd():
+        st = lsp.gspn_bwd(desc, d["x"].data_ptr(), d["logits"].data_ptr(), d["lam"].data_ptr(),
+                          d["dout"].data_ptr(), grads[0].data_ptr(), grads[1].data_ptr(), grads[2].data_ptr(),
+                          wsb.data_ptr() if wsb is not None else 0, wsb.numel() if wsb is not None else 0, sp)
+        if st:
+            raise lsp.GspnError(st, "gspn_bwd")
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(v):
+        if dist is None:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(max(3, args.warmup)):
+        fwd()
+        bwd()
+    barrier()
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e_start.record(stream)
+    for k in range(K):
+        ev[k][0].record(stream)
+        fwd()
+        ev[k][1].record(stream)
+        bwd()
+        ev[k][2].record(stream)
+    e_end.record(stream)
+    barrier()
+    clk = clocks.stop()
+    total_ms = max_over_ranks(e_start.elapsed_time(e_end))
+    fwd_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K)
+    bwd_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / K)
+    ms = total_ms / K
+
+    # end to end: pinned host inputs -> device -> fwd + bwd -> results back to pinned host
+    E = max(1, args.e2e_steps)
+    hout = torch.empty(out.shape, dtype=tdt).pin_memory()
+    hgrads = [torch.empty(g.shape, dtype=tdt).pin_memory() for g in grads]
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = out.numel() * out.element_size() + sum(g.numel() * g.element_size() for g in grads)
+    barrier()
+    e2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+    e2[0].record(stream)
+    for _ in range(E):
+        for k in ("x", "lam", "logits", "dout"):
+            d[k].copy_(h[k], non_blocking=True)
+        fwd()
+        bwd()
+        hout.copy_(out, non_blocking=True)
+        for hg, g in zip(hgrads, grads):
+            hg.copy_(g, non_blocking=True)
+    e2[1].record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(e2[0].elapsed_time(e2[1]) / E)
+
+    fb, bb = pass_bytes(w)
+    peak, peak_src = measured_peaks()
+    n_gpu = world
+    value = (fb + bb) * n_gpu / (ms * 1e-3) / 1e9
+    pixch = w.B * w.C * w.H * w.W
+    fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
+    bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
+    dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
+    dom_gbs = bwd_gbs if dom == "bwd" else fwd_gbs
+    launches = K * (lsp.gspn_launches_per_call(desc, 0) + lsp.gspn_launches_per_call(desc, 1))
+
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            try:
+                s = oracle_sample(w, args.cpu_seconds, os.cpu_count() or 1)
+                cpu = {"value": s["bytes"] / s["seconds"] / 1e9, "unit": "GB/s", "cores": os.cpu_count() or 1,
+                       "kind": "oracle",
+                       "sample": f"fwd+bwd of B=1, C={s['channels']} planes of {w.name} ({s['seconds']:.1f} s)"}
+            except Exception as ex:  # the baseline must not sink the GPU line
+                cpu = {"value": None, "unit": "GB/s", "cores": os.cpu_count() or 1, "kind": "oracle",
+                       "sample": f"failed: {ex!r}"[:200]}
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_gpu, "steps": K,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded numpy PCG64, per-rank seed)",
+            "config": config_of(w, n_gpu),
+            "pct_of_peak": 100.0 * value / n_gpu / peak,
+            "gpix_ch_per_s": pixch * n_gpu / (ms * 1e-3) / 1e9,
+            "fwd": {"ms": fwd_ms, "GB/s": fwd_gbs, "pct_of_peak": 100.0 * fwd_gbs / peak,
+                    "gpix_ch_per_s": pixch / (fwd_ms * 1e-3) / 1e9, "bytes": fb,
+                    "kernel": lsp.gspn_variant_name(desc, 0)},
+            "bwd": {"ms": bwd_ms, "GB/s": bwd_gbs, "pct_of_peak": 100.0 * bwd_gbs / peak,
+                    "gpix_ch_per_s": pixch / (bwd_ms * 1e-3) / 1e9, "bytes": bb,
+                    "kernel": lsp.gspn_variant_name(desc, 1)},
+            "roofline": {"bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": dom_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
+                         "kernel": lsp.gspn_variant_name(desc, 1 if dom == "bwd" else 0),
+                         "traffic": ncu_traffic(dom, w)},
+            "e2e": {"value": (fb + bb) * n_gpu / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": launches,
+            "clocks": clk,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    w = synth.WORKLOADS[args.workload]
+    if not w.backward:
+        w = w.replace(backward=True)
+    if args.impl == "reference":
+        return run_reference(args, w)
+    return run_gpu(args, w)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

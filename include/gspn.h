@@ -1,0 +1,151 @@
+/*
+ * gspn.h -- C ABI of libgspn, the GSPN 2D line-scan propagation on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The operator (cited by page title and section):
+ *
+ *   For one (batch b, channel c) plane and one scan direction, lines are
+ *   visited in scan order and every line i is computed from the previous one:
+ *
+ *       h_i[j] = sum_{k=0..2} w_{i,j,k} * h_{i-1}[j+k-1] + lambda_i[j] * x_i[j]
+ *
+ *   "Parallel Sequence Modeling via Generalized Spatial Propagation Network"
+ *   (GSPN, CVPR 2025 reading notes), Key design 1: the recurrence
+ *   h_i = w_i h_{i-1} + lambda_i (.) x_i with row-stochastic w_i, made so by a
+ *   sigmoid on the non-zero entries of each row and a normalisation of the
+ *   row; Key design 2: w_i is tridiagonal (each pixel reads the three
+ *   adjacent pixels of the previous row or column), four scan directions;
+ *   Key design 3: the local variant propagates each of g groups on its own.
+ *   "GSPN-2: Efficient Parallel Sequence Modeling", Justification for
+ *   Channel-Agnostic Propagation: one tap set shared by all channels
+ *   (W kron I(C)) with per-channel gains lambda.
+ *
+ *   Readings this library fixes (the pages leave them open):
+ *   - weights: s_k = sigmoid(logit_k) for the taps whose source j+k-1 lies in
+ *     the line, w_k = s_k / sum of the valid s; taps outside the line have
+ *     w = 0 and their logits are ignored;
+ *   - h_{-1} = 0, so the first line of a scan (and of each local group) is
+ *     lambda * x;
+ *   - the four directions are merged by an unweighted sum;
+ *   - local groups cut the scan axis into g equal parts; taps still span the
+ *     whole line.
+ *
+ * Directions and coordinates.  Bit d of dir_mask enables direction d:
+ *   GSPN_DIR_T2B (lines = rows, top to bottom),    GSPN_DIR_B2T (bottom to top),
+ *   GSPN_DIR_L2R (lines = columns, left to right), GSPN_DIR_R2L (right to left).
+ * Tap k of a pixel reads the neighbour at offset k-1 along the line (column
+ * offset for row scans, row offset for column scans) in the previous line.
+ * The logits of a pixel's taps are stored at that pixel.
+ *
+ * Layouts (dense, row-major, element type `dtype`):
+ *   x, out, dout, dx   [B, C, H, W]
+ *   lambda, dlambda    [D, B, C, H, W]
+ *   logits, dlogits    [D, B, Cw, 3, H, W]   Cw = 1 when shared_weights, else C
+ * D = popcount(dir_mask); the D axis lists the enabled directions in the bit
+ * order T2B, B2T, L2R, R2L.  Arithmetic is fp32 throughout; bf16 outputs are
+ * rounded to nearest-even once, at the store.
+ *
+ * Ownership and streams.  Every pointer is a device pointer owned by the
+ * caller, including the workspace.  The library allocates no memory, keeps
+ * no state between calls and never synchronises the stream; calls are
+ * asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ * Outputs are overwritten, never accumulated into.  Inputs and outputs must
+ * not alias.  Concurrent calls on different streams may not share a
+ * workspace.
+ *
+ * Errors.  Arguments are checked on the host before any launch; a rejected
+ * call launches nothing and returns:
+ *   GSPN_ERR_INVALID_ARG  null descriptor or pointer, a dimension < 1, a
+ *                         dir_mask of 0 or with bits above 8, groups < 1, or
+ *                         groups not dividing the scan length of an enabled
+ *                         direction (H for T2B/B2T, W for L2R/R2L), or an
+ *                         element count that overflows;
+ *   GSPN_ERR_UNSUPPORTED  an unknown dtype;
+ *   GSPN_ERR_ALIGNMENT    a tensor pointer not 16-byte aligned;
+ *   GSPN_ERR_WORKSPACE    workspace smaller than gspn_workspace_size();
+ *   GSPN_ERR_CUDA         a CUDA runtime error at or before launch (the
+ *                         runtime's own error is left for cudaGetLastError).
+ * No exception or signal crosses the ABI.
+ */
+#ifndef GSPN_H_
+#define GSPN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GSPN_OK = 0,
+    GSPN_ERR_INVALID_ARG = 1,
+    GSPN_ERR_UNSUPPORTED = 2,
+    GSPN_ERR_ALIGNMENT = 3,
+    GSPN_ERR_WORKSPACE = 4,
+    GSPN_ERR_CUDA = 5,
+    GSPN_ERR_TIMEOUT = 6
+} gspn_status;
+
+typedef enum { GSPN_F32 = 0, GSPN_BF16 = 1 } gspn_dtype;
+
+enum { GSPN_DIR_T2B = 1, GSPN_DIR_B2T = 2, GSPN_DIR_L2R = 4, GSPN_DIR_R2L = 8 };
+
+typedef struct {
+    int64_t B, C, H, W;      /* batch, channels, rows, columns; each >= 1 */
+    uint32_t dir_mask;        /* OR of GSPN_DIR_* */
+    int32_t groups;           /* local groups along each scan axis; 1 = global scan */
+    int32_t shared_weights;   /* 1: one tap set per (b, pixel, direction) for all channels */
+    int32_t dtype;            /* gspn_dtype of every tensor */
+} gspn_desc;
+
+/* Bytes of device workspace a gspn_fwd (backward = 0) or gspn_bwd
+ * (backward = 1) call with this descriptor needs; 0 if none.  Returns 0 for a
+ * descriptor gspn_fwd/gspn_bwd would reject.  The workspace must be 256-byte
+ * aligned.  Its contents on entry are irrelevant. */
+size_t gspn_workspace_size(const gspn_desc* desc, int backward);
+
+/* Forward: out = sum over enabled directions d of h^(d), the line scan above
+ * ("Parallel Sequence Modeling via Generalized Spatial Propagation Network",
+ * Key designs 1-3; "GSPN-2: Efficient Parallel Sequence Modeling",
+ * channel-shared taps).  x: [B,C,H,W]; logits: [D,B,Cw,3,H,W] raw
+ * (pre-sigmoid) tap logits; lambda: [D,B,C,H,W]; out: [B,C,H,W].
+ * workspace/ws_bytes: device scratch of at least gspn_workspace_size(desc, 0)
+ * bytes (may be NULL when that is 0). */
+gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda, void* out,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Backward of gspn_fwd for upstream gradient dout ([B,C,H,W]): writes
+ * dx = dL/dx ([B,C,H,W], summed over directions), dlogits = dL/dlogits
+ * ([D,B,Cw,3,H,W]; summed over channels when shared_weights; zero for the
+ * logits of group-start lines and of taps outside the line) and
+ * dlambda = dL/dlambda ([D,B,C,H,W]).  The same kernel-launch design as the
+ * forward ("GSPN-2: Efficient Parallel Sequence Modeling", Backward
+ * Benchmark): each direction's lines are recomputed on chip and its adjoint
+ * h-gradient is run from the last line back to the first.
+ * workspace: at least gspn_workspace_size(desc, 1) bytes. */
+gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda,
+                     const void* dout, void* dx, void* dlogits, void* dlambda, void* workspace, size_t ws_bytes,
+                     void* stream);
+
+/* Number of kernel launches one gspn_fwd (backward = 0) / gspn_bwd
+ * (backward = 1) call with this descriptor issues; 0 for a descriptor the
+ * call would reject. */
+int gspn_launches_per_call(const gspn_desc* desc, int backward);
+
+/* Name of the forward (backward = 0) or backward (backward = 1) kernel
+ * variant this descriptor dispatches to, for logs and benchmarks; a static
+ * string, "invalid" for a rejected descriptor. */
+const char* gspn_variant_name(const gspn_desc* desc, int backward);
+
+/* Static, human-readable text of a status code. */
+const char* gspn_status_string(gspn_status status);
+
+/* Library version as MAJOR*10000 + MINOR*100 + PATCH. */
+int gspn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GSPN_H_ */

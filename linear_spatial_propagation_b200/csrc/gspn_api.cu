@@ -1,0 +1,185 @@
+// gspn_api.cu -- the C ABI of libgspn (declared in include/gspn.h): argument
+// checks, workspace sizing and dispatch to a kernel family.  Every check runs
+// on the host before any launch; no exception crosses the ABI.
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+
+#include "gspn_internal.h"
+
+namespace gspn {
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+constexpr int kMaxAttrSlots = 32;
+
+struct DevCache {
+    std::atomic<int> ready{0};
+    DeviceInfo info{};
+};
+DevCache g_dev[kMaxDevices];
+std::atomic<int> g_attr[kMaxDevices][kMaxAttrSlots];
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+gspn_status validate(const gspn_desc* d, Problem* p) {
+    if (!d) return GSPN_ERR_INVALID_ARG;
+    if (d->B < 1 || d->C < 1 || d->H < 1 || d->W < 1) return GSPN_ERR_INVALID_ARG;
+    if ((d->dir_mask & 15u) == 0 || (d->dir_mask & ~15u)) return GSPN_ERR_INVALID_ARG;
+    if (d->groups < 1) return GSPN_ERR_INVALID_ARG;
+    if ((d->dir_mask & 3u) && d->H % d->groups) return GSPN_ERR_INVALID_ARG;
+    if ((d->dir_mask & 12u) && d->W % d->groups) return GSPN_ERR_INVALID_ARG;
+    if (d->dtype != GSPN_F32 && d->dtype != GSPN_BF16) return GSPN_ERR_UNSUPPORTED;
+    // the kernels index a plane with 32-bit ints and tensors with 64-bit ones
+    if (d->H > (1 << 20) || d->W > (1 << 20) || d->H * d->W > (int64_t)1 << 30) return GSPN_ERR_INVALID_ARG;
+    if (d->B > (1 << 30) || d->C > (1 << 30)) return GSPN_ERR_INVALID_ARG;
+    const int D = __builtin_popcount(d->dir_mask & 15u);
+    const int64_t HW = d->H * d->W;
+    if (d->B * d->C > ((int64_t)1 << 40) / HW / (D * 3)) return GSPN_ERR_INVALID_ARG;
+    if (p) {
+        std::memset(p, 0, sizeof(*p));
+        p->d = *d;
+        p->g.B = (int)d->B;
+        p->g.C = (int)d->C;
+        p->g.H = (int)d->H;
+        p->g.W = (int)d->W;
+        p->g.D = D;
+        int s = 0;
+        for (int k = 0; k < 4; ++k)
+            if (d->dir_mask & (1u << k)) p->g.dirs[s++] = k;
+        p->g.groups = d->groups;
+        p->g.shared = d->shared_weights ? 1 : 0;
+        p->planes = d->B * d->C;
+        p->HW = HW;
+        p->elt = d->dtype == GSPN_F32 ? 4 : 2;
+    }
+    return GSPN_OK;
+}
+
+gspn_status check_ptrs(std::initializer_list<const void*> ptrs) {
+    for (const void* q : ptrs)
+        if (!q) return GSPN_ERR_INVALID_ARG;
+    for (const void* q : ptrs)
+        if (!aligned16(q)) return GSPN_ERR_ALIGNMENT;
+    return GSPN_OK;
+}
+
+gspn_status check_ws(void* ws, size_t have, size_t need) {
+    if (need == 0) return GSPN_OK;
+    if (!ws || have < need) return GSPN_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(ws) % kWsAlign) return GSPN_ERR_ALIGNMENT;
+    return GSPN_OK;
+}
+
+}  // namespace
+
+cudaError_t device_info(DeviceInfo* out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    DevCache& c = g_dev[dev];
+    if (!c.ready.load(std::memory_order_acquire)) {
+        DeviceInfo info;
+        e = cudaDeviceGetAttribute(&info.sm_count, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = cudaDeviceGetAttribute(&info.max_smem_optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+        if (e != cudaSuccess) return e;
+        c.info = info;
+        c.ready.store(1, std::memory_order_release);
+    }
+    *out = c.info;
+    return cudaSuccess;
+}
+
+cudaError_t ensure_smem_attr(const void* fn, int bytes, int slot) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices || slot < 0 || slot >= kMaxAttrSlots) return cudaErrorInvalidValue;
+    std::atomic<int>& a = g_attr[dev][slot];
+    if (a.load(std::memory_order_acquire) >= bytes) return cudaSuccess;
+    // always raise to the device maximum once, so later calls need no attribute change
+    DeviceInfo di;
+    e = device_info(&di);
+    if (e != cudaSuccess) return e;
+    const int want = bytes > di.max_smem_optin ? bytes : di.max_smem_optin;
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, want);
+    if (e != cudaSuccess) return e;
+    a.store(want, std::memory_order_release);
+    return cudaSuccess;
+}
+
+}  // namespace gspn
+
+using namespace gspn;
+
+extern "C" {
+
+int gspn_version(void) { return 100; }
+
+const char* gspn_status_string(gspn_status s) {
+    switch (s) {
+    case GSPN_OK: return "ok";
+    case GSPN_ERR_INVALID_ARG: return "invalid argument";
+    case GSPN_ERR_UNSUPPORTED: return "unsupported configuration";
+    case GSPN_ERR_ALIGNMENT: return "pointer not aligned (tensors: 16 bytes, workspace: 256 bytes)";
+    case GSPN_ERR_WORKSPACE: return "workspace missing or too small";
+    case GSPN_ERR_CUDA: return "CUDA runtime error";
+    case GSPN_ERR_TIMEOUT: return "device-side wait timed out";
+    default: return "unknown status";
+    }
+}
+
+size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
+    Problem p;
+    if (validate(desc, &p) != GSPN_OK) return 0;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess) return 0;
+    return backward ? generic_bwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
+}
+
+int gspn_launches_per_call(const gspn_desc* desc, int backward) {
+    Problem p;
+    if (validate(desc, &p) != GSPN_OK) return 0;
+    return backward ? generic_bwd_launches(p) : 1;
+}
+
+const char* gspn_variant_name(const gspn_desc* desc, int backward) {
+    Problem p;
+    if (validate(desc, &p) != GSPN_OK) return "invalid";
+    return backward ? "generic_bwd" : "generic_fwd";
+}
+
+gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda, void* out,
+                     void* workspace, size_t ws_bytes, void* stream) {
+    Problem p;
+    gspn_status st = validate(desc, &p);
+    if (st != GSPN_OK) return st;
+    st = check_ptrs({x, logits, lambda, out});
+    if (st != GSPN_OK) return st;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, generic_fwd_workspace(p, dev));
+    if (st != GSPN_OK) return st;
+    return generic_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda,
+                     const void* dout, void* dx, void* dlogits, void* dlambda, void* workspace, size_t ws_bytes,
+                     void* stream) {
+    Problem p;
+    gspn_status st = validate(desc, &p);
+    if (st != GSPN_OK) return st;
+    st = check_ptrs({x, logits, lambda, dout, dx, dlogits, dlambda});
+    if (st != GSPN_OK) return st;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
+    st = check_ws(workspace, ws_bytes, generic_bwd_workspace(p, dev));
+    if (st != GSPN_OK) return st;
+    return generic_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
+                       static_cast<cudaStream_t>(stream));
+}
+
+}  // extern "C"

@@ -1,0 +1,58 @@
+// gspn_common.cuh -- device helpers shared by the libgspn kernels.
+//
+// Coordinates (GSPN, "Parallel Sequence Modeling via Generalized Spatial
+// Propagation Network", Key design 2: row and column line scans in four
+// directions).  For direction d, line i in scan order and position j along the
+// line, the image pixel (r, c) is
+//     T2B (i, j) -> (i, j)        B2T (i, j) -> (H-1-i, j)
+//     L2R (i, j) -> (j, i)        R2L (i, j) -> (j, W-1-i)
+// and tap k in {0,1,2} of position j reads position j+k-1 of line i-1.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace gspn {
+
+enum Dir { T2B = 0, B2T = 1, L2R = 2, R2L = 3 };
+
+__host__ __device__ __forceinline__ int scan_len(int d, int H, int W) { return d < 2 ? H : W; }
+__host__ __device__ __forceinline__ int line_len(int d, int H, int W) { return d < 2 ? W : H; }
+
+// offset r*W + c of scan coordinate (i, j) in direction d
+__host__ __device__ __forceinline__ int pix(int d, int H, int W, int i, int j) {
+    switch (d) {
+    case T2B: return i * W + j;
+    case B2T: return (H - 1 - i) * W + j;
+    case L2R: return j * W + i;
+    default: return j * W + (W - 1 - i);
+    }
+}
+
+// ---- element access ---------------------------------------------------------
+// bf16 <-> fp32: a bf16 value is the top 16 bits of the fp32 with the same value.
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t u) { return __uint_as_float(((uint32_t)u) << 16); }
+
+__device__ __forceinline__ float load_elt(const float* p, int64_t i) { return __ldg(p + i); }
+__device__ __forceinline__ float load_elt(const __nv_bfloat16* p, int64_t i) {
+    return bf16_bits_to_float(__ldg(reinterpret_cast<const unsigned short*>(p) + i));
+}
+__device__ __forceinline__ void store_elt(float* p, int64_t i, float v) { p[i] = v; }
+__device__ __forceinline__ void store_elt(__nv_bfloat16* p, int64_t i, float v) { p[i] = __float2bfloat16_rn(v); }
+
+// ---- gate ---------------------------------------------------------------------
+// Sigmoid of a tap logit (GSPN Key design 1: "sigmoid on the non-zero entries
+// of each row, then row normalisation").  __expf's error is a few ulp; the
+// result is exact 0 for logits below about -88.
+__device__ __forceinline__ float sigmoidf(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+struct Launch {
+    int B, C, H, W;
+    int D;            // number of enabled directions
+    int dirs[4];      // direction of each D slot, in bit order
+    int groups;
+    int shared;       // 1: logits have one channel (Cw = 1)
+};
+
+}  // namespace gspn

@@ -1,0 +1,362 @@
+// gspn_generic.cu -- the generic GSPN kernels: any B, C, H, W, dtype, direction
+// set, local-group count and weight mode.
+//
+// One warp owns one (b, c) plane.  For each enabled direction it walks the
+// lines in scan order ("Parallel Sequence Modeling via Generalized Spatial
+// Propagation Network", Key design 2: lines are sequential, the positions of
+// a line are independent); lane l computes positions l, l+32, ... of the
+// line.  The previous line lives in a per-warp shared-memory buffer with a
+// zero halo at both ends, so tap k of position j reads buffer slot j+k.  The
+// four directions are summed (the merge) into an fp32 plane accumulator that
+// lives in shared memory when it fits and in the workspace otherwise; the
+// plane is written once at the end.
+//
+// The tap weights are recomputed from the logits where they are used:
+// s_k = sigmoid(logit_k) for the taps whose source lies in the line,
+// w_k = s_k / sum of those s (Key design 1).
+#include "gspn_internal.h"
+
+namespace gspn {
+
+namespace {
+
+constexpr int kMaxWarps = 8;
+constexpr int kSmemBudget = 200 * 1024;
+
+struct FwdArgs {
+    Launch g;
+    const void* x;
+    const void* logits;
+    const void* lam;
+    void* out;
+    float* acc_ws;
+    int acc_in_smem;
+    int warps_per_cta;
+    int lstride;  // floats per line buffer (N_max + 2)
+};
+
+template <typename T>
+__global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_kernel(FwdArgs a) {
+    extern __shared__ float smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C;
+    const int64_t plane = (int64_t)blockIdx.x * a.warps_per_cta + warp;
+    if (plane >= (int64_t)B * C) return;
+    float* wsm = smem + (size_t)warp * (2 * a.lstride + (a.acc_in_smem ? HW : 0));
+    float* acc = a.acc_in_smem ? wsm + 2 * a.lstride : a.acc_ws + plane * HW;
+    const int64_t b = plane / C, c = plane % C, cw = a.g.shared ? 0 : c;
+    const int Cw = a.g.shared ? 1 : C;
+    const T* x = static_cast<const T*>(a.x) + plane * HW;
+
+    for (int slot = 0; slot < a.g.D; ++slot) {
+        const int d = a.g.dirs[slot];
+        const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
+        const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
+        const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+        float* hp = wsm;
+        float* hc = wsm + a.lstride;
+        if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
+        __syncwarp();
+        for (int i = 0; i < L; ++i) {
+            const bool carry = (i % seg) != 0;
+            for (int j = lane; j < N; j += 32) {
+                const int p = pix(d, H, W, i, j);
+                float v = load_elt(lam, p) * load_elt(x, p);
+                if (carry) {
+                    const float s0 = j > 0 ? sigmoidf(load_elt(lg, p)) : 0.f;
+                    const float s1 = sigmoidf(load_elt(lg, HW + p));
+                    const float s2 = j < N - 1 ? sigmoidf(load_elt(lg, 2 * HW + p)) : 0.f;
+                    const float num = s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2];
+                    v += num / (s0 + s1 + s2);
+                }
+                hc[j + 1] = v;
+                acc[p] = slot == 0 ? v : acc[p] + v;
+            }
+            __syncwarp();
+            float* t = hp; hp = hc; hc = t;
+        }
+    }
+    __syncwarp();
+    T* out = static_cast<T*>(a.out) + plane * HW;
+    for (int q = lane; q < HW; q += 32) store_elt(out, q, acc[q]);
+}
+
+struct BwdArgs {
+    Launch g;
+    const void* x;
+    const void* logits;
+    const void* lam;
+    const void* dout;
+    void* dx;
+    void* dlogits;
+    void* dlam;
+    float* hstore;   // [B*C][HW]: the current direction's lines, scan coordinates
+    float* dx_ws;    // [B*C][HW] when the dx accumulator does not fit in smem
+    float* dlog_ws;  // [D][B][3][HW] fp32 sums over channels (shared mode)
+    int acc_in_smem;
+    int warps_per_cta;
+    int lstride;
+};
+
+// Backward.  With a_i = dL/dh_i in scan coordinates:
+//   a_i[j] = dout_i[j] + sum_k w_{i+1}[j-k+1][k] a_{i+1}[j-k+1]   (no carry into
+//            a line whose successor starts a group),
+//   dx += lam a, dlam = x a, dw_k = a h_{i-1}[j+k-1],
+//   dlogit_k = s_k (1 - s_k) / S (dw_k - sum_m w_m dw_m)   (valid taps; 0 else).
+// The products w_k(i, j) a_i[j] of line i are kept in three shared line buffers
+// so that line i-1 picks up its carry with the transposed taps.
+template <typename T>
+__global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) {
+    extern __shared__ float smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C;
+    const int64_t plane = (int64_t)blockIdx.x * a.warps_per_cta + warp;
+    if (plane >= (int64_t)B * C) return;
+    const int ls = a.lstride;
+    float* wsm = smem + (size_t)warp * (6 * ls + (a.acc_in_smem ? HW : 0));
+    float* dxacc = a.acc_in_smem ? wsm + 6 * ls : a.dx_ws + plane * HW;
+    float* hst = a.hstore + plane * HW;
+    const int64_t b = plane / C, c = plane % C, cw = a.g.shared ? 0 : c;
+    const int Cw = a.g.shared ? 1 : C;
+    const T* x = static_cast<const T*>(a.x) + plane * HW;
+    const T* g = static_cast<const T*>(a.dout) + plane * HW;
+
+    for (int slot = 0; slot < a.g.D; ++slot) {
+        const int d = a.g.dirs[slot];
+        const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
+        const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
+        const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+        T* dlam = static_cast<T*>(a.dlam) + ((slot * (int64_t)B + b) * C + c) * HW;
+
+        // 1. recompute this direction's lines into hst (scan coordinates)
+        {
+            float* hp = wsm;
+            float* hc = wsm + ls;
+            if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
+            __syncwarp();
+            for (int i = 0; i < L; ++i) {
+                const bool carry = (i % seg) != 0;
+                for (int j = lane; j < N; j += 32) {
+                    const int p = pix(d, H, W, i, j);
+                    float v = load_elt(lam, p) * load_elt(x, p);
+                    if (carry) {
+                        const float s0 = j > 0 ? sigmoidf(load_elt(lg, p)) : 0.f;
+                        const float s1 = sigmoidf(load_elt(lg, HW + p));
+                        const float s2 = j < N - 1 ? sigmoidf(load_elt(lg, 2 * HW + p)) : 0.f;
+                        v += (s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2]) / (s0 + s1 + s2);
+                    }
+                    hc[j + 1] = v;
+                    hst[i * N + j] = v;
+                }
+                __syncwarp();
+                float* t = hp; hp = hc; hc = t;
+            }
+        }
+        // 2. reverse scan of the adjoint
+        float* qn = wsm;        // 3 buffers: products of line i+1
+        float* qc = wsm + 3 * ls;  // 3 buffers: products of line i
+        for (int q = lane; q < 6 * ls; q += 32) wsm[q] = 0.f;
+        __syncwarp();
+        for (int i = L - 1; i >= 0; --i) {
+            const bool carry_out = (i % seg) != 0;                 // line i reads line i-1
+            const bool carry_in = (i + 1 < L) && ((i + 1) % seg != 0);  // line i+1 read line i
+            for (int j = lane; j < N; j += 32) {
+                const int p = pix(d, H, W, i, j);
+                float av = load_elt(g, p);
+                if (carry_in) av += qn[j + 2] + qn[ls + j + 1] + qn[2 * ls + j];
+                const float lv = load_elt(lam, p), xv = load_elt(x, p);
+                dxacc[p] = slot == 0 ? lv * av : dxacc[p] + lv * av;
+                store_elt(dlam, p, xv * av);
+                float dl0 = 0.f, dl1 = 0.f, dl2 = 0.f, q0 = 0.f, q1 = 0.f, q2 = 0.f;
+                if (carry_out) {
+                    const float s0 = j > 0 ? sigmoidf(load_elt(lg, p)) : 0.f;
+                    const float s1 = sigmoidf(load_elt(lg, HW + p));
+                    const float s2 = j < N - 1 ? sigmoidf(load_elt(lg, 2 * HW + p)) : 0.f;
+                    const float r = 1.f / (s0 + s1 + s2);
+                    const float w0 = s0 * r, w1 = s1 * r, w2 = s2 * r;
+                    const float* hprev = hst + (i - 1) * N;
+                    const float dw0 = j > 0 ? av * hprev[j - 1] : 0.f;
+                    const float dw1 = av * hprev[j];
+                    const float dw2 = j < N - 1 ? av * hprev[j + 1] : 0.f;
+                    const float tw = w0 * dw0 + w1 * dw1 + w2 * dw2;
+                    dl0 = s0 * (1.f - s0) * r * (dw0 - tw);
+                    dl1 = s1 * (1.f - s1) * r * (dw1 - tw);
+                    dl2 = s2 * (1.f - s2) * r * (dw2 - tw);
+                    q0 = w0 * av; q1 = w1 * av; q2 = w2 * av;
+                }
+                qc[j + 1] = q0;
+                qc[ls + j + 1] = q1;
+                qc[2 * ls + j + 1] = q2;
+                if (a.g.shared) {
+                    if (carry_out) {
+                        float* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
+                        if (j > 0) atomicAdd(dw + p, dl0);
+                        atomicAdd(dw + HW + p, dl1);
+                        if (j < N - 1) atomicAdd(dw + 2 * HW + p, dl2);
+                    }
+                } else {
+                    T* dlg = static_cast<T*>(a.dlogits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+                    store_elt(dlg, p, dl0);
+                    store_elt(dlg, HW + p, dl1);
+                    store_elt(dlg, 2 * HW + p, dl2);
+                }
+            }
+            __syncwarp();
+            float* t = qn; qn = qc; qc = t;
+        }
+        __syncwarp();
+    }
+    T* dx = static_cast<T*>(a.dx) + plane * HW;
+    for (int q = lane; q < HW; q += 32) store_elt(dx, q, dxacc[q]);
+}
+
+__global__ void zero_f32_kernel(float* p, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = 0.f;
+}
+
+template <typename T>
+__global__ void convert_f32_kernel(const float* src, T* dst, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        store_elt(dst, i, src[i]);
+}
+
+struct Plan {
+    int wpc;          // warps per CTA
+    int acc_in_smem;
+    int lstride;
+    size_t smem;      // dynamic smem bytes per CTA
+};
+
+Plan plan_for(const Problem& p, const DeviceInfo& dev, int line_bufs) {
+    Plan pl;
+    const int nmax = p.g.H > p.g.W ? p.g.H : p.g.W;
+    pl.lstride = nmax + 2;
+    const size_t lines = (size_t)line_bufs * pl.lstride * sizeof(float);
+    const size_t acc = (size_t)p.HW * sizeof(float);
+    const size_t budget = dev.max_smem_optin < kSmemBudget ? (size_t)dev.max_smem_optin : (size_t)kSmemBudget;
+    if (lines + acc <= budget) {
+        pl.acc_in_smem = 1;
+        pl.wpc = (int)(budget / (lines + acc));
+    } else {
+        pl.acc_in_smem = 0;
+        pl.wpc = (int)(budget / lines);
+    }
+    if (pl.wpc > kMaxWarps) pl.wpc = kMaxWarps;
+    if (pl.wpc < 1) pl.wpc = 1;
+    if ((int64_t)pl.wpc > p.planes) pl.wpc = (int)p.planes;
+    pl.smem = (size_t)pl.wpc * (lines + (pl.acc_in_smem ? acc : 0));
+    return pl;
+}
+
+bool lines_fit(const Problem& p, const DeviceInfo& dev, int line_bufs) {
+    const int nmax = p.g.H > p.g.W ? p.g.H : p.g.W;
+    return (size_t)line_bufs * (nmax + 2) * sizeof(float) <= (size_t)dev.max_smem_optin;
+}
+
+gspn_status cuda_status(cudaError_t e) { return e == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA; }
+
+int64_t grid_for(int64_t n, int threads) {
+    int64_t g = (n + threads - 1) / threads;
+    if (g > 65535) g = 65535;
+    if (g < 1) g = 1;
+    return g;
+}
+
+}  // namespace
+
+size_t generic_fwd_workspace(const Problem& p, const DeviceInfo& dev) {
+    Plan pl = plan_for(p, dev, 2);
+    return pl.acc_in_smem ? 0 : align_up((size_t)p.planes * p.HW * sizeof(float), kWsAlign);
+}
+
+gspn_status generic_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
+                        const void* lam, void* out, void* ws, cudaStream_t s) {
+    if (!lines_fit(p, dev, 2)) return GSPN_ERR_UNSUPPORTED;
+    Plan pl = plan_for(p, dev, 2);
+    FwdArgs a;
+    a.g = p.g; a.x = x; a.logits = logits; a.lam = lam; a.out = out;
+    a.acc_ws = static_cast<float*>(ws);
+    a.acc_in_smem = pl.acc_in_smem; a.warps_per_cta = pl.wpc; a.lstride = pl.lstride;
+    const int64_t grid = (p.planes + pl.wpc - 1) / pl.wpc;
+    if (grid > 0x7fffffff) return GSPN_ERR_UNSUPPORTED;
+    const void* fn = p.d.dtype == GSPN_F32 ? (const void*)generic_fwd_kernel<float>
+                                           : (const void*)generic_fwd_kernel<__nv_bfloat16>;
+    cudaError_t e = ensure_smem_attr(fn, (int)pl.smem, p.d.dtype == GSPN_F32 ? 0 : 1);
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    if (p.d.dtype == GSPN_F32)
+        generic_fwd_kernel<float><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
+    else
+        generic_fwd_kernel<__nv_bfloat16><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
+    return cuda_status(cudaGetLastError());
+}
+
+namespace {
+struct BwdWs {
+    size_t hstore, dx_ws, dlog_ws, total;
+};
+BwdWs bwd_ws_layout(const Problem& p, const DeviceInfo& dev) {
+    Plan pl = plan_for(p, dev, 6);
+    BwdWs w;
+    const size_t plane_f = (size_t)p.planes * p.HW * sizeof(float);
+    w.hstore = 0;
+    size_t off = align_up(plane_f, kWsAlign);
+    w.dx_ws = off;
+    if (!pl.acc_in_smem) off += align_up(plane_f, kWsAlign);
+    w.dlog_ws = off;
+    if (p.g.shared) off += align_up((size_t)p.g.D * p.g.B * 3 * p.HW * sizeof(float), kWsAlign);
+    w.total = off;
+    return w;
+}
+}  // namespace
+
+size_t generic_bwd_workspace(const Problem& p, const DeviceInfo& dev) { return bwd_ws_layout(p, dev).total; }
+
+int generic_bwd_launches(const Problem& p) { return p.g.shared ? 3 : 1; }
+
+gspn_status generic_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
+                        const void* lam, const void* dout, void* dx, void* dlogits, void* dlam, void* ws,
+                        cudaStream_t s) {
+    if (!lines_fit(p, dev, 6)) return GSPN_ERR_UNSUPPORTED;
+    Plan pl = plan_for(p, dev, 6);
+    BwdWs lay = bwd_ws_layout(p, dev);
+    char* w = static_cast<char*>(ws);
+    BwdArgs a;
+    a.g = p.g; a.x = x; a.logits = logits; a.lam = lam; a.dout = dout;
+    a.dx = dx; a.dlogits = dlogits; a.dlam = dlam;
+    a.hstore = reinterpret_cast<float*>(w + lay.hstore);
+    a.dx_ws = reinterpret_cast<float*>(w + lay.dx_ws);
+    a.dlog_ws = reinterpret_cast<float*>(w + lay.dlog_ws);
+    a.acc_in_smem = pl.acc_in_smem; a.warps_per_cta = pl.wpc; a.lstride = pl.lstride;
+    const int64_t nlog = (int64_t)p.g.D * p.g.B * 3 * p.HW;
+    if (p.g.shared) {
+        zero_f32_kernel<<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(a.dlog_ws, nlog);
+        cudaError_t e0 = cudaGetLastError();
+        if (e0 != cudaSuccess) return GSPN_ERR_CUDA;
+    }
+    const int64_t grid = (p.planes + pl.wpc - 1) / pl.wpc;
+    if (grid > 0x7fffffff) return GSPN_ERR_UNSUPPORTED;
+    const void* fn = p.d.dtype == GSPN_F32 ? (const void*)generic_bwd_kernel<float>
+                                           : (const void*)generic_bwd_kernel<__nv_bfloat16>;
+    cudaError_t e = ensure_smem_attr(fn, (int)pl.smem, p.d.dtype == GSPN_F32 ? 2 : 3);
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    if (p.d.dtype == GSPN_F32)
+        generic_bwd_kernel<float><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
+    else
+        generic_bwd_kernel<__nv_bfloat16><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    if (p.g.shared) {
+        if (p.d.dtype == GSPN_F32)
+            convert_f32_kernel<float><<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(
+                a.dlog_ws, static_cast<float*>(dlogits), nlog);
+        else
+            convert_f32_kernel<__nv_bfloat16><<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(
+                a.dlog_ws, static_cast<__nv_bfloat16*>(dlogits), nlog);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    }
+    return GSPN_OK;
+}
+
+}  // namespace gspn

@@ -1,0 +1,44 @@
+// gspn_internal.h -- host-side interfaces between the C ABI (gspn_api.cu) and
+// the kernel families.  Not part of the public ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "../../include/gspn.h"
+#include "gspn_common.cuh"
+
+namespace gspn {
+
+constexpr size_t kWsAlign = 256;
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// Validated, normalised view of a descriptor.
+struct Problem {
+    gspn_desc d;
+    Launch g;
+    int64_t planes;   // B*C
+    int64_t HW;
+    size_t elt;       // bytes per element
+};
+
+// Device properties the dispatch needs (queried once per device).
+struct DeviceInfo {
+    int sm_count;
+    int max_smem_optin;   // bytes of dynamic shared memory a block may opt in to
+};
+cudaError_t device_info(DeviceInfo* out);
+
+// Sets the max-dynamic-smem attribute of `fn` once per device.
+cudaError_t ensure_smem_attr(const void* fn, int bytes, int slot);
+
+// ---- generic kernels (any shape, dtype, mode) ---------------------------------
+size_t generic_fwd_workspace(const Problem& p, const DeviceInfo& dev);
+gspn_status generic_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
+                        const void* lam, void* out, void* ws, cudaStream_t s);
+size_t generic_bwd_workspace(const Problem& p, const DeviceInfo& dev);
+int generic_bwd_launches(const Problem& p);
+gspn_status generic_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
+                        const void* lam, const void* dout, void* dx, void* dlogits, void* dlam, void* ws,
+                        cudaStream_t s);
+
+}  // namespace gspn

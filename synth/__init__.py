@@ -14,13 +14,15 @@ Draws (each tensor from its own child stream of ``SeedSequence(seed)``, spawned
 in the order x, lambda, logits, dout):
 
 * x ~ N(0, 1), lambda ~ U(0, 1), logits ~ N(0, logit_std), dout ~ N(0, 1),
-  all drawn in float32 by numpy's PCG64 generator;
+  all drawn in float32 by numpy's PCG64 generator, in chunks of 2**22
+  elements, chunk q from child q of the tensor's stream;
 * bf16 tensors are the float32 draws rounded to nearest-even bf16 and are
   stored as ``uint16`` bit patterns (numpy has no bf16 dtype).
 """
 from __future__ import annotations
 
 import dataclasses
+import os
 from typing import Dict, Optional
 
 import numpy as np
@@ -103,18 +105,36 @@ def bf16_bits_to_f32(b: np.ndarray) -> np.ndarray:
     return (np.ascontiguousarray(b, dtype=np.uint16).astype(np.uint32) << np.uint32(16)).view(np.float32)
 
 
-def _draw(rng: np.random.Generator, kind: str, shape: tuple, scale: float = 1.0,
-          chunk: int = 1 << 26) -> np.ndarray:
+CHUNK = 1 << 22
+
+
+def _fill(seq: np.random.SeedSequence, kind: str, shape: tuple, scale: float, bf16: bool) -> np.ndarray:
+    """Draw a tensor in chunks of CHUNK elements; chunk q comes from child q of
+    ``seq``, so the values do not depend on how many threads draw them."""
     n = int(np.prod(shape))
-    out = np.empty(n, dtype=np.float32)
-    for s in range(0, n, chunk):
-        e = min(n, s + chunk)
+    out = np.empty(n, dtype=np.uint16 if bf16 else np.float32)
+    nchunks = max(1, (n + CHUNK - 1) // CHUNK)
+    kids = seq.spawn(nchunks)
+
+    def work(q):
+        s, e = q * CHUNK, min(n, (q + 1) * CHUNK)
+        if e <= s:
+            return
+        rng = np.random.Generator(np.random.PCG64(kids[q]))
         if kind == "normal":
-            rng.standard_normal(e - s, dtype=np.float32, out=out[s:e])
+            v = rng.standard_normal(e - s, dtype=np.float32)
             if scale != 1.0:
-                out[s:e] *= np.float32(scale)
+                v *= np.float32(scale)
         else:
-            rng.random(e - s, dtype=np.float32, out=out[s:e])
+            v = rng.random(e - s, dtype=np.float32)
+        out[s:e] = f32_to_bf16_bits(v) if bf16 else v
+
+    if nchunks == 1:
+        work(0)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(max_workers=min(nchunks, os.cpu_count() or 1)) as ex:
+            list(ex.map(work, range(nchunks)))
     return out.reshape(shape)
 
 
@@ -129,15 +149,14 @@ def make_inputs(w: Workload, with_dout: Optional[bool] = None) -> Dict[str, np.n
         with_dout = w.backward
     kids = np.random.SeedSequence(w.seed).spawn(4)
     shp = w.shapes()
+    bf = w.dtype == "bf16"
     out = {
-        "x": _draw(np.random.Generator(np.random.PCG64(kids[0])), "normal", shp["x"]),
-        "lam": _draw(np.random.Generator(np.random.PCG64(kids[1])), "uniform", shp["lam"]),
-        "logits": _draw(np.random.Generator(np.random.PCG64(kids[2])), "normal", shp["logits"], w.logit_std),
+        "x": _fill(kids[0], "normal", shp["x"], 1.0, bf),
+        "lam": _fill(kids[1], "uniform", shp["lam"], 1.0, bf),
+        "logits": _fill(kids[2], "normal", shp["logits"], w.logit_std, bf),
     }
     if with_dout:
-        out["dout"] = _draw(np.random.Generator(np.random.PCG64(kids[3])), "normal", shp["dout"])
-    if w.dtype == "bf16":
-        out = {k: f32_to_bf16_bits(v) for k, v in out.items()}
+        out["dout"] = _fill(kids[3], "normal", shp["dout"], 1.0, bf)
     return out
 
 

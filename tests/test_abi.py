@@ -1,0 +1,106 @@
+"""CPU checks of the C-ABI library: it loads, exports every symbol that
+include/gspn.h declares, and rejects bad arguments on the host (no GPU, no
+compute)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import linear_spatial_propagation_b200 as lsp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "gspn.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(gspn_\w+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    assert declared_functions() == sorted(lsp.EXPORTS)
+
+
+def test_library_loads_and_exports_every_declared_symbol():
+    lib = lsp.load()
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings():
+    assert lsp.gspn_version() >= 100
+    assert lsp.gspn_status_string(0) == "ok"
+    for s in range(1, 7):
+        assert lsp.gspn_status_string(s) and lsp.gspn_status_string(s) != "unknown status"
+    assert lsp.gspn_status_string(99) == "unknown status"
+
+
+A = 1 << 20  # a 16-byte aligned fake device address: never dereferenced on rejected calls
+
+
+def fwd(desc, x=A, lg=A, lam=A, out=A, ws=0, nbytes=0):
+    return lsp.gspn_fwd(desc, x, lg, lam, out, ws, nbytes, 0)
+
+
+def bwd(desc, ptrs=(A,) * 7):
+    return lsp.gspn_bwd(desc, *ptrs, 0, 0, 0)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(B=0), dict(C=0), dict(H=0), dict(W=-1), dict(dir_mask=0), dict(dir_mask=16), dict(dir_mask=33),
+    dict(groups=0), dict(groups=3),                      # 3 does not divide 8
+    dict(H=6, W=8, groups=4, dir_mask=1),                # T2B needs g | H
+    dict(H=8, W=6, groups=4, dir_mask=4),                # L2R needs g | W
+    dict(H=1 << 21),
+])
+def test_invalid_descriptors_are_rejected_before_launch(kw):
+    base = dict(B=2, C=3, H=8, W=8, dir_mask=15, groups=1, shared=False, dtype="bf16")
+    base.update(kw)
+    d = lsp.make_desc(**base)
+    assert fwd(d) == 1
+    assert bwd(d) == 1
+    assert lsp.gspn_workspace_size(d, 0) == 0 and lsp.gspn_workspace_size(d, 1) == 0
+    assert lsp.gspn_launches_per_call(d, 0) == 0
+    assert lsp.gspn_variant_name(d, 0) == "invalid"
+
+
+def test_groups_only_constrain_enabled_scan_axes():
+    # g = 4 divides H = 8 but not W = 6; a column-free direction set is fine
+    d = lsp.make_desc(1, 1, 8, 6, dir_mask=1 | 2, groups=4)
+    assert lsp.gspn_launches_per_call(d, 0) >= 1
+
+
+def test_unknown_dtype_is_unsupported():
+    d = lsp.make_desc(1, 1, 4, 4, 15, 1, False, 7)
+    assert fwd(d) == 2
+
+
+def test_null_descriptor_and_pointers():
+    lib = lsp.load()
+    assert lib.gspn_fwd(None, A, A, A, A, None, 0, None) == 1
+    d = lsp.make_desc(1, 2, 4, 4)
+    assert fwd(d, x=0) == 1
+    assert fwd(d, out=0) == 1
+    for q in range(7):
+        p = [A] * 7
+        p[q] = 0
+        assert bwd(d, tuple(p)) == 1
+
+
+def test_misaligned_pointers():
+    d = lsp.make_desc(1, 2, 4, 4)
+    assert fwd(d, lam=A + 8) == 3
+    assert fwd(d, out=A + 2) == 3
+    p = [A] * 7
+    p[5] = A + 4
+    assert bwd(d, tuple(p)) == 3
+
+
+def test_python_helpers_raise_on_error():
+    with pytest.raises(lsp.GspnError) as e:
+        st = fwd(lsp.make_desc(1, 1, 4, 4, dir_mask=0))
+        raise lsp.GspnError(st, "gspn_fwd")
+    assert e.value.status == 1
