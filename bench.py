@@ -54,6 +54,9 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target length of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--pass", dest="passes", default="both", choices=["both", "fwd", "bwd"],
+                    help="profiling aid: time only one pass (the JSON line then covers that pass)")
+    ap.add_argument("--batch", type=int, default=0, help="profiling aid: override B (0 = the workload's)")
     return ap.parse_args()
 
 
@@ -212,10 +215,11 @@ def run_reference(args, w):
     return 0
 
 
-def config_of(w, n):
+def config_of(w, n, passes="both"):
     return {"workload": w.name, "B": w.B, "C": w.C, "H": w.H, "W": w.W,
             "directions": "+".join(n_ for b, n_ in ((1, "T2B"), (2, "B2T"), (4, "L2R"), (8, "R2L")) if w.dir_mask & b),
-            "groups": w.groups, "shared_taps": w.shared, "io_dtype": w.dtype, "pass": "fwd+bwd",
+            "groups": w.groups, "shared_taps": w.shared, "io_dtype": w.dtype,
+            "pass": {"both": "fwd+bwd", "fwd": "fwd", "bwd": "bwd"}[passes],
             "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"}
 
 
@@ -287,9 +291,13 @@ def run_gpu(args, w):
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
         return float(t.item())
 
+    do_f = args.passes in ("both", "fwd")
+    do_b = args.passes in ("both", "bwd")
     for _ in range(max(3, args.warmup)):
-        fwd()
-        bwd()
+        if do_f:
+            fwd()
+        if do_b:
+            bwd()
     barrier()
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
@@ -300,9 +308,11 @@ def run_gpu(args, w):
     e_start.record(stream)
     for k in range(K):
         ev[k][0].record(stream)
-        fwd()
+        if do_f:
+            fwd()
         ev[k][1].record(stream)
-        bwd()
+        if do_b:
+            bwd()
         ev[k][2].record(stream)
     e_end.record(stream)
     barrier()
@@ -313,7 +323,7 @@ def run_gpu(args, w):
     ms = total_ms / K
 
     # end to end: pinned host inputs -> device -> fwd + bwd -> results back to pinned host
-    E = max(1, args.e2e_steps)
+    E = args.e2e_steps
     hout = torch.empty(out.shape, dtype=tdt).pin_memory()
     hgrads = [torch.empty(g.shape, dtype=tdt).pin_memory() for g in grads]
     h2d = sum(t.numel() * t.element_size() for t in h.values())
@@ -324,25 +334,31 @@ def run_gpu(args, w):
     for _ in range(E):
         for k in ("x", "lam", "logits", "dout"):
             d[k].copy_(h[k], non_blocking=True)
-        fwd()
-        bwd()
+        if do_f:
+            fwd()
+        if do_b:
+            bwd()
         hout.copy_(out, non_blocking=True)
         for hg, g in zip(hgrads, grads):
             hg.copy_(g, non_blocking=True)
     e2[1].record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e2[0].elapsed_time(e2[1]) / E)
+    e2e_ms = max_over_ranks(e2[0].elapsed_time(e2[1]) / E) if E > 0 else None
 
     fb, bb = pass_bytes(w)
+    if not do_f:
+        fb = 0
+    if not do_b:
+        bb = 0
     peak, peak_src = measured_peaks()
     n_gpu = world
     value = (fb + bb) * n_gpu / (ms * 1e-3) / 1e9
     pixch = w.B * w.C * w.H * w.W
-    fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9
-    bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9
+    fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9 if fb else 0.0
+    bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9 if bb else 0.0
     dom = "bwd" if bwd_ms >= fwd_ms else "fwd"
     dom_gbs = bwd_gbs if dom == "bwd" else fwd_gbs
-    launches = K * (lsp.gspn_launches_per_call(desc, 0) + lsp.gspn_launches_per_call(desc, 1))
+    launches = K * (lsp.gspn_launches_per_call(desc, 0) * do_f + lsp.gspn_launches_per_call(desc, 1) * do_b)
 
     if rank == 0:
         cpu = None
@@ -359,21 +375,22 @@ def run_gpu(args, w):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_gpu, "steps": K,
             "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded numpy PCG64, per-rank seed)",
-            "config": config_of(w, n_gpu),
+            "config": config_of(w, n_gpu, args.passes),
             "pct_of_peak": 100.0 * value / n_gpu / peak,
             "gpix_ch_per_s": pixch * n_gpu / (ms * 1e-3) / 1e9,
             "fwd": {"ms": fwd_ms, "GB/s": fwd_gbs, "pct_of_peak": 100.0 * fwd_gbs / peak,
-                    "gpix_ch_per_s": pixch / (fwd_ms * 1e-3) / 1e9, "bytes": fb,
+                    "gpix_ch_per_s": pixch / (fwd_ms * 1e-3) / 1e9 if fb else 0.0, "bytes": fb,
                     "kernel": lsp.gspn_variant_name(desc, 0)},
             "bwd": {"ms": bwd_ms, "GB/s": bwd_gbs, "pct_of_peak": 100.0 * bwd_gbs / peak,
-                    "gpix_ch_per_s": pixch / (bwd_ms * 1e-3) / 1e9, "bytes": bb,
+                    "gpix_ch_per_s": pixch / (bwd_ms * 1e-3) / 1e9 if bb else 0.0, "bytes": bb,
                     "kernel": lsp.gspn_variant_name(desc, 1)},
             "roofline": {"bound": "hbm", "achieved": dom_gbs, "peak": peak, "unit": "GB/s",
                          "frac": dom_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
                          "kernel": lsp.gspn_variant_name(desc, 1 if dom == "bwd" else 0),
                          "traffic": ncu_traffic(dom, w)},
-            "e2e": {"value": (fb + bb) * n_gpu / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "e2e": ({"value": (fb + bb) * n_gpu / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+                    if e2e_ms else None),
             "gpu_launches": launches,
             "clocks": clk,
             "cpu_baseline": cpu,
@@ -390,6 +407,8 @@ def main():
     w = synth.WORKLOADS[args.workload]
     if not w.backward:
         w = w.replace(backward=True)
+    if args.batch:
+        w = w.replace(B=args.batch, name=f"{w.name}@B{args.batch}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)

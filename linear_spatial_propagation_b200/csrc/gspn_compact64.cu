@@ -1,0 +1,458 @@
+// gspn_compact64.cu -- fast forward for the compact (channel-shared taps)
+// four-direction scan of 64x64 bf16 planes, the 1K foundation shape
+// (C-GSPN, "Scaling Parallel Sequence Models to Vision Foundation Models":
+// batch 32, C = 1152, 1024 px at patch 16).
+//
+// Operator: "Parallel Sequence Modeling via Generalized Spatial Propagation
+// Network" Key designs 1-3 (row-stochastic 3-tap line scan in four directions,
+// summed; local groups) with the channel-shared taps of "GSPN-2: Efficient
+// Parallel Sequence Modeling" (Justification for Channel-Agnostic
+// Propagation: W kron I(C), per-channel lambda).
+//
+// Design (B200):
+// * The tap weights depend only on (b, pixel, direction).  A small pre-kernel
+//   turns the logits into normalised (w0, w2) pairs once per (b, pixel,
+//   direction) -- w1 = 1 - w0 - w2 -- laid out in scan order so that each
+//   scan step reads one contiguous 256-byte row per half-warp.  The main
+//   kernel reads them through L1 and reuses them for every channel.
+// * One warp processes two channels of one batch image at a time (16 lanes
+//   per 64-wide line, 4 positions per lane).  The two directions of a pair
+//   (left->right with right->left, top->bottom with bottom->top) advance
+//   together: lane values are float2 (one direction per half) and the update
+//   uses the packed fp32x2 FMA of sm_100.
+// * Update in difference form, h'[p] = h[p] + lambda x + w2 (h[p+1] - h[p])
+//   - w0 (h[p] - h[p-1]), equal to w0 h[p-1] + w1 h[p] + w2 h[p+1] + lambda x
+//   for w1 = 1 - w0 - w2; the line ends have w0 = 0 / w2 = 0.  Neighbours
+//   across lanes come from two shuffles per direction and step.
+// * Row pass first (left->right and right->left over columns), then column
+//   pass (top->bottom and bottom->top over rows).  The row pass leaves its
+//   sum in an fp32 plane in shared memory (Hacc); the column pass adds its two
+//   directions and writes each output row once, 128 contiguous bytes per line.
+//   In each pass the direction that reaches a pixel first stores, the second
+//   adds, so every Hacc element is written/read the minimum number of times.
+// * All x / lambda traffic is streamed by TMA into a per-warp ring of 8 KB
+//   stages (8 scan steps each): column chunks (8 columns x 64 rows) for the
+//   row pass and row chunks (64 columns x 8 rows) for the column pass.  A
+//   stage is copied to registers at its start and immediately refilled, so
+//   NST-1 stages (16 KB) per warp stay in flight.  Column chunks are fetched
+//   as four boxes of every 4th row (element stride 4), which lays rows
+//   4t..4t+3 of lane t into four separate 512-byte slices: the 16-byte reads
+//   of 8 lanes then hit 8 consecutive bank quads.
+// * Hacc uses an XOR layout of 8-byte units, conflict-free both for the row
+//   pass (each lane stores its 4 rows at one column pair) and for the column
+//   pass (each lane reads 4 columns of one row).
+// * Every mbarrier wait is bounded (2 s); on expiry the warp records an
+//   error word in the workspace, drains its outstanding copies and returns.
+#include "gspn_internal.h"
+#include "gspn_tma.cuh"
+
+namespace gspn {
+
+namespace {
+
+constexpr int S = 64;         // H = W
+constexpr int LPL = 16;       // lanes per line
+constexpr int NWARP = 4;      // warps per CTA (one CTA per SM)
+constexpr int NST = 3;        // ring stages per warp
+constexpr int STAGE = 8192;   // bytes per stage: 4 boxes x 2 planes x 1 KB
+constexpr int BOX = 2048;     // bytes per box (2 planes)
+constexpr int HACC_PLANE = S * S * 4;
+constexpr int WARP_BYTES = NST * STAGE + 2 * HACC_PLANE;
+constexpr int BAR_BYTES = 8 * NST;
+constexpr int SMEM_BYTES = 1024 + NWARP * WARP_BYTES + NWARP * BAR_BYTES;
+constexpr int CHUNKS_PER_UNIT = 16;  // 8 column chunks + 8 row chunks
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+constexpr unsigned FULL = 0xffffffffu;
+
+// ---- weights pre-kernel ----------------------------------------------------------
+// wtab[((b*2 + pass)*64 + s)*64 + p*16 + t] = (-w0_A, -w0_B, w2_A, w2_B) of line
+// position j = 4t + p at scan step s, where pass 0 pairs A = left->right (line s
+// = column s) with B = right->left (column 63-s), positions = rows; pass 1 pairs
+// A = top->bottom (row s) with B = bottom->top (row 63-s), positions = columns.
+template <typename T>
+__device__ __forceinline__ void gate_pair(const T* lg, int pix, int j, float* w0, float* w2) {
+    const float s0 = j > 0 ? sigmoidf(load_elt(lg, pix)) : 0.f;
+    const float s1 = sigmoidf(load_elt(lg, S * S + pix));
+    const float s2 = j < S - 1 ? sigmoidf(load_elt(lg, 2 * S * S + pix)) : 0.f;
+    const float r = 1.f / (s0 + s1 + s2);
+    *w0 = s0 * r;
+    *w2 = s2 * r;
+}
+
+template <typename T>
+__global__ void c64_weights_kernel(const T* __restrict__ logits, float4* __restrict__ wtab, int* err, int B) {
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx == 0) *err = 0;
+    if (idx >= B * 2 * S * S) return;
+    const int j = idx & 63, s = (idx >> 6) & 63, pass = (idx >> 12) & 1, b = idx >> 13;
+    const int slotA = pass ? 0 : 2, slotB = pass ? 1 : 3;
+    const int pixA = pass ? s * S + j : j * S + s;
+    const int pixB = pass ? (S - 1 - s) * S + j : j * S + (S - 1 - s);
+    float w0a, w2a, w0b, w2b;
+    gate_pair(logits + (size_t)(slotA * B + b) * 3 * S * S, pixA, j, &w0a, &w2a);
+    gate_pair(logits + (size_t)(slotB * B + b) * 3 * S * S, pixB, j, &w0b, &w2b);
+    const int t = j >> 2, p = j & 3;
+    wtab[((size_t)(b * 2 + pass) * S + s) * S + p * LPL + t] = make_float4(-w0a, -w0b, w2a, w2b);
+}
+
+// ---- helpers ----------------------------------------------------------------------
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+// element e (0..7) of 8 packed bf16
+__device__ __forceinline__ float bf_at(const uint4& v, int e) {
+    const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
+    return (e & 1) ? bf_hi(w) : bf_lo(w);
+}
+__device__ __forceinline__ float bf_at2(const uint2& v, int e) {
+    const uint32_t w = e < 2 ? v.x : v.y;
+    return (e & 1) ? bf_hi(w) : bf_lo(w);
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t a) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ uint2 lds64(uint32_t a) {
+    uint2 v;
+    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ float2 lds64f(uint32_t a) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
+    return v;
+}
+__device__ __forceinline__ void sts64f(uint32_t a, float2 v) {
+    asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(a), "f"(v.x), "f"(v.y) : "memory");
+}
+__device__ __forceinline__ void stg_cs64(void* p, uint32_t a, uint32_t b) {
+    asm volatile("st.global.cs.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+}
+__device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// Hacc address (bytes from the plane base) of the 8-byte unit holding columns
+// 2u, 2u+1 of row r: unit index XORed with (r / 4) mod 16 and with bit 4 of u.
+__device__ __forceinline__ uint32_t hacc_off(int r, int u) {
+    return (uint32_t)(r * 256 + ((u ^ ((r >> 2) & 15) ^ ((u >> 4) & 1)) << 3));
+}
+
+struct C64Args {
+    const float4* wtab;
+    __nv_bfloat16* out;
+    int* err;
+    int B, C, seg;
+    int units;  // B * C / 2
+};
+
+// a - b, exactly rounded (sm_100 has packed add and fma but no packed subtract)
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
+
+// One scan step for one lane: 4 positions, two directions packed in float2.
+// w[p] = (-w0_A, -w0_B, w2_A, w2_B).
+__device__ __forceinline__ void scan_step(float2 (&h)[4], const float2 (&xl)[4], const float2 (&ll)[4],
+                                          const float4 (&w)[4]) {
+    float2 hl, hr;
+    hl.x = __shfl_up_sync(FULL, h[3].x, 1, LPL);
+    hl.y = __shfl_up_sync(FULL, h[3].y, 1, LPL);
+    hr.x = __shfl_down_sync(FULL, h[0].x, 1, LPL);
+    hr.y = __shfl_down_sync(FULL, h[0].y, 1, LPL);
+    float2 D[5];
+    D[0] = sub2(h[0], hl);
+    D[1] = sub2(h[1], h[0]);
+    D[2] = sub2(h[2], h[1]);
+    D[3] = sub2(h[3], h[2]);
+    D[4] = sub2(hr, h[3]);
+#pragma unroll
+    for (int p = 0; p < 4; ++p) {
+        float2 v = __ffma2_rn(ll[p], xl[p], h[p]);
+        v = __ffma2_rn(make_float2(w[p].z, w[p].w), D[p + 1], v);
+        v = __ffma2_rn(make_float2(w[p].x, w[p].y), D[p], v);
+        h[p] = v;
+    }
+}
+
+__global__ void __launch_bounds__(NWARP * 32, 1)
+    c64_fwd_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
+                   const __grid_constant__ CUtensorMap tm_xr, const __grid_constant__ CUtensorMap tm_lr,
+                   const C64Args a) {
+    extern __shared__ unsigned char smem_raw[];
+    const uint32_t sbase = (tma::smem_u32(smem_raw) + 1023u) & ~1023u;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int g = lane >> 4, t = lane & 15;
+    const uint32_t ring = sbase + warp * WARP_BYTES;
+    const uint32_t hacc = ring + NST * STAGE + g * HACC_PLANE;
+    const uint32_t bar0 = sbase + NWARP * WARP_BYTES + warp * BAR_BYTES;
+    const int wid = blockIdx.x * NWARP + warp;
+    const int wstride = gridDim.x * NWARP;
+    const int half_c = a.C >> 1;
+    if (wid >= a.units) return;
+
+    if (lane == 0) {
+        for (int k = 0; k < NST; ++k) tma::mbar_init(bar0 + 8 * k, 1);
+        tma::fence_barrier_init();
+        tma::prefetch_map(&tm_xc);
+        tma::prefetch_map(&tm_lc);
+        tma::prefetch_map(&tm_xr);
+        tma::prefetch_map(&tm_lr);
+    }
+    __syncwarp();
+
+    // Issue chunk k of this warp's sequence (lane 0 only): unit wid + (k/16)*wstride,
+    // chunk k%16 of it (0..7: column chunks, 8..15: row chunks).
+    auto issue = [&](int k) {
+        const int unit = wid + (k / CHUNKS_PER_UNIT) * wstride;
+        if (unit >= a.units) return;
+        const int local = k % CHUNKS_PER_UNIT, st = k % NST;
+        const uint32_t dst = ring + st * STAGE, bar = bar0 + 8 * st;
+        const int b = unit / half_c, c0 = (unit - b * half_c) * 2;
+        const int plane = b * a.C + c0;
+        const int BC = a.B * a.C;
+        tma::mbar_expect_tx(bar, STAGE);
+        if (local < 8) {
+            const int q = local;
+            // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at 8(7-q)..
+            for (int r = 0; r < 4; ++r) {
+                tma::load_3d(dst + 0 * BOX + r * 512, &tm_xc, 8 * q, r, plane, bar);
+                tma::load_3d(dst + 1 * BOX + r * 512, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
+                tma::load_3d(dst + 2 * BOX + r * 512, &tm_xc, 8 * (7 - q), r, plane, bar);
+                tma::load_3d(dst + 3 * BOX + r * 512, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
+            }
+        } else {
+            const int q = local - 8;
+            // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 56-8q..
+            tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
+            tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, 0 * BC + plane, bar);
+            tma::load_3d(dst + 2 * BOX, &tm_xr, 0, 56 - 8 * q, plane, bar);
+            tma::load_3d(dst + 3 * BOX, &tm_lr, 0, 56 - 8 * q, 1 * BC + plane, bar);
+        }
+    };
+
+    if (lane == 0)
+        for (int k = 0; k < NST; ++k) issue(k);
+
+    int k = 0;  // next chunk to consume
+    auto fail = [&]() {
+        if (lane == 0) atomicExch(a.err, 1);
+        // drain every copy that may still be in flight, with a short bound
+        for (int kk = k; kk < k + NST; ++kk) {
+            const int unit = wid + (kk / CHUNKS_PER_UNIT) * wstride;
+            if (unit < a.units) tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
+        }
+    };
+    // wait for chunk k; false (for every lane) if any lane's wait timed out
+    auto acquire = [&]() -> bool {
+        const bool ok = tma::mbar_wait(bar0 + 8 * (k % NST), (k / NST) & 1);
+        return __all_sync(FULL, ok);
+    };
+    // all lanes done reading stage of chunk k: refill it with chunk k + NST
+    auto release = [&]() {
+        tma::fence_proxy_async();
+        __syncwarp();
+        if (lane == 0) issue(k + NST);
+        ++k;
+    };
+
+    for (int unit = wid; unit < a.units; unit += wstride) {
+        const int b = unit / half_c, c0 = (unit - b * half_c) * 2;
+        const float4* wrow = a.wtab + (size_t)b * 2 * S * S + t;
+        __nv_bfloat16* outp = a.out + (size_t)(b * a.C + c0 + g) * S * S + 4 * t;
+
+        // ---------------- row pass: left->right (x) and right->left (y) ----------------
+        float2 h[4];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
+        for (int q = 0; q < 8; ++q) {
+            if (!acquire()) { fail(); return; }
+            const uint32_t st = ring + (k % NST) * STAGE + g * 256 + t * 16;
+            uint4 XA[4], LA[4], XB[4], LB[4];
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+                XA[p] = lds128(st + 0 * BOX + p * 512);
+                LA[p] = lds128(st + 1 * BOX + p * 512);
+                XB[p] = lds128(st + 2 * BOX + p * 512);
+                LB[p] = lds128(st + 3 * BOX + p * 512);
+            }
+            release();
+            float prevA[4], prevB[4];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int s = 8 * q + e;
+                if (s % a.seg == 0) {
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
+                }
+                float2 xl[4], ll[4];
+                float4 w[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    xl[p] = make_float2(bf_at(XA[p], e), bf_at(XB[p], 7 - e));
+                    ll[p] = make_float2(bf_at(LA[p], e), bf_at(LB[p], 7 - e));
+                    w[p] = __ldg(wrow + s * S + p * LPL);
+                }
+                scan_step(h, xl, ll, w);
+                if (e & 1) {
+                    // left->right covers columns s-1, s; right->left columns 63-s, 64-s
+                    const int uA = s >> 1, uB = (S - 1 - s) >> 1;
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        const int r = 4 * t + p;
+                        const uint32_t adA = hacc + hacc_off(r, uA), adB = hacc + hacc_off(r, uB);
+                        float2 vA = make_float2(prevA[p], h[p].x);
+                        float2 vB = make_float2(h[p].y, prevB[p]);
+                        if (q >= 4) {  // second arrival: add the other direction
+                            const float2 oA = lds64f(adA), oB = lds64f(adB);
+                            vA = __fadd2_rn(vA, oA);
+                            vB = __fadd2_rn(vB, oB);
+                        }
+                        sts64f(adA, vA);
+                        sts64f(adB, vB);
+                    }
+                } else {
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        prevA[p] = h[p].x;
+                        prevB[p] = h[p].y;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+
+        // ---------------- column pass: top->bottom (x) and bottom->top (y) ----------------
+#pragma unroll
+        for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
+        for (int q = 0; q < 8; ++q) {
+            if (!acquire()) { fail(); return; }
+            const uint32_t st = ring + (k % NST) * STAGE + g * 1024 + t * 8;
+            uint2 XA[8], LA[8], XB[8], LB[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                XA[e] = lds64(st + 0 * BOX + e * 128);
+                LA[e] = lds64(st + 1 * BOX + e * 128);
+                XB[e] = lds64(st + 2 * BOX + (7 - e) * 128);
+                LB[e] = lds64(st + 3 * BOX + (7 - e) * 128);
+            }
+            release();
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const int s = 8 * q + e;
+                if (s % a.seg == 0) {
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
+                }
+                float2 xl[4], ll[4];
+                float4 w[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {
+                    xl[p] = make_float2(bf_at2(XA[e], p), bf_at2(XB[e], p));
+                    ll[p] = make_float2(bf_at2(LA[e], p), bf_at2(LB[e], p));
+                    w[p] = __ldg(wrow + (S + s) * S + p * LPL);
+                }
+                scan_step(h, xl, ll, w);
+                const int rA = s, rB = S - 1 - s;
+                const uint32_t a0 = hacc + hacc_off(rA, 2 * t), a1 = hacc + hacc_off(rA, 2 * t + 1);
+                const uint32_t b0 = hacc + hacc_off(rB, 2 * t), b1 = hacc + hacc_off(rB, 2 * t + 1);
+                const float2 vA0 = __fadd2_rn(lds64f(a0), make_float2(h[0].x, h[1].x));
+                const float2 vA1 = __fadd2_rn(lds64f(a1), make_float2(h[2].x, h[3].x));
+                const float2 vB0 = __fadd2_rn(lds64f(b0), make_float2(h[0].y, h[1].y));
+                const float2 vB1 = __fadd2_rn(lds64f(b1), make_float2(h[2].y, h[3].y));
+                if (q < 4) {  // first arrival of this pass: keep the partial sum
+                    sts64f(a0, vA0);
+                    sts64f(a1, vA1);
+                    sts64f(b0, vB0);
+                    sts64f(b1, vB1);
+                } else {      // second arrival: the pixel is complete
+                    stg_cs64(outp + rA * S, pack_bf2(vA0.x, vA0.y), pack_bf2(vA1.x, vA1.y));
+                    stg_cs64(outp + rB * S, pack_bf2(vB0.x, vB0.y), pack_bf2(vB1.x, vB1.y));
+                }
+            }
+        }
+        __syncwarp();
+    }
+}
+
+// ---- host side ----------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 3-D view (column, row, plane) of a stack of 64x64 bf16 planes.
+bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r, uint32_t estride_r,
+              CUtensorMapL2promotion promo) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {S, S, planes};
+    const cuuint64_t strides[2] = {S * 2, S * S * 2};
+    const cuuint32_t box[3] = {box_c, box_r, 2};
+    const cuuint32_t es[3] = {1, estride_r, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool c64_eligible(const Problem& p) {
+    return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
+           (p.g.C % 2) == 0 && encode_fn() != nullptr;
+}
+
+size_t c64_fwd_workspace(const Problem& p) {
+    return kWsAlign + align_up((size_t)p.g.B * 2 * S * S * sizeof(float4), kWsAlign);
+}
+
+gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                    void* out, void* ws, cudaStream_t s) {
+    CUtensorMap xc, lc, xr, lr;
+    const uint64_t BC = (uint64_t)p.planes;
+    // column chunks: 8 columns x every 4th row (16 rows) x 2 planes; row chunks: 64 columns x 8 rows x 2 planes
+    if (!make_map(&xc, x, BC, 8, 64, 4, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&lc, lam, 4 * BC, 8, 64, 4, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&xr, x, BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+        !make_map(&lr, lam, 4 * BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+        return GSPN_ERR_UNSUPPORTED;
+    char* w = static_cast<char*>(ws);
+    C64Args a;
+    a.err = reinterpret_cast<int*>(w);
+    a.wtab = reinterpret_cast<const float4*>(w + kWsAlign);
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.B = p.g.B;
+    a.C = p.g.C;
+    a.seg = S / p.g.groups;
+    a.units = (int)(p.planes / 2);
+    const int nw = p.g.B * 2 * S * S;
+    c64_weights_kernel<__nv_bfloat16><<<(nw + 255) / 256, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.wtab), a.err, p.g.B);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    e = ensure_smem_attr((const void*)c64_fwd_kernel, SMEM_BYTES, 8);
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    int grid = dev.sm_count;
+    const int need = (a.units + NWARP - 1) / NWARP;
+    if (need < grid) grid = need;
+    c64_fwd_kernel<<<grid, NWARP * 32, SMEM_BYTES, s>>>(xc, lc, xr, lr, a);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+}
+
+}  // namespace gspn

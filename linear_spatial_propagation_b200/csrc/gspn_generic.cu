@@ -178,10 +178,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) 
                     const float dw0 = j > 0 ? av * hprev[j - 1] : 0.f;
                     const float dw1 = av * hprev[j];
                     const float dw2 = j < N - 1 ? av * hprev[j + 1] : 0.f;
-                    const float tw = w0 * dw0 + w1 * dw1 + w2 * dw2;
-                    dl0 = s0 * (1.f - s0) * r * (dw0 - tw);
-                    dl1 = s1 * (1.f - s1) * r * (dw1 - tw);
-                    dl2 = s2 * (1.f - s2) * r * (dw2 - tw);
+                    // dw_k - sum_m w_m dw_m = sum_m w_m (dw_k - dw_m) since the w sum to 1;
+                    // the pairwise form is exactly 0 when a single tap is valid
+                    const float r2 = r * r;
+                    dl0 = s0 * (1.f - s0) * r2 * (s1 * (dw0 - dw1) + s2 * (dw0 - dw2));
+                    dl1 = s1 * (1.f - s1) * r2 * (s0 * (dw1 - dw0) + s2 * (dw1 - dw2));
+                    dl2 = s2 * (1.f - s2) * r2 * (s0 * (dw2 - dw0) + s1 * (dw2 - dw1));
                     q0 = w0 * av; q1 = w1 * av; q2 = w2 * av;
                 }
                 qc[j + 1] = q0;

@@ -41,4 +41,10 @@ gspn_status generic_bwd(const Problem& p, const DeviceInfo& dev, const void* x, 
                         const void* lam, const void* dout, void* dx, void* dlogits, void* dlam, void* ws,
                         cudaStream_t s);
 
+// ---- compact 64x64 bf16 forward (TMA-fed, packed fp32x2) ------------------------
+bool c64_eligible(const Problem& p);
+size_t c64_fwd_workspace(const Problem& p);
+gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                    void* out, void* ws, cudaStream_t s);
+
 }  // namespace gspn
