@@ -152,10 +152,33 @@ struct C64Args {
 // a - b, exactly rounded (sm_100 has packed add and fma but no packed subtract)
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
 
+// c + a*b with a, b the low (L) or high (H) bf16 halves of two 32-bit words:
+// the bf16 operands feed the fp32 FMA directly (mixed-precision fma of
+// sm_100), exact products and a single rounding like the fp32 FMA of the
+// widened values.
+__device__ __forceinline__ float fma_bf_lo(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, a0, b0, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fma_bf_hi(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
+        "fma.rn.f32.bf16 %0, a1, b1, %3;\n\t}"
+        : "=f"(d) : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+// `half` is a compile-time constant at every (unrolled) call site
+__device__ __forceinline__ float fma_bf(int half, uint32_t a, uint32_t b, float c) {
+    return half ? fma_bf_hi(a, b, c) : fma_bf_lo(a, b, c);
+}
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
 // One scan step for one lane: 4 positions, two directions packed in float2.
-// w[p] = (-w0_A, -w0_B, w2_A, w2_B).
-__device__ __forceinline__ void scan_step(float2 (&h)[4], const float2 (&xl)[4], const float2 (&ll)[4],
-                                          const float4 (&w)[4]) {
+// base[p] = h[p] + lambda x (both directions), w[p] = (-w0_A, -w0_B, w2_A, w2_B).
+__device__ __forceinline__ void scan_core(float2 (&h)[4], const float2 (&base)[4], const float4 (&w)[4]) {
     float2 hl, hr;
     hl.x = __shfl_up_sync(FULL, h[3].x, 1, LPL);
     hl.y = __shfl_up_sync(FULL, h[3].y, 1, LPL);
@@ -169,10 +192,8 @@ __device__ __forceinline__ void scan_step(float2 (&h)[4], const float2 (&xl)[4],
     D[4] = sub2(hr, h[3]);
 #pragma unroll
     for (int p = 0; p < 4; ++p) {
-        float2 v = __ffma2_rn(ll[p], xl[p], h[p]);
-        v = __ffma2_rn(make_float2(w[p].z, w[p].w), D[p + 1], v);
-        v = __ffma2_rn(make_float2(w[p].x, w[p].y), D[p], v);
-        h[p] = v;
+        float2 v = __ffma2_rn(make_float2(w[p].z, w[p].w), D[p + 1], base[p]);
+        h[p] = __ffma2_rn(make_float2(w[p].x, w[p].y), D[p], v);
     }
 }
 
@@ -190,6 +211,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     const int wid = blockIdx.x * NWARP + warp;
     const int wstride = gridDim.x * NWARP;
     const int half_c = a.C >> 1;
+    const int segmask = a.seg - 1;  // seg divides 64, so it is a power of two
     if (wid >= a.units) return;
 
     if (lane == 0) {
@@ -249,7 +271,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         const bool ok = tma::mbar_wait(bar0 + 8 * (k % NST), (k / NST) & 1);
         return __all_sync(FULL, ok);
     };
-    // all lanes done reading stage of chunk k: refill it with chunk k + NST
+    // all lanes done reading the stage of chunk k: refill it with chunk k + NST
     auto release = [&]() {
         tma::fence_proxy_async();
         __syncwarp();
@@ -257,9 +279,35 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         ++k;
     };
 
+    // Tap weights of the 128 scan steps of a unit (64 row-pass, then 64
+    // column-pass) are table rows b*128 + l; they are prefetched 3 steps ahead
+    // into a 4-deep register ring, continuing into the next unit.
+    float4 wr[4][4];
+    auto wrow_of = [&](int unit) -> const float4* {
+        const int b = unit / half_c;
+        return a.wtab + (size_t)b * 2 * S * S + t;
+    };
+    const float4* wu = wrow_of(wid);
+    const float4* wn = wid + wstride < a.units ? wrow_of(wid + wstride) : wu;
+#pragma unroll
+    for (int l = 0; l < 3; ++l)
+#pragma unroll
+        for (int p = 0; p < 4; ++p) wr[l][p] = __ldg(wu + l * S + p * LPL);
+    // issue the weight loads of unit step l + 3 into ring slot (l + 3) & 3
+    auto prefetch_w = [&](int l, int slot) {
+        const int ls = l + 3;
+        const float4* src = ls < 2 * S ? wu + ls * S : wn + (ls - 2 * S) * S;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) wr[slot][p] = __ldg(src + p * LPL);
+    };
+
+    // Hacc addressing.  Row pass: lane t owns rows 4t..4t+3, whose unit XOR key
+    // is t.  Column pass: lane t owns units 2t, 2t+1 of each row.
+    const uint32_t hrow = hacc + (uint32_t)(4 * t) * 256u;
+    const int u0 = 2 * t;
+
     for (int unit = wid; unit < a.units; unit += wstride) {
         const int b = unit / half_c, c0 = (unit - b * half_c) * 2;
-        const float4* wrow = a.wtab + (size_t)b * 2 * S * S + t;
         __nv_bfloat16* outp = a.out + (size_t)(b * a.C + c0 + g) * S * S + 4 * t;
 
         // ---------------- row pass: left->right (x) and right->left (y) ----------------
@@ -278,46 +326,45 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                 LB[p] = lds128(st + 3 * BOX + p * 512);
             }
             release();
-            float prevA[4], prevB[4];
+            float2 prev[4];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int s = 8 * q + e;
-                if (s % a.seg == 0) {
+                prefetch_w(s, (e + 3) & 3);
+                if ((s & segmask) == 0) {
 #pragma unroll
                     for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
                 }
-                float2 xl[4], ll[4];
-                float4 w[4];
+                // left->right reads column s = element e of the A chunk; right->left
+                // column 63-s = element 7-e of the B chunk
+                float2 base[4];
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    xl[p] = make_float2(bf_at(XA[p], e), bf_at(XB[p], 7 - e));
-                    ll[p] = make_float2(bf_at(LA[p], e), bf_at(LB[p], 7 - e));
-                    w[p] = __ldg(wrow + s * S + p * LPL);
+                    base[p].x = fma_bf(e & 1, word_of(LA[p], e >> 1), word_of(XA[p], e >> 1), h[p].x);
+                    base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1), h[p].y);
                 }
-                scan_step(h, xl, ll, w);
+                scan_core(h, base, wr[e & 3]);
                 if (e & 1) {
-                    // left->right covers columns s-1, s; right->left columns 63-s, 64-s
+                    // left->right covers columns s-1, s (unit s/2); right->left covers
+                    // columns 63-s, 64-s (unit (63-s)/2)
                     const int uA = s >> 1, uB = (S - 1 - s) >> 1;
+                    const uint32_t oA = (uint32_t)((uA ^ t ^ ((uA >> 4) & 1)) << 3);
+                    const uint32_t oB = (uint32_t)((uB ^ t ^ ((uB >> 4) & 1)) << 3);
 #pragma unroll
                     for (int p = 0; p < 4; ++p) {
-                        const int r = 4 * t + p;
-                        const uint32_t adA = hacc + hacc_off(r, uA), adB = hacc + hacc_off(r, uB);
-                        float2 vA = make_float2(prevA[p], h[p].x);
-                        float2 vB = make_float2(h[p].y, prevB[p]);
+                        const uint32_t adA = hrow + p * 256 + oA, adB = hrow + p * 256 + oB;
+                        float2 vA = make_float2(prev[p].x, h[p].x);
+                        float2 vB = make_float2(h[p].y, prev[p].y);
                         if (q >= 4) {  // second arrival: add the other direction
-                            const float2 oA = lds64f(adA), oB = lds64f(adB);
-                            vA = __fadd2_rn(vA, oA);
-                            vB = __fadd2_rn(vB, oB);
+                            vA = __fadd2_rn(vA, lds64f(adA));
+                            vB = __fadd2_rn(vB, lds64f(adB));
                         }
                         sts64f(adA, vA);
                         sts64f(adB, vB);
                     }
                 } else {
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) {
-                        prevA[p] = h[p].x;
-                        prevB[p] = h[p].y;
-                    }
+                    for (int p = 0; p < 4; ++p) prev[p] = h[p];
                 }
             }
         }
@@ -341,22 +388,27 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int s = 8 * q + e;
-                if (s % a.seg == 0) {
+                prefetch_w(S + s, (e + 3) & 3);
+                if ((s & segmask) == 0) {
 #pragma unroll
                     for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
                 }
-                float2 xl[4], ll[4];
-                float4 w[4];
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    xl[p] = make_float2(bf_at2(XA[e], p), bf_at2(XB[e], p));
-                    ll[p] = make_float2(bf_at2(LA[e], p), bf_at2(LB[e], p));
-                    w[p] = __ldg(wrow + (S + s) * S + p * LPL);
-                }
-                scan_step(h, xl, ll, w);
+                float2 base[4];
+                base[0].x = fma_bf(0, LA[e].x, XA[e].x, h[0].x);
+                base[1].x = fma_bf(1, LA[e].x, XA[e].x, h[1].x);
+                base[2].x = fma_bf(0, LA[e].y, XA[e].y, h[2].x);
+                base[3].x = fma_bf(1, LA[e].y, XA[e].y, h[3].x);
+                base[0].y = fma_bf(0, LB[e].x, XB[e].x, h[0].y);
+                base[1].y = fma_bf(1, LB[e].x, XB[e].x, h[1].y);
+                base[2].y = fma_bf(0, LB[e].y, XB[e].y, h[2].y);
+                base[3].y = fma_bf(1, LB[e].y, XB[e].y, h[3].y);
+                scan_core(h, base, wr[e & 3]);
                 const int rA = s, rB = S - 1 - s;
-                const uint32_t a0 = hacc + hacc_off(rA, 2 * t), a1 = hacc + hacc_off(rA, 2 * t + 1);
-                const uint32_t b0 = hacc + hacc_off(rB, 2 * t), b1 = hacc + hacc_off(rB, 2 * t + 1);
+                const int kA = (rA >> 2) & 15, kB = (rB >> 2) & 15;
+                const uint32_t a0 = hacc + rA * 256 + (((u0 ^ kA) ^ (t >> 3)) << 3);
+                const uint32_t a1 = hacc + rA * 256 + ((((u0 + 1) ^ kA) ^ (t >> 3)) << 3);
+                const uint32_t b0 = hacc + rB * 256 + (((u0 ^ kB) ^ (t >> 3)) << 3);
+                const uint32_t b1 = hacc + rB * 256 + ((((u0 + 1) ^ kB) ^ (t >> 3)) << 3);
                 const float2 vA0 = __fadd2_rn(lds64f(a0), make_float2(h[0].x, h[1].x));
                 const float2 vA1 = __fadd2_rn(lds64f(a1), make_float2(h[2].x, h[3].x));
                 const float2 vB0 = __fadd2_rn(lds64f(b0), make_float2(h[0].y, h[1].y));
@@ -373,6 +425,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             }
         }
         __syncwarp();
+        wu = wn;
+        wn = unit + 2 * wstride < a.units ? wrow_of(unit + 2 * wstride) : wu;
     }
 }
 
