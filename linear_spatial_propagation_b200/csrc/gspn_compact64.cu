@@ -10,16 +10,16 @@
 // Propagation: W kron I(C), per-channel lambda).
 //
 // Design (B200):
-// * The tap weights depend only on (b, pixel, direction).  A small pre-kernel
-//   turns the logits into normalised (w0, w2) pairs once per (b, pixel,
-//   direction) -- w1 = 1 - w0 - w2 -- laid out in scan order so that each
-//   scan step reads one contiguous 256-byte row per half-warp.  The main
-//   kernel reads them through L1 and reuses them for every channel.
-// * One warp processes two channels of one batch image at a time (16 lanes
-//   per 64-wide line, 4 positions per lane).  The two directions of a pair
-//   (left->right with right->left, top->bottom with bottom->top) advance
-//   together: lane values are float2 (one direction per half) and the update
-//   uses the packed fp32x2 FMA of sm_100.
+// * The tap weights depend only on (b, pixel, direction).  A pre-kernel turns
+//   the logits into normalised (-w0, w2) pairs once per (b, pixel,
+//   direction) -- w1 = 1 - w0 - w2 -- laid out in scan order, so that each
+//   scan step reads one contiguous 512-byte row per warp; the main kernel
+//   reads them through L1 (prefetched 3 steps ahead) for every channel.
+// * One warp scans one (b, c) plane: 32 lanes per 64-wide line, 2 positions
+//   per lane; 8 warps per SM.  The two directions of a pair (left->right with
+//   right->left, top->bottom with bottom->top) advance together: lane values
+//   are float2 (one direction per half) and the update is the packed fp32x2
+//   FMA of sm_100; lambda*x is one mixed-precision FMA with bf16 inputs.
 // * Update in difference form, h'[p] = h[p] + lambda x + w2 (h[p+1] - h[p])
 //   - w0 (h[p] - h[p-1]), equal to w0 h[p-1] + w1 h[p] + w2 h[p+1] + lambda x
 //   for w1 = 1 - w0 - w2; the line ends have w0 = 0 / w2 = 0.  Neighbours
@@ -27,20 +27,18 @@
 // * Row pass first (left->right and right->left over columns), then column
 //   pass (top->bottom and bottom->top over rows).  The row pass leaves its
 //   sum in an fp32 plane in shared memory (Hacc); the column pass adds its two
-//   directions and writes each output row once, 128 contiguous bytes per line.
-//   In each pass the direction that reaches a pixel first stores, the second
-//   adds, so every Hacc element is written/read the minimum number of times.
-// * All x / lambda traffic is streamed by TMA into a per-warp ring of 8 KB
-//   stages (8 scan steps each): column chunks (8 columns x 64 rows) for the
-//   row pass and row chunks (64 columns x 8 rows) for the column pass.  A
-//   stage is copied to registers at its start and immediately refilled, so
-//   NST-1 stages (16 KB) per warp stay in flight.  Column chunks are fetched
-//   as four boxes of every 4th row (element stride 4), which lays rows
-//   4t..4t+3 of lane t into four separate 512-byte slices: the 16-byte reads
-//   of 8 lanes then hit 8 consecutive bank quads.
-// * Hacc uses an XOR layout of 8-byte units, conflict-free both for the row
-//   pass (each lane stores its 4 rows at one column pair) and for the column
-//   pass (each lane reads 4 columns of one row).
+//   directions and writes each output row once, 128 contiguous bytes.  In
+//   each pass the direction that reaches a pixel first stores, the second
+//   adds, so every Hacc element is stored and loaded the fewest times.
+// * All x / lambda traffic is streamed by TMA into a per-warp ring of 4 KB
+//   stages (8 scan steps each): column chunks (8 columns x 64 rows, one box
+//   per tensor, 128-byte swizzle so that the 16-byte row pieces of 8 lanes
+//   land in 8 different bank quads) for the row pass and row chunks (64
+//   columns x 8 rows) for the column pass.  A stage is copied to registers at
+//   its start and immediately refilled, so NST stages per warp stay in flight.
+// * Hacc uses an XOR layout of 8-byte units, conflict-free for the row pass
+//   (each lane stores rows 2t, 2t+1 at one column pair) and for the column
+//   pass (each lane reads columns 2t, 2t+1 of one row).
 // * Every mbarrier wait is bounded (2 s); on expiry the warp records an
 //   error word in the workspace, drains its outstanding copies and returns.
 #include "gspn_internal.h"
@@ -51,23 +49,24 @@ namespace gspn {
 namespace {
 
 constexpr int S = 64;         // H = W
-constexpr int LPL = 16;       // lanes per line
-constexpr int NWARP = 4;      // warps per CTA (one CTA per SM)
+constexpr int LPL = 32;       // lanes per line (2 positions per lane)
+constexpr int NWARP = 8;      // warps per CTA (one CTA per SM)
 constexpr int NST = 3;        // ring stages per warp
-constexpr int STAGE = 8192;   // bytes per stage: 4 boxes x 2 planes x 1 KB
-constexpr int BOX = 2048;     // bytes per box (2 planes)
-constexpr int HACC_PLANE = S * S * 4;
-constexpr int WARP_BYTES = NST * STAGE + 2 * HACC_PLANE;
+constexpr int BOX = 1024;     // bytes per TMA box (one plane)
+constexpr int STAGE = 4 * BOX;
+constexpr int HACC = S * S * 4;
+constexpr int WARP_BYTES = NST * STAGE + HACC;
 constexpr int BAR_BYTES = 8 * NST;
 constexpr int SMEM_BYTES = 1024 + NWARP * WARP_BYTES + NWARP * BAR_BYTES;
 constexpr int CHUNKS_PER_UNIT = 16;  // 8 column chunks + 8 row chunks
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(WARP_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128-byte swizzle");
 
 constexpr unsigned FULL = 0xffffffffu;
 
 // ---- weights pre-kernel ----------------------------------------------------------
-// wtab[((b*2 + pass)*64 + s)*64 + p*16 + t] = (-w0_A, -w0_B, w2_A, w2_B) of line
-// position j = 4t + p at scan step s, where pass 0 pairs A = left->right (line s
+// wtab[((b*2 + pass)*64 + s)*64 + p*32 + t] = (-w0_A, -w0_B, w2_A, w2_B) of line
+// position j = 2t + p at scan step s, where pass 0 pairs A = left->right (line s
 // = column s) with B = right->left (column 63-s), positions = rows; pass 1 pairs
 // A = top->bottom (row s) with B = bottom->top (row 63-s), positions = columns.
 template <typename T>
@@ -92,31 +91,19 @@ __global__ void c64_weights_kernel(const T* __restrict__ logits, float4* __restr
     float w0a, w2a, w0b, w2b;
     gate_pair(logits + (size_t)(slotA * B + b) * 3 * S * S, pixA, j, &w0a, &w2a);
     gate_pair(logits + (size_t)(slotB * B + b) * 3 * S * S, pixB, j, &w0b, &w2b);
-    const int t = j >> 2, p = j & 3;
+    const int t = j >> 1, p = j & 1;
     wtab[((size_t)(b * 2 + pass) * S + s) * S + p * LPL + t] = make_float4(-w0a, -w0b, w2a, w2b);
 }
 
 // ---- helpers ----------------------------------------------------------------------
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-// element e (0..7) of 8 packed bf16
-__device__ __forceinline__ float bf_at(const uint4& v, int e) {
-    const uint32_t w = e < 2 ? v.x : e < 4 ? v.y : e < 6 ? v.z : v.w;
-    return (e & 1) ? bf_hi(w) : bf_lo(w);
-}
-__device__ __forceinline__ float bf_at2(const uint2& v, int e) {
-    const uint32_t w = e < 2 ? v.x : v.y;
-    return (e & 1) ? bf_hi(w) : bf_lo(w);
-}
-
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
     return v;
 }
-__device__ __forceinline__ uint2 lds64(uint32_t a) {
-    uint2 v;
-    asm volatile("ld.shared.v2.b32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+__device__ __forceinline__ uint32_t lds32(uint32_t a) {
+    uint32_t v;
+    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
 __device__ __forceinline__ float2 lds64f(uint32_t a) {
@@ -127,35 +114,23 @@ __device__ __forceinline__ float2 lds64f(uint32_t a) {
 __device__ __forceinline__ void sts64f(uint32_t a, float2 v) {
     asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(a), "f"(v.x), "f"(v.y) : "memory");
 }
-__device__ __forceinline__ void stg_cs64(void* p, uint32_t a, uint32_t b) {
-    asm volatile("st.global.cs.v2.b32 [%0], {%1,%2};" ::"l"(p), "r"(a), "r"(b) : "memory");
+__device__ __forceinline__ void stg_cs32(void* p, uint32_t v) {
+    asm volatile("st.global.cs.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
 }
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
 }
-
-// Hacc address (bytes from the plane base) of the 8-byte unit holding columns
-// 2u, 2u+1 of row r: unit index XORed with (r / 4) mod 16 and with bit 4 of u.
-__device__ __forceinline__ uint32_t hacc_off(int r, int u) {
-    return (uint32_t)(r * 256 + ((u ^ ((r >> 2) & 15) ^ ((u >> 4) & 1)) << 3));
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) {
+    return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w;
 }
-
-struct C64Args {
-    const float4* wtab;
-    __nv_bfloat16* out;
-    int* err;
-    int B, C, seg;
-    int units;  // B * C / 2
-};
 
 // a - b, exactly rounded (sm_100 has packed add and fma but no packed subtract)
 __device__ __forceinline__ float2 sub2(float2 a, float2 b) { return __ffma2_rn(b, make_float2(-1.f, -1.f), a); }
 
-// c + a*b with a, b the low (L) or high (H) bf16 halves of two 32-bit words:
-// the bf16 operands feed the fp32 FMA directly (mixed-precision fma of
-// sm_100), exact products and a single rounding like the fp32 FMA of the
-// widened values.
+// c + a*b with a, b the low / high bf16 halves of two 32-bit words: the bf16
+// operands feed the fp32 FMA directly (mixed-precision fma of sm_100), exact
+// products and one rounding, like the fp32 FMA of the widened values.
 __device__ __forceinline__ float fma_bf_lo(uint32_t a, uint32_t b, float c) {
     float d;
     asm("{\n\t.reg .b16 a0, a1, b0, b1;\n\tmov.b32 {a0, a1}, %1;\n\tmov.b32 {b0, b1}, %2;\n\t"
@@ -174,28 +149,34 @@ __device__ __forceinline__ float fma_bf_hi(uint32_t a, uint32_t b, float c) {
 __device__ __forceinline__ float fma_bf(int half, uint32_t a, uint32_t b, float c) {
     return half ? fma_bf_hi(a, b, c) : fma_bf_lo(a, b, c);
 }
-__device__ __forceinline__ uint32_t word_of(const uint4& v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
 
-// One scan step for one lane: 4 positions, two directions packed in float2.
+// One scan step for one lane: 2 positions, two directions packed in float2.
 // base[p] = h[p] + lambda x (both directions), w[p] = (-w0_A, -w0_B, w2_A, w2_B).
-__device__ __forceinline__ void scan_core(float2 (&h)[4], const float2 (&base)[4], const float4 (&w)[4]) {
+__device__ __forceinline__ void scan_core(float2 (&h)[2], const float2 (&base)[2], const float4 (&w)[2]) {
     float2 hl, hr;
-    hl.x = __shfl_up_sync(FULL, h[3].x, 1, LPL);
-    hl.y = __shfl_up_sync(FULL, h[3].y, 1, LPL);
-    hr.x = __shfl_down_sync(FULL, h[0].x, 1, LPL);
-    hr.y = __shfl_down_sync(FULL, h[0].y, 1, LPL);
-    float2 D[5];
-    D[0] = sub2(h[0], hl);
-    D[1] = sub2(h[1], h[0]);
-    D[2] = sub2(h[2], h[1]);
-    D[3] = sub2(h[3], h[2]);
-    D[4] = sub2(hr, h[3]);
-#pragma unroll
-    for (int p = 0; p < 4; ++p) {
-        float2 v = __ffma2_rn(make_float2(w[p].z, w[p].w), D[p + 1], base[p]);
-        h[p] = __ffma2_rn(make_float2(w[p].x, w[p].y), D[p], v);
-    }
+    hl.x = __shfl_up_sync(FULL, h[1].x, 1);
+    hl.y = __shfl_up_sync(FULL, h[1].y, 1);
+    hr.x = __shfl_down_sync(FULL, h[0].x, 1);
+    hr.y = __shfl_down_sync(FULL, h[0].y, 1);
+    const float2 D0 = sub2(h[0], hl), D1 = sub2(h[1], h[0]), D2 = sub2(hr, h[1]);
+    const float2 v0 = __ffma2_rn(make_float2(w[0].z, w[0].w), D1, base[0]);
+    const float2 v1 = __ffma2_rn(make_float2(w[1].z, w[1].w), D2, base[1]);
+    h[0] = __ffma2_rn(make_float2(w[0].x, w[0].y), D0, v0);
+    h[1] = __ffma2_rn(make_float2(w[1].x, w[1].y), D1, v1);
 }
+
+// Hacc byte offset of the 8-byte unit u (columns 2u, 2u+1) of row r.
+__device__ __forceinline__ uint32_t hacc_off(int r, int u) {
+    return (uint32_t)(r * 256 + ((u ^ ((r >> 1) & 15)) << 3));
+}
+
+struct C64Args {
+    const float4* wtab;
+    __nv_bfloat16* out;
+    int* err;
+    int B, C, seg;
+    int units;  // B * C planes
+};
 
 __global__ void __launch_bounds__(NWARP * 32, 1)
     c64_fwd_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
@@ -203,18 +184,17 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                    const C64Args a) {
     extern __shared__ unsigned char smem_raw[];
     const uint32_t sbase = (tma::smem_u32(smem_raw) + 1023u) & ~1023u;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int g = lane >> 4, t = lane & 15;
+    const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
     const uint32_t ring = sbase + warp * WARP_BYTES;
-    const uint32_t hacc = ring + NST * STAGE + g * HACC_PLANE;
+    const uint32_t hacc = ring + NST * STAGE;
     const uint32_t bar0 = sbase + NWARP * WARP_BYTES + warp * BAR_BYTES;
     const int wid = blockIdx.x * NWARP + warp;
     const int wstride = gridDim.x * NWARP;
-    const int half_c = a.C >> 1;
     const int segmask = a.seg - 1;  // seg divides 64, so it is a power of two
+    const int BC = a.B * a.C;
     if (wid >= a.units) return;
 
-    if (lane == 0) {
+    if (t == 0) {
         for (int k = 0; k < NST; ++k) tma::mbar_init(bar0 + 8 * k, 1);
         tma::fence_barrier_init();
         tma::prefetch_map(&tm_xc);
@@ -224,26 +204,22 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     }
     __syncwarp();
 
-    // Issue chunk k of this warp's sequence (lane 0 only): unit wid + (k/16)*wstride,
-    // chunk k%16 of it (0..7: column chunks, 8..15: row chunks).
+    // Issue chunk k of this warp's sequence (lane 0 only): plane wid + (k/16)*wstride,
+    // chunk k%16 of it (0..7: column chunks, 8..15: row chunks).  lambda plane
+    // (slot, b, c) is slot*B*C + plane.
     auto issue = [&](int k) {
-        const int unit = wid + (k / CHUNKS_PER_UNIT) * wstride;
-        if (unit >= a.units) return;
+        const int plane = wid + (k / CHUNKS_PER_UNIT) * wstride;
+        if (plane >= a.units) return;
         const int local = k % CHUNKS_PER_UNIT, st = k % NST;
         const uint32_t dst = ring + st * STAGE, bar = bar0 + 8 * st;
-        const int b = unit / half_c, c0 = (unit - b * half_c) * 2;
-        const int plane = b * a.C + c0;
-        const int BC = a.B * a.C;
         tma::mbar_expect_tx(bar, STAGE);
         if (local < 8) {
             const int q = local;
             // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at 8(7-q)..
-            for (int r = 0; r < 4; ++r) {
-                tma::load_3d(dst + 0 * BOX + r * 512, &tm_xc, 8 * q, r, plane, bar);
-                tma::load_3d(dst + 1 * BOX + r * 512, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
-                tma::load_3d(dst + 2 * BOX + r * 512, &tm_xc, 8 * (7 - q), r, plane, bar);
-                tma::load_3d(dst + 3 * BOX + r * 512, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
-            }
+            tma::load_3d(dst + 0 * BOX, &tm_xc, 8 * q, 0, plane, bar);
+            tma::load_3d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 2 * BC + plane, bar);
+            tma::load_3d(dst + 2 * BOX, &tm_xc, 8 * (7 - q), 0, plane, bar);
+            tma::load_3d(dst + 3 * BOX, &tm_lc, 8 * (7 - q), 0, 3 * BC + plane, bar);
         } else {
             const int q = local - 8;
             // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 56-8q..
@@ -254,16 +230,16 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         }
     };
 
-    if (lane == 0)
+    if (t == 0)
         for (int k = 0; k < NST; ++k) issue(k);
 
     int k = 0;  // next chunk to consume
     auto fail = [&]() {
-        if (lane == 0) atomicExch(a.err, 1);
+        if (t == 0) atomicExch(a.err, 1);
         // drain every copy that may still be in flight, with a short bound
         for (int kk = k; kk < k + NST; ++kk) {
-            const int unit = wid + (kk / CHUNKS_PER_UNIT) * wstride;
-            if (unit < a.units) tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
+            const int plane = wid + (kk / CHUNKS_PER_UNIT) * wstride;
+            if (plane < a.units) tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
         }
     };
     // wait for chunk k; false (for every lane) if any lane's wait timed out
@@ -275,83 +251,78 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     auto release = [&]() {
         tma::fence_proxy_async();
         __syncwarp();
-        if (lane == 0) issue(k + NST);
+        if (t == 0) issue(k + NST);
         ++k;
     };
 
-    // Tap weights of the 128 scan steps of a unit (64 row-pass, then 64
+    // Tap weights of the 128 scan steps of a plane (64 row-pass, then 64
     // column-pass) are table rows b*128 + l; they are prefetched 3 steps ahead
-    // into a 4-deep register ring, continuing into the next unit.
-    float4 wr[4][4];
-    auto wrow_of = [&](int unit) -> const float4* {
-        const int b = unit / half_c;
-        return a.wtab + (size_t)b * 2 * S * S + t;
-    };
-    const float4* wu = wrow_of(wid);
-    const float4* wn = wid + wstride < a.units ? wrow_of(wid + wstride) : wu;
+    // into a 4-deep register ring, continuing into the next plane.
+    float4 wr[4][2];
+    auto wbase = [&](int plane) -> const float4* { return a.wtab + (size_t)(plane / a.C) * 2 * S * S + t; };
+    const float4* wu = wbase(wid);
+    const float4* wn = wid + wstride < a.units ? wbase(wid + wstride) : wu;
 #pragma unroll
-    for (int l = 0; l < 3; ++l)
-#pragma unroll
-        for (int p = 0; p < 4; ++p) wr[l][p] = __ldg(wu + l * S + p * LPL);
-    // issue the weight loads of unit step l + 3 into ring slot (l + 3) & 3
+    for (int l = 0; l < 3; ++l) {
+        wr[l][0] = __ldg(wu + l * S);
+        wr[l][1] = __ldg(wu + l * S + LPL);
+    }
+    // load the weights of plane step l + 3 into ring slot `slot`
     auto prefetch_w = [&](int l, int slot) {
         const int ls = l + 3;
         const float4* src = ls < 2 * S ? wu + ls * S : wn + (ls - 2 * S) * S;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) wr[slot][p] = __ldg(src + p * LPL);
+        wr[slot][0] = __ldg(src);
+        wr[slot][1] = __ldg(src + LPL);
     };
 
-    // Hacc addressing.  Row pass: lane t owns rows 4t..4t+3, whose unit XOR key
-    // is t.  Column pass: lane t owns units 2t, 2t+1 of each row.
-    const uint32_t hrow = hacc + (uint32_t)(4 * t) * 256u;
-    const int u0 = 2 * t;
+    // Row pass: lane t owns rows 2t, 2t+1 (unit XOR key t & 15); the 16-byte
+    // piece of row r in a swizzled column-chunk box sits at r*16 ^ ((r>>3)&7)<<4.
+    const uint32_t hrow = hacc + (uint32_t)(2 * t) * 256u;
+    const int tk = t & 15;
+    const uint32_t cpiece0 = (uint32_t)((2 * t) * 16) ^ (uint32_t)(((t >> 2) & 7) << 4);
+    const uint32_t cpiece1 = (uint32_t)((2 * t + 1) * 16) ^ (uint32_t)(((t >> 2) & 7) << 4);
 
-    for (int unit = wid; unit < a.units; unit += wstride) {
-        const int b = unit / half_c, c0 = (unit - b * half_c) * 2;
-        __nv_bfloat16* outp = a.out + (size_t)(b * a.C + c0 + g) * S * S + 4 * t;
+    for (int plane = wid; plane < a.units; plane += wstride) {
+        __nv_bfloat16* outp = a.out + (size_t)plane * S * S + 2 * t;
 
         // ---------------- row pass: left->right (x) and right->left (y) ----------------
-        float2 h[4];
-#pragma unroll
-        for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
+        float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
         for (int q = 0; q < 8; ++q) {
             if (!acquire()) { fail(); return; }
-            const uint32_t st = ring + (k % NST) * STAGE + g * 256 + t * 16;
-            uint4 XA[4], LA[4], XB[4], LB[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                XA[p] = lds128(st + 0 * BOX + p * 512);
-                LA[p] = lds128(st + 1 * BOX + p * 512);
-                XB[p] = lds128(st + 2 * BOX + p * 512);
-                LB[p] = lds128(st + 3 * BOX + p * 512);
-            }
+            const uint32_t st = ring + (k % NST) * STAGE;
+            uint4 XA[2], LA[2], XB[2], LB[2];
+            XA[0] = lds128(st + 0 * BOX + cpiece0);
+            XA[1] = lds128(st + 0 * BOX + cpiece1);
+            LA[0] = lds128(st + 1 * BOX + cpiece0);
+            LA[1] = lds128(st + 1 * BOX + cpiece1);
+            XB[0] = lds128(st + 2 * BOX + cpiece0);
+            XB[1] = lds128(st + 2 * BOX + cpiece1);
+            LB[0] = lds128(st + 3 * BOX + cpiece0);
+            LB[1] = lds128(st + 3 * BOX + cpiece1);
             release();
-            float2 prev[4];
+            float2 prev[2];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int s = 8 * q + e;
                 prefetch_w(s, (e + 3) & 3);
-                if ((s & segmask) == 0) {
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
-                }
+                if ((s & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
                 // left->right reads column s = element e of the A chunk; right->left
                 // column 63-s = element 7-e of the B chunk
-                float2 base[4];
+                float2 base[2];
 #pragma unroll
-                for (int p = 0; p < 4; ++p) {
+                for (int p = 0; p < 2; ++p) {
                     base[p].x = fma_bf(e & 1, word_of(LA[p], e >> 1), word_of(XA[p], e >> 1), h[p].x);
-                    base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1), h[p].y);
+                    base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1),
+                                       h[p].y);
                 }
                 scan_core(h, base, wr[e & 3]);
                 if (e & 1) {
                     // left->right covers columns s-1, s (unit s/2); right->left covers
                     // columns 63-s, 64-s (unit (63-s)/2)
-                    const int uA = s >> 1, uB = (S - 1 - s) >> 1;
-                    const uint32_t oA = (uint32_t)((uA ^ t ^ ((uA >> 4) & 1)) << 3);
-                    const uint32_t oB = (uint32_t)((uB ^ t ^ ((uB >> 4) & 1)) << 3);
+                    const uint32_t oA = (uint32_t)(((s >> 1) ^ tk) << 3);
+                    const uint32_t oB = (uint32_t)((((S - 1 - s) >> 1) ^ tk) << 3);
 #pragma unroll
-                    for (int p = 0; p < 4; ++p) {
+                    for (int p = 0; p < 2; ++p) {
                         const uint32_t adA = hrow + p * 256 + oA, adB = hrow + p * 256 + oB;
                         float2 vA = make_float2(prev[p].x, h[p].x);
                         float2 vB = make_float2(h[p].y, prev[p].y);
@@ -363,70 +334,54 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                         sts64f(adB, vB);
                     }
                 } else {
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) prev[p] = h[p];
+                    prev[0] = h[0];
+                    prev[1] = h[1];
                 }
             }
         }
         __syncwarp();
 
         // ---------------- column pass: top->bottom (x) and bottom->top (y) ----------------
-#pragma unroll
-        for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
+        h[0] = h[1] = make_float2(0.f, 0.f);
         for (int q = 0; q < 8; ++q) {
             if (!acquire()) { fail(); return; }
-            const uint32_t st = ring + (k % NST) * STAGE + g * 1024 + t * 8;
-            uint2 XA[8], LA[8], XB[8], LB[8];
+            const uint32_t st = ring + (k % NST) * STAGE + t * 4;
+            uint32_t XA[8], LA[8], XB[8], LB[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                XA[e] = lds64(st + 0 * BOX + e * 128);
-                LA[e] = lds64(st + 1 * BOX + e * 128);
-                XB[e] = lds64(st + 2 * BOX + (7 - e) * 128);
-                LB[e] = lds64(st + 3 * BOX + (7 - e) * 128);
+                XA[e] = lds32(st + 0 * BOX + e * 128);
+                LA[e] = lds32(st + 1 * BOX + e * 128);
+                XB[e] = lds32(st + 2 * BOX + (7 - e) * 128);
+                LB[e] = lds32(st + 3 * BOX + (7 - e) * 128);
             }
             release();
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
                 const int s = 8 * q + e;
                 prefetch_w(S + s, (e + 3) & 3);
-                if ((s & segmask) == 0) {
-#pragma unroll
-                    for (int p = 0; p < 4; ++p) h[p] = make_float2(0.f, 0.f);
-                }
-                float2 base[4];
-                base[0].x = fma_bf(0, LA[e].x, XA[e].x, h[0].x);
-                base[1].x = fma_bf(1, LA[e].x, XA[e].x, h[1].x);
-                base[2].x = fma_bf(0, LA[e].y, XA[e].y, h[2].x);
-                base[3].x = fma_bf(1, LA[e].y, XA[e].y, h[3].x);
-                base[0].y = fma_bf(0, LB[e].x, XB[e].x, h[0].y);
-                base[1].y = fma_bf(1, LB[e].x, XB[e].x, h[1].y);
-                base[2].y = fma_bf(0, LB[e].y, XB[e].y, h[2].y);
-                base[3].y = fma_bf(1, LB[e].y, XB[e].y, h[3].y);
+                if ((s & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
+                float2 base[2];
+                base[0].x = fma_bf_lo(LA[e], XA[e], h[0].x);
+                base[1].x = fma_bf_hi(LA[e], XA[e], h[1].x);
+                base[0].y = fma_bf_lo(LB[e], XB[e], h[0].y);
+                base[1].y = fma_bf_hi(LB[e], XB[e], h[1].y);
                 scan_core(h, base, wr[e & 3]);
                 const int rA = s, rB = S - 1 - s;
-                const int kA = (rA >> 2) & 15, kB = (rB >> 2) & 15;
-                const uint32_t a0 = hacc + rA * 256 + (((u0 ^ kA) ^ (t >> 3)) << 3);
-                const uint32_t a1 = hacc + rA * 256 + ((((u0 + 1) ^ kA) ^ (t >> 3)) << 3);
-                const uint32_t b0 = hacc + rB * 256 + (((u0 ^ kB) ^ (t >> 3)) << 3);
-                const uint32_t b1 = hacc + rB * 256 + ((((u0 + 1) ^ kB) ^ (t >> 3)) << 3);
-                const float2 vA0 = __fadd2_rn(lds64f(a0), make_float2(h[0].x, h[1].x));
-                const float2 vA1 = __fadd2_rn(lds64f(a1), make_float2(h[2].x, h[3].x));
-                const float2 vB0 = __fadd2_rn(lds64f(b0), make_float2(h[0].y, h[1].y));
-                const float2 vB1 = __fadd2_rn(lds64f(b1), make_float2(h[2].y, h[3].y));
+                const uint32_t adA = hacc + hacc_off(rA, t), adB = hacc + hacc_off(rB, t);
+                const float2 vA = __fadd2_rn(lds64f(adA), make_float2(h[0].x, h[1].x));
+                const float2 vB = __fadd2_rn(lds64f(adB), make_float2(h[0].y, h[1].y));
                 if (q < 4) {  // first arrival of this pass: keep the partial sum
-                    sts64f(a0, vA0);
-                    sts64f(a1, vA1);
-                    sts64f(b0, vB0);
-                    sts64f(b1, vB1);
+                    sts64f(adA, vA);
+                    sts64f(adB, vB);
                 } else {      // second arrival: the pixel is complete
-                    stg_cs64(outp + rA * S, pack_bf2(vA0.x, vA0.y), pack_bf2(vA1.x, vA1.y));
-                    stg_cs64(outp + rB * S, pack_bf2(vB0.x, vB0.y), pack_bf2(vB1.x, vB1.y));
+                    stg_cs32(outp + rA * S, pack_bf2(vA.x, vA.y));
+                    stg_cs32(outp + rB * S, pack_bf2(vB.x, vB.y));
                 }
             }
         }
         __syncwarp();
         wu = wn;
-        wn = unit + 2 * wstride < a.units ? wrow_of(unit + 2 * wstride) : wu;
+        wn = plane + 2 * wstride < a.units ? wbase(plane + 2 * wstride) : wu;
     }
 }
 
@@ -450,25 +405,24 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view (column, row, plane) of a stack of 64x64 bf16 planes.
-bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r, uint32_t estride_r,
-              CUtensorMapL2promotion promo) {
+// 3-D view (column, row, plane) of a stack of 64x64 bf16 planes; one plane per box.
+bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r,
+              CUtensorMapSwizzle swz, CUtensorMapL2promotion promo) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, S * S * 2};
-    const cuuint32_t box[3] = {box_c, box_r, 2};
-    const cuuint32_t es[3] = {1, estride_r, 1};
+    const cuuint32_t box[3] = {box_c, box_r, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
 bool c64_eligible(const Problem& p) {
     return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
-           (p.g.C % 2) == 0 && encode_fn() != nullptr;
+           p.planes <= 0x7fffffff / 4 && encode_fn() != nullptr;
 }
 
 size_t c64_fwd_workspace(const Problem& p) {
@@ -479,11 +433,11 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
                     void* out, void* ws, cudaStream_t s) {
     CUtensorMap xc, lc, xr, lr;
     const uint64_t BC = (uint64_t)p.planes;
-    // column chunks: 8 columns x every 4th row (16 rows) x 2 planes; row chunks: 64 columns x 8 rows x 2 planes
-    if (!make_map(&xc, x, BC, 8, 64, 4, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
-        !make_map(&lc, lam, 4 * BC, 8, 64, 4, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
-        !make_map(&xr, x, BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
-        !make_map(&lr, lam, 4 * BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+    // column chunks: 8 columns x 64 rows (swizzled 16-byte pieces); row chunks: 64 columns x 8 rows
+    if (!make_map(&xc, x, BC, 8, 64, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&lc, lam, 4 * BC, 8, 64, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&xr, x, BC, 64, 8, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+        !make_map(&lr, lam, 4 * BC, 64, 8, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
         return GSPN_ERR_UNSUPPORTED;
     char* w = static_cast<char*>(ws);
     C64Args a;
@@ -493,7 +447,7 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     a.B = p.g.B;
     a.C = p.g.C;
     a.seg = S / p.g.groups;
-    a.units = (int)(p.planes / 2);
+    a.units = (int)p.planes;
     const int nw = p.g.B * 2 * S * S;
     c64_weights_kernel<__nv_bfloat16><<<(nw + 255) / 256, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.wtab), a.err, p.g.B);

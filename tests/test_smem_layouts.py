@@ -11,11 +11,17 @@ import itertools
 
 import pytest
 
-S, LPL, BOX = 64, 16, 2048
+S, LPL, BOX = 64, 32, 1024
 
 
 def hacc_off(r, u):
-    return r * 256 + ((u ^ ((r >> 2) & 15) ^ ((u >> 4) & 1)) << 3)
+    return r * 256 + ((u ^ ((r >> 1) & 15)) << 3)
+
+
+def swz128(a):
+    """TMA 128-byte swizzle: the 16-byte piece index within each 128-byte line
+    is XORed with the line index mod 8 (buffer 1024-byte aligned)."""
+    return a ^ (((a >> 7) & 7) << 4)
 
 
 def wavefronts(addrs, width):
@@ -36,50 +42,46 @@ def optimal(width):
     return 32 * width // 128
 
 
-def lanes():
-    return [(l >> 4, l & 15) for l in range(32)]
-
-
 def test_hacc_is_a_bijection_per_row():
     for r in range(S):
         units = sorted((hacc_off(r, u) - r * 256) >> 3 for u in range(32))
         assert units == list(range(32))
 
 
-@pytest.mark.parametrize("p,u", itertools.product(range(4), range(32)))
+@pytest.mark.parametrize("p,u", list(itertools.product(range(2), range(32))))
 def test_row_pass_hacc_stores(p, u):
-    # lane (g, t) stores the unit u of row 4t+p of its channel plane g
-    addrs = [g * 16384 + hacc_off(4 * t + p, u) for g, t in lanes()]
+    # lane t stores the unit u of row 2t+p
+    addrs = [hacc_off(2 * t + p, u) for t in range(32)]
     assert wavefronts(addrs, 8) == optimal(8)
 
 
-@pytest.mark.parametrize("s,m", itertools.product(range(S), range(2)))
-def test_column_pass_hacc_loads(s, m):
-    # lane (g, t) reads units 2t, 2t+1 (columns 4t..4t+3) of row s
-    addrs = [g * 16384 + hacc_off(s, 2 * t + m) for g, t in lanes()]
+@pytest.mark.parametrize("s", range(S))
+def test_column_pass_hacc_loads(s):
+    # lane t reads unit t (columns 2t, 2t+1) of row s
+    addrs = [hacc_off(s, t) for t in range(32)]
     assert wavefronts(addrs, 8) == optimal(8)
 
 
-@pytest.mark.parametrize("box,p", itertools.product(range(4), range(4)))
+@pytest.mark.parametrize("box,p", list(itertools.product(range(4), range(2))))
 def test_row_pass_stage_reads(box, p):
-    # column chunks: four 512-byte slices (rows 4*r_hi + p), [plane][r_hi][16 B]
-    addrs = [box * BOX + p * 512 + g * 256 + t * 16 for g, t in lanes()]
+    # column chunk box: 64 rows of 16 bytes, 128-byte swizzle; lane t reads rows 2t, 2t+1
+    addrs = [box * BOX + swz128((2 * t + p) * 16) for t in range(32)]
     assert wavefronts(addrs, 16) == optimal(16)
 
 
-@pytest.mark.parametrize("box,e", itertools.product(range(4), range(8)))
+def test_kernel_piece_offsets_match_the_swizzle():
+    # the kernel precomputes (2t+p)*16 ^ ((t>>2)&7)<<4
+    for t in range(32):
+        for p in range(2):
+            assert swz128((2 * t + p) * 16) == ((2 * t + p) * 16) ^ (((t >> 2) & 7) << 4)
+
+
+@pytest.mark.parametrize("box,e", list(itertools.product(range(4), range(8))))
 def test_column_pass_stage_reads(box, e):
-    # row chunks: [plane][8 rows][128 B]; lane (g, t) reads columns 4t..4t+3
-    addrs = [box * BOX + g * 1024 + e * 128 + t * 8 for g, t in lanes()]
-    assert wavefronts(addrs, 8) == optimal(8)
+    # row chunk box: [8 rows][128 B]; lane t reads columns 2t, 2t+1
+    addrs = [box * BOX + e * 128 + t * 4 for t in range(32)]
+    assert wavefronts(addrs, 4) == optimal(4)
 
 
-def test_row_pass_slices_hold_lane_rows():
-    # the element-stride-4 boxes put row 4*r_hi + r_lo of plane g at
-    # slice r_lo, offset g*256 + r_hi*16: lane t's rows 4t..4t+3 are its 4 slices
-    seen = set()
-    for g, r_lo, r_hi in itertools.product(range(2), range(4), range(16)):
-        off = r_lo * 512 + g * 256 + r_hi * 16
-        assert off not in seen
-        seen.add(off)
-    assert len(seen) == 2 * 64 and max(seen) + 16 == BOX
+def test_swizzle_is_a_permutation_of_a_box():
+    assert sorted(swz128(r * 16) for r in range(64)) == [r * 16 for r in range(64)]
