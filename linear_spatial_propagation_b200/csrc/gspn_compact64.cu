@@ -31,11 +31,14 @@
 //   each pass the direction that reaches a pixel first stores, the second
 //   adds, so every Hacc element is stored and loaded the fewest times.
 // * All x / lambda traffic is streamed by TMA into a per-warp ring of 4 KB
-//   stages (8 scan steps each): column chunks (8 columns x 64 rows, one box
-//   per tensor, 128-byte swizzle so that the 16-byte row pieces of 8 lanes
-//   land in 8 different bank quads) for the row pass and row chunks (64
-//   columns x 8 rows) for the column pass.  A stage is copied to registers at
-//   its start and immediately refilled, so NST stages per warp stay in flight.
+//   stages (8 scan steps each): column chunks (8 columns x 64 rows) for the
+//   row pass and row chunks (64 columns x 8 rows) for the column pass.  A
+//   column chunk is fetched as two boxes of every other row (row element
+//   stride 2), so rows 2t and 2t+1 of lane t sit in two 512-byte slices and
+//   the 16-byte reads of 8 lanes cover 128 contiguous bytes.  (A 16-byte wide
+//   box with the 128-byte swizzle would put every row on its own 128-byte
+//   line, eight times the space.)  A stage is copied to registers at its
+//   start and immediately refilled, so NST stages per warp stay in flight.
 // * Hacc uses an XOR layout of 8-byte units, conflict-free for the row pass
 //   (each lane stores rows 2t, 2t+1 at one column pair) and for the column
 //   pass (each lane reads columns 2t, 2t+1 of one row).
@@ -60,7 +63,7 @@ constexpr int BAR_BYTES = 8 * NST;
 constexpr int SMEM_BYTES = 1024 + NWARP * WARP_BYTES + NWARP * BAR_BYTES;
 constexpr int CHUNKS_PER_UNIT = 16;  // 8 column chunks + 8 row chunks
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(WARP_BYTES % 1024 == 0, "stages must stay 1024-byte aligned for the 128-byte swizzle");
+static_assert(WARP_BYTES % 1024 == 0, "per-warp regions keep TMA destinations 1024-byte aligned");
 
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -216,10 +219,13 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         if (local < 8) {
             const int q = local;
             // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at 8(7-q)..
-            tma::load_3d(dst + 0 * BOX, &tm_xc, 8 * q, 0, plane, bar);
-            tma::load_3d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 2 * BC + plane, bar);
-            tma::load_3d(dst + 2 * BOX, &tm_xc, 8 * (7 - q), 0, plane, bar);
-            tma::load_3d(dst + 3 * BOX, &tm_lc, 8 * (7 - q), 0, 3 * BC + plane, bar);
+            // rows r_lo, r_lo + 2, ... of each tensor go to slice r_lo (512 bytes)
+            for (int r = 0; r < 2; ++r) {
+                tma::load_3d(dst + 0 * BOX + r * 512, &tm_xc, 8 * q, r, plane, bar);
+                tma::load_3d(dst + 1 * BOX + r * 512, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
+                tma::load_3d(dst + 2 * BOX + r * 512, &tm_xc, 8 * (7 - q), r, plane, bar);
+                tma::load_3d(dst + 3 * BOX + r * 512, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
+            }
         } else {
             const int q = local - 8;
             // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 56-8q..
@@ -276,11 +282,11 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     };
 
     // Row pass: lane t owns rows 2t, 2t+1 (unit XOR key t & 15); the 16-byte
-    // piece of row r in a swizzled column-chunk box sits at r*16 ^ ((r>>3)&7)<<4.
+    // piece of row 2t + p of a column chunk sits at p*512 + t*16.
     const uint32_t hrow = hacc + (uint32_t)(2 * t) * 256u;
     const int tk = t & 15;
-    const uint32_t cpiece0 = (uint32_t)((2 * t) * 16) ^ (uint32_t)(((t >> 2) & 7) << 4);
-    const uint32_t cpiece1 = (uint32_t)((2 * t + 1) * 16) ^ (uint32_t)(((t >> 2) & 7) << 4);
+    const uint32_t cpiece0 = (uint32_t)(t * 16);
+    const uint32_t cpiece1 = 512u + (uint32_t)(t * 16);
 
     for (int plane = wid; plane < a.units; plane += wstride) {
         __nv_bfloat16* outp = a.out + (size_t)plane * S * S + 2 * t;
@@ -405,17 +411,19 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view (column, row, plane) of a stack of 64x64 bf16 planes; one plane per box.
-bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r,
-              CUtensorMapSwizzle swz, CUtensorMapL2promotion promo) {
+// 3-D view (column, row, plane) of a stack of 64x64 bf16 planes; one plane per
+// box, every `row_step`-th row.
+bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r, uint32_t row_step,
+              CUtensorMapL2promotion promo) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, S * S * 2};
     const cuuint32_t box[3] = {box_c, box_r, 1};
-    const cuuint32_t es[3] = {1, 1, 1};
+    const cuuint32_t es[3] = {1, row_step, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, promo, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
@@ -433,11 +441,11 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
                     void* out, void* ws, cudaStream_t s) {
     CUtensorMap xc, lc, xr, lr;
     const uint64_t BC = (uint64_t)p.planes;
-    // column chunks: 8 columns x 64 rows (swizzled 16-byte pieces); row chunks: 64 columns x 8 rows
-    if (!make_map(&xc, x, BC, 8, 64, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
-        !make_map(&lc, lam, 4 * BC, 8, 64, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
-        !make_map(&xr, x, BC, 64, 8, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
-        !make_map(&lr, lam, 4 * BC, 64, 8, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+    // column chunks: 8 columns x every other row (32 rows); row chunks: 64 columns x 8 rows
+    if (!make_map(&xc, x, BC, 8, 64, 2, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&lc, lam, 4 * BC, 8, 64, 2, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&xr, x, BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+        !make_map(&lr, lam, 4 * BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
         return GSPN_ERR_UNSUPPORTED;
     char* w = static_cast<char*>(ws);
     C64Args a;

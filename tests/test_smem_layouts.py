@@ -18,12 +18,6 @@ def hacc_off(r, u):
     return r * 256 + ((u ^ ((r >> 1) & 15)) << 3)
 
 
-def swz128(a):
-    """TMA 128-byte swizzle: the 16-byte piece index within each 128-byte line
-    is XORed with the line index mod 8 (buffer 1024-byte aligned)."""
-    return a ^ (((a >> 7) & 7) << 4)
-
-
 def wavefronts(addrs, width):
     """Wavefronts a warp access needs: addrs[lane] = byte address."""
     lanes_per_phase = {4: 32, 8: 16, 16: 8}[width]
@@ -64,16 +58,15 @@ def test_column_pass_hacc_loads(s):
 
 @pytest.mark.parametrize("box,p", list(itertools.product(range(4), range(2))))
 def test_row_pass_stage_reads(box, p):
-    # column chunk box: 64 rows of 16 bytes, 128-byte swizzle; lane t reads rows 2t, 2t+1
-    addrs = [box * BOX + swz128((2 * t + p) * 16) for t in range(32)]
+    # column chunk: two boxes of every other row (element stride 2); row
+    # 2*r_hi + r_lo sits at r_lo*512 + r_hi*16; lane t reads rows 2t, 2t+1
+    addrs = [box * BOX + p * 512 + t * 16 for t in range(32)]
     assert wavefronts(addrs, 16) == optimal(16)
 
 
-def test_kernel_piece_offsets_match_the_swizzle():
-    # the kernel precomputes (2t+p)*16 ^ ((t>>2)&7)<<4
-    for t in range(32):
-        for p in range(2):
-            assert swz128((2 * t + p) * 16) == ((2 * t + p) * 16) ^ (((t >> 2) & 7) << 4)
+def test_column_chunk_slices_cover_the_box():
+    offs = sorted(r_lo * 512 + r_hi * 16 for r_lo in range(2) for r_hi in range(32))
+    assert offs == [16 * i for i in range(64)]
 
 
 @pytest.mark.parametrize("box,e", list(itertools.product(range(4), range(8))))
@@ -82,6 +75,3 @@ def test_column_pass_stage_reads(box, e):
     addrs = [box * BOX + e * 128 + t * 4 for t in range(32)]
     assert wavefronts(addrs, 4) == optimal(4)
 
-
-def test_swizzle_is_a_permutation_of_a_box():
-    assert sorted(swz128(r * 16) for r in range(64)) == [r * 16 for r in range(64)]
