@@ -14,7 +14,7 @@
 //   the logits into normalised (-w0, w2) pairs once per (b, pixel,
 //   direction) -- w1 = 1 - w0 - w2 -- laid out in scan order, so that each
 //   scan step reads one contiguous 512-byte row per warp; the main kernel
-//   reads them through L1 (prefetched 3 steps ahead) for every channel.
+//   reads them through L1 (prefetched 8 steps ahead) for every channel.
 // * One warp scans one (b, c) plane: 32 lanes per 64-wide line, 2 positions
 //   per lane; 8 warps per SM.  The two directions of a pair (left->right with
 //   right->left, top->bottom with bottom->top) advance together: lane values
@@ -44,6 +44,8 @@
 //   pass (each lane reads columns 2t, 2t+1 of one row).
 // * Every mbarrier wait is bounded (2 s); on expiry the warp records an
 //   error word in the workspace, drains its outstanding copies and returns.
+#include <type_traits>
+
 #include "gspn_internal.h"
 #include "gspn_tma.cuh"
 
@@ -181,6 +183,7 @@ struct C64Args {
     int units;  // B * C planes
 };
 
+template <bool LOCAL>
 __global__ void __launch_bounds__(NWARP * 32, 1)
     c64_fwd_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
                    const __grid_constant__ CUtensorMap tm_xr, const __grid_constant__ CUtensorMap tm_lr,
@@ -198,7 +201,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     if (wid >= a.units) return;
 
     if (t == 0) {
-        for (int k = 0; k < NST; ++k) tma::mbar_init(bar0 + 8 * k, 1);
+        for (int s = 0; s < NST; ++s) tma::mbar_init(bar0 + 8 * s, 1);
         tma::fence_barrier_init();
         tma::prefetch_map(&tm_xc);
         tma::prefetch_map(&tm_lc);
@@ -207,19 +210,19 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     }
     __syncwarp();
 
-    // Issue chunk k of this warp's sequence (lane 0 only): plane wid + (k/16)*wstride,
-    // chunk k%16 of it (0..7: column chunks, 8..15: row chunks).  lambda plane
+    // Issue chunk kk of this warp's sequence (lane 0 only): plane wid + (kk/16)*wstride,
+    // chunk kk%16 of it (0..7: column chunks, 8..15: row chunks).  lambda plane
     // (slot, b, c) is slot*B*C + plane.
-    auto issue = [&](int k) {
-        const int plane = wid + (k / CHUNKS_PER_UNIT) * wstride;
+    auto issue = [&](int kk) {
+        const int plane = wid + (kk / CHUNKS_PER_UNIT) * wstride;
         if (plane >= a.units) return;
-        const int local = k % CHUNKS_PER_UNIT, st = k % NST;
+        const int local = kk % CHUNKS_PER_UNIT, st = kk % NST;
         const uint32_t dst = ring + st * STAGE, bar = bar0 + 8 * st;
         tma::mbar_expect_tx(bar, STAGE);
         if (local < 8) {
             const int q = local;
-            // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at 8(7-q)..
-            // rows r_lo, r_lo + 2, ... of each tensor go to slice r_lo (512 bytes)
+            // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at
+            // 8(7-q)..; rows r_lo, r_lo + 2, ... of each tensor go to slice r_lo (512 bytes)
             for (int r = 0; r < 2; ++r) {
                 tma::load_3d(dst + 0 * BOX + r * 512, &tm_xc, 8 * q, r, plane, bar);
                 tma::load_3d(dst + 1 * BOX + r * 512, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
@@ -237,9 +240,11 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     };
 
     if (t == 0)
-        for (int k = 0; k < NST; ++k) issue(k);
+        for (int kk = 0; kk < NST; ++kk) issue(kk);
 
-    int k = 0;  // next chunk to consume
+    int k = 0;            // next chunk to consume
+    int stage = 0;        // k % NST
+    uint32_t phase = 0;   // bit s: parity of the next completion of stage s
     auto fail = [&]() {
         if (t == 0) atomicExch(a.err, 1);
         // drain every copy that may still be in flight, with a short bound
@@ -250,7 +255,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     };
     // wait for chunk k; false (for every lane) if any lane's wait timed out
     auto acquire = [&]() -> bool {
-        const bool ok = tma::mbar_wait(bar0 + 8 * (k % NST), (k / NST) & 1);
+        const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
         return __all_sync(FULL, ok);
     };
     // all lanes done reading the stage of chunk k: refill it with chunk k + NST
@@ -258,44 +263,46 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         tma::fence_proxy_async();
         __syncwarp();
         if (t == 0) issue(k + NST);
+        phase ^= 1u << stage;
         ++k;
+        stage = stage == NST - 1 ? 0 : stage + 1;
     };
 
-    // Tap weights of the 128 scan steps of a plane (64 row-pass, then 64
-    // column-pass) are table rows b*128 + l; they are prefetched 3 steps ahead
-    // into a 4-deep register ring, continuing into the next plane.
-    float4 wr[4][2];
+    // Tap weights: a plane's 128 scan steps (64 row-pass, then 64 column-pass)
+    // are table rows b*128 + l.  wr[e] holds the taps of the step l with
+    // l % 8 == e; right after step l uses them it is refilled with step l + 8,
+    // which continues into the next plane of this warp.
+    float4 wr[8][2];
     auto wbase = [&](int plane) -> const float4* { return a.wtab + (size_t)(plane / a.C) * 2 * S * S + t; };
     const float4* wu = wbase(wid);
     const float4* wn = wid + wstride < a.units ? wbase(wid + wstride) : wu;
 #pragma unroll
-    for (int l = 0; l < 3; ++l) {
-        wr[l][0] = __ldg(wu + l * S);
-        wr[l][1] = __ldg(wu + l * S + LPL);
+    for (int e = 0; e < 8; ++e) {
+        wr[e][0] = __ldg(wu + e * S);
+        wr[e][1] = __ldg(wu + e * S + LPL);
     }
-    // load the weights of plane step l + 3 into ring slot `slot`
-    auto prefetch_w = [&](int l, int slot) {
-        const int ls = l + 3;
-        const float4* src = ls < 2 * S ? wu + ls * S : wn + (ls - 2 * S) * S;
-        wr[slot][0] = __ldg(src);
-        wr[slot][1] = __ldg(src + LPL);
-    };
+    // first table row of the refills issued by the chunk starting at plane step l0
+    auto wnext = [&](int l0) -> const float4* { return l0 + 8 < 2 * S ? wu + (l0 + 8) * S : wn; };
 
-    // Row pass: lane t owns rows 2t, 2t+1 (unit XOR key t & 15); the 16-byte
+    // Row pass: lane t owns rows 2t, 2t+1 (Hacc unit XOR key t & 15); the 16-byte
     // piece of row 2t + p of a column chunk sits at p*512 + t*16.
     const uint32_t hrow = hacc + (uint32_t)(2 * t) * 256u;
-    const int tk = t & 15;
+    const uint32_t tk8 = (uint32_t)(t & 15) << 3;
+    const uint32_t t8 = (uint32_t)t << 3;
     const uint32_t cpiece0 = (uint32_t)(t * 16);
     const uint32_t cpiece1 = 512u + (uint32_t)(t * 16);
+    float2 h[2];
+    __nv_bfloat16* outp = nullptr;
 
-    for (int plane = wid; plane < a.units; plane += wstride) {
-        __nv_bfloat16* outp = a.out + (size_t)plane * S * S + 2 * t;
-
-        // ---------------- row pass: left->right (x) and right->left (y) ----------------
-        float2 h[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        for (int q = 0; q < 8; ++q) {
-            if (!acquire()) { fail(); return; }
-            const uint32_t st = ring + (k % NST) * STAGE;
+    // Four column chunks of the row pass: left->right (x) and right->left (y).
+    // SECOND: the chunks q = 4..7, where both directions are the second to reach
+    // their columns and add to Hacc.
+    auto row_half = [&](auto second) -> bool {
+        constexpr bool SECOND = decltype(second)::value;
+        for (int qq = 0; qq < 4; ++qq) {
+            const int q = SECOND ? qq + 4 : qq;
+            if (!acquire()) return false;
+            const uint32_t st = ring + stage * STAGE;
             uint4 XA[2], LA[2], XB[2], LB[2];
             XA[0] = lds128(st + 0 * BOX + cpiece0);
             XA[1] = lds128(st + 0 * BOX + cpiece1);
@@ -306,14 +313,14 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             LB[0] = lds128(st + 3 * BOX + cpiece0);
             LB[1] = lds128(st + 3 * BOX + cpiece1);
             release();
+            const float4* wp = wnext(8 * q);
+            const uint32_t q8 = (uint32_t)(4 * q) << 3;
             float2 prev[2];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int s = 8 * q + e;
-                prefetch_w(s, (e + 3) & 3);
-                if ((s & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
-                // left->right reads column s = element e of the A chunk; right->left
-                // column 63-s = element 7-e of the B chunk
+                if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
+                // left->right reads column 8q+e = element e of the A chunk; right->left
+                // column 63-8q-e = element 7-e of the B chunk
                 float2 base[2];
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {
@@ -321,18 +328,20 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                     base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1),
                                        h[p].y);
                 }
-                scan_core(h, base, wr[e & 3]);
+                scan_core(h, base, wr[e]);
+                wr[e][0] = __ldg(wp + e * S);
+                wr[e][1] = __ldg(wp + e * S + LPL);
                 if (e & 1) {
-                    // left->right covers columns s-1, s (unit s/2); right->left covers
-                    // columns 63-s, 64-s (unit (63-s)/2)
-                    const uint32_t oA = (uint32_t)(((s >> 1) ^ tk) << 3);
-                    const uint32_t oB = (uint32_t)((((S - 1 - s) >> 1) ^ tk) << 3);
+                    // left->right covers columns s-1, s (unit s/2 = 4q + e/2), right->left
+                    // columns 63-s, 64-s (unit 31 - (4q + e/2)); XOR with the row key
+                    const uint32_t oA = (q8 + (uint32_t)((e >> 1) << 3)) ^ tk8;
+                    const uint32_t oB = oA ^ (31u << 3);
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
                         const uint32_t adA = hrow + p * 256 + oA, adB = hrow + p * 256 + oB;
                         float2 vA = make_float2(prev[p].x, h[p].x);
                         float2 vB = make_float2(h[p].y, prev[p].y);
-                        if (q >= 4) {  // second arrival: add the other direction
+                        if (SECOND) {
                             vA = __fadd2_rn(vA, lds64f(adA));
                             vB = __fadd2_rn(vB, lds64f(adB));
                         }
@@ -345,13 +354,17 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                 }
             }
         }
-        __syncwarp();
+        return true;
+    };
 
-        // ---------------- column pass: top->bottom (x) and bottom->top (y) ----------------
-        h[0] = h[1] = make_float2(0.f, 0.f);
-        for (int q = 0; q < 8; ++q) {
-            if (!acquire()) { fail(); return; }
-            const uint32_t st = ring + (k % NST) * STAGE + t * 4;
+    // Four row chunks of the column pass: top->bottom (x) and bottom->top (y).
+    // SECOND: the chunks q = 4..7, which complete their pixels and store them.
+    auto col_half = [&](auto second) -> bool {
+        constexpr bool SECOND = decltype(second)::value;
+        for (int qq = 0; qq < 4; ++qq) {
+            const int q = SECOND ? qq + 4 : qq;
+            if (!acquire()) return false;
+            const uint32_t st = ring + stage * STAGE + t * 4;
             uint32_t XA[8], LA[8], XB[8], LB[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -361,30 +374,49 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                 LB[e] = lds32(st + 3 * BOX + (7 - e) * 128);
             }
             release();
+            const float4* wp = wnext(S + 8 * q);
+            // rows s = 8q + e (top->bottom) and 63 - s (bottom->top); the Hacc unit key
+            // of row s is ((4q) & 15) + e/2, that of row 63 - s is 15 minus it
+            const uint32_t hA = hacc + (uint32_t)(8 * q) * 256u;
+            const uint32_t hB = hacc + (uint32_t)(S - 1 - 8 * q) * 256u;
+            const uint32_t k8 = (uint32_t)((4 * q) & 15) << 3;
+            __nv_bfloat16* oA_row = outp + (8 * q) * S;
+            __nv_bfloat16* oB_row = outp + (S - 1 - 8 * q) * S;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const int s = 8 * q + e;
-                prefetch_w(S + s, (e + 3) & 3);
-                if ((s & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
+                if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
                 float2 base[2];
                 base[0].x = fma_bf_lo(LA[e], XA[e], h[0].x);
                 base[1].x = fma_bf_hi(LA[e], XA[e], h[1].x);
                 base[0].y = fma_bf_lo(LB[e], XB[e], h[0].y);
                 base[1].y = fma_bf_hi(LB[e], XB[e], h[1].y);
-                scan_core(h, base, wr[e & 3]);
-                const int rA = s, rB = S - 1 - s;
-                const uint32_t adA = hacc + hacc_off(rA, t), adB = hacc + hacc_off(rB, t);
+                scan_core(h, base, wr[e]);
+                wr[e][0] = __ldg(wp + e * S);
+                wr[e][1] = __ldg(wp + e * S + LPL);
+                const uint32_t oA = (k8 + (uint32_t)((e >> 1) << 3)) ^ t8;
+                const uint32_t oB = oA ^ (15u << 3);
+                const uint32_t adA = hA + e * 256 + oA, adB = hB - e * 256 + oB;
                 const float2 vA = __fadd2_rn(lds64f(adA), make_float2(h[0].x, h[1].x));
                 const float2 vB = __fadd2_rn(lds64f(adB), make_float2(h[0].y, h[1].y));
-                if (q < 4) {  // first arrival of this pass: keep the partial sum
+                if (!SECOND) {  // first arrival of this pass: keep the partial sum
                     sts64f(adA, vA);
                     sts64f(adB, vB);
-                } else {      // second arrival: the pixel is complete
-                    stg_cs32(outp + rA * S, pack_bf2(vA.x, vA.y));
-                    stg_cs32(outp + rB * S, pack_bf2(vB.x, vB.y));
+                } else {        // second arrival: the pixel is complete
+                    stg_cs32(oA_row + e * S, pack_bf2(vA.x, vA.y));
+                    stg_cs32(oB_row - e * S, pack_bf2(vB.x, vB.y));
                 }
             }
         }
+        return true;
+    };
+
+    for (int plane = wid; plane < a.units; plane += wstride) {
+        outp = a.out + (size_t)plane * S * S + 2 * t;
+        h[0] = h[1] = make_float2(0.f, 0.f);
+        if (!row_half(std::false_type{}) || !row_half(std::true_type{})) { fail(); return; }
+        __syncwarp();
+        h[0] = h[1] = make_float2(0.f, 0.f);
+        if (!col_half(std::false_type{}) || !col_half(std::true_type{})) { fail(); return; }
         __syncwarp();
         wu = wn;
         wn = plane + 2 * wstride < a.units ? wbase(plane + 2 * wstride) : wu;
@@ -461,12 +493,17 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
         static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.wtab), a.err, p.g.B);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
-    e = ensure_smem_attr((const void*)c64_fwd_kernel, SMEM_BYTES, 8);
+    const bool local = p.g.groups > 1;
+    const void* fn = local ? (const void*)c64_fwd_kernel<true> : (const void*)c64_fwd_kernel<false>;
+    e = ensure_smem_attr(fn, SMEM_BYTES, local ? 9 : 8);
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
     int grid = dev.sm_count;
     const int need = (a.units + NWARP - 1) / NWARP;
     if (need < grid) grid = need;
-    c64_fwd_kernel<<<grid, NWARP * 32, SMEM_BYTES, s>>>(xc, lc, xr, lr, a);
+    if (local)
+        c64_fwd_kernel<true><<<grid, NWARP * 32, SMEM_BYTES, s>>>(xc, lc, xr, lr, a);
+    else
+        c64_fwd_kernel<false><<<grid, NWARP * 32, SMEM_BYTES, s>>>(xc, lc, xr, lr, a);
     e = cudaGetLastError();
     return e == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
 }
