@@ -101,26 +101,16 @@ __global__ void c64_weights_kernel(const T* __restrict__ logits, float4* __restr
 }
 
 // ---- helpers ----------------------------------------------------------------------
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-    uint4 v;
-    asm volatile("ld.shared.v4.b32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ float2 lds64f(uint32_t a) {
-    float2 v;
-    asm volatile("ld.shared.v2.f32 {%0,%1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ void sts64f(uint32_t a, float2 v) {
-    asm volatile("st.shared.v2.f32 [%0], {%1,%2};" ::"r"(a), "f"(v.x), "f"(v.y) : "memory");
-}
-__device__ __forceinline__ void stg_cs32(void* p, uint32_t v) {
-    asm volatile("st.global.cs.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+// Shared memory is addressed through ordinary pointers into the dynamic
+// shared array, so the compiler folds constant offsets into the accesses; the
+// TMA-written data is read only after the mbarrier wait (an asm with a memory
+// clobber), which orders these loads behind it.
+__device__ __forceinline__ uint4 lds128(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ uint32_t lds32(const unsigned char* p) { return *reinterpret_cast<const uint32_t*>(p); }
+__device__ __forceinline__ float2 lds64f(const unsigned char* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ void sts64f(unsigned char* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+__device__ __forceinline__ void stg_cs32(__nv_bfloat16* p, uint32_t v) {
+    __stcs(reinterpret_cast<unsigned int*>(p), v);
 }
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
@@ -188,11 +178,13 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
     c64_fwd_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
                    const __grid_constant__ CUtensorMap tm_xr, const __grid_constant__ CUtensorMap tm_lr,
                    const C64Args a) {
-    extern __shared__ unsigned char smem_raw[];
-    const uint32_t sbase = (tma::smem_u32(smem_raw) + 1023u) & ~1023u;
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* const smem = smem_raw + ((1024u - (tma::smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = tma::smem_u32(smem);
     const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
-    const uint32_t ring = sbase + warp * WARP_BYTES;
-    const uint32_t hacc = ring + NST * STAGE;
+    const uint32_t ring = sbase + warp * WARP_BYTES;   // shared-window address (TMA)
+    unsigned char* const ringp = smem + warp * WARP_BYTES;  // same bytes, for loads
+    unsigned char* const haccp = ringp + NST * STAGE;
     const uint32_t bar0 = sbase + NWARP * WARP_BYTES + warp * BAR_BYTES;
     const int wid = blockIdx.x * NWARP + warp;
     const int wstride = gridDim.x * NWARP;
@@ -286,7 +278,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
 
     // Row pass: lane t owns rows 2t, 2t+1 (Hacc unit XOR key t & 15); the 16-byte
     // piece of row 2t + p of a column chunk sits at p*512 + t*16.
-    const uint32_t hrow = hacc + (uint32_t)(2 * t) * 256u;
+    unsigned char* const hrow = haccp + 2 * t * 256;
     const uint32_t tk8 = (uint32_t)(t & 15) << 3;
     const uint32_t t8 = (uint32_t)t << 3;
     const uint32_t cpiece0 = (uint32_t)(t * 16);
@@ -302,7 +294,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         for (int qq = 0; qq < 4; ++qq) {
             const int q = SECOND ? qq + 4 : qq;
             if (!acquire()) return false;
-            const uint32_t st = ring + stage * STAGE;
+            const unsigned char* st = ringp + stage * STAGE;
             uint4 XA[2], LA[2], XB[2], LB[2];
             XA[0] = lds128(st + 0 * BOX + cpiece0);
             XA[1] = lds128(st + 0 * BOX + cpiece1);
@@ -338,7 +330,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                     const uint32_t oB = oA ^ (31u << 3);
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        const uint32_t adA = hrow + p * 256 + oA, adB = hrow + p * 256 + oB;
+                        unsigned char* adA = hrow + p * 256 + oA;
+                        unsigned char* adB = hrow + p * 256 + oB;
                         float2 vA = make_float2(prev[p].x, h[p].x);
                         float2 vB = make_float2(h[p].y, prev[p].y);
                         if (SECOND) {
@@ -364,7 +357,7 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
         for (int qq = 0; qq < 4; ++qq) {
             const int q = SECOND ? qq + 4 : qq;
             if (!acquire()) return false;
-            const uint32_t st = ring + stage * STAGE + t * 4;
+            const unsigned char* st = ringp + stage * STAGE + t * 4;
             uint32_t XA[8], LA[8], XB[8], LB[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
@@ -377,8 +370,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
             const float4* wp = wnext(S + 8 * q);
             // rows s = 8q + e (top->bottom) and 63 - s (bottom->top); the Hacc unit key
             // of row s is ((4q) & 15) + e/2, that of row 63 - s is 15 minus it
-            const uint32_t hA = hacc + (uint32_t)(8 * q) * 256u;
-            const uint32_t hB = hacc + (uint32_t)(S - 1 - 8 * q) * 256u;
+            unsigned char* const hA = haccp + 8 * q * 256;
+            unsigned char* const hB = haccp + (S - 1 - 8 * q) * 256;
             const uint32_t k8 = (uint32_t)((4 * q) & 15) << 3;
             __nv_bfloat16* oA_row = outp + (8 * q) * S;
             __nv_bfloat16* oB_row = outp + (S - 1 - 8 * q) * S;
@@ -395,7 +388,8 @@ __global__ void __launch_bounds__(NWARP * 32, 1)
                 wr[e][1] = __ldg(wp + e * S + LPL);
                 const uint32_t oA = (k8 + (uint32_t)((e >> 1) << 3)) ^ t8;
                 const uint32_t oB = oA ^ (15u << 3);
-                const uint32_t adA = hA + e * 256 + oA, adB = hB - e * 256 + oB;
+                unsigned char* adA = hA + e * 256 + oA;
+                unsigned char* adB = hB - e * 256 + oB;
                 const float2 vA = __fadd2_rn(lds64f(adA), make_float2(h[0].x, h[1].x));
                 const float2 vB = __fadd2_rn(lds64f(adB), make_float2(h[0].y, h[1].y));
                 if (!SECOND) {  // first arrival of this pass: keep the partial sum
