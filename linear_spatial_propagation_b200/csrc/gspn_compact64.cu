@@ -12,16 +12,19 @@
 // Design (B200):
 // * The tap weights depend only on (b, pixel, direction).  A pre-kernel turns
 //   the logits into normalised (-w0, w2) pairs once per (b, pixel,
-//   direction) -- w1 = 1 - w0 - w2 -- laid out in scan order, so that each
-//   scan step reads one contiguous 512-byte row per warp; the main kernel
-//   reads them through L1 (prefetched 8 steps ahead) for every channel.
-// * One warp scans KC (2 when C is even, else 1) planes of one batch image:
-//   32 lanes per 64-wide line, 2 positions per lane, the KC channels in the
-//   same lane so that each step's tap weights are loaded once for all of
-//   them; 8 / KC warps per SM.  The two directions of a pair (left->right with
-//   right->left, top->bottom with bottom->top) advance together: lane values
-//   are float2 (one direction per half) and the update is the packed fp32x2
-//   FMA of sm_100; lambda*x is one mixed-precision FMA with bf16 inputs.
+//   direction) -- w1 = 1 - w0 - w2 -- in scan order: table row b*128 + l
+//   holds the 64 positions of plane step l (64 row-pass then 64 column-pass
+//   steps), 1 KB per row.
+// * A CTA (one per SM) scans groups of 8 consecutive planes of one batch
+//   image, one plane per consumer warp, 32 lanes per 64-wide line and 2
+//   positions per lane.  The 8 warps step through the same sequence of
+//   8-step chunks, so one producer warp streams each chunk's tap weights
+//   (8 table rows, 8 KB) with a single bulk copy into a 2-stage ring that all
+//   8 warps read; each warp copies the chunk to registers and releases it.
+// * The two directions of a pair (left->right with right->left, top->bottom
+//   with bottom->top) advance together: lane values are float2 (one
+//   direction per half) and the update is the packed fp32x2 FMA of sm_100;
+//   lambda*x is one mixed-precision FMA with bf16 inputs.
 // * Update in difference form, h'[p] = h[p] + lambda x + w2 (h[p+1] - h[p])
 //   - w0 (h[p] - h[p-1]), equal to w0 h[p-1] + w1 h[p] + w2 h[p+1] + lambda x
 //   for w1 = 1 - w0 - w2; the line ends have w0 = 0 / w2 = 0.  Neighbours
@@ -32,15 +35,15 @@
 //   directions and writes each output row once, 128 contiguous bytes.  In
 //   each pass the direction that reaches a pixel first stores, the second
 //   adds, so every Hacc element is stored and loaded the fewest times.
-// * All x / lambda traffic is streamed by TMA into a per-warp ring of 4 KB
-//   stages (8 scan steps each): column chunks (8 columns x 64 rows) for the
-//   row pass and row chunks (64 columns x 8 rows) for the column pass.  A
-//   column chunk is fetched as two boxes of every other row (row element
-//   stride 2), so rows 2t and 2t+1 of lane t sit in two 512-byte slices and
-//   the 16-byte reads of 8 lanes cover 128 contiguous bytes.  (A 16-byte wide
-//   box with the 128-byte swizzle would put every row on its own 128-byte
-//   line, eight times the space.)  A stage is copied to registers at its
-//   start and immediately refilled, so NST stages per warp stay in flight.
+// * x / lambda are streamed by TMA into a per-warp ring of 4 KB stages (8
+//   scan steps each): column chunks (8 columns x 64 rows) for the row pass
+//   and row chunks (64 columns x 8 rows) for the column pass.  A column chunk
+//   is fetched as two boxes of every other row (row element stride 2), so
+//   rows 2t and 2t+1 of lane t sit in two 512-byte slices and the 16-byte
+//   reads of 8 lanes cover 128 contiguous bytes.  (A 16-byte wide box with
+//   the 128-byte swizzle would put every row on its own 128-byte line, eight
+//   times the space.)  A stage is copied to registers at its start and
+//   immediately refilled.
 // * Hacc uses an XOR layout of 8-byte units, conflict-free for the row pass
 //   (each lane stores rows 2t, 2t+1 at one column pair) and for the column
 //   pass (each lane reads columns 2t, 2t+1 of one row).
@@ -55,27 +58,25 @@ namespace gspn {
 
 namespace {
 
-constexpr int S = 64;         // H = W
-constexpr int LPL = 32;       // lanes per line (2 positions per lane)
-constexpr int NST = 3;        // ring stages per warp
-constexpr int SLICE = 512;    // bytes of one plane in one element-stride-2 column box
+// ---- kernel configuration ------------------------------------------------------------
+constexpr int S = 64;          // H = W
+constexpr int LPL = 32;        // lanes per line (2 positions per lane)
+constexpr int NCW = 8;         // consumer warps per CTA (one plane each), one CTA per SM
+constexpr int NST = 2;         // x/lambda ring stages per consumer warp
+constexpr int NWS = 2;         // tap-weight ring stages per CTA
+constexpr int BOX = 1024;      // bytes per TMA box (one plane)
+constexpr int SLICE = 512;     // one element-stride-2 column box
+constexpr int STAGE = 4 * BOX;
 constexpr int HACC = S * S * 4;
-constexpr int CHUNKS_PER_UNIT = 16;  // 8 column chunks + 8 row chunks
-constexpr int SMEM_OPTIN = 232448;
-
-// KC channels per lane (the tap weights of a step are loaded once for all of
-// them); 8 / KC warps per CTA, one CTA per SM.
-template <int KC>
-struct Cfg {
-    static constexpr int NWARP = 8 / KC;
-    static constexpr int BOX = KC * 1024;           // bytes per tensor per stage (KC planes)
-    static constexpr int STAGE = 4 * BOX;
-    static constexpr int WARP_BYTES = NST * STAGE + KC * HACC;
-    static constexpr int BAR_BYTES = 8 * NST;
-    static constexpr int SMEM_BYTES = 1024 + NWARP * WARP_BYTES + NWARP * BAR_BYTES;
-    static_assert(SMEM_BYTES <= SMEM_OPTIN, "shared memory budget");
-    static_assert(WARP_BYTES % 1024 == 0, "per-warp regions keep TMA destinations 1024-byte aligned");
-};
+constexpr int WCHUNK = 8 * S * 16;  // tap weights of 8 scan steps (8 table rows)
+constexpr int WARP_BYTES = NST * STAGE + HACC;
+constexpr int WRING = NCW * WARP_BYTES;              // offset of the weight ring
+constexpr int BARS = WRING + NWS * WCHUNK;           // offset of the barriers
+constexpr int SMEM_BYTES = 1024 + BARS + 8 * (NCW * NST + 2 * NWS);
+constexpr int CHUNKS_PER_GROUP = 16;  // 8 column chunks + 8 row chunks
+constexpr int THREADS = (NCW + 1) * 32;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+static_assert(WARP_BYTES % 1024 == 0 && WCHUNK % 1024 == 0, "TMA destinations stay 1024-byte aligned");
 
 constexpr unsigned FULL = 0xffffffffu;
 
@@ -116,6 +117,7 @@ __global__ void c64_weights_kernel(const T* __restrict__ logits, float4* __restr
 // TMA-written data is read only after the mbarrier wait (an asm with a memory
 // clobber), which orders these loads behind it.
 __device__ __forceinline__ uint4 lds128(const unsigned char* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ float4 lds128f(const unsigned char* p) { return *reinterpret_cast<const float4*>(p); }
 __device__ __forceinline__ uint32_t lds32(const unsigned char* p) { return *reinterpret_cast<const uint32_t*>(p); }
 __device__ __forceinline__ float2 lds64f(const unsigned char* p) { return *reinterpret_cast<const float2*>(p); }
 __device__ __forceinline__ void sts64f(unsigned char* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
@@ -180,90 +182,139 @@ struct C64Args {
     __nv_bfloat16* out;
     int* err;
     int B, C, seg;
-    int units;  // B * C / KC units of KC consecutive planes
+    int groups;  // B * C / 8 groups of 8 consecutive planes (one batch image each)
 };
 
-template <int KC, bool LOCAL>
-__global__ void __launch_bounds__(Cfg<KC>::NWARP * 32, 1)
+template <bool LOCAL>
+__global__ void __launch_bounds__(THREADS, 1)
     c64_fwd_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
                    const __grid_constant__ CUtensorMap tm_xr, const __grid_constant__ CUtensorMap tm_lr,
                    const C64Args a) {
-    using K = Cfg<KC>;
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* const smem = smem_raw + ((1024u - (tma::smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = tma::smem_u32(smem);
     const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
-    const uint32_t ring = sbase + warp * K::WARP_BYTES;        // shared-window address (TMA)
-    unsigned char* const ringp = smem + warp * K::WARP_BYTES;  // same bytes, for loads
-    unsigned char* const haccp = ringp + NST * K::STAGE;       // KC planes of fp32
-    const uint32_t bar0 = sbase + K::NWARP * K::WARP_BYTES + warp * K::BAR_BYTES;
-    const int wid = blockIdx.x * K::NWARP + warp;
-    const int wstride = gridDim.x * K::NWARP;
+    const uint32_t wfull0 = sbase + BARS + 8 * NCW * NST;  // NWS "weights landed" barriers
+    const uint32_t wempty0 = wfull0 + 8 * NWS;             // NWS "weights consumed" barriers
+    if ((int)blockIdx.x >= a.groups) return;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NCW * NST; ++s) tma::mbar_init(sbase + BARS + 8 * s, 1);
+        for (int s = 0; s < NWS; ++s) {
+            tma::mbar_init(wfull0 + 8 * s, 1);
+            tma::mbar_init(wempty0 + 8 * s, NCW);
+        }
+        tma::fence_barrier_init();
+    }
+    __syncthreads();
+
+    const int ngroups_here = (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int nchunks = ngroups_here * CHUNKS_PER_GROUP;
+
+    // ---------------- producer warp: tap-weight chunks of this CTA's groups ----------------
+    if (warp == NCW) {
+        if (t == 0) {
+            for (int kc = 0; kc < nchunks; ++kc) {
+                const int ws = kc % NWS;
+                if (!tma::mbar_wait(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1)) {
+                    atomicExch(a.err, 1);
+                    break;
+                }
+                const int group = (int)blockIdx.x + (kc / CHUNKS_PER_GROUP) * (int)gridDim.x;
+                const int b = (8 * group) / a.C;
+                const float4* src = a.wtab + ((size_t)b * 2 * S + 8 * (kc % CHUNKS_PER_GROUP)) * S;
+                tma::mbar_expect_tx(wfull0 + 8 * ws, WCHUNK);
+                tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumer warps: one plane each ----------------
+    const uint32_t ring = sbase + warp * WARP_BYTES;        // shared-window address (TMA)
+    unsigned char* const ringp = smem + warp * WARP_BYTES;  // same bytes, for loads
+    unsigned char* const haccp = ringp + NST * STAGE;
+    const unsigned char* const wring = smem + WRING;
+    const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
     const int segmask = a.seg - 1;  // seg divides 64, so it is a power of two
     const int BC = a.B * a.C;
-    if (wid >= a.units) return;
 
     if (t == 0) {
-        for (int s = 0; s < NST; ++s) tma::mbar_init(bar0 + 8 * s, 1);
-        tma::fence_barrier_init();
         tma::prefetch_map(&tm_xc);
         tma::prefetch_map(&tm_lc);
         tma::prefetch_map(&tm_xr);
         tma::prefetch_map(&tm_lr);
     }
-    __syncwarp();
 
-    // Issue chunk kk of this warp's sequence (lane 0 only): unit wid + (kk/16)*wstride
-    // (planes KC*unit ..), chunk kk%16 of it (0..7: column chunks, 8..15: row
-    // chunks).  lambda plane (slot, b, c) is slot*B*C + plane.
+    // Issue chunk kk of this warp's sequence (lane 0 only): plane 8*group + warp of
+    // group blockIdx.x + (kk/16)*gridDim.x, chunk kk%16 (0..7: column chunks,
+    // 8..15: row chunks).  lambda plane (slot, b, c) is slot*B*C + plane.
     auto issue = [&](int kk) {
-        const int unit = wid + (kk / CHUNKS_PER_UNIT) * wstride;
-        if (unit >= a.units) return;
-        const int plane = KC * unit;
-        const int local = kk % CHUNKS_PER_UNIT, st = kk % NST;
-        const uint32_t dst = ring + st * K::STAGE, bar = bar0 + 8 * st;
-        tma::mbar_expect_tx(bar, K::STAGE);
+        if (kk >= nchunks) return;
+        const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
+        const int plane = 8 * group + warp;
+        const int local = kk % CHUNKS_PER_GROUP, st = kk % NST;
+        const uint32_t dst = ring + st * STAGE, bar = bar0 + 8 * st;
+        tma::mbar_expect_tx(bar, STAGE);
         if (local < 8) {
             const int q = local;
             // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at
-            // 8(7-q)..; rows r_lo, r_lo + 2, ... of the KC planes go to slice r_lo
+            // 8(7-q)..; rows r_lo, r_lo + 2, ... go to slice r_lo
             for (int r = 0; r < 2; ++r) {
-                const uint32_t o = r * KC * SLICE;
-                tma::load_3d(dst + 0 * K::BOX + o, &tm_xc, 8 * q, r, plane, bar);
-                tma::load_3d(dst + 1 * K::BOX + o, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
-                tma::load_3d(dst + 2 * K::BOX + o, &tm_xc, 8 * (7 - q), r, plane, bar);
-                tma::load_3d(dst + 3 * K::BOX + o, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
+                tma::load_3d(dst + 0 * BOX + r * SLICE, &tm_xc, 8 * q, r, plane, bar);
+                tma::load_3d(dst + 1 * BOX + r * SLICE, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
+                tma::load_3d(dst + 2 * BOX + r * SLICE, &tm_xc, 8 * (7 - q), r, plane, bar);
+                tma::load_3d(dst + 3 * BOX + r * SLICE, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
             }
         } else {
             const int q = local - 8;
             // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 56-8q..
-            tma::load_3d(dst + 0 * K::BOX, &tm_xr, 0, 8 * q, plane, bar);
-            tma::load_3d(dst + 1 * K::BOX, &tm_lr, 0, 8 * q, 0 * BC + plane, bar);
-            tma::load_3d(dst + 2 * K::BOX, &tm_xr, 0, 56 - 8 * q, plane, bar);
-            tma::load_3d(dst + 3 * K::BOX, &tm_lr, 0, 56 - 8 * q, 1 * BC + plane, bar);
+            tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
+            tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, 0 * BC + plane, bar);
+            tma::load_3d(dst + 2 * BOX, &tm_xr, 0, 56 - 8 * q, plane, bar);
+            tma::load_3d(dst + 3 * BOX, &tm_lr, 0, 56 - 8 * q, 1 * BC + plane, bar);
         }
     };
 
     if (t == 0)
         for (int kk = 0; kk < NST; ++kk) issue(kk);
 
-    int k = 0;            // next chunk to consume
+    int k = 0;            // next chunk to consume (same sequence for data and weights)
     int stage = 0;        // k % NST
-    uint32_t phase = 0;   // bit s: parity of the next completion of stage s
+    uint32_t phase = 0;   // bit s: parity of the next completion of data stage s
     auto fail = [&]() {
         if (t == 0) atomicExch(a.err, 1);
-        // drain every copy that may still be in flight, with a short bound
-        for (int kk = k; kk < k + NST; ++kk) {
-            const int unit = wid + (kk / CHUNKS_PER_UNIT) * wstride;
-            if (unit < a.units) tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
-        }
+        // drain every data copy that may still be in flight, with a short bound
+        for (int kk = k; kk < k + NST && kk < nchunks; ++kk)
+            tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
+        // and the weight chunks this warp has not consumed (the producer issues at
+        // most NWS ahead of the slowest consumer)
+        for (int kk = k; kk < k + NWS && kk < nchunks; ++kk)
+            tma::mbar_wait(wfull0 + 8 * (kk % NWS), (kk / NWS) & 1, 100000000ull);
     };
-    // wait for chunk k; false (for every lane) if any lane's wait timed out
+
+    // Chunk start: wait for the data stage and the weight stage of chunk k, copy
+    // both to registers, hand both stages back (data: refill with chunk k + NST;
+    // weights: one arrival per warp on the stage's "consumed" barrier).
+    float4 wr[8][2];
+    auto weights_in = [&]() -> bool {
+        const int ws = k % NWS;
+        const bool ok = tma::mbar_wait(wfull0 + 8 * ws, (k / NWS) & 1);
+        if (!__all_sync(FULL, ok)) return false;
+        const unsigned char* wsrc = wring + ws * WCHUNK + t * 16;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            wr[e][0] = lds128f(wsrc + e * 1024);
+            wr[e][1] = lds128f(wsrc + e * 1024 + 512);
+        }
+        __syncwarp();
+        if (t == 0) tma::mbar_arrive(wempty0 + 8 * ws);
+        return true;
+    };
     auto acquire = [&]() -> bool {
         const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
         return __all_sync(FULL, ok);
     };
-    // all lanes done reading the stage of chunk k: refill it with chunk k + NST
     auto release = [&]() {
         tma::fence_proxy_async();
         __syncwarp();
@@ -273,31 +324,12 @@ __global__ void __launch_bounds__(Cfg<KC>::NWARP * 32, 1)
         stage = stage == NST - 1 ? 0 : stage + 1;
     };
 
-    // Tap weights: a unit's 128 scan steps (64 row-pass, then 64 column-pass)
-    // are table rows b*128 + l.  wr[e] holds the taps of the step l with
-    // l % 8 == e; right after step l uses them it is refilled with step l + 8,
-    // which continues into the next unit of this warp.
-    float4 wr[8][2];
-    auto wbase = [&](int unit) -> const float4* {
-        return a.wtab + (size_t)((KC * unit) / a.C) * 2 * S * S + t;
-    };
-    const float4* wu = wbase(wid);
-    const float4* wn = wid + wstride < a.units ? wbase(wid + wstride) : wu;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-        wr[e][0] = __ldg(wu + e * S);
-        wr[e][1] = __ldg(wu + e * S + LPL);
-    }
-    // first table row of the refills issued by the chunk starting at unit step l0
-    auto wnext = [&](int l0) -> const float4* { return l0 + 8 < 2 * S ? wu + (l0 + 8) * S : wn; };
-
-    // Row pass: lane t owns rows 2t, 2t+1 of each of its KC planes (Hacc unit
-    // XOR key t & 15); row 2t + p of plane c of a column chunk sits at
-    // p*KC*512 + c*512 + t*16.
+    // Row pass: lane t owns rows 2t, 2t+1 (Hacc unit XOR key t & 15); row 2t + p
+    // of a column chunk sits at p*512 + t*16.
     unsigned char* const hrow = haccp + 2 * t * 256;
     const uint32_t tk8 = (uint32_t)(t & 15) << 3;
     const uint32_t t8 = (uint32_t)t << 3;
-    float2 h[KC][2];
+    float2 h[2];
     __nv_bfloat16* outp = nullptr;
 
     // Four column chunks of the row pass: left->right (x) and right->left (y).
@@ -307,70 +339,53 @@ __global__ void __launch_bounds__(Cfg<KC>::NWARP * 32, 1)
         constexpr bool SECOND = decltype(second)::value;
         for (int qq = 0; qq < 4; ++qq) {
             const int q = SECOND ? qq + 4 : qq;
-            if (!acquire()) return false;
-            const unsigned char* st = ringp + stage * K::STAGE + t * 16;
-            uint4 XA[KC][2], LA[KC][2], XB[KC][2], LB[KC][2];
+            if (!weights_in() || !acquire()) return false;
+            const unsigned char* st = ringp + stage * STAGE + t * 16;
+            uint4 XA[2], LA[2], XB[2], LB[2];
 #pragma unroll
-            for (int c = 0; c < KC; ++c)
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const int o = p * KC * SLICE + c * SLICE;
-                    XA[c][p] = lds128(st + 0 * K::BOX + o);
-                    LA[c][p] = lds128(st + 1 * K::BOX + o);
-                    XB[c][p] = lds128(st + 2 * K::BOX + o);
-                    LB[c][p] = lds128(st + 3 * K::BOX + o);
-                }
+            for (int p = 0; p < 2; ++p) {
+                XA[p] = lds128(st + 0 * BOX + p * SLICE);
+                LA[p] = lds128(st + 1 * BOX + p * SLICE);
+                XB[p] = lds128(st + 2 * BOX + p * SLICE);
+                LB[p] = lds128(st + 3 * BOX + p * SLICE);
+            }
             release();
-            const float4* wp = wnext(8 * q);
             const uint32_t q8 = (uint32_t)(4 * q) << 3;
-            float2 prev[KC][2];
+            float2 prev[2];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                if (LOCAL && ((8 * q + e) & segmask) == 0) {
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) h[c][0] = h[c][1] = make_float2(0.f, 0.f);
-                }
+                if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
                 // left->right reads column 8q+e = element e of the A chunk; right->left
                 // column 63-8q-e = element 7-e of the B chunk
+                float2 base[2];
 #pragma unroll
-                for (int c = 0; c < KC; ++c) {
-                    float2 base[2];
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        base[p].x = fma_bf(e & 1, word_of(LA[c][p], e >> 1), word_of(XA[c][p], e >> 1), h[c][p].x);
-                        base[p].y = fma_bf((7 - e) & 1, word_of(LB[c][p], (7 - e) >> 1),
-                                           word_of(XB[c][p], (7 - e) >> 1), h[c][p].y);
-                    }
-                    scan_core(h[c], base, wr[e]);
+                for (int p = 0; p < 2; ++p) {
+                    base[p].x = fma_bf(e & 1, word_of(LA[p], e >> 1), word_of(XA[p], e >> 1), h[p].x);
+                    base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1),
+                                       h[p].y);
                 }
-                wr[e][0] = __ldg(wp + e * S);
-                wr[e][1] = __ldg(wp + e * S + LPL);
+                scan_core(h, base, wr[e]);
                 if (e & 1) {
                     // left->right covers columns s-1, s (unit s/2 = 4q + e/2), right->left
                     // columns 63-s, 64-s (unit 31 - (4q + e/2)); XOR with the row key
                     const uint32_t oA = (q8 + (uint32_t)((e >> 1) << 3)) ^ tk8;
                     const uint32_t oB = oA ^ (31u << 3);
 #pragma unroll
-                    for (int c = 0; c < KC; ++c)
-#pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            unsigned char* adA = hrow + c * HACC + p * 256 + oA;
-                            unsigned char* adB = hrow + c * HACC + p * 256 + oB;
-                            float2 vA = make_float2(prev[c][p].x, h[c][p].x);
-                            float2 vB = make_float2(h[c][p].y, prev[c][p].y);
-                            if (SECOND) {
-                                vA = __fadd2_rn(vA, lds64f(adA));
-                                vB = __fadd2_rn(vB, lds64f(adB));
-                            }
-                            sts64f(adA, vA);
-                            sts64f(adB, vB);
+                    for (int p = 0; p < 2; ++p) {
+                        unsigned char* adA = hrow + p * 256 + oA;
+                        unsigned char* adB = hrow + p * 256 + oB;
+                        float2 vA = make_float2(prev[p].x, h[p].x);
+                        float2 vB = make_float2(h[p].y, prev[p].y);
+                        if (SECOND) {
+                            vA = __fadd2_rn(vA, lds64f(adA));
+                            vB = __fadd2_rn(vB, lds64f(adB));
                         }
-                } else {
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) {
-                        prev[c][0] = h[c][0];
-                        prev[c][1] = h[c][1];
+                        sts64f(adA, vA);
+                        sts64f(adB, vB);
                     }
+                } else {
+                    prev[0] = h[0];
+                    prev[1] = h[1];
                 }
             }
         }
@@ -383,20 +398,17 @@ __global__ void __launch_bounds__(Cfg<KC>::NWARP * 32, 1)
         constexpr bool SECOND = decltype(second)::value;
         for (int qq = 0; qq < 4; ++qq) {
             const int q = SECOND ? qq + 4 : qq;
-            if (!acquire()) return false;
-            const unsigned char* st = ringp + stage * K::STAGE + t * 4;
-            uint32_t XA[KC][8], LA[KC][8], XB[KC][8], LB[KC][8];
+            if (!weights_in() || !acquire()) return false;
+            const unsigned char* st = ringp + stage * STAGE + t * 4;
+            uint32_t XA[8], LA[8], XB[8], LB[8];
 #pragma unroll
-            for (int c = 0; c < KC; ++c)
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    XA[c][e] = lds32(st + 0 * K::BOX + c * 1024 + e * 128);
-                    LA[c][e] = lds32(st + 1 * K::BOX + c * 1024 + e * 128);
-                    XB[c][e] = lds32(st + 2 * K::BOX + c * 1024 + (7 - e) * 128);
-                    LB[c][e] = lds32(st + 3 * K::BOX + c * 1024 + (7 - e) * 128);
-                }
+            for (int e = 0; e < 8; ++e) {
+                XA[e] = lds32(st + 0 * BOX + e * 128);
+                LA[e] = lds32(st + 1 * BOX + e * 128);
+                XB[e] = lds32(st + 2 * BOX + (7 - e) * 128);
+                LB[e] = lds32(st + 3 * BOX + (7 - e) * 128);
+            }
             release();
-            const float4* wp = wnext(S + 8 * q);
             // rows s = 8q + e (top->bottom) and 63 - s (bottom->top); the Hacc unit key
             // of row s is ((4q) & 15) + e/2, that of row 63 - s is 15 minus it
             unsigned char* const hA = haccp + 8 * q * 256;
@@ -406,54 +418,39 @@ __global__ void __launch_bounds__(Cfg<KC>::NWARP * 32, 1)
             __nv_bfloat16* const oB_row = outp + (S - 1 - 8 * q) * S;
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                if (LOCAL && ((8 * q + e) & segmask) == 0) {
-#pragma unroll
-                    for (int c = 0; c < KC; ++c) h[c][0] = h[c][1] = make_float2(0.f, 0.f);
-                }
-#pragma unroll
-                for (int c = 0; c < KC; ++c) {
-                    float2 base[2];
-                    base[0].x = fma_bf_lo(LA[c][e], XA[c][e], h[c][0].x);
-                    base[1].x = fma_bf_hi(LA[c][e], XA[c][e], h[c][1].x);
-                    base[0].y = fma_bf_lo(LB[c][e], XB[c][e], h[c][0].y);
-                    base[1].y = fma_bf_hi(LB[c][e], XB[c][e], h[c][1].y);
-                    scan_core(h[c], base, wr[e]);
-                }
-                wr[e][0] = __ldg(wp + e * S);
-                wr[e][1] = __ldg(wp + e * S + LPL);
+                if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
+                float2 base[2];
+                base[0].x = fma_bf_lo(LA[e], XA[e], h[0].x);
+                base[1].x = fma_bf_hi(LA[e], XA[e], h[1].x);
+                base[0].y = fma_bf_lo(LB[e], XB[e], h[0].y);
+                base[1].y = fma_bf_hi(LB[e], XB[e], h[1].y);
+                scan_core(h, base, wr[e]);
                 const uint32_t oA = (k8 + (uint32_t)((e >> 1) << 3)) ^ t8;
                 const uint32_t oB = oA ^ (15u << 3);
-#pragma unroll
-                for (int c = 0; c < KC; ++c) {
-                    unsigned char* adA = hA + c * HACC + e * 256 + oA;
-                    unsigned char* adB = hB + c * HACC - e * 256 + oB;
-                    const float2 vA = __fadd2_rn(lds64f(adA), make_float2(h[c][0].x, h[c][1].x));
-                    const float2 vB = __fadd2_rn(lds64f(adB), make_float2(h[c][0].y, h[c][1].y));
-                    if (!SECOND) {  // first arrival of this pass: keep the partial sum
-                        sts64f(adA, vA);
-                        sts64f(adB, vB);
-                    } else {        // second arrival: the pixel is complete
-                        stg_cs32(oA_row + c * S * S + e * S, pack_bf2(vA.x, vA.y));
-                        stg_cs32(oB_row + c * S * S - e * S, pack_bf2(vB.x, vB.y));
-                    }
+                unsigned char* adA = hA + e * 256 + oA;
+                unsigned char* adB = hB - e * 256 + oB;
+                const float2 vA = __fadd2_rn(lds64f(adA), make_float2(h[0].x, h[1].x));
+                const float2 vB = __fadd2_rn(lds64f(adB), make_float2(h[0].y, h[1].y));
+                if (!SECOND) {  // first arrival of this pass: keep the partial sum
+                    sts64f(adA, vA);
+                    sts64f(adB, vB);
+                } else {        // second arrival: the pixel is complete
+                    stg_cs32(oA_row + e * S, pack_bf2(vA.x, vA.y));
+                    stg_cs32(oB_row - e * S, pack_bf2(vB.x, vB.y));
                 }
             }
         }
         return true;
     };
 
-    for (int unit = wid; unit < a.units; unit += wstride) {
-        outp = a.out + (size_t)(KC * unit) * S * S + 2 * t;
-#pragma unroll
-        for (int c = 0; c < KC; ++c) h[c][0] = h[c][1] = make_float2(0.f, 0.f);
+    for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
+        outp = a.out + (size_t)(8 * group + warp) * S * S + 2 * t;
+        h[0] = h[1] = make_float2(0.f, 0.f);
         if (!row_half(std::false_type{}) || !row_half(std::true_type{})) { fail(); return; }
         __syncwarp();
-#pragma unroll
-        for (int c = 0; c < KC; ++c) h[c][0] = h[c][1] = make_float2(0.f, 0.f);
+        h[0] = h[1] = make_float2(0.f, 0.f);
         if (!col_half(std::false_type{}) || !col_half(std::true_type{})) { fail(); return; }
         __syncwarp();
-        wu = wn;
-        wn = unit + 2 * wstride < a.units ? wbase(unit + 2 * wstride) : wu;
     }
 }
 
@@ -477,32 +474,29 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// 3-D view (column, row, plane) of a stack of 64x64 bf16 planes; boxes of
-// box_c columns x box_r rows (every row_step-th row) x box_p planes.
+// 3-D view (column, row, plane) of a stack of 64x64 bf16 planes; one plane per
+// box of box_c columns x box_r rows (every row_step-th row).
 bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r, uint32_t row_step,
-              uint32_t box_p, CUtensorMapL2promotion promo) {
+              CUtensorMapL2promotion promo) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, S * S * 2};
-    const cuuint32_t box[3] = {box_c, box_r, box_p};
+    const cuuint32_t box[3] = {box_c, box_r, 1};
     const cuuint32_t es[3] = {1, row_step, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, promo,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int KC, bool LOCAL>
+template <bool LOCAL>
 gspn_status launch_c64(const DeviceInfo& dev, const CUtensorMap& xc, const CUtensorMap& lc, const CUtensorMap& xr,
                        const CUtensorMap& lr, const C64Args& a, cudaStream_t s) {
-    using K = Cfg<KC>;
-    const void* fn = (const void*)c64_fwd_kernel<KC, LOCAL>;
-    cudaError_t e = ensure_smem_attr(fn, K::SMEM_BYTES, 8 + 2 * (KC - 1) + (LOCAL ? 1 : 0));
+    const void* fn = (const void*)c64_fwd_kernel<LOCAL>;
+    cudaError_t e = ensure_smem_attr(fn, SMEM_BYTES, LOCAL ? 9 : 8);
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
-    int grid = dev.sm_count;
-    const int need = (a.units + K::NWARP - 1) / K::NWARP;
-    if (need < grid) grid = need;
-    c64_fwd_kernel<KC, LOCAL><<<grid, K::NWARP * 32, K::SMEM_BYTES, s>>>(xc, lc, xr, lr, a);
+    const int grid = a.groups < dev.sm_count ? a.groups : dev.sm_count;
+    c64_fwd_kernel<LOCAL><<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, xr, lr, a);
     return cudaGetLastError() == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
 }
 
@@ -510,7 +504,7 @@ gspn_status launch_c64(const DeviceInfo& dev, const CUtensorMap& xc, const CUten
 
 bool c64_eligible(const Problem& p) {
     return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
-           p.planes <= 0x7fffffff / 4 && encode_fn() != nullptr;
+           p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_fn() != nullptr;
 }
 
 size_t c64_fwd_workspace(const Problem& p) {
@@ -519,15 +513,13 @@ size_t c64_fwd_workspace(const Problem& p) {
 
 gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
                     void* out, void* ws, cudaStream_t s) {
-    // two channels per lane when C is even (the pair shares one batch image)
-    const int kc = (p.g.C % 2 == 0) ? 2 : 1;
     CUtensorMap xc, lc, xr, lr;
     const uint64_t BC = (uint64_t)p.planes;
     // column chunks: 8 columns x every other row (32 rows); row chunks: 64 columns x 8 rows
-    if (!make_map(&xc, x, BC, 8, 64, 2, kc, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
-        !make_map(&lc, lam, 4 * BC, 8, 64, 2, kc, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
-        !make_map(&xr, x, BC, 64, 8, 1, kc, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
-        !make_map(&lr, lam, 4 * BC, 64, 8, 1, kc, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
+    if (!make_map(&xc, x, BC, 8, 64, 2, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&lc, lam, 4 * BC, 8, 64, 2, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+        !make_map(&xr, x, BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
+        !make_map(&lr, lam, 4 * BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
         return GSPN_ERR_UNSUPPORTED;
     char* w = static_cast<char*>(ws);
     C64Args a;
@@ -537,15 +529,12 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     a.B = p.g.B;
     a.C = p.g.C;
     a.seg = S / p.g.groups;
-    a.units = (int)(p.planes / kc);
+    a.groups = (int)(p.planes / 8);
     const int nw = p.g.B * 2 * S * S;
     c64_weights_kernel<__nv_bfloat16><<<(nw + 255) / 256, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.wtab), a.err, p.g.B);
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
-    const bool local = p.g.groups > 1;
-    if (kc == 2)
-        return local ? launch_c64<2, true>(dev, xc, lc, xr, lr, a, s) : launch_c64<2, false>(dev, xc, lc, xr, lr, a, s);
-    return local ? launch_c64<1, true>(dev, xc, lc, xr, lr, a, s) : launch_c64<1, false>(dev, xc, lc, xr, lr, a, s);
+    return p.g.groups > 1 ? launch_c64<true>(dev, xc, lc, xr, lr, a, s) : launch_c64<false>(dev, xc, lc, xr, lr, a, s);
 }
 
 }  // namespace gspn

@@ -81,3 +81,21 @@ __device__ __forceinline__ void prefetch_map(const CUtensorMap* map) {
 
 }  // namespace tma
 }  // namespace gspn
+
+namespace gspn {
+namespace tma {
+
+// plain 1-D bulk copy global -> shared (16-byte aligned, size a multiple of 16),
+// completion counted on `bar` (bytes)
+__device__ __forceinline__ void load_1d(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+                 "l"(src), "r"(bytes), "r"(bar)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+}  // namespace tma
+}  // namespace gspn

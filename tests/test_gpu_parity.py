@@ -36,7 +36,7 @@ REDUCED = {
     "t2b_f32_b1c4_16x16": dict(),
     "4dir_f32_b8c96_56x56": dict(B=2, C=10),
     "4dir_local4_bf16_b32c192_28x28": dict(B=2, C=18),
-    "compact_4dir_bf16_b32c1152_64x64": dict(B=2, C=37),
+    "compact_4dir_bf16_b32c1152_64x64": dict(B=3, C=40),
     "compact_4dir_bf16_b2c1152_128x128_fwdbwd": dict(B=1, C=7),
 }
 
@@ -107,6 +107,11 @@ SHAPES = [
     (3, 9, 64, 64, 15, 1, True, "bf16"),
     (1, 6, 64, 64, 5, 2, True, "f32"),
     (1, 2, 97, 41, 9, 1, False, "f32"),
+    (2, 37, 64, 64, 15, 1, True, "bf16"),
+    (2, 16, 64, 64, 15, 1, True, "bf16"),
+    (1, 8, 64, 64, 15, 4, True, "bf16"),
+    (3, 24, 64, 64, 15, 64, True, "bf16"),
+    (5, 8, 64, 64, 15, 2, True, "bf16"),
     (1, 2, 130, 70, 15, 1, True, "bf16"),
     (1, 1, 257, 33, 3, 1, False, "f32"),
 ]
