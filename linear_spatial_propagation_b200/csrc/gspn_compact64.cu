@@ -19,7 +19,7 @@
 //   image, one plane per consumer warp, 32 lanes per 64-wide line and 2
 //   positions per lane.  The 8 warps step through the same sequence of
 //   8-step chunks, so one producer warp streams each chunk's tap weights
-//   (8 table rows, 8 KB) with a single bulk copy into a 2-stage ring that all
+//   (8 table rows, 8 KB) with a single bulk copy into a 4-stage ring that all
 //   8 warps read; each warp copies the chunk to registers and releases it.
 // * The two directions of a pair (left->right with right->left, top->bottom
 //   with bottom->top) advance together: lane values are float2 (one
@@ -63,7 +63,7 @@ constexpr int S = 64;          // H = W
 constexpr int LPL = 32;        // lanes per line (2 positions per lane)
 constexpr int NCW = 8;         // consumer warps per CTA (one plane each), one CTA per SM
 constexpr int NST = 2;         // x/lambda ring stages per consumer warp
-constexpr int NWS = 2;         // tap-weight ring stages per CTA
+constexpr int NWS = 4;         // tap-weight ring stages per CTA
 constexpr int BOX = 1024;      // bytes per TMA box (one plane)
 constexpr int SLICE = 512;     // one element-stride-2 column box
 constexpr int STAGE = 4 * BOX;
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (t == 0) {
             for (int kc = 0; kc < nchunks; ++kc) {
                 const int ws = kc % NWS;
-                if (!tma::mbar_wait(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1)) {
+                if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1, 200)) {
                     atomicExch(a.err, 1);
                     break;
                 }

@@ -66,6 +66,20 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_
     return true;
 }
 
+// The same wait for a thread that has nothing else to do: it sleeps `ns`
+// between polls so that its spinning does not take issue slots from the warps
+// that compute.
+__device__ __forceinline__ bool mbar_wait_sleep(uint32_t bar, uint32_t parity, unsigned ns,
+                                                uint64_t limit_ns = kTimeoutNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const uint64_t t0 = globaltimer();
+    while (!mbar_try_wait(bar, parity)) {
+        __nanosleep(ns);
+        if (globaltimer() - t0 > limit_ns) return false;
+    }
+    return true;
+}
+
 // 3-D tiled load global -> shared, completion counted on `bar` (bytes).
 __device__ __forceinline__ void load_3d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, uint32_t bar) {
     asm volatile(
