@@ -64,7 +64,9 @@
  *   GSPN_ERR_ALIGNMENT    a tensor pointer not 16-byte aligned;
  *   GSPN_ERR_WORKSPACE    workspace smaller than gspn_workspace_size();
  *   GSPN_ERR_CUDA         a CUDA runtime error at or before launch (the
- *                         runtime's own error is left for cudaGetLastError).
+ *                         runtime's own error is left for cudaGetLastError);
+ *   GSPN_ERR_SCRATCH_LIMIT  (gspn_fwd_noalloc only) the problem does not fit
+ *                         the library's fixed scratch.
  * No exception or signal crosses the ABI.
  */
 #ifndef GSPN_H_
@@ -84,7 +86,8 @@ typedef enum {
     GSPN_ERR_ALIGNMENT = 3,
     GSPN_ERR_WORKSPACE = 4,
     GSPN_ERR_CUDA = 5,
-    GSPN_ERR_TIMEOUT = 6
+    GSPN_ERR_TIMEOUT = 6,
+    GSPN_ERR_SCRATCH_LIMIT = 7
 } gspn_status;
 
 typedef enum { GSPN_F32 = 0, GSPN_BF16 = 1 } gspn_dtype;
@@ -127,6 +130,34 @@ gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, c
 gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda,
                      const void* dout, void* dx, void* dlogits, void* dlambda, void* workspace, size_t ws_bytes,
                      void* stream);
+
+/* Forward without any caller-provided workspace and without allocating.
+ *
+ * No counterpart in the GSPN pages: this is a convenience of this library for
+ * callers that cannot allocate device memory -- code that runs under a host
+ * framework which owns all device memory through its own pool and forbids
+ * direct cudaMalloc, code on a latency-critical path where cudaMalloc/cudaFree
+ * would block or synchronize the device, and plugins handed only the tensors
+ * they read and write.  Such callers pass inputs and outputs only.
+ *
+ * The scratch this forward needs (an error word and the normalised tap-weight
+ * table, 128 KB per batch image) lives in a fixed array in the library's
+ * device memory, 4 MiB + 256 bytes, which every GPU that loads the library
+ * holds until the process exits.  Hence the limits: only descriptors that run
+ * the compact 64x64 forward (bf16, shared_weights = 1, dir_mask = 15,
+ * H = W = 64, C a multiple of 8) are accepted, with B <= 32.  Larger batches
+ * return GSPN_ERR_SCRATCH_LIMIT and other descriptors GSPN_ERR_UNSUPPORTED,
+ * both before any launch; argument errors are reported as by gspn_fwd.
+ *
+ * The first call on a device looks up the array's device address for that
+ * device (cudaGetSymbolAddress) and caches it; make that first call before
+ * any stream capture begins.  All calls share the one array and each call
+ * rewrites what it reads, so results never depend on an earlier call, but
+ * calls whose execution overlaps on the GPU (different streams, or graphs
+ * replayed concurrently) race on it: serialise them.  Nothing is allocated
+ * or freed, here or in any library routine this calls. */
+gspn_status gspn_fwd_noalloc(const gspn_desc* desc, const void* x, const void* logits, const void* lambda,
+                             void* out, void* stream);
 
 /* Number of kernel launches one gspn_fwd (backward = 0) / gspn_bwd
  * (backward = 1) call with this descriptor issues; 0 for a descriptor the

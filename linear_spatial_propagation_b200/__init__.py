@@ -21,12 +21,12 @@ GSPN_F32, GSPN_BF16 = 0, 1
 
 STATUS = {
     0: "GSPN_OK", 1: "GSPN_ERR_INVALID_ARG", 2: "GSPN_ERR_UNSUPPORTED", 3: "GSPN_ERR_ALIGNMENT",
-    4: "GSPN_ERR_WORKSPACE", 5: "GSPN_ERR_CUDA", 6: "GSPN_ERR_TIMEOUT",
+    4: "GSPN_ERR_WORKSPACE", 5: "GSPN_ERR_CUDA", 6: "GSPN_ERR_TIMEOUT", 7: "GSPN_ERR_SCRATCH_LIMIT",
 }
 
 # every symbol include/gspn.h declares
-EXPORTS = ("gspn_workspace_size", "gspn_fwd", "gspn_bwd", "gspn_launches_per_call", "gspn_variant_name",
-           "gspn_status_string", "gspn_version")
+EXPORTS = ("gspn_workspace_size", "gspn_fwd", "gspn_bwd", "gspn_fwd_noalloc", "gspn_launches_per_call",
+           "gspn_variant_name", "gspn_status_string", "gspn_version")
 
 
 class GspnError(RuntimeError):
@@ -67,6 +67,8 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gspn_fwd.restype = ctypes.c_int
     lib.gspn_bwd.argtypes = [dp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.gspn_bwd.restype = ctypes.c_int
+    lib.gspn_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
+    lib.gspn_fwd_noalloc.restype = ctypes.c_int
     lib.gspn_launches_per_call.argtypes = [dp, ctypes.c_int]
     lib.gspn_launches_per_call.restype = ctypes.c_int
     lib.gspn_variant_name.argtypes = [dp, ctypes.c_int]
@@ -98,6 +100,12 @@ def gspn_bwd(desc: gspn_desc, x: int, logits: int, lam: int, dout: int, dx: int,
              workspace: int, ws_bytes: int, stream: int) -> int:
     return int(load().gspn_bwd(ctypes.byref(desc), x, logits, lam, dout, dx, dlogits, dlam, workspace or None,
                                int(ws_bytes), stream or None))
+
+
+def gspn_fwd_noalloc(desc: gspn_desc, x: int, logits: int, lam: int, out: int, stream: int) -> int:
+    """Forward on the library's fixed device scratch: for callers that cannot
+    allocate device memory (no workspace argument).  See include/gspn.h."""
+    return int(load().gspn_fwd_noalloc(ctypes.byref(desc), x, logits, lam, out, stream or None))
 
 
 def gspn_launches_per_call(desc: gspn_desc, backward: int = 0) -> int:

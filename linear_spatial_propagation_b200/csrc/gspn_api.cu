@@ -128,6 +128,8 @@ const char* gspn_status_string(gspn_status s) {
     case GSPN_ERR_WORKSPACE: return "workspace missing or too small";
     case GSPN_ERR_CUDA: return "CUDA runtime error";
     case GSPN_ERR_TIMEOUT: return "device-side wait timed out";
+    case GSPN_ERR_SCRATCH_LIMIT:
+        return "problem exceeds the fixed scratch of gspn_fwd_noalloc (compact 64x64 bf16 forward, B <= 32)";
     default: return "unknown status";
     }
 }
@@ -169,6 +171,18 @@ gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, c
     if (st != GSPN_OK) return st;
     if (fast) return c64_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
     return generic_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
+}
+
+gspn_status gspn_fwd_noalloc(const gspn_desc* desc, const void* x, const void* logits, const void* lambda, void* out,
+                             void* stream) {
+    Problem p;
+    gspn_status st = validate(desc, &p);
+    if (st != GSPN_OK) return st;
+    st = check_ptrs({x, logits, lambda, out});
+    if (st != GSPN_OK) return st;
+    DeviceInfo dev;
+    if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
+    return c64_fwd_noalloc(p, dev, x, logits, lambda, out, static_cast<cudaStream_t>(stream));
 }
 
 gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda,

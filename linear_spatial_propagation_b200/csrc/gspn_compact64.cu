@@ -49,6 +49,7 @@
 //   pass (each lane reads columns 2t, 2t+1 of one row).
 // * Every mbarrier wait is bounded (2 s); on expiry the warp records an
 //   error word in the workspace, drains its outstanding copies and returns.
+#include <atomic>
 #include <type_traits>
 
 #include "gspn_internal.h"
@@ -170,11 +171,6 @@ __device__ __forceinline__ void scan_core(float2 (&h)[2], const float2 (&base)[2
     const float2 v1 = __ffma2_rn(make_float2(w[1].z, w[1].w), D2, base[1]);
     h[0] = __ffma2_rn(make_float2(w[0].x, w[0].y), D0, v0);
     h[1] = __ffma2_rn(make_float2(w[1].x, w[1].y), D1, v1);
-}
-
-// Hacc byte offset of the 8-byte unit u (columns 2u, 2u+1) of row r.
-__device__ __forceinline__ uint32_t hacc_off(int r, int u) {
-    return (uint32_t)(r * 256 + ((u ^ ((r >> 1) & 15)) << 3));
 }
 
 struct C64Args {
@@ -535,6 +531,36 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
         static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.wtab), a.err, p.g.B);
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
     return p.g.groups > 1 ? launch_c64<true>(dev, xc, lc, xr, lr, a, s) : launch_c64<false>(dev, xc, lc, xr, lr, a, s);
+}
+
+// ---- allocation-free entry (gspn_fwd_noalloc) ------------------------------------
+// Fixed scratch of the forward for callers that cannot allocate device memory:
+// the error word and the tap-weight table of up to kNoAllocMaxBatch batch
+// images (4 MiB + 256 bytes).  Every GPU that loads the library holds it until
+// the process exits; all calls share it (the weights pre-kernel rewrites both
+// the error word and every table row a call reads).
+namespace {
+constexpr int kNoAllocMaxBatch = 32;
+constexpr size_t kNoAllocBytes = kWsAlign + (size_t)kNoAllocMaxBatch * 2 * S * S * sizeof(float4);
+__device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
+constexpr int kMaxNoAllocDevices = 64;
+std::atomic<void*> g_noalloc_ptr[kMaxNoAllocDevices];
+}  // namespace
+
+gspn_status c64_fwd_noalloc(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
+                            const void* lam, void* out, cudaStream_t s) {
+    if (!c64_eligible(p)) return GSPN_ERR_UNSUPPORTED;
+    if (p.g.B > kNoAllocMaxBatch || c64_fwd_workspace(p) > kNoAllocBytes) return GSPN_ERR_SCRATCH_LIMIT;
+    int d = 0;
+    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxNoAllocDevices) return GSPN_ERR_CUDA;
+    // set-up, once per device with that device current: the device address of
+    // the array (in host code its name is only a host-side stand-in)
+    void* ptr = g_noalloc_ptr[d].load(std::memory_order_acquire);
+    if (!ptr) {
+        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return GSPN_ERR_CUDA;
+        g_noalloc_ptr[d].store(ptr, std::memory_order_release);
+    }
+    return c64_fwd(p, dev, x, logits, lam, out, ptr, s);
 }
 
 }  // namespace gspn

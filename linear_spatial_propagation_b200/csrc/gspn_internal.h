@@ -46,5 +46,8 @@ bool c64_eligible(const Problem& p);
 size_t c64_fwd_workspace(const Problem& p);
 gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
                     void* out, void* ws, cudaStream_t s);
+// the same forward on the library's fixed device scratch (no workspace argument)
+gspn_status c64_fwd_noalloc(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
+                            const void* lam, void* out, cudaStream_t s);
 
 }  // namespace gspn
