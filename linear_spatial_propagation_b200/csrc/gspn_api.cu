@@ -139,21 +139,21 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     if (validate(desc, &p) != GSPN_OK) return 0;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return 0;
-    if (backward) return generic_bwd_workspace(p, dev);
+    if (backward) return c64_bwd_eligible(p) ? c64_bwd_workspace(p) : generic_bwd_workspace(p, dev);
     return c64_eligible(p) ? c64_fwd_workspace(p) : generic_fwd_workspace(p, dev);
 }
 
 int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return 0;
-    if (backward) return generic_bwd_launches(p);
+    if (backward) return c64_bwd_eligible(p) ? 3 : generic_bwd_launches(p);
     return c64_eligible(p) ? 2 : 1;
 }
 
 const char* gspn_variant_name(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return "invalid";
-    if (backward) return "generic_bwd";
+    if (backward) return c64_bwd_eligible(p) ? "compact64_tma_bwd" : "generic_bwd";
     return c64_eligible(p) ? "compact64_tma_fwd" : "generic_fwd";
 }
 
@@ -195,8 +195,12 @@ gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, c
     if (st != GSPN_OK) return st;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
-    st = check_ws(workspace, ws_bytes, generic_bwd_workspace(p, dev));
+    const bool fast = c64_bwd_eligible(p);
+    st = check_ws(workspace, ws_bytes, fast ? c64_bwd_workspace(p) : generic_bwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
+    if (fast)
+        return c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
+                       static_cast<cudaStream_t>(stream));
     return generic_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
                        static_cast<cudaStream_t>(stream));
 }

@@ -1,0 +1,723 @@
+// gspn_compact64_bwd.cu -- fast backward for the compact (channel-shared taps)
+// four-direction global scan of 64x64 bf16 planes (the 1K foundation shape of
+// C-GSPN, "Scaling Parallel Sequence Models to Vision Foundation Models").
+//
+// The gradient of the line scan ("Parallel Sequence Modeling via Generalized
+// Spatial Propagation Network", Key designs 1-2) is its adjoint run from the
+// last line to the first ("GSPN-2: Efficient Parallel Sequence Modeling",
+// Backward Benchmark: the same kernel-launch design as the forward).  With
+// a_i = dL/dh_i, per direction and line:
+//   a_i[j]   = G_i[j] + sum_k w_{i+1}[j-k+1][k] a_{i+1}[j-k+1]
+//            = G_i[j] + a_{i+1}[j] - p0[j] - p2[j] + p0[j+1] + p2[j-1],
+//              p0 = w0 a_{i+1}, p2 = w2 a_{i+1} (weights of line i+1; w1 = 1-w0-w2)
+//   dlambda  = x a,   dx += lambda a,
+//   D_k[j]   = sum over channels of a_i[j] h_{i-1}[j+k-1]   (tap products)
+// and dlogits follow from D in a finalize kernel (the sigmoid-and-normalise
+// chain rule, channel independent in compact mode).
+//
+// Design (B200), per plane and per pass (row pass: A = left->right,
+// B = right->left over columns s; column pass: A = top->bottom,
+// B = bottom->top over rows s):
+// * Sweep 1, s ascending: the forward scan of A (h_A) and the adjoint of B
+//   (a_B, whose last line is s = 0) both advance with s.  They are kept only
+//   as checkpoints at the end of every 8-step chunk (registers).
+// * Sweep 2, s descending, chunk by chunk: h_A and a_B of the chunk are
+//   recomputed from their checkpoints (forward in s), then the chunk is
+//   walked backwards running the adjoint of A and the forward of B.  At every
+//   s all four of h_A(s-1), a_A(s), h_B(s+1), a_B(s) are at hand, so dlambda
+//   of both directions, the pass's share of dx and the tap products of both
+//   directions are produced without storing any plane of h or a.
+// * dx: the row pass's share goes to an fp32 shared plane (XOR layout of
+//   8-byte units); the column pass adds its share and stores dx once.
+// * Tap products: the 8 warps of a CTA (8 channels of one image) add theirs
+//   into one shared buffer per chunk; the last warp to finish the chunk sends
+//   it with a bulk shared->global fp32 reduce-add into an L2-resident sum.
+// * x, lambda and dout are streamed by TMA exactly as in the compact forward
+//   (per-warp ring of 8-step chunks); the normalised tap weights (a table
+//   written by a pre-kernel, one row per scan step with both directions at
+//   the same column) by a producer warp into a ring shared by the CTA.
+// * Every wait is bounded (2 s); on expiry the warp records an error word,
+//   drains its copies and returns.
+#include <atomic>
+#include <type_traits>
+
+#include "gspn_internal.h"
+#include "gspn_lane.cuh"
+#include "gspn_tma.cuh"
+
+namespace gspn {
+
+namespace {
+
+using namespace lane;
+
+constexpr int S = 64;           // H = W
+constexpr int LPL = 32;         // lanes per line, 2 positions each
+constexpr int NCW = 8;          // consumer warps (one plane each)
+constexpr int NST = 2;          // data ring stages per warp
+constexpr int NWS = 2;          // weight ring stages per CTA
+constexpr int BOX = 1024;       // one plane of one tensor per chunk
+constexpr int SLICE = 512;
+constexpr int STAGE = 4 * BOX;  // x, lambda_A, lambda_B, dout
+constexpr int DACC = S * S * 4;
+constexpr int WCHUNK = 8 * S * 16;
+constexpr int DBUF = 2 * 3 * 8 * S * 4;  // [dir][tap][step][position] fp32
+constexpr int WARP_BYTES = NST * STAGE + DACC;
+constexpr int WRING = NCW * WARP_BYTES;
+constexpr int DBUFO = WRING + NWS * WCHUNK;
+constexpr int BARS = DBUFO + DBUF;
+constexpr int NBAR = NCW * NST + 2 * NWS + 1;
+constexpr int CNT = BARS + 8 * NBAR;
+constexpr int SMEM_BYTES = 1024 + CNT + 16;
+constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
+constexpr int THREADS = (NCW + 1) * 32;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// ---- backward tap table ---------------------------------------------------------------
+// btab[((b*2 + pass)*64 + s)*64 + p*32 + t] = (w0_A, w0_B, w2_A, w2_B) of position
+// j = 2t + p where both directions' lines sit at column (row pass) or row
+// (column pass) s: pass 0 A = left->right (slot 2), B = right->left (slot 3),
+// pixel (j, s); pass 1 A = top->bottom (slot 0), B = bottom->top (slot 1), pixel (s, j).
+template <typename T>
+__device__ __forceinline__ void gate_w(const T* lg, int pix, int j, float* w0, float* w2) {
+    const float s0 = j > 0 ? sigmoidf(load_elt(lg, pix)) : 0.f;
+    const float s1 = sigmoidf(load_elt(lg, S * S + pix));
+    const float s2 = j < S - 1 ? sigmoidf(load_elt(lg, 2 * S * S + pix)) : 0.f;
+    const float r = 1.f / (s0 + s1 + s2);
+    *w0 = s0 * r;
+    *w2 = s2 * r;
+}
+
+template <typename T>
+__global__ void c64b_table_kernel(const T* __restrict__ logits, float4* __restrict__ btab, float* __restrict__ dsum,
+                                  int* err, int B) {
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx == 0) *err = 0;
+    const int n = B * 2 * S * S;
+    // the tap-product sums start at zero: 2 directions x 3 taps per table entry
+    for (int q = idx; q < n * 6; q += gridDim.x * blockDim.x) dsum[q] = 0.f;
+    if (idx >= n) return;
+    const int j = idx & 63, s = (idx >> 6) & 63, pass = (idx >> 12) & 1, b = idx >> 13;
+    const int slotA = pass ? 0 : 2, slotB = pass ? 1 : 3;
+    const int pix = pass ? s * S + j : j * S + s;
+    float w0a, w2a, w0b, w2b;
+    gate_w(logits + (size_t)(slotA * B + b) * 3 * S * S, pix, j, &w0a, &w2a);
+    gate_w(logits + (size_t)(slotB * B + b) * 3 * S * S, pix, j, &w0b, &w2b);
+    const int t = j >> 1, p = j & 1;
+    btab[((size_t)(b * 2 + pass) * S + s) * S + p * LPL + t] = make_float4(w0a, w0b, w2a, w2b);
+}
+
+// dlogits from the tap-product sums: for the pixel's valid taps with sigmoids s_k
+// and normalised weights w_k, dlogit_k = w_k (1 - s_k) sum_m w_m (D_k - D_m)
+// (the chain rule through w_k = s_k / sum s, s_k = sigmoid(logit_k)); zero on the
+// first line of each direction (its taps are never used) and on invalid taps.
+template <typename T>
+__global__ void c64b_dlogits_kernel(const T* __restrict__ logits, const float* __restrict__ dsum,
+                                    T* __restrict__ dlogits, int B) {
+    const int idx = blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= 4 * B * S * S) return;
+    const int pix = idx & (S * S - 1), b = (idx >> 12) % B, slot = (idx >> 12) / B;
+    const int r = pix >> 6, c = pix & 63;
+    const int pass = slot < 2 ? 1 : 0, dir = slot & 1;  // dir 0 = A, 1 = B
+    // scan coordinates: row pass (s = column, j = row), column pass (s = row, j = column)
+    const int s = pass ? r : c, j = pass ? c : r;
+    const bool first_line = dir == 0 ? s == 0 : s == S - 1;
+    const T* lg = logits + (size_t)(slot * B + b) * 3 * S * S;
+    T* out = dlogits + (size_t)(slot * B + b) * 3 * S * S;
+    float d[3] = {0.f, 0.f, 0.f}, sg[3], w[3];
+    const bool valid[3] = {j > 0, true, j < S - 1};
+    float sum = 0.f;
+    for (int k = 0; k < 3; ++k) {
+        sg[k] = valid[k] ? sigmoidf(load_elt(lg, k * S * S + pix)) : 0.f;
+        sum += sg[k];
+    }
+    const float rs = 1.f / sum;
+    const size_t base = (((size_t)(b * 2 + pass) * 2 + dir) * 3) * S * S + (size_t)s * S + (j & 1) * LPL + (j >> 1);
+    for (int k = 0; k < 3; ++k) {
+        w[k] = sg[k] * rs;
+        d[k] = dsum[base + (size_t)k * S * S];
+    }
+    for (int k = 0; k < 3; ++k) {
+        float v = 0.f;
+        if (!first_line && valid[k]) {
+            float acc = 0.f;
+            for (int m = 0; m < 3; ++m) acc += w[m] * (d[k] - d[m]);
+            v = w[k] * (1.f - sg[k]) * acc;
+        }
+        store_elt(out, (size_t)k * S * S + pix, v);
+    }
+}
+
+struct C64BArgs {
+    const float4* btab;
+    float* dsum;  // [B][pass][dir][tap][s][p*32 + t]
+    __nv_bfloat16* dx;
+    __nv_bfloat16* dlam;
+    int* err;
+    int B, C;
+    int groups;  // B * C / 8
+};
+
+__device__ __forceinline__ float bfv(const uint4& v, int e) {
+    const uint32_t w = word_of(v, e >> 1);
+    return (e & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
+}
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// Forward step: h(s) of both positions from h(s-1) = h; w0/w2 at own positions.
+__device__ __forceinline__ void fwd_step(float (&h)[2], const float (&lx)[2], const float (&w0)[2],
+                                         const float (&w2)[2], float* nb /* out: hl, h0, h1, hr of h(s-1) */) {
+    const float hl = __shfl_up_sync(FULL, h[1], 1);
+    const float hr = __shfl_down_sync(FULL, h[0], 1);
+    nb[0] = hl;
+    nb[1] = h[0];
+    nb[2] = h[1];
+    nb[3] = hr;
+    const float n0 = h[0] + lx[0] + w2[0] * (h[1] - h[0]) - w0[0] * (h[0] - hl);
+    const float n1 = h[1] + lx[1] + w2[1] * (hr - h[1]) - w0[1] * (h[1] - h[0]);
+    h[0] = n0;
+    h[1] = n1;
+}
+
+// Adjoint step: a(line i) from a = a(line i+1) with the weights of line i+1.
+__device__ __forceinline__ void adj_step(float (&a)[2], const float (&g)[2], const float (&w0)[2],
+                                         const float (&w2)[2], int t) {
+    const float p00 = w0[0] * a[0], p01 = w0[1] * a[1];
+    const float p20 = w2[0] * a[0], p21 = w2[1] * a[1];
+    float p0r = __shfl_down_sync(FULL, p00, 1);  // p0 at j = 2t+2
+    float p2l = __shfl_up_sync(FULL, p21, 1);    // p2 at j = 2t-1
+    if (t == LPL - 1) p0r = 0.f;
+    if (t == 0) p2l = 0.f;
+    const float n0 = g[0] + a[0] - p00 - p20 + p01 + p2l;
+    const float n1 = g[1] + a[1] - p01 - p21 + p0r + p20;
+    a[0] = n0;
+    a[1] = n1;
+}
+
+__global__ void __launch_bounds__(THREADS, 1)
+    c64b_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
+                const __grid_constant__ CUtensorMap tm_gc, const __grid_constant__ CUtensorMap tm_xr,
+                const __grid_constant__ CUtensorMap tm_lr, const __grid_constant__ CUtensorMap tm_gr,
+                const C64BArgs a) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    unsigned char* const smem = smem_raw + ((1024u - (tma::smem_u32(smem_raw) & 1023u)) & 1023u);
+    const uint32_t sbase = tma::smem_u32(smem);
+    const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
+    const uint32_t wfull0 = sbase + BARS + 8 * NCW * NST;
+    const uint32_t wempty0 = wfull0 + 8 * NWS;
+    const uint32_t dempty = wempty0 + 8 * NWS;
+    unsigned int* const dcount = reinterpret_cast<unsigned int*>(smem + CNT);
+    float* const dbuf = reinterpret_cast<float*>(smem + DBUFO);
+    if ((int)blockIdx.x >= a.groups) return;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NCW * NST; ++s) tma::mbar_init(sbase + BARS + 8 * s, 1);
+        for (int s = 0; s < NWS; ++s) {
+            tma::mbar_init(wfull0 + 8 * s, 1);
+            tma::mbar_init(wempty0 + 8 * s, NCW);
+        }
+        tma::mbar_init(dempty, 1);
+        *dcount = 0;
+        tma::fence_barrier_init();
+    }
+    // the tap-product buffer starts at zero
+    for (int q = threadIdx.x; q < DBUF / 4; q += THREADS) dbuf[q] = 0.f;
+    __syncthreads();
+
+    const int ngroups_here = (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int nchunks = ngroups_here * CHUNKS_PER_GROUP;
+    const int BC = a.B * a.C;
+
+    // chunk kk of the CTA sequence: pass, sweep, chunk index q of 8 steps
+    auto chunk_info = [](int kk, int& pass, int& sweep, int& q) {
+        const int l = kk % CHUNKS_PER_GROUP;
+        pass = l >> 4;
+        sweep = (l >> 3) & 1;
+        q = sweep ? 7 - (l & 7) : (l & 7);
+    };
+
+    // ---------------- producer warp: tap-table chunks ----------------
+    if (warp == NCW) {
+        if (t == 0) {
+            for (int kc = 0; kc < nchunks; ++kc) {
+                const int ws = kc % NWS;
+                if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1, 200)) {
+                    atomicExch(a.err, 1);
+                    break;
+                }
+                const int group = (int)blockIdx.x + (kc / CHUNKS_PER_GROUP) * (int)gridDim.x;
+                const int b = (8 * group) / a.C;
+                int pass, sweep, q;
+                chunk_info(kc, pass, sweep, q);
+                const float4* src = a.btab + ((size_t)(b * 2 + pass) * S + 8 * q) * S;
+                tma::mbar_expect_tx(wfull0 + 8 * ws, WCHUNK);
+                tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumer warps ----------------
+    const uint32_t ring = sbase + warp * WARP_BYTES;
+    unsigned char* const ringp = smem + warp * WARP_BYTES;
+    unsigned char* const daccp = ringp + NST * STAGE;
+    const unsigned char* const wring = smem + WRING;
+    const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
+
+    if (t == 0) {
+        tma::prefetch_map(&tm_xc);
+        tma::prefetch_map(&tm_lc);
+        tma::prefetch_map(&tm_gc);
+        tma::prefetch_map(&tm_xr);
+        tma::prefetch_map(&tm_lr);
+        tma::prefetch_map(&tm_gr);
+    }
+
+    // Data of chunk kk (lane 0): x, lambda_A, lambda_B (sweep 2 only), dout of
+    // the chunk's 8 columns (row pass) or rows (column pass).
+    auto issue = [&](int kk) {
+        if (kk >= nchunks) return;
+        const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
+        const int plane = 8 * group + warp;
+        int pass, sweep, q;
+        chunk_info(kk, pass, sweep, q);
+        const int st = kk % NST;
+        const uint32_t dst = ring + st * STAGE, bar = bar0 + 8 * st;
+        tma::mbar_expect_tx(bar, sweep ? 4 * BOX : 3 * BOX);
+        const int la = pass ? 0 : 2, lb = pass ? 1 : 3;  // lambda slots of A and B
+        if (pass == 0) {
+            for (int r = 0; r < 2; ++r) {
+                tma::load_3d(dst + 0 * BOX + r * SLICE, &tm_xc, 8 * q, r, plane, bar);
+                tma::load_3d(dst + 1 * BOX + r * SLICE, &tm_lc, 8 * q, r, la * BC + plane, bar);
+                if (sweep) tma::load_3d(dst + 2 * BOX + r * SLICE, &tm_lc, 8 * q, r, lb * BC + plane, bar);
+                tma::load_3d(dst + 3 * BOX + r * SLICE, &tm_gc, 8 * q, r, plane, bar);
+            }
+        } else {
+            tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
+            tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, la * BC + plane, bar);
+            if (sweep) tma::load_3d(dst + 2 * BOX, &tm_lr, 0, 8 * q, lb * BC + plane, bar);
+            tma::load_3d(dst + 3 * BOX, &tm_gr, 0, 8 * q, plane, bar);
+        }
+    };
+    if (t == 0)
+        for (int kk = 0; kk < NST; ++kk) issue(kk);
+
+    int k = 0, stage = 0;
+    uint32_t phase = 0;
+    int dchunk = 0;  // sweep-2 chunks done (tap-product buffer uses)
+    auto fail = [&]() {
+        if (t == 0) atomicExch(a.err, 1);
+        for (int kk = k; kk < k + NST && kk < nchunks; ++kk)
+            tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
+        for (int kk = k; kk < k + NWS && kk < nchunks; ++kk)
+            tma::mbar_wait(wfull0 + 8 * (kk % NWS), (kk / NWS) & 1, 100000000ull);
+    };
+    auto acquire = [&]() -> bool {
+        const bool ok1 = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
+        const bool ok2 = tma::mbar_wait(wfull0 + 8 * (k % NWS), (k / NWS) & 1);
+        return __all_sync(FULL, ok1 && ok2);
+    };
+    // the data stage is in registers: refill it
+    auto release_data = [&]() {
+        tma::fence_proxy_async();
+        __syncwarp();
+        if (t == 0) issue(k + NST);
+        phase ^= 1u << stage;
+        stage = stage == NST - 1 ? 0 : stage + 1;
+    };
+    // done with the weight stage of chunk k
+    auto release_w = [&]() {
+        __syncwarp();
+        if (t == 0) tma::mbar_arrive(wempty0 + 8 * (k % NWS));
+        ++k;
+    };
+    // tap weights of row e of the current weight stage, positions 2t, 2t+1
+    auto wrow = [&](int e, float (&w0A)[2], float (&w0B)[2], float (&w2A)[2], float (&w2B)[2]) {
+        const unsigned char* src = wring + (k % NWS) * WCHUNK + e * 1024 + t * 16;
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+            const float4 v = lds128f(src + p * 512);
+            w0A[p] = v.x;
+            w0B[p] = v.y;
+            w2A[p] = v.z;
+            w2B[p] = v.w;
+        }
+    };
+    // tap products of one direction/tap/position into the CTA buffer
+    auto dadd = [&](int dir, int kt, int e, int p, float v) {
+        atomicAdd(dbuf + ((dir * 3 + kt) * 8 + e) * S + p * LPL + t, v);
+    };
+    // the warp is done with the tap-product buffer of this sweep-2 chunk; the last
+    // of the 8 warps sends it to the global sums, clears it and frees it
+    auto dflush = [&](float* gdst) -> bool {
+        __threadfence_block();
+        tma::fence_proxy_async();
+        __syncwarp();
+        unsigned last = 0;
+        if (t == 0) last = atomicAdd(dcount, 1u) == NCW - 1 ? 1u : 0u;
+        last = __shfl_sync(FULL, last, 0);
+        if (last) {
+            __threadfence_block();
+            tma::fence_proxy_async();
+            if (t == 0) {
+                for (int r = 0; r < 6; ++r)
+                    tma::reduce_add_f32(gdst + (size_t)r * S * S, sbase + DBUFO + r * 8 * S * 4, 8 * S * 4);
+                tma::bulk_commit();
+                tma::bulk_wait_read();
+                *dcount = 0;
+            }
+            __syncwarp();
+            for (int q = t; q < DBUF / 16; q += 32) reinterpret_cast<float4*>(dbuf)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+            __threadfence_block();
+            __syncwarp();
+            if (t == 0) tma::mbar_arrive(dempty);
+        }
+        ++dchunk;
+        return true;
+    };
+    // before the first tap product of a sweep-2 chunk: the buffer is free again
+    auto dacquire = [&]() -> bool {
+        if (dchunk == 0) return true;
+        const bool ok = tma::mbar_wait(dempty, (dchunk - 1) & 1);
+        return __all_sync(FULL, ok);
+    };
+
+    const int tk = t & 15;
+    unsigned char* const drow = daccp + 2 * t * 256;  // row pass: rows 2t, 2t+1
+
+    for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
+        const int plane = 8 * group + warp;
+        const int b = plane / a.C;
+        const float4* const btab_b = a.btab + (size_t)b * 2 * S * S;
+
+        auto run_pass = [&](auto pass_c) -> bool {
+            constexpr int pass = decltype(pass_c)::value;
+            const int la = pass ? 0 : 2, lb = pass ? 1 : 3;
+            __nv_bfloat16* const dlamA = a.dlam + ((size_t)la * BC + plane) * S * S;
+            __nv_bfloat16* const dlamB = a.dlam + ((size_t)lb * BC + plane) * S * S;
+            float* const dsum = a.dsum + ((size_t)(b * 2 + pass) * 2) * 3 * S * S;
+
+            // ---------------- sweep 1: h_A forward and a_B adjoint, s ascending ----------------
+            float hA[2] = {0.f, 0.f}, aB[2] = {0.f, 0.f};
+            float ckA[8][2], ckB[8][2];
+            float w0Bp[2] = {0.f, 0.f}, w2Bp[2] = {0.f, 0.f};  // B taps of line s-1
+            for (int q = 0; q < 8; ++q) {
+                if (!acquire()) { fail(); return false; }
+                uint4 X[2] = {}, LA[2] = {}, G[2] = {};
+                uint32_t Xr[8] = {}, LAr[8] = {}, Gr[8] = {};
+                if constexpr (decltype(pass_c)::value == 0) {
+                    const unsigned char* st = ringp + stage * STAGE + t * 16;
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        X[p] = lds128(st + 0 * BOX + p * SLICE);
+                        LA[p] = lds128(st + 1 * BOX + p * SLICE);
+                        G[p] = lds128(st + 3 * BOX + p * SLICE);
+                    }
+                } else {
+                    const unsigned char* st = ringp + stage * STAGE + t * 4;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        Xr[e] = lds32(st + 0 * BOX + e * 128);
+                        LAr[e] = lds32(st + 1 * BOX + e * 128);
+                        Gr[e] = lds32(st + 3 * BOX + e * 128);
+                    }
+                }
+                release_data();
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int s = 8 * q + e;
+                    float w0A[2], w0B[2], w2A[2], w2B[2];
+                    wrow(e, w0A, w0B, w2A, w2B);
+                    float lx[2], g[2];
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        if constexpr (decltype(pass_c)::value == 0) {
+                            lx[p] = bfv(LA[p], e) * bfv(X[p], e);
+                            g[p] = bfv(G[p], e);
+                        } else {
+                            lx[p] = (p ? bf_hi(LAr[e]) : bf_lo(LAr[e])) * (p ? bf_hi(Xr[e]) : bf_lo(Xr[e]));
+                            g[p] = p ? bf_hi(Gr[e]) : bf_lo(Gr[e]);
+                        }
+                    }
+                    float nb[4];
+                    fwd_step(hA, lx, w0A, w2A, nb);
+                    if (s > 0) {
+                        adj_step(aB, g, w0Bp, w2Bp, t);
+                    } else {
+                        aB[0] = g[0];
+                        aB[1] = g[1];
+                    }
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        w0Bp[p] = w0B[p];
+                        w2Bp[p] = w2B[p];
+                    }
+                }
+                ckA[q][0] = hA[0];
+                ckA[q][1] = hA[1];
+                ckB[q][0] = aB[0];
+                ckB[q][1] = aB[1];
+                release_w();
+            }
+
+            // ---------------- sweep 2: s descending ----------------
+            float aA[2] = {0.f, 0.f}, hB[2] = {0.f, 0.f};
+            float w0An[2] = {0.f, 0.f}, w2An[2] = {0.f, 0.f};  // A taps of line s+1
+            for (int qq = 0; qq < 8; ++qq) {
+                const int q = 7 - qq;
+                // B taps of line 8q-1 for the a_B recompute (previous chunk in s, not in this ring)
+                float w0Bm[2] = {0.f, 0.f}, w2Bm[2] = {0.f, 0.f};
+                if (q > 0) {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const float4 v = __ldg(btab_b + ((size_t)pass * S + 8 * q - 1) * S + p * LPL + t);
+                        w0Bm[p] = v.y;
+                        w2Bm[p] = v.w;
+                    }
+                }
+                if (!acquire()) { fail(); return false; }
+                uint4 X[2] = {}, LA[2] = {}, LB[2] = {}, G[2] = {};
+                uint32_t Xr[8] = {}, LAr[8] = {}, LBr[8] = {}, Gr[8] = {};
+                if constexpr (decltype(pass_c)::value == 0) {
+                    const unsigned char* st = ringp + stage * STAGE + t * 16;
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        X[p] = lds128(st + 0 * BOX + p * SLICE);
+                        LA[p] = lds128(st + 1 * BOX + p * SLICE);
+                        LB[p] = lds128(st + 2 * BOX + p * SLICE);
+                        G[p] = lds128(st + 3 * BOX + p * SLICE);
+                    }
+                } else {
+                    const unsigned char* st = ringp + stage * STAGE + t * 4;
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        Xr[e] = lds32(st + 0 * BOX + e * 128);
+                        LAr[e] = lds32(st + 1 * BOX + e * 128);
+                        LBr[e] = lds32(st + 2 * BOX + e * 128);
+                        Gr[e] = lds32(st + 3 * BOX + e * 128);
+                    }
+                }
+                release_data();
+                auto xv = [&](int e, int p) {
+                    return pass == 0 ? bfv(X[p], e) : (p ? bf_hi(Xr[e]) : bf_lo(Xr[e]));
+                };
+                auto lav = [&](int e, int p) {
+                    return pass == 0 ? bfv(LA[p], e) : (p ? bf_hi(LAr[e]) : bf_lo(LAr[e]));
+                };
+                auto lbv = [&](int e, int p) {
+                    return pass == 0 ? bfv(LB[p], e) : (p ? bf_hi(LBr[e]) : bf_lo(LBr[e]));
+                };
+                auto gv = [&](int e, int p) { return pass == 0 ? bfv(G[p], e) : (p ? bf_hi(Gr[e]) : bf_lo(Gr[e])); };
+
+                // recompute h_A (with the neighbours of h_A(s-1)) and a_B over the chunk
+                float hs[8][4], aBs[8][2];
+                {
+                    float h[2] = {q > 0 ? ckA[q - 1][0] : 0.f, q > 0 ? ckA[q - 1][1] : 0.f};
+                    float ab[2] = {q > 0 ? ckB[q - 1][0] : 0.f, q > 0 ? ckB[q - 1][1] : 0.f};
+                    float w0Bq[2] = {w0Bm[0], w0Bm[1]}, w2Bq[2] = {w2Bm[0], w2Bm[1]};
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        float w0A[2], w0B[2], w2A[2], w2B[2];
+                        wrow(e, w0A, w0B, w2A, w2B);
+                        float lx[2] = {lav(e, 0) * xv(e, 0), lav(e, 1) * xv(e, 1)};
+                        float g[2] = {gv(e, 0), gv(e, 1)};
+                        fwd_step(h, lx, w0A, w2A, hs[e]);
+                        if (8 * q + e > 0) {
+                            adj_step(ab, g, w0Bq, w2Bq, t);
+                        } else {
+                            ab[0] = g[0];
+                            ab[1] = g[1];
+                        }
+                        aBs[e][0] = ab[0];
+                        aBs[e][1] = ab[1];
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            w0Bq[p] = w0B[p];
+                            w2Bq[p] = w2B[p];
+                        }
+                    }
+                }
+                if (!dacquire()) { fail(); return false; }
+                uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns
+                float dxp[2];                    // row pass: dx share of column s+1 (pairs)
+#pragma unroll
+                for (int ee = 0; ee < 8; ++ee) {
+                    const int e = 7 - ee;
+                    const int s = 8 * q + e;
+                    float w0A[2], w0B[2], w2A[2], w2B[2];
+                    wrow(e, w0A, w0B, w2A, w2B);
+                    float g[2] = {gv(e, 0), gv(e, 1)};
+                    // adjoint of A at s from s+1 (taps of line s+1)
+                    if (s < S - 1) {
+                        adj_step(aA, g, w0An, w2An, t);
+                    } else {
+                        aA[0] = g[0];
+                        aA[1] = g[1];
+                    }
+                    // forward of B at s from s+1 (taps of B's line at s)
+                    float lxb[2] = {lbv(e, 0) * xv(e, 0), lbv(e, 1) * xv(e, 1)};
+                    float nbB[4];
+                    fwd_step(hB, lxb, w0B, w2B, nbB);
+                    // tap products: A's line s reads h_A(s-1); B's line (column/row s)
+                    // reads h_B(s+1); the first line of each direction has none
+                    if (s > 0) {
+                        dadd(0, 0, e, 0, aA[0] * hs[e][0]);
+                        dadd(0, 1, e, 0, aA[0] * hs[e][1]);
+                        dadd(0, 2, e, 0, aA[0] * hs[e][2]);
+                        dadd(0, 0, e, 1, aA[1] * hs[e][1]);
+                        dadd(0, 1, e, 1, aA[1] * hs[e][2]);
+                        dadd(0, 2, e, 1, aA[1] * hs[e][3]);
+                    }
+                    if (s < S - 1) {
+                        const float* ab = aBs[e];
+                        dadd(1, 0, e, 0, ab[0] * nbB[0]);
+                        dadd(1, 1, e, 0, ab[0] * nbB[1]);
+                        dadd(1, 2, e, 0, ab[0] * nbB[2]);
+                        dadd(1, 0, e, 1, ab[1] * nbB[1]);
+                        dadd(1, 1, e, 1, ab[1] * nbB[2]);
+                        dadd(1, 2, e, 1, ab[1] * nbB[3]);
+                    }
+                    // dlambda of both directions and this pass's share of dx
+                    float dla[2], dlb[2], dxs[2];
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const float xx = xv(e, p);
+                        dla[p] = xx * aA[p];
+                        dlb[p] = xx * aBs[e][p];
+                        dxs[p] = lav(e, p) * aA[p] + lbv(e, p) * aBs[e][p];
+                    }
+                    if constexpr (decltype(pass_c)::value == 0) {
+                        // rows 2t+p, column s: pack 8 columns of each row, store at chunk end
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            if (e & 1) {
+                                dlA[p][e >> 1] = pack_bf2(0.f, dla[p]);
+                                dlB[p][e >> 1] = pack_bf2(0.f, dlb[p]);
+                            } else {
+                                dlA[p][e >> 1] = (dlA[p][e >> 1] & 0xffff0000u) | (pack_bf2(dla[p], 0.f) & 0xffffu);
+                                dlB[p][e >> 1] = (dlB[p][e >> 1] & 0xffff0000u) | (pack_bf2(dlb[p], 0.f) & 0xffffu);
+                            }
+                        }
+                        // dx share into the fp32 plane, columns s, s+1 per 8-byte unit
+                        if (e & 1) {
+                            dxp[0] = dxs[0];
+                            dxp[1] = dxs[1];
+                        } else {
+                            const uint32_t o = (uint32_t)(((s >> 1) ^ tk) << 3);
+#pragma unroll
+                            for (int p = 0; p < 2; ++p) sts64f(drow + p * 256 + o, make_float2(dxs[p], dxp[p]));
+                        }
+                    } else {
+                        // row s, columns 2t, 2t+1: complete dx, dlambda of both directions
+                        const float2 prev = lds64f(daccp + s * 256 + ((t ^ ((s >> 1) & 15)) << 3));
+                        stg_cs32(a.dx + (size_t)plane * S * S + s * S + 2 * t,
+                                 pack_bf2(prev.x + dxs[0], prev.y + dxs[1]));
+                        stg_cs32(dlamA + s * S + 2 * t, pack_bf2(dla[0], dla[1]));
+                        stg_cs32(dlamB + s * S + 2 * t, pack_bf2(dlb[0], dlb[1]));
+                    }
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        w0An[p] = w0A[p];
+                        w2An[p] = w2A[p];
+                    }
+                }
+                if constexpr (decltype(pass_c)::value == 0) {
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const int r = 2 * t + p;
+                        uint4 va = make_uint4(dlA[p][0], dlA[p][1], dlA[p][2], dlA[p][3]);
+                        uint4 vb = make_uint4(dlB[p][0], dlB[p][1], dlB[p][2], dlB[p][3]);
+                        __stcs(reinterpret_cast<uint4*>(dlamA + r * S + 8 * q), va);
+                        __stcs(reinterpret_cast<uint4*>(dlamB + r * S + 8 * q), vb);
+                    }
+                }
+                dflush(dsum + (size_t)8 * q * S);
+                release_w();
+            }
+            __syncwarp();
+            return true;
+        };
+        if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) return;
+    }
+}
+
+// ---- host side ----------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn_b() {
+    static EncodeTiledFn fn = nullptr;
+    static bool tried = false;
+    if (!tried) {
+        tried = true;
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+bool make_map_b(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r, uint32_t row_step) {
+    EncodeTiledFn fn = encode_fn_b();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {S, S, planes};
+    const cuuint64_t strides[2] = {S * 2, S * S * 2};
+    const cuuint32_t box[3] = {box_c, box_r, 1};
+    const cuuint32_t es[3] = {1, row_step, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool c64_bwd_eligible(const Problem& p) {
+    return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
+           p.g.groups == 1 && p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_fn_b() != nullptr;
+}
+
+size_t c64_bwd_workspace(const Problem& p) {
+    // error word | tap table (B*2*64*64 float4) | tap-product sums (B*2*2*3*64*64 fp32)
+    return kWsAlign + align_up((size_t)p.g.B * 2 * S * S * sizeof(float4), kWsAlign) +
+           align_up((size_t)p.g.B * 2 * 2 * 3 * S * S * sizeof(float), kWsAlign);
+}
+
+gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                    const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s) {
+    CUtensorMap xc, lc, gc, xr, lr, gr;
+    const uint64_t BC = (uint64_t)p.planes;
+    if (!make_map_b(&xc, x, BC, 8, 64, 2) || !make_map_b(&lc, lam, 4 * BC, 8, 64, 2) ||
+        !make_map_b(&gc, dout, BC, 8, 64, 2) || !make_map_b(&xr, x, BC, 64, 8, 1) ||
+        !make_map_b(&lr, lam, 4 * BC, 64, 8, 1) || !make_map_b(&gr, dout, BC, 64, 8, 1))
+        return GSPN_ERR_UNSUPPORTED;
+    char* w = static_cast<char*>(ws);
+    C64BArgs a;
+    a.err = reinterpret_cast<int*>(w);
+    a.btab = reinterpret_cast<const float4*>(w + kWsAlign);
+    a.dsum = reinterpret_cast<float*>(w + kWsAlign + align_up((size_t)p.g.B * 2 * S * S * sizeof(float4), kWsAlign));
+    a.dx = static_cast<__nv_bfloat16*>(dx);
+    a.dlam = static_cast<__nv_bfloat16*>(dlam);
+    a.B = p.g.B;
+    a.C = p.g.C;
+    a.groups = (int)(p.planes / 8);
+    const int nt = p.g.B * 2 * S * S;
+    c64b_table_kernel<__nv_bfloat16><<<(nt + 255) / 256, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.btab), a.dsum, a.err, p.g.B);
+    if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
+    cudaError_t e = ensure_smem_attr((const void*)c64b_kernel, SMEM_BYTES, 10);
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
+    const int grid = a.groups < dev.sm_count ? a.groups : dev.sm_count;
+    c64b_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, gc, xr, lr, gr, a);
+    if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
+    const int nl = 4 * p.g.B * S * S;
+    c64b_dlogits_kernel<__nv_bfloat16><<<(nl + 255) / 256, 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(logits), a.dsum, static_cast<__nv_bfloat16*>(dlogits), p.g.B);
+    return cudaGetLastError() == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+}
+
+}  // namespace gspn

@@ -50,4 +50,10 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
 gspn_status c64_fwd_noalloc(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
                             const void* lam, void* out, cudaStream_t s);
 
+// ---- compact 64x64 bf16 backward (TMA-fed, checkpointed sweeps) ------------------
+bool c64_bwd_eligible(const Problem& p);
+size_t c64_bwd_workspace(const Problem& p);
+gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                    const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s);
+
 }  // namespace gspn

@@ -113,3 +113,22 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 
 }  // namespace tma
 }  // namespace gspn
+
+namespace gspn {
+namespace tma {
+
+// shared -> global bulk reduction (fp32 add performed at the destination);
+// 16-byte aligned, size a multiple of 16
+__device__ __forceinline__ void reduce_add_f32(void* gdst, uint32_t ssrc, uint32_t bytes) {
+    asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;" ::"l"(gdst),
+                 "r"(ssrc), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk operation of this thread has finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// wait until every committed bulk operation of this thread has completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+}  // namespace tma
+}  // namespace gspn
