@@ -139,7 +139,7 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     if (validate(desc, &p) != GSPN_OK) return 0;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return 0;
-    if (backward) return c64_bwd_eligible(p) ? c64_bwd_workspace(p) : generic_bwd_workspace(p, dev);
+    if (backward) return c64_bwd_eligible(p) ? c64_bwd_workspace(p, dev) : generic_bwd_workspace(p, dev);
     return c64_eligible(p) ? c64_fwd_workspace(p) : generic_fwd_workspace(p, dev);
 }
 
@@ -196,7 +196,7 @@ gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, c
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
     const bool fast = c64_bwd_eligible(p);
-    st = check_ws(workspace, ws_bytes, fast ? c64_bwd_workspace(p) : generic_bwd_workspace(p, dev));
+    st = check_ws(workspace, ws_bytes, fast ? c64_bwd_workspace(p, dev) : generic_bwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
     if (fast)
         return c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,

@@ -11,9 +11,13 @@
 //            = G_i[j] + a_{i+1}[j] - p0[j] - p2[j] + p0[j+1] + p2[j-1],
 //              p0 = w0 a_{i+1}, p2 = w2 a_{i+1} (weights of line i+1; w1 = 1-w0-w2)
 //   dlambda  = x a,   dx += lambda a,
-//   D_k[j]   = sum over channels of a_i[j] h_{i-1}[j+k-1]   (tap products)
-// and dlogits follow from D in a finalize kernel (the sigmoid-and-normalise
-// chain rule, channel independent in compact mode).
+//   dw_k[j]  = a_i[j] h_{i-1}[j+k-1]   (tap products)
+// and dlogit_k = w_k (1 - s_k) E_k with E_k = sum over channels of
+// (dw_k - sum_m w_m dw_m) (chain rule through w_k = s_k / sum s, s_k =
+// sigmoid(logit_k); the taps are channel independent in compact mode).
+// Since sum_k w_k E_k = 0, only E_0 and E_2 are summed:
+//   E_0 = w_1 (dw_0 - dw_1) + w_2 (dw_0 - dw_2),  E_2 = w_0 (dw_2 - dw_0) + w_1 (dw_2 - dw_1),
+//   dlogit_1 = -(1 - s_1) (w_0 E_0 + w_2 E_2).
 //
 // Design (B200), per plane and per pass (row pass: A = left->right,
 // B = right->left over columns s; column pass: A = top->bottom,
@@ -27,11 +31,14 @@
 //   s all four of h_A(s-1), a_A(s), h_B(s+1), a_B(s) are at hand, so dlambda
 //   of both directions, the pass's share of dx and the tap products of both
 //   directions are produced without storing any plane of h or a.
-// * dx: the row pass's share goes to an fp32 shared plane (XOR layout of
-//   8-byte units); the column pass adds its share and stores dx once.
-// * Tap products: the 8 warps of a CTA (8 channels of one image) add theirs
-//   into one shared buffer per chunk; the last warp to finish the chunk sends
-//   it with a bulk shared->global fp32 reduce-add into an L2-resident sum.
+// * dx: the row pass's share goes to a per-warp fp32 plane in the workspace
+//   (rewritten for every plane, so it stays in L2); the column pass adds its
+//   share and stores dx once.
+// * Tap values E_0, E_2: each of the 8 warps of a CTA (8 channels of one
+//   image) stores its chunk of values into its own shared slot; after a
+//   barrier of the 8 warps, warp w sums step w of the chunk over the 8 slots
+//   and adds it with a bulk shared->global fp32 reduce-add to L2-resident
+//   sums.  Slots alternate between two sets, so no warp waits for the sums.
 // * x, lambda and dout are streamed by TMA exactly as in the compact forward
 //   (per-warp ring of 8-step chunks); the normalised tap weights (a table
 //   written by a pre-kernel, one row per scan step with both directions at
@@ -59,16 +66,15 @@ constexpr int NWS = 2;          // weight ring stages per CTA
 constexpr int BOX = 1024;       // one plane of one tensor per chunk
 constexpr int SLICE = 512;
 constexpr int STAGE = 4 * BOX;  // x, lambda_A, lambda_B, dout
-constexpr int DACC = S * S * 4;
 constexpr int WCHUNK = 8 * S * 16;
-constexpr int DBUF = 2 * 3 * 8 * S * 4;  // [dir][tap][step][position] fp32
-constexpr int WARP_BYTES = NST * STAGE + DACC;
+constexpr int DSLOT = 8 * 4 * S * 4;      // one warp's tap values of a chunk: [step][dir*2 + value][position]
+constexpr int WARP_BYTES = NST * STAGE;   // data ring per warp
 constexpr int WRING = NCW * WARP_BYTES;
-constexpr int DBUFO = WRING + NWS * WCHUNK;
-constexpr int BARS = DBUFO + DBUF;
+constexpr int DSTG = WRING + NWS * WCHUNK;    // 2 sets x NCW slots
+constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // NCW reduced one-step slices (1 KB)
+constexpr int BARS = DOUT + NCW * 1024;
 constexpr int NBAR = NCW * NST + 2 * NWS + 1;
-constexpr int CNT = BARS + 8 * NBAR;
-constexpr int SMEM_BYTES = 1024 + CNT + 16;
+constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR;
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
 constexpr int THREADS = (NCW + 1) * 32;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -94,8 +100,8 @@ __global__ void c64b_table_kernel(const T* __restrict__ logits, float4* __restri
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx == 0) *err = 0;
     const int n = B * 2 * S * S;
-    // the tap-product sums start at zero: 2 directions x 3 taps per table entry
-    for (int q = idx; q < n * 6; q += gridDim.x * blockDim.x) dsum[q] = 0.f;
+    // the tap sums start at zero: 2 directions x 2 values per table entry
+    for (int q = idx; q < n * 4; q += gridDim.x * blockDim.x) dsum[q] = 0.f;
     if (idx >= n) return;
     const int j = idx & 63, s = (idx >> 6) & 63, pass = (idx >> 12) & 1, b = idx >> 13;
     const int slotA = pass ? 0 : 2, slotB = pass ? 1 : 3;
@@ -107,10 +113,10 @@ __global__ void c64b_table_kernel(const T* __restrict__ logits, float4* __restri
     btab[((size_t)(b * 2 + pass) * S + s) * S + p * LPL + t] = make_float4(w0a, w0b, w2a, w2b);
 }
 
-// dlogits from the tap-product sums: for the pixel's valid taps with sigmoids s_k
-// and normalised weights w_k, dlogit_k = w_k (1 - s_k) sum_m w_m (D_k - D_m)
-// (the chain rule through w_k = s_k / sum s, s_k = sigmoid(logit_k)); zero on the
-// first line of each direction (its taps are never used) and on invalid taps.
+// dlogits from the tap sums: with the pixel's sigmoids s_k and normalised
+// weights w_k over its valid taps, dlogit_0 = w_0 (1 - s_0) E_0,
+// dlogit_2 = w_2 (1 - s_2) E_2, dlogit_1 = -(1 - s_1) (w_0 E_0 + w_2 E_2); zero on
+// the first line of each direction (its taps are never used) and on invalid taps.
 template <typename T>
 __global__ void c64b_dlogits_kernel(const T* __restrict__ logits, const float* __restrict__ dsum,
                                     T* __restrict__ dlogits, int B) {
@@ -124,33 +130,24 @@ __global__ void c64b_dlogits_kernel(const T* __restrict__ logits, const float* _
     const bool first_line = dir == 0 ? s == 0 : s == S - 1;
     const T* lg = logits + (size_t)(slot * B + b) * 3 * S * S;
     T* out = dlogits + (size_t)(slot * B + b) * 3 * S * S;
-    float d[3] = {0.f, 0.f, 0.f}, sg[3], w[3];
-    const bool valid[3] = {j > 0, true, j < S - 1};
-    float sum = 0.f;
-    for (int k = 0; k < 3; ++k) {
-        sg[k] = valid[k] ? sigmoidf(load_elt(lg, k * S * S + pix)) : 0.f;
-        sum += sg[k];
-    }
-    const float rs = 1.f / sum;
-    const size_t base = (((size_t)(b * 2 + pass) * 2 + dir) * 3) * S * S + (size_t)s * S + (j & 1) * LPL + (j >> 1);
-    for (int k = 0; k < 3; ++k) {
-        w[k] = sg[k] * rs;
-        d[k] = dsum[base + (size_t)k * S * S];
-    }
-    for (int k = 0; k < 3; ++k) {
-        float v = 0.f;
-        if (!first_line && valid[k]) {
-            float acc = 0.f;
-            for (int m = 0; m < 3; ++m) acc += w[m] * (d[k] - d[m]);
-            v = w[k] * (1.f - sg[k]) * acc;
-        }
-        store_elt(out, (size_t)k * S * S + pix, v);
-    }
+    const bool v0 = j > 0, v2 = j < S - 1;
+    const float s0 = v0 ? sigmoidf(load_elt(lg, pix)) : 0.f;
+    const float s1 = sigmoidf(load_elt(lg, S * S + pix));
+    const float s2 = v2 ? sigmoidf(load_elt(lg, 2 * S * S + pix)) : 0.f;
+    const float rs = 1.f / (s0 + s1 + s2);
+    const float w0 = s0 * rs, w2 = s2 * rs;
+    const size_t base = (((size_t)(b * 2 + pass) * 4 + dir * 2) * S + s) * S + (j & 1) * LPL + (j >> 1);
+    const float e0 = first_line ? 0.f : dsum[base];
+    const float e2 = first_line ? 0.f : dsum[base + (size_t)S * S];
+    store_elt(out, pix, v0 ? w0 * (1.f - s0) * e0 : 0.f);
+    store_elt(out, (size_t)S * S + pix, -(1.f - s1) * (w0 * e0 + w2 * e2));
+    store_elt(out, (size_t)2 * S * S + pix, v2 ? w2 * (1.f - s2) * e2 : 0.f);
 }
 
 struct C64BArgs {
     const float4* btab;
-    float* dsum;  // [B][pass][dir][tap][s][p*32 + t]
+    float* dsum;  // [B][pass][dir*2 + value][s][p*32 + t]: E_0, E_2 sums
+    float* dxh;   // per-warp fp32 planes: the row pass's share of dx
     __nv_bfloat16* dx;
     __nv_bfloat16* dlam;
     int* err;
@@ -206,9 +203,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
     const uint32_t wfull0 = sbase + BARS + 8 * NCW * NST;
     const uint32_t wempty0 = wfull0 + 8 * NWS;
-    const uint32_t dempty = wempty0 + 8 * NWS;
-    unsigned int* const dcount = reinterpret_cast<unsigned int*>(smem + CNT);
-    float* const dbuf = reinterpret_cast<float*>(smem + DBUFO);
+    const uint32_t dbar = wempty0 + 8 * NWS;  // the consumer warps' slots of a chunk are written
     if ((int)blockIdx.x >= a.groups) return;
 
     if (threadIdx.x == 0) {
@@ -217,12 +212,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_init(wfull0 + 8 * s, 1);
             tma::mbar_init(wempty0 + 8 * s, NCW);
         }
-        tma::mbar_init(dempty, 1);
-        *dcount = 0;
+        tma::mbar_init(dbar, NCW * 32);
         tma::fence_barrier_init();
     }
-    // the tap-product buffer starts at zero
-    for (int q = threadIdx.x; q < DBUF / 4; q += THREADS) dbuf[q] = 0.f;
     __syncthreads();
 
     const int ngroups_here = (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
@@ -261,7 +253,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------- consumer warps ----------------
     const uint32_t ring = sbase + warp * WARP_BYTES;
     unsigned char* const ringp = smem + warp * WARP_BYTES;
-    unsigned char* const daccp = ringp + NST * STAGE;
+    float* const dxslot = a.dxh + ((size_t)blockIdx.x * NCW + warp) * S * S;
     const unsigned char* const wring = smem + WRING;
     const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
 
@@ -305,7 +297,6 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     int k = 0, stage = 0;
     uint32_t phase = 0;
-    int dchunk = 0;  // sweep-2 chunks done (tap-product buffer uses)
     auto fail = [&]() {
         if (t == 0) atomicExch(a.err, 1);
         for (int kk = k; kk < k + NST && kk < nchunks; ++kk)
@@ -344,47 +335,42 @@ __global__ void __launch_bounds__(THREADS, 1)
             w2B[p] = v.w;
         }
     };
-    // tap products of one direction/tap/position into the CTA buffer
-    auto dadd = [&](int dir, int kt, int e, int p, float v) {
-        atomicAdd(dbuf + ((dir * 3 + kt) * 8 + e) * S + p * LPL + t, v);
+    // tap values of sweep-2 chunk number dchunk: this warp's slot in set dchunk & 1
+    int dchunk = 0;
+    auto dslot = [&]() -> float* {
+        return reinterpret_cast<float*>(smem + DSTG + ((dchunk & 1) * NCW + warp) * DSLOT);
     };
-    // the warp is done with the tap-product buffer of this sweep-2 chunk; the last
-    // of the 8 warps sends it to the global sums, clears it and frees it
-    auto dflush = [&](float* gdst) -> bool {
-        __threadfence_block();
+    // end of a sweep-2 chunk: after the 8 warps have stored their slots, warp w
+    // sums step w of the chunk over the 8 slots and adds its 4 rows (direction x
+    // value, 64 positions) to the global sums at rows gdst + w*64.  A warp can be
+    // at most one chunk ahead of the slowest (it waits here for all of them), so
+    // one barrier's phase parity tells the chunks apart and two slot sets suffice.
+    auto dreduce = [&](float* gdst) -> bool {
+        tma::mbar_arrive(dbar);
+        const bool ok = tma::mbar_wait(dbar, dchunk & 1);
+        if (!__all_sync(FULL, ok)) return false;
+        const float* set = reinterpret_cast<const float*>(smem + DSTG + (dchunk & 1) * NCW * DSLOT) + warp * 256;
+        float* outp = reinterpret_cast<float*>(smem + DOUT + warp * 1024);
+        if (t == 0) tma::bulk_wait_read();  // the previous reduce has read this slice
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float acc = 0.f;
+#pragma unroll
+            for (int w = 0; w < NCW; ++w) acc += set[w * (DSLOT / 4) + i * 32 + t];
+            outp[i * 32 + t] = acc;
+        }
         tma::fence_proxy_async();
         __syncwarp();
-        unsigned last = 0;
-        if (t == 0) last = atomicAdd(dcount, 1u) == NCW - 1 ? 1u : 0u;
-        last = __shfl_sync(FULL, last, 0);
-        if (last) {
-            __threadfence_block();
-            tma::fence_proxy_async();
-            if (t == 0) {
-                for (int r = 0; r < 6; ++r)
-                    tma::reduce_add_f32(gdst + (size_t)r * S * S, sbase + DBUFO + r * 8 * S * 4, 8 * S * 4);
-                tma::bulk_commit();
-                tma::bulk_wait_read();
-                *dcount = 0;
-            }
-            __syncwarp();
-            for (int q = t; q < DBUF / 16; q += 32) reinterpret_cast<float4*>(dbuf)[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-            __threadfence_block();
-            __syncwarp();
-            if (t == 0) tma::mbar_arrive(dempty);
+        if (t == 0) {
+            for (int r = 0; r < 4; ++r)
+                tma::reduce_add_f32(gdst + (size_t)r * S * S + warp * S, sbase + DOUT + warp * 1024 + r * 256, 256);
+            tma::bulk_commit();
         }
         ++dchunk;
         return true;
     };
-    // before the first tap product of a sweep-2 chunk: the buffer is free again
-    auto dacquire = [&]() -> bool {
-        if (dchunk == 0) return true;
-        const bool ok = tma::mbar_wait(dempty, (dchunk - 1) & 1);
-        return __all_sync(FULL, ok);
-    };
 
-    const int tk = t & 15;
-    unsigned char* const drow = daccp + 2 * t * 256;  // row pass: rows 2t, 2t+1
 
     for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
         const int plane = 8 * group + warp;
@@ -396,7 +382,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int la = pass ? 0 : 2, lb = pass ? 1 : 3;
             __nv_bfloat16* const dlamA = a.dlam + ((size_t)la * BC + plane) * S * S;
             __nv_bfloat16* const dlamB = a.dlam + ((size_t)lb * BC + plane) * S * S;
-            float* const dsum = a.dsum + ((size_t)(b * 2 + pass) * 2) * 3 * S * S;
+            float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S;
 
             // ---------------- sweep 1: h_A forward and a_B adjoint, s ascending ----------------
             float hA[2] = {0.f, 0.f}, aB[2] = {0.f, 0.f};
@@ -426,7 +412,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                 release_data();
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    const int s = 8 * q + e;
                     float w0A[2], w0B[2], w2A[2], w2B[2];
                     wrow(e, w0A, w0B, w2A, w2B);
                     float lx[2], g[2];
@@ -442,12 +427,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     float nb[4];
                     fwd_step(hA, lx, w0A, w2A, nb);
-                    if (s > 0) {
-                        adj_step(aB, g, w0Bp, w2Bp, t);
-                    } else {
-                        aB[0] = g[0];
-                        aB[1] = g[1];
-                    }
+                    // s = 0 (B's last line) has no carry: aB and the taps of line -1 are 0
+                    adj_step(aB, g, w0Bp, w2Bp, t);
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
                         w0Bp[p] = w0B[p];
@@ -523,12 +504,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         float lx[2] = {lav(e, 0) * xv(e, 0), lav(e, 1) * xv(e, 1)};
                         float g[2] = {gv(e, 0), gv(e, 1)};
                         fwd_step(h, lx, w0A, w2A, hs[e]);
-                        if (8 * q + e > 0) {
-                            adj_step(ab, g, w0Bq, w2Bq, t);
-                        } else {
-                            ab[0] = g[0];
-                            ab[1] = g[1];
-                        }
+                        adj_step(ab, g, w0Bq, w2Bq, t);  // zero state and taps before s = 0
                         aBs[e][0] = ab[0];
                         aBs[e][1] = ab[1];
 #pragma unroll
@@ -538,9 +514,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                     }
                 }
-                if (!dacquire()) { fail(); return false; }
                 uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns
-                float dxp[2];                    // row pass: dx share of column s+1 (pairs)
+                float dxr[2][8];                 // row pass: dx share of rows 2t+p, 8 columns
+                float2 dxin[8];                  // column pass: row pass's dx share, rows 8q+e
+                if constexpr (decltype(pass_c)::value == 1) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        dxin[e] = *reinterpret_cast<const float2*>(dxslot + (8 * q + e) * S + 2 * t);
+                }
+                float* const ds = dslot();
 #pragma unroll
                 for (int ee = 0; ee < 8; ++ee) {
                     const int e = 7 - ee;
@@ -548,35 +530,33 @@ __global__ void __launch_bounds__(THREADS, 1)
                     float w0A[2], w0B[2], w2A[2], w2B[2];
                     wrow(e, w0A, w0B, w2A, w2B);
                     float g[2] = {gv(e, 0), gv(e, 1)};
-                    // adjoint of A at s from s+1 (taps of line s+1)
-                    if (s < S - 1) {
-                        adj_step(aA, g, w0An, w2An, t);
-                    } else {
-                        aA[0] = g[0];
-                        aA[1] = g[1];
-                    }
+                    // adjoint of A at s from s+1 (taps of line s+1; zero state and taps at s = 63)
+                    adj_step(aA, g, w0An, w2An, t);
                     // forward of B at s from s+1 (taps of B's line at s)
                     float lxb[2] = {lbv(e, 0) * xv(e, 0), lbv(e, 1) * xv(e, 1)};
                     float nbB[4];
                     fwd_step(hB, lxb, w0B, w2B, nbB);
-                    // tap products: A's line s reads h_A(s-1); B's line (column/row s)
-                    // reads h_B(s+1); the first line of each direction has none
-                    if (s > 0) {
-                        dadd(0, 0, e, 0, aA[0] * hs[e][0]);
-                        dadd(0, 1, e, 0, aA[0] * hs[e][1]);
-                        dadd(0, 2, e, 0, aA[0] * hs[e][2]);
-                        dadd(0, 0, e, 1, aA[1] * hs[e][1]);
-                        dadd(0, 1, e, 1, aA[1] * hs[e][2]);
-                        dadd(0, 2, e, 1, aA[1] * hs[e][3]);
-                    }
-                    if (s < S - 1) {
-                        const float* ab = aBs[e];
-                        dadd(1, 0, e, 0, ab[0] * nbB[0]);
-                        dadd(1, 1, e, 0, ab[0] * nbB[1]);
-                        dadd(1, 2, e, 0, ab[0] * nbB[2]);
-                        dadd(1, 0, e, 1, ab[1] * nbB[1]);
-                        dadd(1, 1, e, 1, ab[1] * nbB[2]);
-                        dadd(1, 2, e, 1, ab[1] * nbB[3]);
+                    // tap values: A's line s reads h_A(s-1) (neighbours hs[e]) with taps
+                    // w0A, w2A; B's line at s reads h_B(s+1) (nbB) with w0B, w2B.  On the
+                    // first line of each direction the read state is zero, so they are 0.
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        {
+                            const float hl = hs[e][p], hc = hs[e][p + 1], hr = hs[e][p + 2];
+                            const float w0 = w0A[p], w2 = w2A[p], w1 = 1.f - w0 - w2;
+                            const float u0 = w1 * (hl - hc) + w2 * (hl - hr);
+                            const float u2 = w0 * (hr - hl) + w1 * (hr - hc);
+                            ds[(e * 4 + 0) * S + p * LPL + t] = aA[p] * u0;
+                            ds[(e * 4 + 1) * S + p * LPL + t] = aA[p] * u2;
+                        }
+                        {
+                            const float hl = nbB[p], hc = nbB[p + 1], hr = nbB[p + 2];
+                            const float w0 = w0B[p], w2 = w2B[p], w1 = 1.f - w0 - w2;
+                            const float u0 = w1 * (hl - hc) + w2 * (hl - hr);
+                            const float u2 = w0 * (hr - hl) + w1 * (hr - hc);
+                            ds[(e * 4 + 2) * S + p * LPL + t] = aBs[e][p] * u0;
+                            ds[(e * 4 + 3) * S + p * LPL + t] = aBs[e][p] * u2;
+                        }
                     }
                     // dlambda of both directions and this pass's share of dx
                     float dla[2], dlb[2], dxs[2];
@@ -599,20 +579,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 dlB[p][e >> 1] = (dlB[p][e >> 1] & 0xffff0000u) | (pack_bf2(dlb[p], 0.f) & 0xffffu);
                             }
                         }
-                        // dx share into the fp32 plane, columns s, s+1 per 8-byte unit
-                        if (e & 1) {
-                            dxp[0] = dxs[0];
-                            dxp[1] = dxs[1];
-                        } else {
-                            const uint32_t o = (uint32_t)(((s >> 1) ^ tk) << 3);
-#pragma unroll
-                            for (int p = 0; p < 2; ++p) sts64f(drow + p * 256 + o, make_float2(dxs[p], dxp[p]));
-                        }
+                        dxr[0][e] = dxs[0];
+                        dxr[1][e] = dxs[1];
                     } else {
                         // row s, columns 2t, 2t+1: complete dx, dlambda of both directions
-                        const float2 prev = lds64f(daccp + s * 256 + ((t ^ ((s >> 1) & 15)) << 3));
                         stg_cs32(a.dx + (size_t)plane * S * S + s * S + 2 * t,
-                                 pack_bf2(prev.x + dxs[0], prev.y + dxs[1]));
+                                 pack_bf2(dxin[e].x + dxs[0], dxin[e].y + dxs[1]));
                         stg_cs32(dlamA + s * S + 2 * t, pack_bf2(dla[0], dla[1]));
                         stg_cs32(dlamB + s * S + 2 * t, pack_bf2(dlb[0], dlb[1]));
                     }
@@ -630,16 +602,27 @@ __global__ void __launch_bounds__(THREADS, 1)
                         uint4 vb = make_uint4(dlB[p][0], dlB[p][1], dlB[p][2], dlB[p][3]);
                         __stcs(reinterpret_cast<uint4*>(dlamA + r * S + 8 * q), va);
                         __stcs(reinterpret_cast<uint4*>(dlamB + r * S + 8 * q), vb);
+                        float4* dxo = reinterpret_cast<float4*>(dxslot + r * S + 8 * q);
+                        dxo[0] = make_float4(dxr[p][0], dxr[p][1], dxr[p][2], dxr[p][3]);
+                        dxo[1] = make_float4(dxr[p][4], dxr[p][5], dxr[p][6], dxr[p][7]);
                     }
                 }
-                dflush(dsum + (size_t)8 * q * S);
+                if (!dreduce(dsum + (size_t)8 * q * S)) {
+                    ++k;  // the data and weight stages of this chunk were consumed
+                    fail();
+                    return false;
+                }
                 release_w();
             }
             __syncwarp();
             return true;
         };
-        if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) return;
+        if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) {
+            if (t == 0) tma::bulk_wait_all();
+            return;
+        }
     }
+    if (t == 0) tma::bulk_wait_all();  // the last reduces have read their shared slices
 }
 
 // ---- host side ----------------------------------------------------------------------
@@ -681,10 +664,19 @@ bool c64_bwd_eligible(const Problem& p) {
            p.g.groups == 1 && p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_fn_b() != nullptr;
 }
 
-size_t c64_bwd_workspace(const Problem& p) {
-    // error word | tap table (B*2*64*64 float4) | tap-product sums (B*2*2*3*64*64 fp32)
-    return kWsAlign + align_up((size_t)p.g.B * 2 * S * S * sizeof(float4), kWsAlign) +
-           align_up((size_t)p.g.B * 2 * 2 * 3 * S * S * sizeof(float), kWsAlign);
+namespace {
+size_t tab_bytes(const Problem& p) { return align_up((size_t)p.g.B * 2 * S * S * sizeof(float4), kWsAlign); }
+size_t sum_bytes(const Problem& p) { return align_up((size_t)p.g.B * 2 * 4 * S * S * sizeof(float), kWsAlign); }
+int bwd_grid(const Problem& p, const DeviceInfo& dev) {
+    const int groups = (int)(p.planes / 8);
+    return groups < dev.sm_count ? groups : dev.sm_count;
+}
+}  // namespace
+
+size_t c64_bwd_workspace(const Problem& p, const DeviceInfo& dev) {
+    // error word | tap table (B*2*64*64 float4) | E sums (B*2*4*64*64 fp32) |
+    // per-warp dx planes (grid*8 x 64*64 fp32)
+    return kWsAlign + tab_bytes(p) + sum_bytes(p) + (size_t)bwd_grid(p, dev) * NCW * S * S * sizeof(float);
 }
 
 gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
@@ -699,7 +691,8 @@ gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     C64BArgs a;
     a.err = reinterpret_cast<int*>(w);
     a.btab = reinterpret_cast<const float4*>(w + kWsAlign);
-    a.dsum = reinterpret_cast<float*>(w + kWsAlign + align_up((size_t)p.g.B * 2 * S * S * sizeof(float4), kWsAlign));
+    a.dsum = reinterpret_cast<float*>(w + kWsAlign + tab_bytes(p));
+    a.dxh = reinterpret_cast<float*>(w + kWsAlign + tab_bytes(p) + sum_bytes(p));
     a.dx = static_cast<__nv_bfloat16*>(dx);
     a.dlam = static_cast<__nv_bfloat16*>(dlam);
     a.B = p.g.B;
@@ -711,7 +704,7 @@ gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
     cudaError_t e = ensure_smem_attr((const void*)c64b_kernel, SMEM_BYTES, 10);
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
-    const int grid = a.groups < dev.sm_count ? a.groups : dev.sm_count;
+    const int grid = bwd_grid(p, dev);
     c64b_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, gc, xr, lr, gr, a);
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
     const int nl = 4 * p.g.B * S * S;

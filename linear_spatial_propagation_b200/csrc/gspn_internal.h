@@ -52,7 +52,7 @@ gspn_status c64_fwd_noalloc(const Problem& p, const DeviceInfo& dev, const void*
 
 // ---- compact 64x64 bf16 backward (TMA-fed, checkpointed sweeps) ------------------
 bool c64_bwd_eligible(const Problem& p);
-size_t c64_bwd_workspace(const Problem& p);
+size_t c64_bwd_workspace(const Problem& p, const DeviceInfo& dev);
 gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
                     const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s);
 
