@@ -35,10 +35,11 @@
 //   (rewritten for every plane, so it stays in L2); the column pass adds its
 //   share and stores dx once.
 // * Tap values E_0, E_2: each of the 8 warps of a CTA (8 channels of one
-//   image) stores its chunk of values into its own shared slot; after a
-//   barrier of the 8 warps, warp w sums step w of the chunk over the 8 slots
-//   and adds it with a bulk shared->global fp32 reduce-add to L2-resident
-//   sums.  Slots alternate between two sets, so no warp waits for the sums.
+//   image) stores its chunk of values into its own shared slot; a reducer
+//   warp sums the 8 slots of a chunk and adds the result with bulk
+//   shared->global fp32 reduce-adds to L2-resident sums.  Slots alternate
+//   between two sets, so a compute warp waits only if it runs two chunks
+//   ahead of the reducer.
 // * x, lambda and dout are streamed by TMA exactly as in the compact forward
 //   (per-warp ring of 8-step chunks); the normalised tap weights (a table
 //   written by a pre-kernel, one row per scan step with both directions at
@@ -67,16 +68,16 @@ constexpr int BOX = 1024;       // one plane of one tensor per chunk
 constexpr int SLICE = 512;
 constexpr int STAGE = 4 * BOX;  // x, lambda_A, lambda_B, dout
 constexpr int WCHUNK = 8 * S * 16;
-constexpr int DSLOT = 8 * 4 * S * 4;      // one warp's tap values of a chunk: [step][dir*2 + value][position]
+constexpr int DSLOT = 8 * 4 * S * 4;      // one warp's tap values of a chunk: [step][dir*2 + value][position j]
 constexpr int WARP_BYTES = NST * STAGE;   // data ring per warp
 constexpr int WRING = NCW * WARP_BYTES;
 constexpr int DSTG = WRING + NWS * WCHUNK;    // 2 sets x NCW slots
-constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // NCW reduced one-step slices (1 KB)
-constexpr int BARS = DOUT + NCW * 1024;
-constexpr int NBAR = NCW * NST + 2 * NWS + 1;
+constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // the reduced chunk: [dir*2 + value][step][position j]
+constexpr int BARS = DOUT + DSLOT;
+constexpr int NBAR = NCW * NST + 2 * NWS + 4;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR;
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
-constexpr int THREADS = (NCW + 1) * 32;
+constexpr int THREADS = (NCW + 2) * 32;  // compute warps, tap-table producer, tap-value reducer
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ---- backward tap table ---------------------------------------------------------------
@@ -136,7 +137,7 @@ __global__ void c64b_dlogits_kernel(const T* __restrict__ logits, const float* _
     const float s2 = v2 ? sigmoidf(load_elt(lg, 2 * S * S + pix)) : 0.f;
     const float rs = 1.f / (s0 + s1 + s2);
     const float w0 = s0 * rs, w2 = s2 * rs;
-    const size_t base = (((size_t)(b * 2 + pass) * 4 + dir * 2) * S + s) * S + (j & 1) * LPL + (j >> 1);
+    const size_t base = (((size_t)(b * 2 + pass) * 4 + dir * 2) * S + s) * S + j;
     const float e0 = first_line ? 0.f : dsum[base];
     const float e2 = first_line ? 0.f : dsum[base + (size_t)S * S];
     store_elt(out, pix, v0 ? w0 * (1.f - s0) * e0 : 0.f);
@@ -146,7 +147,7 @@ __global__ void c64b_dlogits_kernel(const T* __restrict__ logits, const float* _
 
 struct C64BArgs {
     const float4* btab;
-    float* dsum;  // [B][pass][dir*2 + value][s][p*32 + t]: E_0, E_2 sums
+    float* dsum;  // [B][pass][dir*2 + value][s][j]: E_0, E_2 sums
     float* dxh;   // per-warp fp32 planes: the row pass's share of dx
     __nv_bfloat16* dx;
     __nv_bfloat16* dlam;
@@ -203,7 +204,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
     const uint32_t wfull0 = sbase + BARS + 8 * NCW * NST;
     const uint32_t wempty0 = wfull0 + 8 * NWS;
-    const uint32_t dbar = wempty0 + 8 * NWS;  // the consumer warps' slots of a chunk are written
+    const uint32_t dfull0 = wempty0 + 8 * NWS;  // [set]: the compute warps' slots of a chunk are written
+    const uint32_t dempty0 = dfull0 + 16;       // [set]: the reducer has read the set
     if ((int)blockIdx.x >= a.groups) return;
 
     if (threadIdx.x == 0) {
@@ -212,7 +214,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_init(wfull0 + 8 * s, 1);
             tma::mbar_init(wempty0 + 8 * s, NCW);
         }
-        tma::mbar_init(dbar, NCW * 32);
+        for (int s = 0; s < 2; ++s) {
+            tma::mbar_init(dfull0 + 8 * s, NCW * 32);
+            tma::mbar_init(dempty0 + 8 * s, 1);
+        }
         tma::fence_barrier_init();
     }
     __syncthreads();
@@ -250,10 +255,67 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
     }
 
+    // ---------------- reducer warp: tap values of each sweep-2 chunk ----------------
+    // Sweep-2 chunk n of the CTA (pass-major within a group, q descending) sits in
+    // slot set n & 1.  The 8 slots are summed into the reduced chunk, the set is
+    // handed back, and the chunk is added to the image's sums (rows 8q..8q+7 of
+    // each of the 4 [s][j] planes) by 4 bulk reduce-adds of 2 KB.
+    if (warp == NCW + 1) {
+        const float4* const sets = reinterpret_cast<const float4*>(smem + DSTG);
+        float4* const outp = reinterpret_cast<float4*>(smem + DOUT);
+        int n = 0;
+        bool ok = true;
+        for (int group = blockIdx.x; ok && group < a.groups; group += gridDim.x) {
+            const int b = (8 * group) / a.C;
+            for (int pass = 0; ok && pass < 2; ++pass) {
+                float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S;
+                for (int qq = 0; qq < 8; ++qq, ++n) {
+                    const int q = 7 - qq, set = n & 1;
+                    if (!__all_sync(FULL, tma::mbar_wait(dfull0 + 8 * set, (n >> 1) & 1))) {
+                        ok = false;
+                        break;
+                    }
+                    if (t == 0) tma::bulk_wait_read();  // the previous chunk's reduces have read outp
+                    __syncwarp();
+                    const float4* const src = sets + set * NCW * (DSLOT / 16);
+#pragma unroll 4
+                    for (int i = 0; i < DSLOT / 16 / 32; ++i) {
+                        const int f = i * 32 + t;  // float4 f of a slot: step f >> 6, row (f >> 4) & 3, j = 4 (f & 15)
+                        float4 acc = src[f];
+#pragma unroll
+                        for (int w = 1; w < NCW; ++w) {
+                            const float4 v = src[w * (DSLOT / 16) + f];
+                            acc.x += v.x;
+                            acc.y += v.y;
+                            acc.z += v.z;
+                            acc.w += v.w;
+                        }
+                        outp[(((f >> 4) & 3) * 8 + (f >> 6)) * 16 + (f & 15)] = acc;
+                    }
+                    __syncwarp();
+                    if (t == 0) tma::mbar_arrive(dempty0 + 8 * set);
+                    tma::fence_proxy_async();
+                    __syncwarp();
+                    if (t == 0) {
+                        for (int r = 0; r < 4; ++r)
+                            tma::reduce_add_f32(dsum + (size_t)r * S * S + 8 * q * S, sbase + DOUT + r * 2048, 2048);
+                        tma::bulk_commit();
+                    }
+                }
+            }
+        }
+        if (t == 0) {
+            if (!ok) atomicExch(a.err, 1);
+            tma::bulk_wait_all();
+        }
+        return;
+    }
+
     // ---------------- consumer warps ----------------
     const uint32_t ring = sbase + warp * WARP_BYTES;
     unsigned char* const ringp = smem + warp * WARP_BYTES;
     float* const dxslot = a.dxh + ((size_t)blockIdx.x * NCW + warp) * S * S;
+    const uint64_t keep = l2_evict_last_policy();
     const unsigned char* const wring = smem + WRING;
     const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
 
@@ -335,42 +397,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             w2B[p] = v.w;
         }
     };
-    // tap values of sweep-2 chunk number dchunk: this warp's slot in set dchunk & 1
+    // tap values of sweep-2 chunk number dchunk: this warp's slot in set dchunk & 1,
+    // free once the reducer has handed the set back
     int dchunk = 0;
     auto dslot = [&]() -> float* {
+        const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk & 1), ((dchunk >> 1) & 1) ^ 1);
+        if (!__all_sync(FULL, ok)) return nullptr;
         return reinterpret_cast<float*>(smem + DSTG + ((dchunk & 1) * NCW + warp) * DSLOT);
     };
-    // end of a sweep-2 chunk: after the 8 warps have stored their slots, warp w
-    // sums step w of the chunk over the 8 slots and adds its 4 rows (direction x
-    // value, 64 positions) to the global sums at rows gdst + w*64.  A warp can be
-    // at most one chunk ahead of the slowest (it waits here for all of them), so
-    // one barrier's phase parity tells the chunks apart and two slot sets suffice.
-    auto dreduce = [&](float* gdst) -> bool {
-        tma::mbar_arrive(dbar);
-        const bool ok = tma::mbar_wait(dbar, dchunk & 1);
-        if (!__all_sync(FULL, ok)) return false;
-        const float* set = reinterpret_cast<const float*>(smem + DSTG + (dchunk & 1) * NCW * DSLOT) + warp * 256;
-        float* outp = reinterpret_cast<float*>(smem + DOUT + warp * 1024);
-        if (t == 0) tma::bulk_wait_read();  // the previous reduce has read this slice
-        __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            float acc = 0.f;
-#pragma unroll
-            for (int w = 0; w < NCW; ++w) acc += set[w * (DSLOT / 4) + i * 32 + t];
-            outp[i * 32 + t] = acc;
-        }
-        tma::fence_proxy_async();
-        __syncwarp();
-        if (t == 0) {
-            for (int r = 0; r < 4; ++r)
-                tma::reduce_add_f32(gdst + (size_t)r * S * S + warp * S, sbase + DOUT + warp * 1024 + r * 256, 256);
-            tma::bulk_commit();
-        }
+    auto dpublish = [&]() {
+        tma::mbar_arrive(dfull0 + 8 * (dchunk & 1));  // every lane: its stores are released
         ++dchunk;
-        return true;
     };
-
 
     for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
         const int plane = 8 * group + warp;
@@ -382,7 +420,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int la = pass ? 0 : 2, lb = pass ? 1 : 3;
             __nv_bfloat16* const dlamA = a.dlam + ((size_t)la * BC + plane) * S * S;
             __nv_bfloat16* const dlamB = a.dlam + ((size_t)lb * BC + plane) * S * S;
-            float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S;
 
             // ---------------- sweep 1: h_A forward and a_B adjoint, s ascending ----------------
             float hA[2] = {0.f, 0.f}, aB[2] = {0.f, 0.f};
@@ -457,6 +494,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         w2Bm[p] = v.w;
                     }
                 }
+                float2 dxin[8];  // column pass: the row pass's dx share, rows 8q+e (loaded early)
+                if constexpr (decltype(pass_c)::value == 1) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) dxin[e] = ldg64_keep(dxslot + (8 * q + e) * S + 2 * t, keep);
+                }
                 if (!acquire()) { fail(); return false; }
                 uint4 X[2] = {}, LA[2] = {}, LB[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, LBr[8] = {}, Gr[8] = {};
@@ -516,13 +558,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns
                 float dxr[2][8];                 // row pass: dx share of rows 2t+p, 8 columns
-                float2 dxin[8];                  // column pass: row pass's dx share, rows 8q+e
-                if constexpr (decltype(pass_c)::value == 1) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        dxin[e] = *reinterpret_cast<const float2*>(dxslot + (8 * q + e) * S + 2 * t);
-                }
                 float* const ds = dslot();
+                if (ds == nullptr) {
+                    ++k;  // the data and weight stages of this chunk were consumed
+                    fail();
+                    return false;
+                }
 #pragma unroll
                 for (int ee = 0; ee < 8; ++ee) {
                     const int e = 7 - ee;
@@ -539,24 +580,26 @@ __global__ void __launch_bounds__(THREADS, 1)
                     // tap values: A's line s reads h_A(s-1) (neighbours hs[e]) with taps
                     // w0A, w2A; B's line at s reads h_B(s+1) (nbB) with w0B, w2B.  On the
                     // first line of each direction the read state is zero, so they are 0.
+                    {
+                        float v[4][2];
 #pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        {
-                            const float hl = hs[e][p], hc = hs[e][p + 1], hr = hs[e][p + 2];
-                            const float w0 = w0A[p], w2 = w2A[p], w1 = 1.f - w0 - w2;
-                            const float u0 = w1 * (hl - hc) + w2 * (hl - hr);
-                            const float u2 = w0 * (hr - hl) + w1 * (hr - hc);
-                            ds[(e * 4 + 0) * S + p * LPL + t] = aA[p] * u0;
-                            ds[(e * 4 + 1) * S + p * LPL + t] = aA[p] * u2;
+                        for (int p = 0; p < 2; ++p) {
+                            {
+                                const float hl = hs[e][p], hc = hs[e][p + 1], hr = hs[e][p + 2];
+                                const float w0 = w0A[p], w2 = w2A[p], w1 = 1.f - w0 - w2;
+                                v[0][p] = aA[p] * (w1 * (hl - hc) + w2 * (hl - hr));
+                                v[1][p] = aA[p] * (w0 * (hr - hl) + w1 * (hr - hc));
+                            }
+                            {
+                                const float hl = nbB[p], hc = nbB[p + 1], hr = nbB[p + 2];
+                                const float w0 = w0B[p], w2 = w2B[p], w1 = 1.f - w0 - w2;
+                                v[2][p] = aBs[e][p] * (w1 * (hl - hc) + w2 * (hl - hr));
+                                v[3][p] = aBs[e][p] * (w0 * (hr - hl) + w1 * (hr - hc));
+                            }
                         }
-                        {
-                            const float hl = nbB[p], hc = nbB[p + 1], hr = nbB[p + 2];
-                            const float w0 = w0B[p], w2 = w2B[p], w1 = 1.f - w0 - w2;
-                            const float u0 = w1 * (hl - hc) + w2 * (hl - hr);
-                            const float u2 = w0 * (hr - hl) + w1 * (hr - hc);
-                            ds[(e * 4 + 2) * S + p * LPL + t] = aBs[e][p] * u0;
-                            ds[(e * 4 + 3) * S + p * LPL + t] = aBs[e][p] * u2;
-                        }
+#pragma unroll
+                        for (int r = 0; r < 4; ++r)
+                            *reinterpret_cast<float2*>(ds + (e * 4 + r) * S + 2 * t) = make_float2(v[r][0], v[r][1]);
                     }
                     // dlambda of both directions and this pass's share of dx
                     float dla[2], dlb[2], dxs[2];
@@ -602,27 +645,25 @@ __global__ void __launch_bounds__(THREADS, 1)
                         uint4 vb = make_uint4(dlB[p][0], dlB[p][1], dlB[p][2], dlB[p][3]);
                         __stcs(reinterpret_cast<uint4*>(dlamA + r * S + 8 * q), va);
                         __stcs(reinterpret_cast<uint4*>(dlamB + r * S + 8 * q), vb);
-                        float4* dxo = reinterpret_cast<float4*>(dxslot + r * S + 8 * q);
-                        dxo[0] = make_float4(dxr[p][0], dxr[p][1], dxr[p][2], dxr[p][3]);
-                        dxo[1] = make_float4(dxr[p][4], dxr[p][5], dxr[p][6], dxr[p][7]);
+                        float* dxo = dxslot + r * S + 8 * q;
+                        stg128_keep(dxo, make_float4(dxr[p][0], dxr[p][1], dxr[p][2], dxr[p][3]), keep);
+                        stg128_keep(dxo + 4, make_float4(dxr[p][4], dxr[p][5], dxr[p][6], dxr[p][7]), keep);
                     }
                 }
-                if (!dreduce(dsum + (size_t)8 * q * S)) {
-                    ++k;  // the data and weight stages of this chunk were consumed
-                    fail();
-                    return false;
+                if constexpr (decltype(pass_c)::value == 1) {
+                    // every lane has used its loads of rows 8q..8q+7 of the dx plane:
+                    // the rows are dead, drop their 16 lines of 128 bytes from L2
+                    __syncwarp();
+                    if (t < 16) l2_discard128(dxslot + (8 * q + (t >> 1)) * S + (t & 1) * 32);
                 }
+                dpublish();
                 release_w();
             }
             __syncwarp();
             return true;
         };
-        if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) {
-            if (t == 0) tma::bulk_wait_all();
-            return;
-        }
+        if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) return;
     }
-    if (t == 0) tma::bulk_wait_all();  // the last reduces have read their shared slices
 }
 
 // ---- host side ----------------------------------------------------------------------

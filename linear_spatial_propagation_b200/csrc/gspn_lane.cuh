@@ -56,5 +56,28 @@ __device__ __forceinline__ float fma_bf(int half, uint32_t a, uint32_t b, float 
     return half ? fma_bf_hi(a, b, c) : fma_bf_lo(a, b, c);
 }
 
+// Scratch that lives in L2 between two phases of a kernel: stored with the
+// evict-last priority, read back once, then discarded (the dead lines are
+// dropped without a write-back to DRAM).
+__device__ __forceinline__ uint64_t l2_evict_last_policy() {
+    uint64_t pol;
+    asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+    return pol;
+}
+__device__ __forceinline__ void stg128_keep(float* p, float4 v, uint64_t pol) {
+    asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w), "l"(pol)
+                 : "memory");
+}
+__device__ __forceinline__ float2 ldg64_keep(const float* p, uint64_t pol) {
+    float2 v;
+    asm volatile("ld.global.L2::cache_hint.v2.f32 {%0, %1}, [%2], %3;" : "=f"(v.x), "=f"(v.y) : "l"(p), "l"(pol) : "memory");
+    return v;
+}
+// drop one 128-byte L2 line (128-byte aligned address); its contents become undefined
+__device__ __forceinline__ void l2_discard128(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 }  // namespace lane
 }  // namespace gspn
