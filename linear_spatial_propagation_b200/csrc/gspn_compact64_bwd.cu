@@ -63,17 +63,18 @@ constexpr int S = 64;           // H = W
 constexpr int LPL = 32;         // lanes per line, 2 positions each
 constexpr int NCW = 8;          // consumer warps (one plane each)
 constexpr int NST = 2;          // data ring stages per warp
-constexpr int NWS = 2;          // weight ring stages per CTA
+constexpr int NWS = 4;          // weight ring stages per CTA
 constexpr int BOX = 1024;       // one plane of one tensor per chunk
 constexpr int SLICE = 512;
 constexpr int STAGE = 4 * BOX;  // x, lambda_A, lambda_B, dout
 constexpr int WCHUNK = 8 * S * 16;
-constexpr int DSLOT = 8 * 4 * S * 4;      // one warp's tap values of a chunk: [step][dir*2 + value][position j]
+constexpr int DSLOT = 4 * 4 * S * 4;      // one warp's tap values of half a chunk: [step][dir*2 + value][position j]
 constexpr int WARP_BYTES = NST * STAGE;   // data ring per warp
 constexpr int WRING = NCW * WARP_BYTES;
 constexpr int DSTG = WRING + NWS * WCHUNK;    // 2 sets x NCW slots
-constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // the reduced chunk: [dir*2 + value][step][position j]
-constexpr int BARS = DOUT + DSLOT;
+constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // 2 reduced half chunks: [dir*2 + value][step][position j]
+constexpr int CKO = DOUT + 2 * DSLOT;          // per warp: sweep-1 checkpoints (h_A, a_B) of the 8 chunks
+constexpr int BARS = CKO + NCW * 8 * 32 * 16;
 constexpr int NBAR = NCW * NST + 2 * NWS + 4;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR;
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
@@ -81,10 +82,12 @@ constexpr int THREADS = (NCW + 2) * 32;  // compute warps, tap-table producer, t
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ---- backward tap table ---------------------------------------------------------------
-// btab[((b*2 + pass)*64 + s)*64 + p*32 + t] = (w0_A, w0_B, w2_A, w2_B) of position
-// j = 2t + p where both directions' lines sit at column (row pass) or row
-// (column pass) s: pass 0 A = left->right (slot 2), B = right->left (slot 3),
-// pixel (j, s); pass 1 A = top->bottom (slot 0), B = bottom->top (slot 1), pixel (s, j).
+// Row (b, pass, s) of the table holds the taps of both directions' lines at
+// column (row pass) or row (column pass) s, as pairs over the positions
+// j = 2t, 2t+1 of lane t: float4 t = (w0_A, w0_A', w2_A, w2_A') and float4
+// 32 + t = (w0_B, w0_B', w2_B, w2_B') (' = position 2t+1).  Pass 0: A =
+// left->right (slot 2), B = right->left (slot 3), pixel (j, s); pass 1: A =
+// top->bottom (slot 0), B = bottom->top (slot 1), pixel (s, j).
 template <typename T>
 __device__ __forceinline__ void gate_w(const T* lg, int pix, int j, float* w0, float* w2) {
     const float s0 = j > 0 ? sigmoidf(load_elt(lg, pix)) : 0.f;
@@ -100,18 +103,21 @@ __global__ void c64b_table_kernel(const T* __restrict__ logits, float4* __restri
                                   int* err, int B) {
     const int idx = blockIdx.x * blockDim.x + threadIdx.x;
     if (idx == 0) *err = 0;
-    const int n = B * 2 * S * S;
-    // the tap sums start at zero: 2 directions x 2 values per table entry
-    for (int q = idx; q < n * 4; q += gridDim.x * blockDim.x) dsum[q] = 0.f;
+    const int n = B * 2 * S * LPL;  // one thread per (b, pass, s, lane)
+    // the tap sums start at zero: 2 directions x 2 values per pixel of each pass
+    for (int q = idx; q < n * 8; q += gridDim.x * blockDim.x) dsum[q] = 0.f;
     if (idx >= n) return;
-    const int j = idx & 63, s = (idx >> 6) & 63, pass = (idx >> 12) & 1, b = idx >> 13;
+    const int t = idx & 31, s = (idx >> 5) & 63, pass = (idx >> 11) & 1, b = idx >> 12;
     const int slotA = pass ? 0 : 2, slotB = pass ? 1 : 3;
-    const int pix = pass ? s * S + j : j * S + s;
-    float w0a, w2a, w0b, w2b;
-    gate_w(logits + (size_t)(slotA * B + b) * 3 * S * S, pix, j, &w0a, &w2a);
-    gate_w(logits + (size_t)(slotB * B + b) * 3 * S * S, pix, j, &w0b, &w2b);
-    const int t = j >> 1, p = j & 1;
-    btab[((size_t)(b * 2 + pass) * S + s) * S + p * LPL + t] = make_float4(w0a, w0b, w2a, w2b);
+    float w[2][2][2];  // [dir][position][w0, w2]
+    for (int p = 0; p < 2; ++p) {
+        const int j = 2 * t + p, pix = pass ? s * S + j : j * S + s;
+        gate_w(logits + (size_t)(slotA * B + b) * 3 * S * S, pix, j, &w[0][p][0], &w[0][p][1]);
+        gate_w(logits + (size_t)(slotB * B + b) * 3 * S * S, pix, j, &w[1][p][0], &w[1][p][1]);
+    }
+    float4* row = btab + ((size_t)(b * 2 + pass) * S + s) * S;
+    row[t] = make_float4(w[0][0][0], w[0][1][0], w[0][0][1], w[0][1][1]);
+    row[LPL + t] = make_float4(w[1][0][0], w[1][1][0], w[1][0][1], w[1][1][1]);
 }
 
 // dlogits from the tap sums: with the pixel's sigmoids s_k and normalised
@@ -156,43 +162,51 @@ struct C64BArgs {
     int groups;  // B * C / 8
 };
 
+// bf16 element e of 8 packed in a uint4, widened
 __device__ __forceinline__ float bfv(const uint4& v, int e) {
     const uint32_t w = word_of(v, e >> 1);
     return (e & 1) ? __uint_as_float(w & 0xffff0000u) : __uint_as_float(w << 16);
 }
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-
-// Forward step: h(s) of both positions from h(s-1) = h; w0/w2 at own positions.
-__device__ __forceinline__ void fwd_step(float (&h)[2], const float (&lx)[2], const float (&w0)[2],
-                                         const float (&w2)[2], float* nb /* out: hl, h0, h1, hr of h(s-1) */) {
-    const float hl = __shfl_up_sync(FULL, h[1], 1);
-    const float hr = __shfl_down_sync(FULL, h[0], 1);
-    nb[0] = hl;
-    nb[1] = h[0];
-    nb[2] = h[1];
-    nb[3] = hr;
-    const float n0 = h[0] + lx[0] + w2[0] * (h[1] - h[0]) - w0[0] * (h[0] - hl);
-    const float n1 = h[1] + lx[1] + w2[1] * (hr - h[1]) - w0[1] * (h[1] - h[0]);
-    h[0] = n0;
-    h[1] = n1;
+// the two bf16 halves of a word, widened: (low, high)
+__device__ __forceinline__ float2 bf2(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
 }
 
-// Adjoint step: a(line i) from a = a(line i+1) with the weights of line i+1.
-__device__ __forceinline__ void adj_step(float (&a)[2], const float (&g)[2], const float (&w0)[2],
-                                         const float (&w2)[2], int t) {
-    const float p00 = w0[0] * a[0], p01 = w0[1] * a[1];
-    const float p20 = w2[0] * a[0], p21 = w2[1] * a[1];
-    float p0r = __shfl_down_sync(FULL, p00, 1);  // p0 at j = 2t+2
-    float p2l = __shfl_up_sync(FULL, p21, 1);    // p2 at j = 2t-1
-    if (t == LPL - 1) p0r = 0.f;
-    if (t == 0) p2l = 0.f;
-    const float n0 = g[0] + a[0] - p00 - p20 + p01 + p2l;
-    const float n1 = g[1] + a[1] - p01 - p21 + p0r + p20;
-    a[0] = n0;
-    a[1] = n1;
+// Lane t holds positions j = 2t, 2t+1 of a line as a float2; all arithmetic
+// below is packed over the pair.
+__device__ __forceinline__ float2 add2(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+
+// Tap weights of a line for this lane's pair of positions.
+struct Taps {
+    float2 w0, w2;
+};
+
+// Neighbour mix of the previous state h: m[j] = sum_k w_k[j] h[j+k-1],
+// written as h + w2 (hR - h) + w0 (hL - h) with w1 = 1 - w0 - w2; hL, hR
+// are h shifted by one position.  The shuffles rotate, so lane 0 reads
+// position 63 as its left neighbour and lane 31 position 0 as its right
+// one: both meet a zero tap weight (w0 at j = 0, w2 at j = 63).
+__device__ __forceinline__ float2 mix(float2 h, const Taps& w, int t, float2& hL, float2& hR) {
+    hL = make_float2(__shfl_sync(FULL, h.y, (t + 31) & 31), h.x);
+    hR = make_float2(h.y, __shfl_sync(FULL, h.x, (t + 1) & 31));
+    return fma2(w.w0, sub2(hL, h), fma2(w.w2, sub2(hR, h), h));
 }
 
+// Adjoint step: a(line i) = g + W_{i+1}^T a(line i+1), with w the taps of
+// line i+1: a'[j] = g[j] + w1[j] a[j] + w0[j+1] a[j+1] + w2[j-1] a[j-1].  The
+// rotated shuffles bring in w0 a at j = 0 and w2 a at j = 63, both zero.
+__device__ __forceinline__ float2 adjoint(float2 a, float2 g, const Taps& w, int t) {
+    const float2 p0 = mul2(w.w0, a), p2 = mul2(w.w2, a);
+    const float p0r = __shfl_sync(FULL, p0.x, (t + 1) & 31);  // w0 a at j = 2t+2
+    const float p2l = __shfl_sync(FULL, p2.y, (t + 31) & 31); // w2 a at j = 2t-1
+    float2 n = fma2(make_float2(-1.f, -1.f), p2, fma2(make_float2(-1.f, -1.f), p0, add2(g, a)));
+    return add2(n, add2(make_float2(p0.y, p0r), make_float2(p2l, p2.x)));
+}
+
+// 10 warps put 3 on two of the SM's four schedulers, each with a quarter of
+// the register file: at most 16384 / (3 * 32) -> 168 registers per thread
 __global__ void __launch_bounds__(THREADS, 1)
     c64b_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
                 const __grid_constant__ CUtensorMap tm_gc, const __grid_constant__ CUtensorMap tm_xr,
@@ -255,52 +269,51 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
     }
 
-    // ---------------- reducer warp: tap values of each sweep-2 chunk ----------------
-    // Sweep-2 chunk n of the CTA (pass-major within a group, q descending) sits in
-    // slot set n & 1.  The 8 slots are summed into the reduced chunk, the set is
-    // handed back, and the chunk is added to the image's sums (rows 8q..8q+7 of
-    // each of the 4 [s][j] planes) by 4 bulk reduce-adds of 2 KB.
+    // ---------------- reducer warp: tap values of each sweep-2 half chunk ----------------
+    // Half chunk n of the CTA (pass-major within a group, q descending, the upper
+    // 4 steps of a chunk first) sits in slot set n & 1.  The 8 slots are summed
+    // into reduced buffer n & 1, the set is handed back, and the half chunk is
+    // added to the image's sums (rows 8q+4h..8q+4h+3 of each of the 4 [s][j]
+    // planes) by 4 bulk reduce-adds of 1 KB.
     if (warp == NCW + 1) {
         const float4* const sets = reinterpret_cast<const float4*>(smem + DSTG);
-        float4* const outp = reinterpret_cast<float4*>(smem + DOUT);
         int n = 0;
         bool ok = true;
         for (int group = blockIdx.x; ok && group < a.groups; group += gridDim.x) {
             const int b = (8 * group) / a.C;
-            for (int pass = 0; ok && pass < 2; ++pass) {
-                float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S;
-                for (int qq = 0; qq < 8; ++qq, ++n) {
-                    const int q = 7 - qq, set = n & 1;
-                    if (!__all_sync(FULL, tma::mbar_wait(dfull0 + 8 * set, (n >> 1) & 1))) {
-                        ok = false;
-                        break;
-                    }
-                    if (t == 0) tma::bulk_wait_read();  // the previous chunk's reduces have read outp
-                    __syncwarp();
-                    const float4* const src = sets + set * NCW * (DSLOT / 16);
+            for (int l = 0; l < 32; ++l, ++n) {
+                const int pass = l >> 4, q = 7 - ((l >> 1) & 7), h = 1 - (l & 1), set = n & 1;
+                float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S + (8 * q + 4 * h) * S;
+                if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n >> 1) & 1, 128))) {
+                    ok = false;
+                    break;
+                }
+                if (t == 0) tma::bulk_wait_read_n<1>();  // the reduces of half chunk n-2 have read its buffer
+                __syncwarp();
+                const float4* const src = sets + set * NCW * (DSLOT / 16);
+                float4* const outp = reinterpret_cast<float4*>(smem + DOUT + set * DSLOT);
 #pragma unroll 4
-                    for (int i = 0; i < DSLOT / 16 / 32; ++i) {
-                        const int f = i * 32 + t;  // float4 f of a slot: step f >> 6, row (f >> 4) & 3, j = 4 (f & 15)
-                        float4 acc = src[f];
+                for (int i = 0; i < DSLOT / 16 / 32; ++i) {
+                    const int f = i * 32 + t;  // float4 f of a slot: step f >> 6, row (f >> 4) & 3, j = 4 (f & 15)
+                    float4 acc = src[f];
 #pragma unroll
-                        for (int w = 1; w < NCW; ++w) {
-                            const float4 v = src[w * (DSLOT / 16) + f];
-                            acc.x += v.x;
-                            acc.y += v.y;
-                            acc.z += v.z;
-                            acc.w += v.w;
-                        }
-                        outp[(((f >> 4) & 3) * 8 + (f >> 6)) * 16 + (f & 15)] = acc;
+                    for (int w = 1; w < NCW; ++w) {
+                        const float4 v = src[w * (DSLOT / 16) + f];
+                        acc.x += v.x;
+                        acc.y += v.y;
+                        acc.z += v.z;
+                        acc.w += v.w;
                     }
-                    __syncwarp();
-                    if (t == 0) tma::mbar_arrive(dempty0 + 8 * set);
-                    tma::fence_proxy_async();
-                    __syncwarp();
-                    if (t == 0) {
-                        for (int r = 0; r < 4; ++r)
-                            tma::reduce_add_f32(dsum + (size_t)r * S * S + 8 * q * S, sbase + DOUT + r * 2048, 2048);
-                        tma::bulk_commit();
-                    }
+                    outp[(((f >> 4) & 3) * 4 + (f >> 6)) * 16 + (f & 15)] = acc;
+                }
+                __syncwarp();
+                if (t == 0) tma::mbar_arrive(dempty0 + 8 * set);
+                tma::fence_proxy_async();
+                __syncwarp();
+                if (t == 0) {
+                    for (int r = 0; r < 4; ++r)
+                        tma::reduce_add_f32(dsum + (size_t)r * S * S, sbase + DOUT + set * DSLOT + r * 1024, 1024);
+                    tma::bulk_commit();
                 }
             }
         }
@@ -315,6 +328,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t ring = sbase + warp * WARP_BYTES;
     unsigned char* const ringp = smem + warp * WARP_BYTES;
     float* const dxslot = a.dxh + ((size_t)blockIdx.x * NCW + warp) * S * S;
+    float4* const ck = reinterpret_cast<float4*>(smem + CKO) + warp * 8 * 32 + t;  // [chunk][lane]
     const uint64_t keep = l2_evict_last_policy();
     const unsigned char* const wring = smem + WRING;
     const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
@@ -385,20 +399,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (t == 0) tma::mbar_arrive(wempty0 + 8 * (k % NWS));
         ++k;
     };
-    // tap weights of row e of the current weight stage, positions 2t, 2t+1
-    auto wrow = [&](int e, float (&w0A)[2], float (&w0B)[2], float (&w2A)[2], float (&w2B)[2]) {
+    // tap weights of row e of the current weight stage (line 8q+e of both directions)
+    auto wrow = [&](int e, Taps& A, Taps& Bt) {
         const unsigned char* src = wring + (k % NWS) * WCHUNK + e * 1024 + t * 16;
-#pragma unroll
-        for (int p = 0; p < 2; ++p) {
-            const float4 v = lds128f(src + p * 512);
-            w0A[p] = v.x;
-            w0B[p] = v.y;
-            w2A[p] = v.z;
-            w2B[p] = v.w;
-        }
+        const float4 va = lds128f(src), vb = lds128f(src + 512);
+        A.w0 = make_float2(va.x, va.y);
+        A.w2 = make_float2(va.z, va.w);
+        Bt.w0 = make_float2(vb.x, vb.y);
+        Bt.w2 = make_float2(vb.z, vb.w);
     };
-    // tap values of sweep-2 chunk number dchunk: this warp's slot in set dchunk & 1,
-    // free once the reducer has handed the set back
+    // tap values of sweep-2 half chunk number dchunk: this warp's slot in set
+    // dchunk & 1, free once the reducer has handed the set back
     int dchunk = 0;
     auto dslot = [&]() -> float* {
         const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk & 1), ((dchunk >> 1) & 1) ^ 1);
@@ -412,24 +423,22 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
         const int plane = 8 * group + warp;
-        const int b = plane / a.C;
-        const float4* const btab_b = a.btab + (size_t)b * 2 * S * S;
 
         auto run_pass = [&](auto pass_c) -> bool {
             constexpr int pass = decltype(pass_c)::value;
             const int la = pass ? 0 : 2, lb = pass ? 1 : 3;
             __nv_bfloat16* const dlamA = a.dlam + ((size_t)la * BC + plane) * S * S;
             __nv_bfloat16* const dlamB = a.dlam + ((size_t)lb * BC + plane) * S * S;
+            const Taps zero_taps = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 
             // ---------------- sweep 1: h_A forward and a_B adjoint, s ascending ----------------
-            float hA[2] = {0.f, 0.f}, aB[2] = {0.f, 0.f};
-            float ckA[8][2], ckB[8][2];
-            float w0Bp[2] = {0.f, 0.f}, w2Bp[2] = {0.f, 0.f};  // B taps of line s-1
+            float2 hA = make_float2(0.f, 0.f), aB = make_float2(0.f, 0.f);
+            Taps WBp = zero_taps;  // B taps of line s-1 (none before s = 0: a_B(-1) = 0)
             for (int q = 0; q < 8; ++q) {
                 if (!acquire()) { fail(); return false; }
                 uint4 X[2] = {}, LA[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, Gr[8] = {};
-                if constexpr (decltype(pass_c)::value == 0) {
+                if constexpr (pass == 0) {
                     const unsigned char* st = ringp + stage * STAGE + t * 16;
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
@@ -449,60 +458,42 @@ __global__ void __launch_bounds__(THREADS, 1)
                 release_data();
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                    float w0A[2], w0B[2], w2A[2], w2B[2];
-                    wrow(e, w0A, w0B, w2A, w2B);
-                    float lx[2], g[2];
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        if constexpr (decltype(pass_c)::value == 0) {
-                            lx[p] = bfv(LA[p], e) * bfv(X[p], e);
-                            g[p] = bfv(G[p], e);
-                        } else {
-                            lx[p] = (p ? bf_hi(LAr[e]) : bf_lo(LAr[e])) * (p ? bf_hi(Xr[e]) : bf_lo(Xr[e]));
-                            g[p] = p ? bf_hi(Gr[e]) : bf_lo(Gr[e]);
-                        }
+                    Taps WA, WB;
+                    wrow(e, WA, WB);
+                    float2 x, lam, g;
+                    if constexpr (pass == 0) {
+                        x = make_float2(bfv(X[0], e), bfv(X[1], e));
+                        lam = make_float2(bfv(LA[0], e), bfv(LA[1], e));
+                        g = make_float2(bfv(G[0], e), bfv(G[1], e));
+                    } else {
+                        x = bf2(Xr[e]);
+                        lam = bf2(LAr[e]);
+                        g = bf2(Gr[e]);
                     }
-                    float nb[4];
-                    fwd_step(hA, lx, w0A, w2A, nb);
-                    // s = 0 (B's last line) has no carry: aB and the taps of line -1 are 0
-                    adj_step(aB, g, w0Bp, w2Bp, t);
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        w0Bp[p] = w0B[p];
-                        w2Bp[p] = w2B[p];
-                    }
+                    float2 hL, hR;
+                    hA = add2(mix(hA, WA, t, hL, hR), mul2(lam, x));
+                    aB = adjoint(aB, g, WBp, t);
+                    WBp = WB;
                 }
-                ckA[q][0] = hA[0];
-                ckA[q][1] = hA[1];
-                ckB[q][0] = aB[0];
-                ckB[q][1] = aB[1];
+                ck[q * 32] = make_float4(hA.x, hA.y, aB.x, aB.y);
                 release_w();
             }
 
             // ---------------- sweep 2: s descending ----------------
-            float aA[2] = {0.f, 0.f}, hB[2] = {0.f, 0.f};
-            float w0An[2] = {0.f, 0.f}, w2An[2] = {0.f, 0.f};  // A taps of line s+1
+            float2 aA = make_float2(0.f, 0.f), hB = make_float2(0.f, 0.f);
+            Taps WAn = zero_taps;  // A taps of line s+1 (none after s = 63: a_A(64) = 0)
             for (int qq = 0; qq < 8; ++qq) {
                 const int q = 7 - qq;
                 // B taps of line 8q-1 for the a_B recompute (previous chunk in s, not in this ring)
-                float w0Bm[2] = {0.f, 0.f}, w2Bm[2] = {0.f, 0.f};
-                if (q > 0) {
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        const float4 v = __ldg(btab_b + ((size_t)pass * S + 8 * q - 1) * S + p * LPL + t);
-                        w0Bm[p] = v.y;
-                        w2Bm[p] = v.w;
-                    }
-                }
                 float2 dxin[8];  // column pass: the row pass's dx share, rows 8q+e (loaded early)
-                if constexpr (decltype(pass_c)::value == 1) {
+                if constexpr (pass == 1) {
 #pragma unroll
                     for (int e = 0; e < 8; ++e) dxin[e] = ldg64_keep(dxslot + (8 * q + e) * S + 2 * t, keep);
                 }
                 if (!acquire()) { fail(); return false; }
                 uint4 X[2] = {}, LA[2] = {}, LB[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, LBr[8] = {}, Gr[8] = {};
-                if constexpr (decltype(pass_c)::value == 0) {
+                if constexpr (pass == 0) {
                     const unsigned char* st = ringp + stage * STAGE + t * 16;
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
@@ -522,43 +513,47 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
                 release_data();
-                auto xv = [&](int e, int p) {
-                    return pass == 0 ? bfv(X[p], e) : (p ? bf_hi(Xr[e]) : bf_lo(Xr[e]));
-                };
-                auto lav = [&](int e, int p) {
-                    return pass == 0 ? bfv(LA[p], e) : (p ? bf_hi(LAr[e]) : bf_lo(LAr[e]));
-                };
-                auto lbv = [&](int e, int p) {
-                    return pass == 0 ? bfv(LB[p], e) : (p ? bf_hi(LBr[e]) : bf_lo(LBr[e]));
-                };
-                auto gv = [&](int e, int p) { return pass == 0 ? bfv(G[p], e) : (p ? bf_hi(Gr[e]) : bf_lo(Gr[e])); };
+                // B taps of line 8q-1: the last row of the next chunk's weight stage
+                Taps WBm = zero_taps;
+                if (q > 0) {
+                    const int kn = k + 1;
+                    if (!__all_sync(FULL, tma::mbar_wait(wfull0 + 8 * (kn % NWS), (kn / NWS) & 1))) {
+                        ++k;
+                        fail();
+                        return false;
+                    }
+                    const float4 v = lds128f(wring + (kn % NWS) * WCHUNK + 7 * 1024 + 512 + t * 16);
+                    WBm.w0 = make_float2(v.x, v.y);
+                    WBm.w2 = make_float2(v.z, v.w);
+                }
+                auto xv = [&](int e) { return pass == 0 ? make_float2(bfv(X[0], e), bfv(X[1], e)) : bf2(Xr[e]); };
+                auto lav = [&](int e) { return pass == 0 ? make_float2(bfv(LA[0], e), bfv(LA[1], e)) : bf2(LAr[e]); };
+                auto lbv = [&](int e) { return pass == 0 ? make_float2(bfv(LB[0], e), bfv(LB[1], e)) : bf2(LBr[e]); };
+                auto gv = [&](int e) { return pass == 0 ? make_float2(bfv(G[0], e), bfv(G[1], e)) : bf2(Gr[e]); };
 
-                // recompute h_A (with the neighbours of h_A(s-1)) and a_B over the chunk
-                float hs[8][4], aBs[8][2];
+                // recompute h_A and a_B over the chunk from the checkpoints, keeping
+                // h_A(s-1) (the state line s reads) and a_B(s)
+                float2 hAp[8], aBs[8];
                 {
-                    float h[2] = {q > 0 ? ckA[q - 1][0] : 0.f, q > 0 ? ckA[q - 1][1] : 0.f};
-                    float ab[2] = {q > 0 ? ckB[q - 1][0] : 0.f, q > 0 ? ckB[q - 1][1] : 0.f};
-                    float w0Bq[2] = {w0Bm[0], w0Bm[1]}, w2Bq[2] = {w2Bm[0], w2Bm[1]};
+                    const float4 c = q > 0 ? ck[(q - 1) * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
+                    float2 h = make_float2(c.x, c.y), ab = make_float2(c.z, c.w);
+                    Taps WBq = WBm;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        float w0A[2], w0B[2], w2A[2], w2B[2];
-                        wrow(e, w0A, w0B, w2A, w2B);
-                        float lx[2] = {lav(e, 0) * xv(e, 0), lav(e, 1) * xv(e, 1)};
-                        float g[2] = {gv(e, 0), gv(e, 1)};
-                        fwd_step(h, lx, w0A, w2A, hs[e]);
-                        adj_step(ab, g, w0Bq, w2Bq, t);  // zero state and taps before s = 0
-                        aBs[e][0] = ab[0];
-                        aBs[e][1] = ab[1];
-#pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            w0Bq[p] = w0B[p];
-                            w2Bq[p] = w2B[p];
-                        }
+                        Taps WA, WB;
+                        wrow(e, WA, WB);
+                        float2 hL, hR;
+                        hAp[e] = h;
+                        h = add2(mix(h, WA, t, hL, hR), mul2(lav(e), xv(e)));
+                        ab = adjoint(ab, gv(e), WBq, t);
+                        aBs[e] = ab;
+                        WBq = WB;
                     }
                 }
-                uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns
-                float dxr[2][8];                 // row pass: dx share of rows 2t+p, 8 columns
-                float* const ds = dslot();
+                uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns (bf16 pairs)
+                float2 dlAo, dlBo;               // row pass: dlambda of the odd column of a pair
+                float2 dxr[8];                   // row pass: dx share of rows 2t, 2t+1 at column 8q+e
+                float* ds = dslot();  // upper half chunk (steps 7..4) first
                 if (ds == nullptr) {
                     ++k;  // the data and weight stages of this chunk were consumed
                     fail();
@@ -568,76 +563,60 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int ee = 0; ee < 8; ++ee) {
                     const int e = 7 - ee;
                     const int s = 8 * q + e;
-                    float w0A[2], w0B[2], w2A[2], w2B[2];
-                    wrow(e, w0A, w0B, w2A, w2B);
-                    float g[2] = {gv(e, 0), gv(e, 1)};
-                    // adjoint of A at s from s+1 (taps of line s+1; zero state and taps at s = 63)
-                    adj_step(aA, g, w0An, w2An, t);
-                    // forward of B at s from s+1 (taps of B's line at s)
-                    float lxb[2] = {lbv(e, 0) * xv(e, 0), lbv(e, 1) * xv(e, 1)};
-                    float nbB[4];
-                    fwd_step(hB, lxb, w0B, w2B, nbB);
-                    // tap values: A's line s reads h_A(s-1) (neighbours hs[e]) with taps
-                    // w0A, w2A; B's line at s reads h_B(s+1) (nbB) with w0B, w2B.  On the
-                    // first line of each direction the read state is zero, so they are 0.
-                    {
-                        float v[4][2];
-#pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            {
-                                const float hl = hs[e][p], hc = hs[e][p + 1], hr = hs[e][p + 2];
-                                const float w0 = w0A[p], w2 = w2A[p], w1 = 1.f - w0 - w2;
-                                v[0][p] = aA[p] * (w1 * (hl - hc) + w2 * (hl - hr));
-                                v[1][p] = aA[p] * (w0 * (hr - hl) + w1 * (hr - hc));
-                            }
-                            {
-                                const float hl = nbB[p], hc = nbB[p + 1], hr = nbB[p + 2];
-                                const float w0 = w0B[p], w2 = w2B[p], w1 = 1.f - w0 - w2;
-                                v[2][p] = aBs[e][p] * (w1 * (hl - hc) + w2 * (hl - hr));
-                                v[3][p] = aBs[e][p] * (w0 * (hr - hl) + w1 * (hr - hc));
-                            }
+                    if (ee == 4) {
+                        dpublish();
+                        ds = dslot();
+                        if (ds == nullptr) {
+                            ++k;
+                            fail();
+                            return false;
                         }
-#pragma unroll
-                        for (int r = 0; r < 4; ++r)
-                            *reinterpret_cast<float2*>(ds + (e * 4 + r) * S + 2 * t) = make_float2(v[r][0], v[r][1]);
+                    }
+                    Taps WA, WB;
+                    wrow(e, WA, WB);
+                    const float2 x = xv(e), lamA = lav(e), lamB = lbv(e), ab = aBs[e];
+                    // adjoint of A at s from s+1 (taps of line s+1)
+                    aA = adjoint(aA, gv(e), WAn, t);
+                    WAn = WA;
+                    // forward of B at s from s+1 (taps of B's line at s) and B's tap values
+                    float2 hL, hR;
+                    const float2 m = mix(hB, WB, t, hL, hR);
+                    hB = add2(m, mul2(lamB, x));
+                    // tap values E = a (h_k - m): A's line s with a_A(s), B's with a_B(s).
+                    // On each direction's first line the state read is zero and so are they.
+                    float* const d = ds + (e & 3) * 4 * S + 2 * t;
+                    *reinterpret_cast<float2*>(d + 2 * S) = mul2(ab, sub2(hL, m));
+                    *reinterpret_cast<float2*>(d + 3 * S) = mul2(ab, sub2(hR, m));
+                    {
+                        float2 aL, aR;
+                        const float2 mA = mix(hAp[e], WA, t, aL, aR);
+                        *reinterpret_cast<float2*>(d + 0 * S) = mul2(aA, sub2(aL, mA));
+                        *reinterpret_cast<float2*>(d + 1 * S) = mul2(aA, sub2(aR, mA));
                     }
                     // dlambda of both directions and this pass's share of dx
-                    float dla[2], dlb[2], dxs[2];
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        const float xx = xv(e, p);
-                        dla[p] = xx * aA[p];
-                        dlb[p] = xx * aBs[e][p];
-                        dxs[p] = lav(e, p) * aA[p] + lbv(e, p) * aBs[e][p];
-                    }
-                    if constexpr (decltype(pass_c)::value == 0) {
-                        // rows 2t+p, column s: pack 8 columns of each row, store at chunk end
-#pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            if (e & 1) {
-                                dlA[p][e >> 1] = pack_bf2(0.f, dla[p]);
-                                dlB[p][e >> 1] = pack_bf2(0.f, dlb[p]);
-                            } else {
-                                dlA[p][e >> 1] = (dlA[p][e >> 1] & 0xffff0000u) | (pack_bf2(dla[p], 0.f) & 0xffffu);
-                                dlB[p][e >> 1] = (dlB[p][e >> 1] & 0xffff0000u) | (pack_bf2(dlb[p], 0.f) & 0xffffu);
-                            }
+                    const float2 dla = mul2(x, aA), dlb = mul2(x, ab);
+                    const float2 dxs = fma2(lamB, ab, mul2(lamA, aA));
+                    if constexpr (pass == 0) {
+                        // rows 2t, 2t+1, column s: bf16 pairs of columns (even, odd), odd first
+                        if (e & 1) {
+                            dlAo = dla;
+                            dlBo = dlb;
+                        } else {
+                            dlA[0][e >> 1] = pack_bf2(dla.x, dlAo.x);
+                            dlA[1][e >> 1] = pack_bf2(dla.y, dlAo.y);
+                            dlB[0][e >> 1] = pack_bf2(dlb.x, dlBo.x);
+                            dlB[1][e >> 1] = pack_bf2(dlb.y, dlBo.y);
                         }
-                        dxr[0][e] = dxs[0];
-                        dxr[1][e] = dxs[1];
+                        dxr[e] = dxs;
                     } else {
                         // row s, columns 2t, 2t+1: complete dx, dlambda of both directions
-                        stg_cs32(a.dx + (size_t)plane * S * S + s * S + 2 * t,
-                                 pack_bf2(dxin[e].x + dxs[0], dxin[e].y + dxs[1]));
-                        stg_cs32(dlamA + s * S + 2 * t, pack_bf2(dla[0], dla[1]));
-                        stg_cs32(dlamB + s * S + 2 * t, pack_bf2(dlb[0], dlb[1]));
-                    }
-#pragma unroll
-                    for (int p = 0; p < 2; ++p) {
-                        w0An[p] = w0A[p];
-                        w2An[p] = w2A[p];
+                        const float2 dxt = add2(dxin[e], dxs);
+                        stg_cs32(a.dx + (size_t)plane * S * S + s * S + 2 * t, pack_bf2(dxt.x, dxt.y));
+                        stg_cs32(dlamA + s * S + 2 * t, pack_bf2(dla.x, dla.y));
+                        stg_cs32(dlamB + s * S + 2 * t, pack_bf2(dlb.x, dlb.y));
                     }
                 }
-                if constexpr (decltype(pass_c)::value == 0) {
+                if constexpr (pass == 0) {
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
                         const int r = 2 * t + p;
@@ -646,11 +625,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                         __stcs(reinterpret_cast<uint4*>(dlamA + r * S + 8 * q), va);
                         __stcs(reinterpret_cast<uint4*>(dlamB + r * S + 8 * q), vb);
                         float* dxo = dxslot + r * S + 8 * q;
-                        stg128_keep(dxo, make_float4(dxr[p][0], dxr[p][1], dxr[p][2], dxr[p][3]), keep);
-                        stg128_keep(dxo + 4, make_float4(dxr[p][4], dxr[p][5], dxr[p][6], dxr[p][7]), keep);
+                        const float c[8] = {p ? dxr[0].y : dxr[0].x, p ? dxr[1].y : dxr[1].x,
+                                            p ? dxr[2].y : dxr[2].x, p ? dxr[3].y : dxr[3].x,
+                                            p ? dxr[4].y : dxr[4].x, p ? dxr[5].y : dxr[5].x,
+                                            p ? dxr[6].y : dxr[6].x, p ? dxr[7].y : dxr[7].x};
+                        stg128_keep(dxo, make_float4(c[0], c[1], c[2], c[3]), keep);
+                        stg128_keep(dxo + 4, make_float4(c[4], c[5], c[6], c[7]), keep);
                     }
-                }
-                if constexpr (decltype(pass_c)::value == 1) {
+                } else {
                     // every lane has used its loads of rows 8q..8q+7 of the dx plane:
                     // the rows are dead, drop their 16 lines of 128 bytes from L2
                     __syncwarp();
@@ -739,7 +721,7 @@ gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     a.B = p.g.B;
     a.C = p.g.C;
     a.groups = (int)(p.planes / 8);
-    const int nt = p.g.B * 2 * S * S;
+    const int nt = p.g.B * 2 * S * LPL;
     c64b_table_kernel<__nv_bfloat16><<<(nt + 255) / 256, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.btab), a.dsum, a.err, p.g.B);
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
