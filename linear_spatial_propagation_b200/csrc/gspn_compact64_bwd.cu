@@ -65,7 +65,6 @@ constexpr int NCW = 8;          // consumer warps (one plane each)
 constexpr int NST = 2;          // data ring stages per warp
 constexpr int NWS = 4;          // weight ring stages per CTA
 constexpr int BOX = 1024;       // one plane of one tensor per chunk
-constexpr int SLICE = 512;
 constexpr int STAGE = 4 * BOX;  // x, lambda_A, lambda_B, dout
 constexpr int WCHUNK = 8 * S * 16;
 constexpr int DSLOT = 4 * 4 * S * 4;      // one warp's tap values of half a chunk: [step][dir*2 + value][position j]
@@ -74,7 +73,8 @@ constexpr int WRING = NCW * WARP_BYTES;
 constexpr int DSTG = WRING + NWS * WCHUNK;    // 2 sets x NCW slots
 constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // 2 reduced half chunks: [dir*2 + value][step][position j]
 constexpr int CKO = DOUT + 2 * DSLOT;          // per warp: sweep-1 checkpoints (h_A, a_B) of the 8 chunks
-constexpr int BARS = CKO + NCW * 8 * 32 * 16;
+constexpr int DLS = CKO + NCW * 8 * 32 * 16;  // per warp: row-pass dlambda of a chunk, A then B, [row][8 columns]
+constexpr int BARS = DLS + NCW * 2 * BOX;
 constexpr int NBAR = NCW * NST + 2 * NWS + 4;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR;
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     c64b_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
                 const __grid_constant__ CUtensorMap tm_gc, const __grid_constant__ CUtensorMap tm_xr,
                 const __grid_constant__ CUtensorMap tm_lr, const __grid_constant__ CUtensorMap tm_gr,
-                const C64BArgs a) {
+                const __grid_constant__ CUtensorMap tm_dl, const C64BArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* const smem = smem_raw + ((1024u - (tma::smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = tma::smem_u32(smem);
@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     unsigned char* const ringp = smem + warp * WARP_BYTES;
     float* const dxslot = a.dxh + ((size_t)blockIdx.x * NCW + warp) * S * S;
     float4* const ck = reinterpret_cast<float4*>(smem + CKO) + warp * 8 * 32 + t;  // [chunk][lane]
+    unsigned char* const dlst = smem + DLS + warp * 2 * BOX;
+    const uint32_t dlsa = sbase + DLS + warp * 2 * BOX;
     const uint64_t keep = l2_evict_last_policy();
     const unsigned char* const wring = smem + WRING;
     const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
@@ -340,10 +342,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma::prefetch_map(&tm_xr);
         tma::prefetch_map(&tm_lr);
         tma::prefetch_map(&tm_gr);
+        tma::prefetch_map(&tm_dl);
     }
 
     // Data of chunk kk (lane 0): x, lambda_A, lambda_B (sweep 2 only), dout of
-    // the chunk's 8 columns (row pass) or rows (column pass).
+    // the chunk's 8 columns (row pass: [64 rows][8 columns]) or rows (column
+    // pass: [8 rows][64 columns]).
     auto issue = [&](int kk) {
         if (kk >= nchunks) return;
         const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
@@ -355,12 +359,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma::mbar_expect_tx(bar, sweep ? 4 * BOX : 3 * BOX);
         const int la = pass ? 0 : 2, lb = pass ? 1 : 3;  // lambda slots of A and B
         if (pass == 0) {
-            for (int r = 0; r < 2; ++r) {
-                tma::load_3d(dst + 0 * BOX + r * SLICE, &tm_xc, 8 * q, r, plane, bar);
-                tma::load_3d(dst + 1 * BOX + r * SLICE, &tm_lc, 8 * q, r, la * BC + plane, bar);
-                if (sweep) tma::load_3d(dst + 2 * BOX + r * SLICE, &tm_lc, 8 * q, r, lb * BC + plane, bar);
-                tma::load_3d(dst + 3 * BOX + r * SLICE, &tm_gc, 8 * q, r, plane, bar);
-            }
+            tma::load_3d(dst + 0 * BOX, &tm_xc, 8 * q, 0, plane, bar);
+            tma::load_3d(dst + 1 * BOX, &tm_lc, 8 * q, 0, la * BC + plane, bar);
+            if (sweep) tma::load_3d(dst + 2 * BOX, &tm_lc, 8 * q, 0, lb * BC + plane, bar);
+            tma::load_3d(dst + 3 * BOX, &tm_gc, 8 * q, 0, plane, bar);
         } else {
             tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
             tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, la * BC + plane, bar);
@@ -439,12 +441,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint4 X[2] = {}, LA[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, Gr[8] = {};
                 if constexpr (pass == 0) {
-                    const unsigned char* st = ringp + stage * STAGE + t * 16;
+                    const unsigned char* st = ringp + stage * STAGE + t * 32;  // rows 2t, 2t+1
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        X[p] = lds128(st + 0 * BOX + p * SLICE);
-                        LA[p] = lds128(st + 1 * BOX + p * SLICE);
-                        G[p] = lds128(st + 3 * BOX + p * SLICE);
+                        X[p] = lds128(st + 0 * BOX + p * 16);
+                        LA[p] = lds128(st + 1 * BOX + p * 16);
+                        G[p] = lds128(st + 3 * BOX + p * 16);
                     }
                 } else {
                     const unsigned char* st = ringp + stage * STAGE + t * 4;
@@ -485,22 +487,26 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int qq = 0; qq < 8; ++qq) {
                 const int q = 7 - qq;
                 // B taps of line 8q-1 for the a_B recompute (previous chunk in s, not in this ring)
-                float2 dxin[8];  // column pass: the row pass's dx share, rows 8q+e (loaded early)
+                // column pass: the row pass's dx share of columns 2t, 2t+1, rows 8q..8q+7
+                // (loaded early; the scratch plane is column-major)
+                float4 dxc[2][2];
                 if constexpr (pass == 1) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) dxin[e] = ldg64_keep(dxslot + (8 * q + e) * S + 2 * t, keep);
+                    for (int p = 0; p < 2; ++p)
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) dxc[p][h] = ldg128_keep(dxslot + (2 * t + p) * S + 8 * q + 4 * h, keep);
                 }
                 if (!acquire()) { fail(); return false; }
                 uint4 X[2] = {}, LA[2] = {}, LB[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, LBr[8] = {}, Gr[8] = {};
                 if constexpr (pass == 0) {
-                    const unsigned char* st = ringp + stage * STAGE + t * 16;
+                    const unsigned char* st = ringp + stage * STAGE + t * 32;  // rows 2t, 2t+1
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        X[p] = lds128(st + 0 * BOX + p * SLICE);
-                        LA[p] = lds128(st + 1 * BOX + p * SLICE);
-                        LB[p] = lds128(st + 2 * BOX + p * SLICE);
-                        G[p] = lds128(st + 3 * BOX + p * SLICE);
+                        X[p] = lds128(st + 0 * BOX + p * 16);
+                        LA[p] = lds128(st + 1 * BOX + p * 16);
+                        LB[p] = lds128(st + 2 * BOX + p * 16);
+                        G[p] = lds128(st + 3 * BOX + p * 16);
                     }
                 } else {
                     const unsigned char* st = ringp + stage * STAGE + t * 4;
@@ -552,7 +558,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns (bf16 pairs)
                 float2 dlAo, dlBo;               // row pass: dlambda of the odd column of a pair
-                float2 dxr[8];                   // row pass: dx share of rows 2t, 2t+1 at column 8q+e
                 float* ds = dslot();  // upper half chunk (steps 7..4) first
                 if (ds == nullptr) {
                     ++k;  // the data and weight stages of this chunk were consumed
@@ -607,36 +612,46 @@ __global__ void __launch_bounds__(THREADS, 1)
                             dlB[0][e >> 1] = pack_bf2(dlb.x, dlBo.x);
                             dlB[1][e >> 1] = pack_bf2(dlb.y, dlBo.y);
                         }
-                        dxr[e] = dxs;
+                        // dx share of column s, rows 2t, 2t+1 into the column-major scratch
+                        stg64_keep(dxslot + s * S + 2 * t, dxs, keep);
                     } else {
                         // row s, columns 2t, 2t+1: complete dx, dlambda of both directions
-                        const float2 dxt = add2(dxin[e], dxs);
+                        const float4& c0 = dxc[0][e >> 2];
+                        const float4& c1 = dxc[1][e >> 2];
+                        const int i = e & 3;
+                        const float2 prev = make_float2(i == 0 ? c0.x : i == 1 ? c0.y : i == 2 ? c0.z : c0.w,
+                                                        i == 0 ? c1.x : i == 1 ? c1.y : i == 2 ? c1.z : c1.w);
+                        const float2 dxt = add2(prev, dxs);
                         stg_cs32(a.dx + (size_t)plane * S * S + s * S + 2 * t, pack_bf2(dxt.x, dxt.y));
                         stg_cs32(dlamA + s * S + 2 * t, pack_bf2(dla.x, dla.y));
                         stg_cs32(dlamB + s * S + 2 * t, pack_bf2(dlb.x, dlb.y));
                     }
                 }
                 if constexpr (pass == 0) {
+                    // dlambda of the chunk's 8 columns: staged [row][8 columns] and
+                    // written by two tiled bulk stores
+                    if (t == 0) tma::bulk_wait_read();  // the previous chunk's stores have read the stage
+                    __syncwarp();
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        const int r = 2 * t + p;
-                        uint4 va = make_uint4(dlA[p][0], dlA[p][1], dlA[p][2], dlA[p][3]);
-                        uint4 vb = make_uint4(dlB[p][0], dlB[p][1], dlB[p][2], dlB[p][3]);
-                        __stcs(reinterpret_cast<uint4*>(dlamA + r * S + 8 * q), va);
-                        __stcs(reinterpret_cast<uint4*>(dlamB + r * S + 8 * q), vb);
-                        float* dxo = dxslot + r * S + 8 * q;
-                        const float c[8] = {p ? dxr[0].y : dxr[0].x, p ? dxr[1].y : dxr[1].x,
-                                            p ? dxr[2].y : dxr[2].x, p ? dxr[3].y : dxr[3].x,
-                                            p ? dxr[4].y : dxr[4].x, p ? dxr[5].y : dxr[5].x,
-                                            p ? dxr[6].y : dxr[6].x, p ? dxr[7].y : dxr[7].x};
-                        stg128_keep(dxo, make_float4(c[0], c[1], c[2], c[3]), keep);
-                        stg128_keep(dxo + 4, make_float4(c[4], c[5], c[6], c[7]), keep);
+                        *reinterpret_cast<uint4*>(dlst + t * 32 + p * 16) =
+                            make_uint4(dlA[p][0], dlA[p][1], dlA[p][2], dlA[p][3]);
+                        *reinterpret_cast<uint4*>(dlst + BOX + t * 32 + p * 16) =
+                            make_uint4(dlB[p][0], dlB[p][1], dlB[p][2], dlB[p][3]);
                     }
-                } else {
-                    // every lane has used its loads of rows 8q..8q+7 of the dx plane:
-                    // the rows are dead, drop their 16 lines of 128 bytes from L2
+                    tma::fence_proxy_async();
                     __syncwarp();
-                    if (t < 16) l2_discard128(dxslot + (8 * q + (t >> 1)) * S + (t & 1) * 32);
+                    if (t == 0) {
+                        tma::store_3d(&tm_dl, dlsa, 8 * q, 0, la * BC + plane);
+                        tma::store_3d(&tm_dl, dlsa + BOX, 8 * q, 0, lb * BC + plane);
+                        tma::bulk_commit();
+                    }
+                } else if (q == 4 || q == 0) {
+                    // every lane has used its loads of rows 32..63 (q = 4) or 0..31 (q = 0)
+                    // of the dx plane: drop those dead 128-byte lines of columns 2t, 2t+1
+                    __syncwarp();
+                    l2_discard128(dxslot + (2 * t) * S + 8 * q);
+                    l2_discard128(dxslot + (2 * t + 1) * S + 8 * q);
                 }
                 dpublish();
                 release_w();
@@ -644,8 +659,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             __syncwarp();
             return true;
         };
-        if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) return;
+        if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) break;
     }
+    if (t == 0) tma::bulk_wait_all();  // the dlambda stores have read shared memory
 }
 
 // ---- host side ----------------------------------------------------------------------
@@ -668,13 +684,13 @@ EncodeTiledFn encode_fn_b() {
     return fn;
 }
 
-bool make_map_b(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r, uint32_t row_step) {
+bool make_map_b(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r) {
     EncodeTiledFn fn = encode_fn_b();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, S * S * 2};
     const cuuint32_t box[3] = {box_c, box_r, 1};
-    const cuuint32_t es[3] = {1, row_step, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
     return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -704,11 +720,11 @@ size_t c64_bwd_workspace(const Problem& p, const DeviceInfo& dev) {
 
 gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
                     const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s) {
-    CUtensorMap xc, lc, gc, xr, lr, gr;
+    CUtensorMap xc, lc, gc, xr, lr, gr, dl;
     const uint64_t BC = (uint64_t)p.planes;
-    if (!make_map_b(&xc, x, BC, 8, 64, 2) || !make_map_b(&lc, lam, 4 * BC, 8, 64, 2) ||
-        !make_map_b(&gc, dout, BC, 8, 64, 2) || !make_map_b(&xr, x, BC, 64, 8, 1) ||
-        !make_map_b(&lr, lam, 4 * BC, 64, 8, 1) || !make_map_b(&gr, dout, BC, 64, 8, 1))
+    if (!make_map_b(&xc, x, BC, 8, 64) || !make_map_b(&lc, lam, 4 * BC, 8, 64) || !make_map_b(&gc, dout, BC, 8, 64) ||
+        !make_map_b(&xr, x, BC, 64, 8) || !make_map_b(&lr, lam, 4 * BC, 64, 8) || !make_map_b(&gr, dout, BC, 64, 8) ||
+        !make_map_b(&dl, dlam, 4 * BC, 8, 64))
         return GSPN_ERR_UNSUPPORTED;
     char* w = static_cast<char*>(ws);
     C64BArgs a;
@@ -728,7 +744,7 @@ gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     cudaError_t e = ensure_smem_attr((const void*)c64b_kernel, SMEM_BYTES, 10);
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
     const int grid = bwd_grid(p, dev);
-    c64b_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, gc, xr, lr, gr, a);
+    c64b_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, gc, xr, lr, gr, dl, a);
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
     const int nl = 4 * p.g.B * S * S;
     c64b_dlogits_kernel<__nv_bfloat16><<<(nl + 255) / 256, 256, 0, s>>>(
