@@ -76,9 +76,10 @@ constexpr int WCHUNK = 8 * S * 16;  // tap weights of 8 scan steps (8 table rows
 constexpr int WARP_BYTES = NST * STAGE + HACC;
 constexpr int WRING = NCW * WARP_BYTES;              // offset of the weight ring
 constexpr int BARS = WRING + NWS * WCHUNK;           // offset of the barriers
-constexpr int SMEM_BYTES = 1024 + BARS + 8 * (NCW * NST + 2 * NWS);
+constexpr int SMEM_BYTES = 1024 + BARS + 8 * (2 * NCW * NST + 2 * NWS);
 constexpr int CHUNKS_PER_GROUP = 16;  // 8 column chunks + 8 row chunks
-constexpr int THREADS = (NCW + 1) * 32;
+constexpr int NPW = NCW / 2;  // producer warps, each feeding two consumer warps
+constexpr int THREADS = (NCW + NPW) * 32;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(WARP_BYTES % 1024 == 0 && WCHUNK % 1024 == 0, "TMA destinations stay 1024-byte aligned");
 
@@ -146,12 +147,17 @@ __global__ void __launch_bounds__(THREADS, 1)
     unsigned char* const smem = smem_raw + ((1024u - (tma::smem_u32(smem_raw) & 1023u)) & 1023u);
     const uint32_t sbase = tma::smem_u32(smem);
     const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
-    const uint32_t wfull0 = sbase + BARS + 8 * NCW * NST;  // NWS "weights landed" barriers
+    const uint32_t xfull0 = sbase + BARS;                  // [warp][stage] "data landed"
+    const uint32_t xempty0 = xfull0 + 8 * NCW * NST;       // [warp][stage] "data read"
+    const uint32_t wfull0 = xempty0 + 8 * NCW * NST;       // NWS "weights landed" barriers
     const uint32_t wempty0 = wfull0 + 8 * NWS;             // NWS "weights consumed" barriers
     if ((int)blockIdx.x >= a.groups) return;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < NCW * NST; ++s) tma::mbar_init(sbase + BARS + 8 * s, 1);
+        for (int s = 0; s < NCW * NST; ++s) {
+            tma::mbar_init(xfull0 + 8 * s, 1);
+            tma::mbar_init(xempty0 + 8 * s, 32);
+        }
         for (int s = 0; s < NWS; ++s) {
             tma::mbar_init(wfull0 + 8 * s, 1);
             tma::mbar_init(wempty0 + 8 * s, NCW);
@@ -163,73 +169,78 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int ngroups_here = (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const int nchunks = ngroups_here * CHUNKS_PER_GROUP;
 
-    // ---------------- producer warp: tap-weight chunks of this CTA's groups ----------------
-    if (warp == NCW) {
+    const int BC = a.B * a.C;
+
+    // ---------------- producer warps ----------------
+    // Lane 0 of producer warp p streams the x / lambda chunks of consumer warps
+    // 2p and 2p+1: chunk kk of warp w (plane 8*group + w of group blockIdx.x +
+    // (kk/16)*gridDim.x; chunk kk%16: 0..7 column chunks, 8..15 row chunks;
+    // lambda plane (slot, b, c) at slot*B*C + plane) goes to stage kk % NST of the
+    // warp's ring once the warp has read what the stage held.  Producer 0 also
+    // streams the tap-weight chunks, each one into the ring shared by the CTA.
+    if (warp >= NCW) {
         if (t == 0) {
-            for (int kc = 0; kc < nchunks; ++kc) {
-                const int ws = kc % NWS;
-                if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1, 200)) {
-                    atomicExch(a.err, 1);
-                    break;
-                }
-                const int group = (int)blockIdx.x + (kc / CHUNKS_PER_GROUP) * (int)gridDim.x;
-                const int b = (8 * group) / a.C;
-                const float4* src = a.wtab + ((size_t)b * 2 * S + 8 * (kc % CHUNKS_PER_GROUP)) * S;
-                tma::mbar_expect_tx(wfull0 + 8 * ws, WCHUNK);
-                tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
+            const int pw = warp - NCW;
+            if (pw == 0) {
+                tma::prefetch_map(&tm_xc);
+                tma::prefetch_map(&tm_lc);
+                tma::prefetch_map(&tm_xr);
+                tma::prefetch_map(&tm_lr);
             }
+            bool ok = true;
+            for (int kk = 0; ok && kk < nchunks; ++kk) {
+                const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
+                const int local = kk % CHUNKS_PER_GROUP, st = kk % NST;
+                if (pw == 0) {
+                    const int ws = kk % NWS;
+                    if (!tma::mbar_wait(wempty0 + 8 * ws, ((kk / NWS) & 1) ^ 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const int b = (8 * group) / a.C;
+                    const float4* src = a.wtab + ((size_t)b * 2 * S + 8 * local) * S;
+                    tma::mbar_expect_tx(wfull0 + 8 * ws, WCHUNK);
+                    tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
+                }
+                for (int w = 2 * pw; w < 2 * pw + 2; ++w) {
+                    if (!tma::mbar_wait(xempty0 + 8 * (w * NST + st), ((kk / NST) & 1) ^ 1)) {
+                        ok = false;
+                        break;
+                    }
+                    const int plane = 8 * group + w;
+                    const uint32_t dst = sbase + w * WARP_BYTES + st * STAGE, bar = xfull0 + 8 * (w * NST + st);
+                    tma::mbar_expect_tx(bar, STAGE);
+                    if (local < 8) {
+                        const int q = local;
+                        // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at
+                        // 8(7-q)..; rows r_lo, r_lo + 2, ... go to slice r_lo
+                        for (int r = 0; r < 2; ++r) {
+                            tma::load_3d(dst + 0 * BOX + r * SLICE, &tm_xc, 8 * q, r, plane, bar);
+                            tma::load_3d(dst + 1 * BOX + r * SLICE, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
+                            tma::load_3d(dst + 2 * BOX + r * SLICE, &tm_xc, 8 * (7 - q), r, plane, bar);
+                            tma::load_3d(dst + 3 * BOX + r * SLICE, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
+                        }
+                    } else {
+                        const int q = local - 8;
+                        // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 56-8q..
+                        tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
+                        tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, 0 * BC + plane, bar);
+                        tma::load_3d(dst + 2 * BOX, &tm_xr, 0, 56 - 8 * q, plane, bar);
+                        tma::load_3d(dst + 3 * BOX, &tm_lr, 0, 56 - 8 * q, 1 * BC + plane, bar);
+                    }
+                }
+            }
+            if (!ok) atomicExch(a.err, 1);
         }
         return;
     }
 
     // ---------------- consumer warps: one plane each ----------------
-    const uint32_t ring = sbase + warp * WARP_BYTES;        // shared-window address (TMA)
-    unsigned char* const ringp = smem + warp * WARP_BYTES;  // same bytes, for loads
+    unsigned char* const ringp = smem + warp * WARP_BYTES;
     unsigned char* const haccp = ringp + NST * STAGE;
     const unsigned char* const wring = smem + WRING;
-    const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
+    const uint32_t bar0 = xfull0 + 8 * NST * warp, ebar0 = xempty0 + 8 * NST * warp;
     const int segmask = a.seg - 1;  // seg divides 64, so it is a power of two
-    const int BC = a.B * a.C;
-
-    if (t == 0) {
-        tma::prefetch_map(&tm_xc);
-        tma::prefetch_map(&tm_lc);
-        tma::prefetch_map(&tm_xr);
-        tma::prefetch_map(&tm_lr);
-    }
-
-    // Issue chunk kk of this warp's sequence (lane 0 only): plane 8*group + warp of
-    // group blockIdx.x + (kk/16)*gridDim.x, chunk kk%16 (0..7: column chunks,
-    // 8..15: row chunks).  lambda plane (slot, b, c) is slot*B*C + plane.
-    auto issue = [&](int kk) {
-        if (kk >= nchunks) return;
-        const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
-        const int plane = 8 * group + warp;
-        const int local = kk % CHUNKS_PER_GROUP, st = kk % NST;
-        const uint32_t dst = ring + st * STAGE, bar = bar0 + 8 * st;
-        tma::mbar_expect_tx(bar, STAGE);
-        if (local < 8) {
-            const int q = local;
-            // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at
-            // 8(7-q)..; rows r_lo, r_lo + 2, ... go to slice r_lo
-            for (int r = 0; r < 2; ++r) {
-                tma::load_3d(dst + 0 * BOX + r * SLICE, &tm_xc, 8 * q, r, plane, bar);
-                tma::load_3d(dst + 1 * BOX + r * SLICE, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
-                tma::load_3d(dst + 2 * BOX + r * SLICE, &tm_xc, 8 * (7 - q), r, plane, bar);
-                tma::load_3d(dst + 3 * BOX + r * SLICE, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
-            }
-        } else {
-            const int q = local - 8;
-            // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 56-8q..
-            tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
-            tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, 0 * BC + plane, bar);
-            tma::load_3d(dst + 2 * BOX, &tm_xr, 0, 56 - 8 * q, plane, bar);
-            tma::load_3d(dst + 3 * BOX, &tm_lr, 0, 56 - 8 * q, 1 * BC + plane, bar);
-        }
-    };
-
-    if (t == 0)
-        for (int kk = 0; kk < NST; ++kk) issue(kk);
 
     int k = 0;            // next chunk to consume (same sequence for data and weights)
     int stage = 0;        // k % NST
@@ -267,10 +278,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
         return __all_sync(FULL, ok);
     };
+    // the stage is in registers: hand it back to its producer
     auto release = [&]() {
-        tma::fence_proxy_async();
-        __syncwarp();
-        if (t == 0) issue(k + NST);
+        tma::mbar_arrive(ebar0 + 8 * stage);
         phase ^= 1u << stage;
         ++k;
         stage = stage == NST - 1 ? 0 : stage + 1;
