@@ -215,6 +215,23 @@ def run_reference(args, w):
     return 0
 
 
+def max_over_ranks(dist, v: float, device) -> float:
+    """The maximum of v over the ranks of the process group (v itself when
+    there is none); every rank calls it at the same point."""
+    if dist is None:
+        return v
+    import torch
+
+    t = torch.tensor([v], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(bytes_per_rank: int, n_ranks: int, ms: float) -> float:
+    """Whole-job GB/s: the bytes every rank moved over the slowest rank's time."""
+    return bytes_per_rank * n_ranks / (ms * 1e-3) / 1e9
+
+
 def config_of(w, n, passes="both"):
     return {"workload": w.name, "B": w.B, "C": w.C, "H": w.H, "W": w.W,
             "directions": "+".join(n_ for b, n_ in ((1, "T2B"), (2, "B2T"), (4, "L2R"), (8, "R2L")) if w.dir_mask & b),
@@ -284,12 +301,8 @@ def run_gpu(args, w):
             dist.barrier()
         torch.cuda.synchronize()
 
-    def max_over_ranks(v):
-        if dist is None:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def rank_max(v):
+        return max_over_ranks(dist, v, dev)
 
     do_f = args.passes in ("both", "fwd")
     do_b = args.passes in ("both", "bwd")
@@ -317,9 +330,9 @@ def run_gpu(args, w):
     e_end.record(stream)
     barrier()
     clk = clocks.stop()
-    total_ms = max_over_ranks(e_start.elapsed_time(e_end))
-    fwd_ms = max_over_ranks(sum(e[0].elapsed_time(e[1]) for e in ev) / K)
-    bwd_ms = max_over_ranks(sum(e[1].elapsed_time(e[2]) for e in ev) / K)
+    total_ms = rank_max(e_start.elapsed_time(e_end))
+    fwd_ms = rank_max(sum(e[0].elapsed_time(e[1]) for e in ev) / K)
+    bwd_ms = rank_max(sum(e[1].elapsed_time(e[2]) for e in ev) / K)
     ms = total_ms / K
 
     # end to end: pinned host inputs -> device -> fwd + bwd -> results back to pinned host
@@ -343,7 +356,7 @@ def run_gpu(args, w):
             hg.copy_(g, non_blocking=True)
     e2[1].record(stream)
     barrier()
-    e2e_ms = max_over_ranks(e2[0].elapsed_time(e2[1]) / E) if E > 0 else None
+    e2e_ms = rank_max(e2[0].elapsed_time(e2[1]) / E) if E > 0 else None
 
     fb, bb = pass_bytes(w)
     if not do_f:
@@ -352,7 +365,7 @@ def run_gpu(args, w):
         bb = 0
     peak, peak_src = measured_peaks()
     n_gpu = world
-    value = (fb + bb) * n_gpu / (ms * 1e-3) / 1e9
+    value = job_gbs(fb + bb, n_gpu, ms)
     pixch = w.B * w.C * w.H * w.W
     fwd_gbs = fb / (fwd_ms * 1e-3) / 1e9 if fb else 0.0
     bwd_gbs = bb / (bwd_ms * 1e-3) / 1e9 if bb else 0.0
@@ -388,7 +401,7 @@ def run_gpu(args, w):
                          "frac": dom_gbs / peak, "peak_source": f"{peak_src} copy bandwidth",
                          "kernel": lsp.gspn_variant_name(desc, 1 if dom == "bwd" else 0),
                          "traffic": ncu_traffic(dom, w)},
-            "e2e": ({"value": (fb + bb) * n_gpu / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "e2e": ({"value": job_gbs(fb + bb, n_gpu, e2e_ms), "unit": "GB/s",
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
                     if e2e_ms else None),
             "gpu_launches": launches,
