@@ -81,6 +81,83 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_kernel(FwdArgs a) 
     for (int q = lane; q < HW; q += 32) store_elt(out, q, acc[q]);
 }
 
+// The same forward for lines of at most 32*P positions, with the loads of line
+// i+1 issued before line i is computed: lane l holds positions l + 32r (r < P)
+// of the line in registers, so each line's global loads overlap the previous
+// line's arithmetic instead of stalling it.
+template <typename T, int P>
+__global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_pipelined_kernel(FwdArgs a) {
+    extern __shared__ float smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C;
+    const int64_t plane = (int64_t)blockIdx.x * a.warps_per_cta + warp;
+    if (plane >= (int64_t)B * C) return;
+    float* wsm = smem + (size_t)warp * (2 * a.lstride + (a.acc_in_smem ? HW : 0));
+    float* acc = a.acc_in_smem ? wsm + 2 * a.lstride : a.acc_ws + plane * HW;
+    const int64_t b = plane / C, c = plane % C, cw = a.g.shared ? 0 : c;
+    const int Cw = a.g.shared ? 1 : C;
+    const T* x = static_cast<const T*>(a.x) + plane * HW;
+
+    for (int slot = 0; slot < a.g.D; ++slot) {
+        const int d = a.g.dirs[slot];
+        const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
+        const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
+        const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+        float* hp = wsm;
+        float* hc = wsm + a.lstride;
+        if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
+        __syncwarp();
+        // inputs of the line in flight: lambda*x and the three raw tap logits
+        float lx[P], g0[P], g1[P], g2[P];
+        auto fetch = [&](int i, float (&flx)[P], float (&f0)[P], float (&f1)[P], float (&f2)[P]) {
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                const int j = lane + 32 * r;
+                const int pp = j < N ? pix(d, H, W, i, j) : 0;  // in bounds for idle lanes
+                flx[r] = load_elt(lam, pp) * load_elt(x, pp);
+                f0[r] = load_elt(lg, pp);
+                f1[r] = load_elt(lg, HW + pp);
+                f2[r] = load_elt(lg, 2 * HW + pp);
+            }
+        };
+        fetch(0, lx, g0, g1, g2);
+        for (int i = 0; i < L; ++i) {
+            float nlx[P], n0[P], n1[P], n2[P];
+            if (i + 1 < L) fetch(i + 1, nlx, n0, n1, n2);
+            const bool carry = (i % seg) != 0;
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                const int j = lane + 32 * r;
+                if (j < N) {
+                    float v = lx[r];
+                    if (carry) {
+                        const float s0 = j > 0 ? sigmoidf(g0[r]) : 0.f;
+                        const float s1 = sigmoidf(g1[r]);
+                        const float s2 = j < N - 1 ? sigmoidf(g2[r]) : 0.f;
+                        const float num = s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2];
+                        v += num / (s0 + s1 + s2);
+                    }
+                    hc[j + 1] = v;
+                    const int pp = pix(d, H, W, i, j);
+                    acc[pp] = slot == 0 ? v : acc[pp] + v;
+                }
+            }
+            __syncwarp();
+            float* tswap = hp; hp = hc; hc = tswap;
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                lx[r] = nlx[r];
+                g0[r] = n0[r];
+                g1[r] = n1[r];
+                g2[r] = n2[r];
+            }
+        }
+    }
+    __syncwarp();
+    T* out = static_cast<T*>(a.out) + plane * HW;
+    for (int q = lane; q < HW; q += 32) store_elt(out, q, acc[q]);
+}
+
 struct BwdArgs {
     Launch g;
     const void* x;
@@ -282,15 +359,32 @@ gspn_status generic_fwd(const Problem& p, const DeviceInfo& dev, const void* x, 
     a.acc_in_smem = pl.acc_in_smem; a.warps_per_cta = pl.wpc; a.lstride = pl.lstride;
     const int64_t grid = (p.planes + pl.wpc - 1) / pl.wpc;
     if (grid > 0x7fffffff) return GSPN_ERR_UNSUPPORTED;
-    const void* fn = p.d.dtype == GSPN_F32 ? (const void*)generic_fwd_kernel<float>
-                                           : (const void*)generic_fwd_kernel<__nv_bfloat16>;
-    cudaError_t e = ensure_smem_attr(fn, (int)pl.smem, p.d.dtype == GSPN_F32 ? 0 : 1);
+    const int nmax = p.g.H > p.g.W ? p.g.H : p.g.W;
+    const bool f32 = p.d.dtype == GSPN_F32;
+    // lines of up to 128 positions: the pipelined kernel with 1, 2 or 4 positions per lane
+    const void* fn;
+    int slot;
+    if (nmax <= 32) {
+        fn = f32 ? (const void*)generic_fwd_pipelined_kernel<float, 1>
+                 : (const void*)generic_fwd_pipelined_kernel<__nv_bfloat16, 1>;
+        slot = f32 ? 11 : 12;
+    } else if (nmax <= 64) {
+        fn = f32 ? (const void*)generic_fwd_pipelined_kernel<float, 2>
+                 : (const void*)generic_fwd_pipelined_kernel<__nv_bfloat16, 2>;
+        slot = f32 ? 13 : 14;
+    } else if (nmax <= 128) {
+        fn = f32 ? (const void*)generic_fwd_pipelined_kernel<float, 4>
+                 : (const void*)generic_fwd_pipelined_kernel<__nv_bfloat16, 4>;
+        slot = f32 ? 15 : 16;
+    } else {
+        fn = f32 ? (const void*)generic_fwd_kernel<float> : (const void*)generic_fwd_kernel<__nv_bfloat16>;
+        slot = f32 ? 0 : 1;
+    }
+    cudaError_t e = ensure_smem_attr(fn, (int)pl.smem, slot);
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
-    if (p.d.dtype == GSPN_F32)
-        generic_fwd_kernel<float><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
-    else
-        generic_fwd_kernel<__nv_bfloat16><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
-    return cuda_status(cudaGetLastError());
+    void* args[] = {&a};
+    e = cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(pl.wpc * 32), args, pl.smem, s);
+    return cuda_status(e);
 }
 
 namespace {
