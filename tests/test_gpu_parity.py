@@ -91,6 +91,45 @@ def test_backward_workload_full_size():
     check_bwd(w, nthreads=max(1, oracle.max_threads()))
 
 
+def test_headline_backward_full_size_sampled():
+    """The 32x1152x64x64 backward in its bench launch configuration.  dx and
+    dlambda of sampled planes against the oracle plane by plane; dlogits (a
+    sum over all channels) through a second full-size launch whose upstream
+    gradient is zero outside the sampled planes, so that the oracle needs only
+    those planes: planes with a zero gradient contribute nothing to any
+    gradient."""
+    t = gu.torch()
+    w = synth.WORKLOADS["compact_4dir_bf16_b32c1152_64x64"].replace(backward=True)
+    inp = synth.make_inputs(w, with_dout=True)
+    rng = np.random.default_rng(11)
+    picks = {(0, 0), (w.B - 1, w.C - 1), (5, 17)}
+    while len(picks) < 8:
+        picks.add((int(rng.integers(w.B)), int(rng.integers(w.C))))
+    one = w.replace(B=1, C=1)
+    dinp = gu.dev_inputs(w, inp)
+    dx, _, dlam = gu.run_bwd(w, dinp)
+    for b, c in sorted(picks):
+        rdx, _, rdlam = oracle.bwd_workload(one, synth.plane_slice(w, inp, b, c))
+        gu.assert_close(gu.from_dev(dx[b:b + 1, c:c + 1]), rdx, w.dtype, f"dx plane ({b},{c})")
+        gu.assert_close(gu.from_dev(dlam[:, b:b + 1, c:c + 1]), rdlam, w.dtype, f"dlam plane ({b},{c})")
+    # dlogits with the upstream gradient restricted to the sampled planes
+    mask = np.zeros((w.B, w.C, 1, 1), dtype=bool)
+    for b, c in picks:
+        mask[b, c] = True
+    sparse = dict(inp)
+    sparse["dout"] = np.where(mask, inp["dout"], np.zeros_like(inp["dout"]))
+    dinp["dout"] = gu.to_dev(sparse["dout"], w.dtype)
+    dx2, dlg2, _ = gu.run_bwd(w, dinp)
+    want = np.zeros(tuple(dlg2.shape))
+    for b, c in sorted(picks):
+        _, rdlg, _ = oracle.bwd_workload(one, synth.plane_slice(w, sparse, b, c))
+        want[:, b:b + 1] += rdlg
+    gu.assert_close(gu.from_dev(dlg2), want, w.dtype, "dlogits (sampled upstream gradient)")
+    # and a plane outside the sample gets no gradient
+    b, c = next((b, c) for b in range(w.B) for c in range(w.C) if (b, c) not in picks)
+    assert float(t.count_nonzero(dx2[b, c]).item()) == 0.0
+
+
 SHAPES = [
     # B, C, H, W, mask, groups, shared, dtype
     (1, 1, 1, 1, 15, 1, False, "f32"),
