@@ -52,6 +52,7 @@
 #include "gspn_internal.h"
 #include "gspn_lane.cuh"
 #include "gspn_tma.cuh"
+#include "gspn_tmem.cuh"
 
 namespace gspn {
 
@@ -72,11 +73,10 @@ constexpr int WARP_BYTES = NST * STAGE;   // data ring per warp
 constexpr int WRING = NCW * WARP_BYTES;
 constexpr int DSTG = WRING + NWS * WCHUNK;    // 2 sets x NCW slots
 constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // 2 reduced half chunks: [dir*2 + value][step][position j]
-constexpr int CKO = DOUT + 2 * DSLOT;          // per warp: sweep-1 checkpoints (h_A, a_B) of the 8 chunks
-constexpr int DLS = CKO + NCW * 8 * 32 * 16;  // per warp: row-pass dlambda of a chunk, A then B, [row][8 columns]
+constexpr int DLS = DOUT + 2 * DSLOT;          // per warp: row-pass dlambda of a chunk, A then B, [row][8 columns]
 constexpr int BARS = DLS + NCW * 2 * BOX;
-constexpr int NBAR = NCW * NST + 2 * NWS + 4;
-constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR;
+constexpr int NBAR = NCW * NST + 2 * NWS + 4 + 1;
+constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
 constexpr int THREADS = (NCW + 2) * 32;  // compute warps, tap-table producer, tap-value reducer
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
@@ -220,6 +220,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t wempty0 = wfull0 + 8 * NWS;
     const uint32_t dfull0 = wempty0 + 8 * NWS;  // [set]: the compute warps' slots of a chunk are written
     const uint32_t dempty0 = dfull0 + 16;       // [set]: the reducer has read the set
+    const uint32_t done0 = dempty0 + 16;        // every compute warp is done with the tensor memory
+    uint32_t* const tslot = reinterpret_cast<uint32_t*>(smem + BARS + 8 * NBAR);
     if ((int)blockIdx.x >= a.groups) return;
 
     if (threadIdx.x == 0) {
@@ -232,9 +234,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_init(dfull0 + 8 * s, NCW * 32);
             tma::mbar_init(dempty0 + 8 * s, 1);
         }
+        tma::mbar_init(done0, NCW);
         tma::fence_barrier_init();
     }
+    if (warp == 0) {  // compute warp 0 owns the CTA's tensor memory: all 512 columns
+        tmem::alloc(tma::smem_u32(tslot), 512);
+        tmem::relinquish();
+    }
+    tmem::fence_before();
     __syncthreads();
+    tmem::fence_after();
+    const uint32_t taddr = *tslot;
 
     const int ngroups_here = (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const int nchunks = ngroups_here * CHUNKS_PER_GROUP;
@@ -328,7 +338,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t ring = sbase + warp * WARP_BYTES;
     unsigned char* const ringp = smem + warp * WARP_BYTES;
     float* const dxslot = a.dxh + ((size_t)blockIdx.x * NCW + warp) * S * S;
-    float4* const ck = reinterpret_cast<float4*>(smem + CKO) + warp * 8 * 32 + t;  // [chunk][lane]
+    // sweep-1 states of this warp's plane: lane t of TMEM quarter warp % 4,
+    // columns 256 * (warp / 4) + 4s .. +3 = (h_A(s-1), a_B(s)) at positions 2t, 2t+1
+    const uint32_t tstate = taddr + ((uint32_t)(32 * (warp & 3)) << 16) + 256u * (uint32_t)(warp >> 2);
     unsigned char* const dlst = smem + DLS + warp * 2 * BOX;
     const uint32_t dlsa = sbase + DLS + warp * 2 * BOX;
     const uint64_t keep = l2_evict_last_policy();
@@ -377,6 +389,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t phase = 0;
     auto fail = [&]() {
         if (t == 0) atomicExch(a.err, 1);
+        tmem::wait_st();  // no TMEM store may outlive the warp
         for (int kk = k; kk < k + NST && kk < nchunks; ++kk)
             tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
         for (int kk = k; kk < k + NWS && kk < nchunks; ++kk)
@@ -440,6 +453,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             float2 hA = make_float2(0.f, 0.f), aB = make_float2(0.f, 0.f);
             Taps WBp = zero_taps;  // B taps of line s-1 (none before s = 0: a_B(-1) = 0)
             for (int q = 0; q < 8; ++q) {
+                uint32_t sv[32];  // (h_A(s-1), a_B(s)) of the chunk's 8 steps, for TMEM
                 if (!acquire()) { fail(); return false; }
                 uint4 X[2] = {}, LA[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, Gr[8] = {};
@@ -476,20 +490,24 @@ __global__ void __launch_bounds__(THREADS, 1)
                         g = bf2(Gr[e]);
                     }
                     float2 hL, hR;
+                    sv[4 * e] = __float_as_uint(hA.x);
+                    sv[4 * e + 1] = __float_as_uint(hA.y);
                     hA = add2(mix(hA, WA, t, hL, hR), mul2(lam, x));
                     aB = adjoint(aB, g, WBp, t);
+                    sv[4 * e + 2] = __float_as_uint(aB.x);
+                    sv[4 * e + 3] = __float_as_uint(aB.y);
                     WBp = WB;
                 }
-                ck[q * 32] = make_float4(hA.x, hA.y, aB.x, aB.y);
+                tmem::st_x32(tstate + 32 * q, sv);
                 release_w();
             }
+            tmem::wait_st();  // sweep 2 reads what sweep 1 stored
 
             // ---------------- sweep 2: s descending ----------------
             float2 aA = make_float2(0.f, 0.f), hB = make_float2(0.f, 0.f);
             Taps WAn = zero_taps;  // A taps of line s+1 (none after s = 63: a_A(64) = 0)
             for (int qq = 0; qq < 8; ++qq) {
                 const int q = 7 - qq;
-                // B taps of line 8q-1 for the a_B recompute (previous chunk in s, not in this ring)
                 // column pass: the row pass's dx share of columns 2t, 2t+1, rows 8q..8q+7
                 // (loaded early; the scratch plane is column-major)
                 float4 dxc[2][2];
@@ -522,41 +540,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
                 release_data();
-                // B taps of line 8q-1: the last row of the next chunk's weight stage
-                Taps WBm = zero_taps;
-                if (q > 0) {
-                    const int kn = k + 1;
-                    if (!__all_sync(FULL, tma::mbar_wait(wfull0 + 8 * (kn % NWS), (kn / NWS) & 1))) {
-                        ++k;
-                        fail();
-                        return false;
-                    }
-                    const float4 v = lds128f(wring + (kn % NWS) * WCHUNK + 7 * 1024 + 512 + t * 16);
-                    WBm.w0 = make_float2(v.x, v.y);
-                    WBm.w2 = make_float2(v.z, v.w);
-                }
                 auto xv = [&](int e) { return pass == 0 ? make_float2(bfv(X[0], e), bfv(X[1], e)) : bf2(Xr[e]); };
                 auto lav = [&](int e) { return pass == 0 ? make_float2(bfv(LA[0], e), bfv(LA[1], e)) : bf2(LAr[e]); };
                 auto lbv = [&](int e) { return pass == 0 ? make_float2(bfv(LB[0], e), bfv(LB[1], e)) : bf2(LBr[e]); };
                 auto gv = [&](int e) { return pass == 0 ? make_float2(bfv(G[0], e), bfv(G[1], e)) : bf2(Gr[e]); };
 
-                // recompute h_A and a_B over the chunk from the checkpoints, keeping
-                // h_A(s-1) (the state line s reads) and a_B(s)
+                // h_A(s-1) (the state line s reads) and a_B(s) of the chunk, from sweep 1
                 float2 hAp[8], aBs[8];
                 {
-                    const float4 c = q > 0 ? ck[(q - 1) * 32] : make_float4(0.f, 0.f, 0.f, 0.f);
-                    float2 h = make_float2(c.x, c.y), ab = make_float2(c.z, c.w);
-                    Taps WBq = WBm;
+                    uint32_t sv[32];
+                    tmem::ld_x32(tstate + 32 * q, sv);
+                    tmem::wait_ld(sv);
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        Taps WA, WB;
-                        wrow(e, WA, WB);
-                        float2 hL, hR;
-                        hAp[e] = h;
-                        h = add2(mix(h, WA, t, hL, hR), mul2(lav(e), xv(e)));
-                        ab = adjoint(ab, gv(e), WBq, t);
-                        aBs[e] = ab;
-                        WBq = WB;
+                        hAp[e] = make_float2(__uint_as_float(sv[4 * e]), __uint_as_float(sv[4 * e + 1]));
+                        aBs[e] = make_float2(__uint_as_float(sv[4 * e + 2]), __uint_as_float(sv[4 * e + 3]));
                     }
                 }
                 uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns (bf16 pairs)
@@ -665,6 +663,16 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!run_pass(std::integral_constant<int, 0>{}) || !run_pass(std::integral_constant<int, 1>{})) break;
     }
     if (t == 0) tma::bulk_wait_all();  // the dlambda stores have read shared memory
+    // this warp no longer touches the tensor memory; warp 0 frees it after all
+    tmem::fence_before();
+    __syncwarp();
+    if (t == 0) tma::mbar_arrive(done0);
+    if (warp == 0) {
+        if (!tma::mbar_wait(done0, 0, 10 * tma::kTimeoutNs) && t == 0) atomicExch(a.err, 1);
+        __syncwarp();
+        tmem::fence_after();
+        tmem::dealloc(taddr, 512);
+    }
 }
 
 // ---- host side ----------------------------------------------------------------------
