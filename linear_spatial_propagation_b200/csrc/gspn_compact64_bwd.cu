@@ -78,7 +78,7 @@ constexpr int BARS = DLS + NCW * 2 * BOX;
 constexpr int NBAR = NCW * NST + 2 * NWS + 4 + 1;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
-constexpr int THREADS = (NCW + 2) * 32;  // compute warps, tap-table producer, tap-value reducer
+constexpr int THREADS = (NCW + 3) * 32;  // compute warps, tap-table producer, two tap-value reducers
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ---- backward tap table ---------------------------------------------------------------
@@ -205,7 +205,7 @@ __device__ __forceinline__ float2 adjoint(float2 a, float2 g, const Taps& w, int
     return add2(n, add2(make_float2(p0.y, p0r), make_float2(p2l, p2.x)));
 }
 
-// 10 warps put 3 on two of the SM's four schedulers, each with a quarter of
+// 11 warps put 3 on three of the SM's four schedulers, each with a quarter of
 // the register file: at most 16384 / (3 * 32) -> 168 registers per thread
 __global__ void __launch_bounds__(THREADS, 1)
     c64b_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
@@ -285,7 +285,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // into reduced buffer n & 1, the set is handed back, and the half chunk is
     // added to the image's sums (rows 8q+4h..8q+4h+3 of each of the 4 [s][j]
     // planes) by 4 bulk reduce-adds of 1 KB.
-    if (warp == NCW + 1) {
+    if (warp >= NCW + 1) {
+        // reducer r takes the pieces of slot set r (every other half chunk)
+        const int r = warp - (NCW + 1);
         const float4* const sets = reinterpret_cast<const float4*>(smem + DSTG);
         int n = 0;
         bool ok = true;
@@ -293,12 +295,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int b = (8 * group) / a.C;
             for (int l = 0; l < 32; ++l, ++n) {
                 const int pass = l >> 4, q = 7 - ((l >> 1) & 7), h = 1 - (l & 1), set = n & 1;
+                if (set != r) continue;
                 float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S + (8 * q + 4 * h) * S;
                 if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n >> 1) & 1, 128))) {
                     ok = false;
                     break;
                 }
-                if (t == 0) tma::bulk_wait_read_n<1>();  // the reduces of half chunk n-2 have read its buffer
+                if (t == 0) tma::bulk_wait_read();  // this reducer's previous reduces have read its buffer
                 __syncwarp();
                 const float4* const src = sets + set * NCW * (DSLOT / 16);
                 float4* const outp = reinterpret_cast<float4*>(smem + DOUT + set * DSLOT);
