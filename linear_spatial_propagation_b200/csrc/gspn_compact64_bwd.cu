@@ -35,11 +35,11 @@
 //   (rewritten for every plane, so it stays in L2); the column pass adds its
 //   share and stores dx once.
 // * Tap values E_0, E_2: each of the 8 warps of a CTA (8 channels of one
-//   image) stores its chunk of values into its own shared slot; a reducer
-//   warp sums the 8 slots of a chunk and adds the result with bulk
-//   shared->global fp32 reduce-adds to L2-resident sums.  Slots alternate
-//   between two sets, so a compute warp waits only if it runs two chunks
-//   ahead of the reducer.
+//   image) stores each half chunk of values into its own shared slot; a
+//   reducer warp sums the 8 slots and adds the result with bulk
+//   shared->global fp32 reduce-adds to L2-resident sums.  Half chunks rotate
+//   over three slot sets, each with its own reducer warp, so the reductions
+//   overlap and a compute warp rarely waits for a set.
 // * x, lambda and dout are streamed by TMA exactly as in the compact forward
 //   (per-warp ring of 8-step chunks); the normalised tap weights (a table
 //   written by a pre-kernel, one row per scan step with both directions at
@@ -72,13 +72,14 @@ constexpr int DSLOT = 4 * 4 * S * 4;      // one warp's tap values of half a chu
 constexpr int WARP_BYTES = NST * STAGE;   // data ring per warp
 constexpr int WRING = NCW * WARP_BYTES;
 constexpr int DSTG = WRING + NWS * WCHUNK;    // 2 sets x NCW slots
-constexpr int DOUT = DSTG + 2 * NCW * DSLOT;  // 2 reduced half chunks: [dir*2 + value][step][position j]
-constexpr int DLS = DOUT + 2 * DSLOT;          // per warp: row-pass dlambda of a chunk, A then B, [row][8 columns]
+constexpr int NSET = 3;                         // slot sets, one reducer warp each
+constexpr int DOUT = DSTG + NSET * NCW * DSLOT;  // a reduced half chunk per set: [dir*2 + value][step][position j]
+constexpr int DLS = DOUT + NSET * DSLOT;          // per warp: row-pass dlambda of a chunk, A then B, [row][8 columns]
 constexpr int BARS = DLS + NCW * 2 * BOX;
-constexpr int NBAR = NCW * NST + 2 * NWS + 4 + 1;
+constexpr int NBAR = NCW * NST + 2 * NWS + 2 * NSET + 1;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
-constexpr int THREADS = (NCW + 3) * 32;  // compute warps, tap-table producer, two tap-value reducers
+constexpr int THREADS = (NCW + 1 + NSET) * 32;  // compute warps, tap-table producer, tap-value reducers
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ---- backward tap table ---------------------------------------------------------------
@@ -205,7 +206,7 @@ __device__ __forceinline__ float2 adjoint(float2 a, float2 g, const Taps& w, int
     return add2(n, add2(make_float2(p0.y, p0r), make_float2(p2l, p2.x)));
 }
 
-// 11 warps put 3 on three of the SM's four schedulers, each with a quarter of
+// 12 warps put 3 on each of the SM's four schedulers, each with a quarter of
 // the register file: at most 16384 / (3 * 32) -> 168 registers per thread
 __global__ void __launch_bounds__(THREADS, 1)
     c64b_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
@@ -219,8 +220,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t wfull0 = sbase + BARS + 8 * NCW * NST;
     const uint32_t wempty0 = wfull0 + 8 * NWS;
     const uint32_t dfull0 = wempty0 + 8 * NWS;  // [set]: the compute warps' slots of a chunk are written
-    const uint32_t dempty0 = dfull0 + 16;       // [set]: the reducer has read the set
-    const uint32_t done0 = dempty0 + 16;        // every compute warp is done with the tensor memory
+    const uint32_t dempty0 = dfull0 + 8 * NSET;  // [set]: the reducer has read the set
+    const uint32_t done0 = dempty0 + 8 * NSET;   // every compute warp is done with the tensor memory
     uint32_t* const tslot = reinterpret_cast<uint32_t*>(smem + BARS + 8 * NBAR);
     if ((int)blockIdx.x >= a.groups) return;
 
@@ -230,7 +231,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_init(wfull0 + 8 * s, 1);
             tma::mbar_init(wempty0 + 8 * s, NCW);
         }
-        for (int s = 0; s < 2; ++s) {
+        for (int s = 0; s < NSET; ++s) {
             tma::mbar_init(dfull0 + 8 * s, NCW * 32);
             tma::mbar_init(dempty0 + 8 * s, 1);
         }
@@ -279,25 +280,25 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
     }
 
-    // ---------------- reducer warp: tap values of each sweep-2 half chunk ----------------
+    // ---------------- reducer warps: tap values of each sweep-2 half chunk ----------------
     // Half chunk n of the CTA (pass-major within a group, q descending, the upper
-    // 4 steps of a chunk first) sits in slot set n & 1.  The 8 slots are summed
-    // into reduced buffer n & 1, the set is handed back, and the half chunk is
-    // added to the image's sums (rows 8q+4h..8q+4h+3 of each of the 4 [s][j]
-    // planes) by 4 bulk reduce-adds of 1 KB.
+    // 4 steps of a chunk first) sits in slot set n % NSET, which reducer warp
+    // n % NSET owns.  It sums the 8 slots into its reduced buffer, hands the set
+    // back, and adds the half chunk to the image's sums (rows 8q+4h..8q+4h+3 of
+    // each of the 4 [s][j] planes) by 4 bulk reduce-adds of 1 KB.
     if (warp >= NCW + 1) {
-        // reducer r takes the pieces of slot set r (every other half chunk)
-        const int r = warp - (NCW + 1);
+        // reducer rid takes the pieces of slot set rid (every NSET-th half chunk)
+        const int rid = warp - (NCW + 1);
         const float4* const sets = reinterpret_cast<const float4*>(smem + DSTG);
         int n = 0;
         bool ok = true;
         for (int group = blockIdx.x; ok && group < a.groups; group += gridDim.x) {
             const int b = (8 * group) / a.C;
             for (int l = 0; l < 32; ++l, ++n) {
-                const int pass = l >> 4, q = 7 - ((l >> 1) & 7), h = 1 - (l & 1), set = n & 1;
-                if (set != r) continue;
+                const int pass = l >> 4, q = 7 - ((l >> 1) & 7), h = 1 - (l & 1), set = n % NSET;
+                if (set != rid) continue;
                 float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S + (8 * q + 4 * h) * S;
-                if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n >> 1) & 1, 128))) {
+                if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n / NSET) & 1, 128))) {
                     ok = false;
                     break;
                 }
@@ -430,15 +431,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         Bt.w2 = make_float2(vb.z, vb.w);
     };
     // tap values of sweep-2 half chunk number dchunk: this warp's slot in set
-    // dchunk & 1, free once the reducer has handed the set back
+    // dchunk % NSET, free once the reducer has handed the set back
     int dchunk = 0;
     auto dslot = [&]() -> float* {
-        const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk & 1), ((dchunk >> 1) & 1) ^ 1);
+        const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk % NSET), ((dchunk / NSET) & 1) ^ 1);
         if (!__all_sync(FULL, ok)) return nullptr;
-        return reinterpret_cast<float*>(smem + DSTG + ((dchunk & 1) * NCW + warp) * DSLOT);
+        return reinterpret_cast<float*>(smem + DSTG + ((dchunk % NSET) * NCW + warp) * DSLOT);
     };
     auto dpublish = [&]() {
-        tma::mbar_arrive(dfull0 + 8 * (dchunk & 1));  // every lane: its stores are released
+        tma::mbar_arrive(dfull0 + 8 * (dchunk % NSET));  // every lane: its stores are released
         ++dchunk;
     };
 
