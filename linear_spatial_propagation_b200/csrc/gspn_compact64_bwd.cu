@@ -160,7 +160,8 @@ struct C64BArgs {
     __nv_bfloat16* dlam;
     int* err;
     int B, C;
-    int groups;  // B * C / 8
+    int groups;   // B * C / 8
+    int segmask;  // local groups: lines per group - 1 (a power of two minus one; 63 = global)
 };
 
 // bf16 element e of 8 packed in a uint4, widened
@@ -208,6 +209,7 @@ __device__ __forceinline__ float2 adjoint(float2 a, float2 g, const Taps& w, int
 
 // 12 warps put 3 on each of the SM's four schedulers, each with a quarter of
 // the register file: at most 16384 / (3 * 32) -> 168 registers per thread
+template <bool LOCAL>
 __global__ void __launch_bounds__(THREADS, 1)
     c64b_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
                 const __grid_constant__ CUtensorMap tm_gc, const __grid_constant__ CUtensorMap tm_xr,
@@ -494,6 +496,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                         g = bf2(Gr[e]);
                     }
                     float2 hL, hR;
+                    // local groups: line s of A starts a group, and line s-1 of B (the
+                    // next in B's order) starts one, exactly when s is a multiple of seg
+                    if (LOCAL && ((8 * q + e) & a.segmask) == 0) {
+                        hA = make_float2(0.f, 0.f);
+                        aB = make_float2(0.f, 0.f);
+                    }
                     sv[4 * e] = __float_as_uint(hA.x);
                     sv[4 * e + 1] = __float_as_uint(hA.y);
                     hA = add2(mix(hA, WA, t, hL, hR), mul2(lam, x));
@@ -585,6 +593,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     Taps WA, WB;
                     wrow(e, WA, WB);
                     const float2 x = xv(e), lamA = lav(e), lamB = lbv(e), ab = aBs[e];
+                    // local groups: line s+1 of A starts a group, and line s of B does,
+                    // exactly when s+1 is a multiple of seg
+                    if (LOCAL && ((s + 1) & a.segmask) == 0) {
+                        aA = make_float2(0.f, 0.f);
+                        hB = make_float2(0.f, 0.f);
+                    }
                     // adjoint of A at s from s+1 (taps of line s+1)
                     aA = adjoint(aA, gv(e), WAn, t);
                     WAn = WA;
@@ -715,7 +729,7 @@ bool make_map_b(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_
 
 bool c64_bwd_eligible(const Problem& p) {
     return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
-           p.g.groups == 1 && p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_fn_b() != nullptr;
+           S % p.g.groups == 0 && p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_fn_b() != nullptr;
 }
 
 namespace {
@@ -752,14 +766,20 @@ gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     a.B = p.g.B;
     a.C = p.g.C;
     a.groups = (int)(p.planes / 8);
+    a.segmask = S / p.g.groups - 1;
     const int nt = p.g.B * 2 * S * LPL;
     c64b_table_kernel<__nv_bfloat16><<<(nt + 255) / 256, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.btab), a.dsum, a.err, p.g.B);
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
-    cudaError_t e = ensure_smem_attr((const void*)c64b_kernel, SMEM_BYTES, 10);
+    const bool local = p.g.groups > 1;
+    const void* fn = local ? (const void*)c64b_kernel<true> : (const void*)c64b_kernel<false>;
+    cudaError_t e = ensure_smem_attr(fn, SMEM_BYTES, local ? 17 : 10);
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
     const int grid = bwd_grid(p, dev);
-    c64b_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, gc, xr, lr, gr, dl, a);
+    if (local)
+        c64b_kernel<true><<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, gc, xr, lr, gr, dl, a);
+    else
+        c64b_kernel<false><<<grid, THREADS, SMEM_BYTES, s>>>(xc, lc, gc, xr, lr, gr, dl, a);
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
     const int nl = 4 * p.g.B * S * S;
     c64b_dlogits_kernel<__nv_bfloat16><<<(nl + 255) / 256, 256, 0, s>>>(
