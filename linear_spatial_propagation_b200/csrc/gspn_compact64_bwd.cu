@@ -196,6 +196,19 @@ __device__ __forceinline__ float2 mix(float2 h, const Taps& w, int t, float2& hL
     return fma2(w.w0, sub2(hL, h), fma2(w.w2, sub2(hR, h), h));
 }
 
+// Forward step h' = w0 hL + w1 h + w2 hR + lx written so that only two FMAs
+// follow the shuffles (w1 h + lx is formed while they are in flight); m =
+// h' - lx is the neighbour mix, for the tap values.
+__device__ __forceinline__ float2 fwd_step(float2 h, float2 lx, const Taps& w, int t, float2& hL, float2& hR,
+                                           float2& m) {
+    hL = make_float2(__shfl_sync(FULL, h.y, (t + 31) & 31), h.x);
+    hR = make_float2(h.y, __shfl_sync(FULL, h.x, (t + 1) & 31));
+    const float2 w1 = sub2(sub2(make_float2(1.f, 1.f), w.w0), w.w2);
+    const float2 hn = fma2(w.w2, hR, fma2(w.w0, hL, fma2(w1, h, lx)));
+    m = sub2(hn, lx);
+    return hn;
+}
+
 // Adjoint step: a(line i) = g + W_{i+1}^T a(line i+1), with w the taps of
 // line i+1: a'[j] = g[j] + w1[j] a[j] + w0[j+1] a[j+1] + w2[j-1] a[j-1].  The
 // rotated shuffles bring in w0 a at j = 0 and w2 a at j = 63, both zero.
@@ -203,8 +216,10 @@ __device__ __forceinline__ float2 adjoint(float2 a, float2 g, const Taps& w, int
     const float2 p0 = mul2(w.w0, a), p2 = mul2(w.w2, a);
     const float p0r = __shfl_sync(FULL, p0.x, (t + 1) & 31);  // w0 a at j = 2t+2
     const float p2l = __shfl_sync(FULL, p2.y, (t + 31) & 31); // w2 a at j = 2t-1
-    float2 n = fma2(make_float2(-1.f, -1.f), p2, fma2(make_float2(-1.f, -1.f), p0, add2(g, a)));
-    return add2(n, add2(make_float2(p0.y, p0r), make_float2(p2l, p2.x)));
+    // the in-lane terms are summed while the shuffles are in flight
+    const float2 n = add2(fma2(make_float2(-1.f, -1.f), p2, fma2(make_float2(-1.f, -1.f), p0, add2(g, a))),
+                          make_float2(p0.y, p2.x));
+    return add2(n, make_float2(p2l, p0r));
 }
 
 // 12 warps put 3 on each of the SM's four schedulers, each with a quarter of
@@ -504,7 +519,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     sv[4 * e] = __float_as_uint(hA.x);
                     sv[4 * e + 1] = __float_as_uint(hA.y);
-                    hA = add2(mix(hA, WA, t, hL, hR), mul2(lam, x));
+                    float2 mA_;
+                    hA = fwd_step(hA, mul2(lam, x), WA, t, hL, hR, mA_);
                     aB = adjoint(aB, g, WBp, t);
                     sv[4 * e + 2] = __float_as_uint(aB.x);
                     sv[4 * e + 3] = __float_as_uint(aB.y);
@@ -603,9 +619,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     aA = adjoint(aA, gv(e), WAn, t);
                     WAn = WA;
                     // forward of B at s from s+1 (taps of B's line at s) and B's tap values
-                    float2 hL, hR;
-                    const float2 m = mix(hB, WB, t, hL, hR);
-                    hB = add2(m, mul2(lamB, x));
+                    float2 hL, hR, m;
+                    hB = fwd_step(hB, mul2(lamB, x), WB, t, hL, hR, m);
                     // tap values E = a (h_k - m): A's line s with a_A(s), B's with a_B(s).
                     // On each direction's first line the state read is zero and so are they.
                     float* const d = ds + (e & 3) * 4 * S + 2 * t;
