@@ -23,11 +23,13 @@
 // B = right->left over columns s; column pass: A = top->bottom,
 // B = bottom->top over rows s):
 // * Sweep 1, s ascending: the forward scan of A (h_A) and the adjoint of B
-//   (a_B, whose last line is s = 0) both advance with s.  They are kept only
-//   as checkpoints at the end of every 8-step chunk (registers).
-// * Sweep 2, s descending, chunk by chunk: h_A and a_B of the chunk are
-//   recomputed from their checkpoints (forward in s), then the chunk is
-//   walked backwards running the adjoint of A and the forward of B.  At every
+//   (a_B, whose last line is s = 0) both advance with s.  Every step's pair
+//   (h_A(s-1), a_B(s)) is parked in tensor memory (TMEM, 512 columns per CTA:
+//   each warp owns a 32-lane x 256-column block, lane t = plane columns 2t, 2t+1),
+//   so nothing is recomputed and no shared memory is spent on states.
+// * Sweep 2, s descending, chunk by chunk: the chunk's states are read back
+//   from TMEM, then the chunk is walked backwards running the adjoint of A
+//   and the forward of B.  At every
 //   s all four of h_A(s-1), a_A(s), h_B(s+1), a_B(s) are at hand, so dlambda
 //   of both directions, the pass's share of dx and the tap products of both
 //   directions are produced without storing any plane of h or a.
