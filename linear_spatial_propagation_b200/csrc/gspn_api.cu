@@ -140,21 +140,23 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return 0;
     if (backward) return c64_bwd_eligible(p) ? c64_bwd_workspace(p, dev) : generic_bwd_workspace(p, dev);
-    return c64_eligible(p) ? c64_fwd_workspace(p) : generic_fwd_workspace(p, dev);
+    if (c64_eligible(p)) return c64_fwd_workspace(p);
+    return c128_eligible(p) ? c128_fwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
 }
 
 int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return 0;
     if (backward) return c64_bwd_eligible(p) ? 3 : generic_bwd_launches(p);
-    return c64_eligible(p) ? 2 : 1;
+    return c64_eligible(p) || c128_eligible(p) ? 2 : 1;
 }
 
 const char* gspn_variant_name(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return "invalid";
     if (backward) return c64_bwd_eligible(p) ? "compact64_tma_bwd" : "generic_bwd";
-    return c64_eligible(p) ? "compact64_tma_fwd" : "generic_fwd";
+    if (c64_eligible(p)) return "compact64_tma_fwd";
+    return c128_eligible(p) ? "compact128_tma_fwd" : "generic_fwd";
 }
 
 gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda, void* out,
@@ -166,10 +168,12 @@ gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, c
     if (st != GSPN_OK) return st;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
-    const bool fast = c64_eligible(p);
-    st = check_ws(workspace, ws_bytes, fast ? c64_fwd_workspace(p) : generic_fwd_workspace(p, dev));
+    const bool fast = c64_eligible(p), fast128 = !fast && c128_eligible(p);
+    st = check_ws(workspace, ws_bytes,
+                  fast ? c64_fwd_workspace(p) : fast128 ? c128_fwd_workspace(p, dev) : generic_fwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
     if (fast) return c64_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
+    if (fast128) return c128_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
     return generic_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
 }
 

@@ -270,6 +270,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             wr[e][0] = lds128f(wsrc + e * 1024);
             wr[e][1] = lds128f(wsrc + e * 1024 + 512);
         }
+        // every lane's reads of the stage come before the async-proxy refill
+        tma::fence_proxy_async();
         __syncwarp();
         if (t == 0) tma::mbar_arrive(wempty0 + 8 * ws);
         return true;
@@ -280,6 +282,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
     // the stage is in registers: hand it back to its producer
     auto release = [&]() {
+        tma::fence_proxy_async();  // this lane's reads of the stage come before its refill
         tma::mbar_arrive(ebar0 + 8 * stage);
         phase ^= 1u << stage;
         ++k;

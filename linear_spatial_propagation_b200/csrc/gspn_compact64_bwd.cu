@@ -423,19 +423,18 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool ok2 = tma::mbar_wait(wfull0 + 8 * (k % NWS), (k / NWS) & 1);
         return __all_sync(FULL, ok1 && ok2);
     };
-    // the data stage is in registers: refill it (the warp's reads of the stage
-    // happen before lane 0's proxy fence and the async-proxy writes after it)
+    // the data stage is in registers: refill it (every lane orders its reads of
+    // the stage before the async-proxy writes with a proxy fence of its own)
     auto release_data = [&]() {
+        tma::fence_proxy_async();
         __syncwarp();
-        if (t == 0) {
-            tma::fence_proxy_async();
-            issue(k + NST);
-        }
+        if (t == 0) issue(k + NST);
         phase ^= 1u << stage;
         stage = stage == NST - 1 ? 0 : stage + 1;
     };
     // done with the weight stage of chunk k
     auto release_w = [&]() {
+        tma::fence_proxy_async();
         __syncwarp();
         if (t == 0) tma::mbar_arrive(wempty0 + 8 * (k % NWS));
         ++k;

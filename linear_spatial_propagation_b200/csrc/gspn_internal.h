@@ -50,6 +50,12 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
 gspn_status c64_fwd_noalloc(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
                             const void* lam, void* out, cudaStream_t s);
 
+// ---- compact 128x128 bf16 forward (TMA-fed, first arrivals in TMEM) ------------------
+bool c128_eligible(const Problem& p);
+size_t c128_fwd_workspace(const Problem& p, const DeviceInfo& dev);
+gspn_status c128_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                     void* out, void* ws, cudaStream_t s);
+
 // ---- compact 64x64 bf16 backward (TMA-fed, checkpointed sweeps) ------------------
 bool c64_bwd_eligible(const Problem& p);
 size_t c64_bwd_workspace(const Problem& p, const DeviceInfo& dev);

@@ -152,6 +152,12 @@ SHAPES = [
     (3, 24, 64, 64, 15, 64, True, "bf16"),
     (5, 8, 64, 64, 15, 2, True, "bf16"),
     (1, 2, 130, 70, 15, 1, True, "bf16"),
+    # 128x128 compact bf16 with C % 4 == 0: the TMA-fed 128x128 forward
+    (1, 4, 128, 128, 15, 1, True, "bf16"),
+    (2, 12, 128, 128, 15, 1, True, "bf16"),
+    (1, 8, 128, 128, 15, 4, True, "bf16"),
+    (1, 4, 128, 128, 15, 128, True, "bf16"),
+    (1, 600, 128, 128, 15, 2, True, "bf16"),  # 150 groups of 4 planes: CTAs take more than one
     (1, 1, 257, 33, 3, 1, False, "f32"),
 ]
 
@@ -223,3 +229,33 @@ def test_workspace_errors_on_gpu():
     ws = t.empty(need, dtype=t.uint8, device="cuda")
     st = lsp.gspn_bwd(d, *(x.data_ptr(),) * 7, ws.data_ptr(), need - 1, 0)
     assert st == 4
+
+
+def test_compact128_forward_dispatch_guards_and_repeats():
+    """The 128x128 compact forward: its dispatch, out-of-bounds canaries around
+    the output and after the exact workspace (which holds its row-sum scratch
+    planes), and bit-identical repeats on a side stream."""
+    import linear_spatial_propagation_b200 as lsp
+    t = gu.torch()
+    w = shape_workload(1, 8, 128, 128, 15, 1, True, "bf16", 501)
+    d = lsp.make_desc(w.B, w.C, w.H, w.W, w.dir_mask, w.groups, w.shared, w.dtype)
+    assert lsp.gspn_variant_name(d, 0) == "compact128_tma_fwd"
+    assert lsp.gspn_launches_per_call(d, 0) == 2
+    inp = synth.make_inputs(w, with_dout=False)
+    dinp = gu.dev_inputs(w, inp)
+    guard = 4096
+    n = w.B * w.C * w.H * w.W
+    buf = t.full((n + 2 * guard,), 7.0, dtype=t.bfloat16, device="cuda")
+    out = buf[guard:guard + n].view(w.B, w.C, w.H, w.W)
+    need = lsp.gspn_workspace_size(d, 0)
+    wsbuf = t.full((need + guard,), 0x5A, dtype=t.uint8, device="cuda")
+    s = t.cuda.Stream()
+    s.wait_stream(t.cuda.current_stream())  # the inputs and canaries are written on the default stream
+    with t.cuda.stream(s):
+        lsp.forward(dinp["x"], dinp["logits"], dinp["lam"], dir_mask=15, shared=True, out=out, ws=wsbuf[:need])
+        again = lsp.forward(dinp["x"], dinp["logits"], dinp["lam"], dir_mask=15, shared=True)
+    s.synchronize()
+    assert bool((buf[:guard] == 7.0).all()) and bool((buf[guard + n:] == 7.0).all())
+    assert bool((wsbuf[need:] == 0x5A).all())
+    assert bool(t.equal(out, again))
+    gu.assert_close(gu.from_dev(out), oracle.fwd_workload(w, inp), w.dtype, "128x128 compact forward")
