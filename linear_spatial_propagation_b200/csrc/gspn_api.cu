@@ -139,7 +139,10 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     if (validate(desc, &p) != GSPN_OK) return 0;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return 0;
-    if (backward) return c64_bwd_eligible(p) ? c64_bwd_workspace(p, dev) : generic_bwd_workspace(p, dev);
+    if (backward) {
+        if (c64_bwd_eligible(p)) return c64_bwd_workspace(p, dev);
+        return c128_bwd_eligible(p) ? c128_bwd_workspace(p, dev) : generic_bwd_workspace(p, dev);
+    }
     if (c64_eligible(p)) return c64_fwd_workspace(p);
     return c128_eligible(p) ? c128_fwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
 }
@@ -147,14 +150,17 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
 int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return 0;
-    if (backward) return c64_bwd_eligible(p) ? 3 : generic_bwd_launches(p);
+    if (backward) return c64_bwd_eligible(p) || c128_bwd_eligible(p) ? 3 : generic_bwd_launches(p);
     return c64_eligible(p) || c128_eligible(p) ? 2 : 1;
 }
 
 const char* gspn_variant_name(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return "invalid";
-    if (backward) return c64_bwd_eligible(p) ? "compact64_tma_bwd" : "generic_bwd";
+    if (backward) {
+        if (c64_bwd_eligible(p)) return "compact64_tma_bwd";
+        return c128_bwd_eligible(p) ? "compact128_tma_bwd" : "generic_bwd";
+    }
     if (c64_eligible(p)) return "compact64_tma_fwd";
     return c128_eligible(p) ? "compact128_tma_fwd" : "generic_fwd";
 }
@@ -199,12 +205,18 @@ gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, c
     if (st != GSPN_OK) return st;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
-    const bool fast = c64_bwd_eligible(p);
-    st = check_ws(workspace, ws_bytes, fast ? c64_bwd_workspace(p, dev) : generic_bwd_workspace(p, dev));
+    const bool fast = c64_bwd_eligible(p), fast128 = !fast && c128_bwd_eligible(p);
+    st = check_ws(workspace, ws_bytes,
+                  fast      ? c64_bwd_workspace(p, dev)
+                  : fast128 ? c128_bwd_workspace(p, dev)
+                            : generic_bwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
     if (fast)
         return c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
                        static_cast<cudaStream_t>(stream));
+    if (fast128)
+        return c128_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
+                        static_cast<cudaStream_t>(stream));
     return generic_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
                        static_cast<cudaStream_t>(stream));
 }

@@ -151,16 +151,6 @@ __device__ __forceinline__ uint2 lds64u(const unsigned char* p) { return *reinte
 // order this thread's generic-proxy accesses (global and shared) before later async-proxy ones
 __device__ __forceinline__ void fence_proxy_async_all() { asm volatile("fence.proxy.async;" ::: "memory"); }
 
-// 4-D tiled load global -> shared, completion counted on `bar` (bytes).
-__device__ __forceinline__ void load_4d(uint32_t dst, const CUtensorMap* map, int c0, int c1, int c2, int c3,
-                                        uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(dst),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar)
-        : "memory");
-}
-
 struct C128Args {
     const float4* wtab;
     float* rsum;  // per consumer warp of the grid: one 128x128 fp32 scratch plane
@@ -254,10 +244,10 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (pass == 0) {
                     // x and lambda(left->right) at columns 8q.., x and lambda(right->left)
                     // at columns 120-8q..; all 128 rows through the (column, row/4, row%4) view
-                    load_4d(dst + 0 * BOX, &tm_xc, 8 * q, 0, 0, plane, bar);
-                    load_4d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 0, 2 * BC + plane, bar);
-                    load_4d(dst + 2 * BOX, &tm_xc, S - 8 - 8 * q, 0, 0, plane, bar);
-                    load_4d(dst + 3 * BOX, &tm_lc, S - 8 - 8 * q, 0, 0, 3 * BC + plane, bar);
+                    tma::load_4d(dst + 0 * BOX, &tm_xc, 8 * q, 0, 0, plane, bar);
+                    tma::load_4d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 0, 2 * BC + plane, bar);
+                    tma::load_4d(dst + 2 * BOX, &tm_xc, S - 8 - 8 * q, 0, 0, plane, bar);
+                    tma::load_4d(dst + 3 * BOX, &tm_lc, S - 8 - 8 * q, 0, 0, 3 * BC + plane, bar);
                 } else {
                     // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 120-8q..
                     tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);

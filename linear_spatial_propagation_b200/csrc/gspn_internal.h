@@ -56,6 +56,12 @@ size_t c128_fwd_workspace(const Problem& p, const DeviceInfo& dev);
 gspn_status c128_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
                      void* out, void* ws, cudaStream_t s);
 
+// ---- compact 128x128 bf16 backward (TMA-fed; h_A states in TMEM, a_B through L2) ------
+bool c128_bwd_eligible(const Problem& p);
+size_t c128_bwd_workspace(const Problem& p, const DeviceInfo& dev);
+gspn_status c128_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                     const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s);
+
 // ---- compact 64x64 bf16 backward (TMA-fed, checkpointed sweeps) ------------------
 bool c64_bwd_eligible(const Problem& p);
 size_t c64_bwd_workspace(const Problem& p, const DeviceInfo& dev);

@@ -259,3 +259,34 @@ def test_compact128_forward_dispatch_guards_and_repeats():
     assert bool((wsbuf[need:] == 0x5A).all())
     assert bool(t.equal(out, again))
     gu.assert_close(gu.from_dev(out), oracle.fwd_workload(w, inp), w.dtype, "128x128 compact forward")
+
+
+def test_compact128_backward_dispatch_and_guards():
+    """The 128x128 compact backward: its dispatch, canaries around every
+    gradient and after the exact workspace (tap table, tap sums and the
+    per-warp dx and a_B scratch planes), and the oracle's gradients."""
+    import linear_spatial_propagation_b200 as lsp
+    t = gu.torch()
+    w = shape_workload(1, 8, 128, 128, 15, 1, True, "bf16", 601)
+    d = lsp.make_desc(w.B, w.C, w.H, w.W, w.dir_mask, w.groups, w.shared, w.dtype)
+    assert lsp.gspn_variant_name(d, 1) == "compact128_tma_bwd"
+    assert lsp.gspn_launches_per_call(d, 1) == 3
+    inp = synth.make_inputs(w, with_dout=True)
+    dinp = gu.dev_inputs(w, inp)
+    guard = 4096
+    bufs = [t.full((x.numel() + 2 * guard,), -3.0, dtype=t.bfloat16, device="cuda") for x in
+            (dinp["x"], dinp["logits"], dinp["lam"])]
+    views = [b[guard:guard + x.numel()].view(x.shape) for b, x in zip(bufs, (dinp["x"], dinp["logits"], dinp["lam"]))]
+    need = lsp.gspn_workspace_size(d, 1)
+    wsbuf = t.full((need + guard,), 0x5A, dtype=t.uint8, device="cuda")
+    lsp.backward(dinp["x"], dinp["logits"], dinp["lam"], dinp["dout"], dir_mask=15, shared=True, grads=tuple(views),
+                 ws=wsbuf[:need])
+    t.cuda.synchronize()
+    for b, v in zip(bufs, views):
+        assert bool((b[:guard] == -3.0).all()) and bool((b[guard + v.numel():] == -3.0).all())
+    assert bool((wsbuf[need:] == 0x5A).all())
+    assert int(wsbuf[:4].view(t.int32).item()) == 0  # no device-side wait gave up
+    rdx, rdlg, rdlam = oracle.bwd_workload(w, inp, nthreads=8)
+    gu.assert_close(gu.from_dev(views[0]), rdx, w.dtype, "dx")
+    gu.assert_close(gu.from_dev(views[1]), rdlg, w.dtype, "dlogits")
+    gu.assert_close(gu.from_dev(views[2]), rdlam, w.dtype, "dlam")
