@@ -55,6 +55,7 @@
 #include "gspn_internal.h"
 #include "gspn_lane.cuh"
 #include "gspn_tma.cuh"
+#include "gspn_tmem.cuh"
 
 namespace gspn {
 
@@ -76,7 +77,8 @@ constexpr int WCHUNK = 8 * S * 16;  // tap weights of 8 scan steps (8 table rows
 constexpr int WARP_BYTES = NST * STAGE + HACC;
 constexpr int WRING = NCW * WARP_BYTES;              // offset of the weight ring
 constexpr int BARS = WRING + NWS * WCHUNK;           // offset of the barriers
-constexpr int SMEM_BYTES = 1024 + BARS + 8 * (2 * NCW * NST + 2 * NWS);
+constexpr int NBAR = 2 * NCW * NST + 2 * NWS + 1;
+constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
 constexpr int CHUNKS_PER_GROUP = 16;  // 8 column chunks + 8 row chunks
 constexpr int NPW = NCW / 2;  // producer warps, each feeding two consumer warps
 constexpr int THREADS = (NCW + NPW) * 32;
@@ -151,6 +153,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t xempty0 = xfull0 + 8 * NCW * NST;       // [warp][stage] "data read"
     const uint32_t wfull0 = xempty0 + 8 * NCW * NST;       // NWS "weights landed" barriers
     const uint32_t wempty0 = wfull0 + 8 * NWS;             // NWS "weights consumed" barriers
+    const uint32_t done0 = wempty0 + 8 * NWS;              // every consumer is done with the tensor memory
+    uint32_t* const tslot = reinterpret_cast<uint32_t*>(smem + BARS + 8 * NBAR);
     if ((int)blockIdx.x >= a.groups) return;
 
     if (threadIdx.x == 0) {
@@ -162,9 +166,17 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_init(wfull0 + 8 * s, 1);
             tma::mbar_init(wempty0 + 8 * s, NCW);
         }
+        tma::mbar_init(done0, NCW);
         tma::fence_barrier_init();
     }
+    if (warp == 0) {  // consumer warp 0 owns 256 TMEM columns: 128 per consumer warp
+        tmem::alloc(tma::smem_u32(tslot), 256);
+        tmem::relinquish();
+    }
+    tmem::fence_before();
     __syncthreads();
+    tmem::fence_after();
+    const uint32_t taddr = *tslot;
 
     const int ngroups_here = (a.groups - (int)blockIdx.x + (int)gridDim.x - 1) / (int)gridDim.x;
     const int nchunks = ngroups_here * CHUNKS_PER_GROUP;
@@ -247,6 +259,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t phase = 0;   // bit s: parity of the next completion of data stage s
     auto fail = [&]() {
         if (t == 0) atomicExch(a.err, 1);
+        tmem::wait_st();  // no TMEM access outlives the warp
+        tmem::wait_ld_all();
         // drain every data copy that may still be in flight, with a short bound
         for (int kk = k; kk < k + NST && kk < nchunks; ++kk)
             tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
@@ -292,6 +306,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     // Row pass: lane t owns rows 2t, 2t+1 (Hacc unit XOR key t & 15); row 2t + p
     // of a column chunk sits at p*512 + t*16.
     unsigned char* const hrow = haccp + 2 * t * 256;
+    // First arrivals of a pass (its steps 0..31) wait in TMEM for the second:
+    // lane t of lane quarter warp % 4, 128 columns from 128 * (warp / 4); a half
+    // chunk (4 steps) is 16 columns [step][position][direction].
+    const uint32_t tcol = taddr + ((uint32_t)(32 * (warp & 3)) << 16) + 128u * (uint32_t)(warp >> 2);
     const uint32_t tk8 = (uint32_t)(t & 15) << 3;
     const uint32_t t8 = (uint32_t)t << 3;
     float2 h[2];
@@ -318,40 +336,60 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t q8 = (uint32_t)(4 * q) << 3;
             float2 prev[2];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
-                // left->right reads column 8q+e = element e of the A chunk; right->left
-                // column 63-8q-e = element 7-e of the B chunk
-                float2 base[2];
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    base[p].x = fma_bf(e & 1, word_of(LA[p], e >> 1), word_of(XA[p], e >> 1), h[p].x);
-                    base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1),
-                                       h[p].y);
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t tv[16];  // first arrivals of a half chunk: [step][position][direction]
+                if (SECOND) {
+                    // the first arrivals these steps meet were made at steps 63-s:
+                    // half 1-hh of chunk 7-q
+                    tmem::ld_x16(tcol + 32 * (7 - q) + 16 * (1 - hh), tv);
+                    tmem::wait_ld16(tv);
                 }
-                scan_core(h, base, wr[e]);
-                if (e & 1) {
-                    // left->right covers columns s-1, s (unit s/2 = 4q + e/2), right->left
-                    // columns 63-s, 64-s (unit 31 - (4q + e/2)); XOR with the row key
-                    const uint32_t oA = (q8 + (uint32_t)((e >> 1) << 3)) ^ tk8;
-                    const uint32_t oB = oA ^ (31u << 3);
+#pragma unroll
+                for (int ee = 0; ee < 4; ++ee) {
+                    const int e = 4 * hh + ee;
+                    if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
+                    // left->right reads column 8q+e = element e of the A chunk; right->left
+                    // column 63-8q-e = element 7-e of the B chunk
+                    float2 base[2];
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        unsigned char* adA = hrow + p * 256 + oA;
-                        unsigned char* adB = hrow + p * 256 + oB;
-                        float2 vA = make_float2(prev[p].x, h[p].x);
-                        float2 vB = make_float2(h[p].y, prev[p].y);
-                        if (SECOND) {
-                            vA = __fadd2_rn(vA, lds64f(adA));
-                            vB = __fadd2_rn(vB, lds64f(adB));
-                        }
-                        sts64f(adA, vA);
-                        sts64f(adB, vB);
+                        base[p].x = fma_bf(e & 1, word_of(LA[p], e >> 1), word_of(XA[p], e >> 1), h[p].x);
+                        base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1),
+                                           h[p].y);
                     }
-                } else {
-                    prev[0] = h[0];
-                    prev[1] = h[1];
+                    scan_core(h, base, wr[e]);
+                    if (!SECOND) {
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            tv[ee * 4 + p * 2] = __float_as_uint(h[p].x);
+                            tv[ee * 4 + p * 2 + 1] = __float_as_uint(h[p].y);
+                        }
+                        continue;
+                    }
+                    // left->right at column s meets right->left's first arrival there
+                    // (element 3-ee of the loaded half), right->left at column 63-s
+                    // meets left->right's: the completed row sums
+                    float2 sum[2];
+#pragma unroll
+                    for (int p = 0; p < 2; ++p)
+                        sum[p] = __fadd2_rn(h[p], make_float2(__uint_as_float(tv[(3 - ee) * 4 + p * 2 + 1]),
+                                                              __uint_as_float(tv[(3 - ee) * 4 + p * 2])));
+                    if (e & 1) {
+                        // left->right covers columns s-1, s (unit s/2 = 4q + e/2), right->left
+                        // columns 63-s, 64-s (unit 31 - (4q + e/2)); XOR with the row key
+                        const uint32_t oA = (q8 + (uint32_t)((e >> 1) << 3)) ^ tk8;
+                        const uint32_t oB = oA ^ (31u << 3);
+#pragma unroll
+                        for (int p = 0; p < 2; ++p) {
+                            sts64f(hrow + p * 256 + oA, make_float2(prev[p].x, sum[p].x));
+                            sts64f(hrow + p * 256 + oB, make_float2(sum[p].y, prev[p].y));
+                        }
+                    } else {
+                        prev[0] = sum[0];
+                        prev[1] = sum[1];
+                    }
                 }
+                if (!SECOND) tmem::st_x16(tcol + 32 * q + 16 * hh, tv);
             }
         }
         return true;
@@ -382,40 +420,76 @@ __global__ void __launch_bounds__(THREADS, 1)
             __nv_bfloat16* const oA_row = outp + (8 * q) * S;
             __nv_bfloat16* const oB_row = outp + (S - 1 - 8 * q) * S;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
-                float2 base[2];
-                base[0].x = fma_bf_lo(LA[e], XA[e], h[0].x);
-                base[1].x = fma_bf_hi(LA[e], XA[e], h[1].x);
-                base[0].y = fma_bf_lo(LB[e], XB[e], h[0].y);
-                base[1].y = fma_bf_hi(LB[e], XB[e], h[1].y);
-                scan_core(h, base, wr[e]);
-                const uint32_t oA = (k8 + (uint32_t)((e >> 1) << 3)) ^ t8;
-                const uint32_t oB = oA ^ (15u << 3);
-                unsigned char* adA = hA + e * 256 + oA;
-                unsigned char* adB = hB - e * 256 + oB;
-                const float2 vA = __fadd2_rn(lds64f(adA), make_float2(h[0].x, h[1].x));
-                const float2 vB = __fadd2_rn(lds64f(adB), make_float2(h[0].y, h[1].y));
-                if (!SECOND) {  // first arrival of this pass: keep the partial sum
-                    sts64f(adA, vA);
-                    sts64f(adB, vB);
-                } else {        // second arrival: the pixel is complete
-                    stg_cs32(oA_row + e * S, pack_bf2(vA.x, vA.y));
-                    stg_cs32(oB_row - e * S, pack_bf2(vB.x, vB.y));
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t tv[16];  // first arrivals of a half chunk: [step][top->bottom, bottom->top][position]
+                if (SECOND) {
+                    tmem::ld_x16(tcol + 32 * (7 - q) + 16 * (1 - hh), tv);
+                    tmem::wait_ld16(tv);
                 }
+#pragma unroll
+                for (int ee = 0; ee < 4; ++ee) {
+                    const int e = 4 * hh + ee;
+                    if (LOCAL && ((8 * q + e) & segmask) == 0) h[0] = h[1] = make_float2(0.f, 0.f);
+                    float2 base[2];
+                    base[0].x = fma_bf_lo(LA[e], XA[e], h[0].x);
+                    base[1].x = fma_bf_hi(LA[e], XA[e], h[1].x);
+                    base[0].y = fma_bf_lo(LB[e], XB[e], h[0].y);
+                    base[1].y = fma_bf_hi(LB[e], XB[e], h[1].y);
+                    scan_core(h, base, wr[e]);
+                    if (!SECOND) {
+                        // first arrival of this pass: the row sum of the pixel plus this
+                        // direction's value, parked in TMEM
+                        const uint32_t oA = (k8 + (uint32_t)((e >> 1) << 3)) ^ t8;
+                        const uint32_t oB = oA ^ (15u << 3);
+                        const float2 vA = __fadd2_rn(lds64f(hA + e * 256 + oA), make_float2(h[0].x, h[1].x));
+                        const float2 vB = __fadd2_rn(lds64f(hB - e * 256 + oB), make_float2(h[0].y, h[1].y));
+                        tv[ee * 4 + 0] = __float_as_uint(vA.x);
+                        tv[ee * 4 + 1] = __float_as_uint(vA.y);
+                        tv[ee * 4 + 2] = __float_as_uint(vB.x);
+                        tv[ee * 4 + 3] = __float_as_uint(vB.y);
+                    } else {
+                        // second arrival: top->bottom at row s meets bottom->top's first
+                        // arrival there (element 3-ee of the loaded half), and vice versa
+                        const int f = (3 - ee) * 4;
+                        const float2 vA = __fadd2_rn(make_float2(__uint_as_float(tv[f + 2]), __uint_as_float(tv[f + 3])),
+                                                     make_float2(h[0].x, h[1].x));
+                        const float2 vB = __fadd2_rn(make_float2(__uint_as_float(tv[f]), __uint_as_float(tv[f + 1])),
+                                                     make_float2(h[0].y, h[1].y));
+                        stg_cs32(oA_row + e * S, pack_bf2(vA.x, vA.y));
+                        stg_cs32(oB_row - e * S, pack_bf2(vB.x, vB.y));
+                    }
+                }
+                if (!SECOND) tmem::st_x16(tcol + 32 * q + 16 * hh, tv);
             }
         }
         return true;
     };
 
-    for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
+    bool ok = true;
+    for (int group = blockIdx.x; ok && group < a.groups; group += gridDim.x) {
         outp = a.out + (size_t)(8 * group + warp) * S * S + 2 * t;
         h[0] = h[1] = make_float2(0.f, 0.f);
-        if (!row_half(std::false_type{}) || !row_half(std::true_type{})) { fail(); return; }
+        ok = row_half(std::false_type{});
+        tmem::wait_st();  // the second half reads what the first half parked
+        ok = ok && row_half(std::true_type{});
         __syncwarp();
         h[0] = h[1] = make_float2(0.f, 0.f);
-        if (!col_half(std::false_type{}) || !col_half(std::true_type{})) { fail(); return; }
+        ok = ok && col_half(std::false_type{});
+        tmem::wait_st();
+        ok = ok && col_half(std::true_type{});
         __syncwarp();
+    }
+    if (!ok) fail();
+    // this warp no longer touches the tensor memory; warp 0 frees it after all
+    tmem::wait_st();
+    tmem::fence_before();
+    __syncwarp();
+    if (t == 0) tma::mbar_arrive(done0);
+    if (warp == 0) {
+        if (!tma::mbar_wait(done0, 0, 10 * tma::kTimeoutNs) && t == 0) atomicExch(a.err, 1);
+        __syncwarp();
+        tmem::fence_after();
+        tmem::dealloc(taddr, 256);
     }
 }
 
