@@ -72,6 +72,17 @@ gspn_status check_ws(void* ws, size_t have, size_t need) {
     return GSPN_OK;
 }
 
+// The kernel family a descriptor runs on: the TMA-fed compact kernels for their
+// shapes, the one-CTA-per-plane kernels for planes of at most 64x64, the generic
+// kernels for everything else.
+enum class Path { kC64, kC128, kSmall, kGeneric };
+Path pick(const Problem& p, int backward) {
+    if (backward ? c64_bwd_eligible(p) : c64_eligible(p)) return Path::kC64;
+    if (backward ? c128_bwd_eligible(p) : c128_eligible(p)) return Path::kC128;
+    if (small_eligible(p, backward)) return Path::kSmall;
+    return Path::kGeneric;
+}
+
 }  // namespace
 
 cudaError_t device_info(DeviceInfo* out) {
@@ -139,30 +150,34 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     if (validate(desc, &p) != GSPN_OK) return 0;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return 0;
-    if (backward) {
-        if (c64_bwd_eligible(p)) return c64_bwd_workspace(p, dev);
-        return c128_bwd_eligible(p) ? c128_bwd_workspace(p, dev) : generic_bwd_workspace(p, dev);
+    switch (pick(p, backward)) {
+    case Path::kC64: return backward ? c64_bwd_workspace(p, dev) : c64_fwd_workspace(p);
+    case Path::kC128: return backward ? c128_bwd_workspace(p, dev) : c128_fwd_workspace(p, dev);
+    case Path::kSmall: return backward ? small_bwd_workspace(p) : 0;
+    default: return backward ? generic_bwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
     }
-    if (c64_eligible(p)) return c64_fwd_workspace(p);
-    return c128_eligible(p) ? c128_fwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
 }
 
 int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return 0;
-    if (backward) return c64_bwd_eligible(p) || c128_bwd_eligible(p) ? 3 : generic_bwd_launches(p);
-    return c64_eligible(p) || c128_eligible(p) ? 2 : 1;
+    switch (pick(p, backward)) {
+    case Path::kC64:
+    case Path::kC128: return backward ? 3 : 2;
+    case Path::kSmall: return backward ? small_bwd_launches(p) : 1;
+    default: return backward ? generic_bwd_launches(p) : 1;
+    }
 }
 
 const char* gspn_variant_name(const gspn_desc* desc, int backward) {
     Problem p;
     if (validate(desc, &p) != GSPN_OK) return "invalid";
-    if (backward) {
-        if (c64_bwd_eligible(p)) return "compact64_tma_bwd";
-        return c128_bwd_eligible(p) ? "compact128_tma_bwd" : "generic_bwd";
+    switch (pick(p, backward)) {
+    case Path::kC64: return backward ? "compact64_tma_bwd" : "compact64_tma_fwd";
+    case Path::kC128: return backward ? "compact128_tma_bwd" : "compact128_tma_fwd";
+    case Path::kSmall: return backward ? "small_plane_bwd" : "small_plane_fwd";
+    default: return backward ? "generic_bwd" : "generic_fwd";
     }
-    if (c64_eligible(p)) return "compact64_tma_fwd";
-    return c128_eligible(p) ? "compact128_tma_fwd" : "generic_fwd";
 }
 
 gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda, void* out,
@@ -174,12 +189,17 @@ gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, c
     if (st != GSPN_OK) return st;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
-    const bool fast = c64_eligible(p), fast128 = !fast && c128_eligible(p);
+    const Path path = pick(p, 0);
     st = check_ws(workspace, ws_bytes,
-                  fast ? c64_fwd_workspace(p) : fast128 ? c128_fwd_workspace(p, dev) : generic_fwd_workspace(p, dev));
+                  path == Path::kC64    ? c64_fwd_workspace(p)
+                  : path == Path::kC128 ? c128_fwd_workspace(p, dev)
+                  : path == Path::kSmall ? 0
+                                         : generic_fwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
-    if (fast) return c64_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
-    if (fast128) return c128_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (path == Path::kC64) return c64_fwd(p, dev, x, logits, lambda, out, workspace, cs);
+    if (path == Path::kC128) return c128_fwd(p, dev, x, logits, lambda, out, workspace, cs);
+    if (path == Path::kSmall) return small_fwd(p, dev, x, logits, lambda, out, cs);
     return generic_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
 }
 
@@ -205,18 +225,17 @@ gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, c
     if (st != GSPN_OK) return st;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
-    const bool fast = c64_bwd_eligible(p), fast128 = !fast && c128_bwd_eligible(p);
+    const Path path = pick(p, 1);
     st = check_ws(workspace, ws_bytes,
-                  fast      ? c64_bwd_workspace(p, dev)
-                  : fast128 ? c128_bwd_workspace(p, dev)
-                            : generic_bwd_workspace(p, dev));
+                  path == Path::kC64     ? c64_bwd_workspace(p, dev)
+                  : path == Path::kC128  ? c128_bwd_workspace(p, dev)
+                  : path == Path::kSmall ? small_bwd_workspace(p)
+                                         : generic_bwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
-    if (fast)
-        return c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
-                       static_cast<cudaStream_t>(stream));
-    if (fast128)
-        return c128_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
-                        static_cast<cudaStream_t>(stream));
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    if (path == Path::kC64) return c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
+    if (path == Path::kC128) return c128_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
+    if (path == Path::kSmall) return small_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
     return generic_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
                        static_cast<cudaStream_t>(stream));
 }

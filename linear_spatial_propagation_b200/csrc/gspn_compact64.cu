@@ -358,35 +358,35 @@ __global__ void __launch_bounds__(THREADS, 1)
                                            h[p].y);
                     }
                     scan_core(h, base, wr[e]);
-                    if (!SECOND) {
+                    if constexpr (!SECOND) {
 #pragma unroll
                         for (int p = 0; p < 2; ++p) {
                             tv[ee * 4 + p * 2] = __float_as_uint(h[p].x);
                             tv[ee * 4 + p * 2 + 1] = __float_as_uint(h[p].y);
                         }
-                        continue;
-                    }
-                    // left->right at column s meets right->left's first arrival there
-                    // (element 3-ee of the loaded half), right->left at column 63-s
-                    // meets left->right's: the completed row sums
-                    float2 sum[2];
-#pragma unroll
-                    for (int p = 0; p < 2; ++p)
-                        sum[p] = __fadd2_rn(h[p], make_float2(__uint_as_float(tv[(3 - ee) * 4 + p * 2 + 1]),
-                                                              __uint_as_float(tv[(3 - ee) * 4 + p * 2])));
-                    if (e & 1) {
-                        // left->right covers columns s-1, s (unit s/2 = 4q + e/2), right->left
-                        // columns 63-s, 64-s (unit 31 - (4q + e/2)); XOR with the row key
-                        const uint32_t oA = (q8 + (uint32_t)((e >> 1) << 3)) ^ tk8;
-                        const uint32_t oB = oA ^ (31u << 3);
-#pragma unroll
-                        for (int p = 0; p < 2; ++p) {
-                            sts64f(hrow + p * 256 + oA, make_float2(prev[p].x, sum[p].x));
-                            sts64f(hrow + p * 256 + oB, make_float2(sum[p].y, prev[p].y));
-                        }
                     } else {
-                        prev[0] = sum[0];
-                        prev[1] = sum[1];
+                        // left->right at column s meets right->left's first arrival there
+                        // (element 3-ee of the loaded half), right->left at column 63-s
+                        // meets left->right's: the completed row sums
+                        float2 sum[2];
+#pragma unroll
+                        for (int p = 0; p < 2; ++p)
+                            sum[p] = __fadd2_rn(h[p], make_float2(__uint_as_float(tv[(3 - ee) * 4 + p * 2 + 1]),
+                                                                  __uint_as_float(tv[(3 - ee) * 4 + p * 2])));
+                        if (e & 1) {
+                            // left->right covers columns s-1, s (unit s/2 = 4q + e/2), right->left
+                            // columns 63-s, 64-s (unit 31 - (4q + e/2)); XOR with the row key
+                            const uint32_t oA = (q8 + (uint32_t)((e >> 1) << 3)) ^ tk8;
+                            const uint32_t oB = oA ^ (31u << 3);
+#pragma unroll
+                            for (int p = 0; p < 2; ++p) {
+                                sts64f(hrow + p * 256 + oA, make_float2(prev[p].x, sum[p].x));
+                                sts64f(hrow + p * 256 + oB, make_float2(sum[p].y, prev[p].y));
+                            }
+                        } else {
+                            prev[0] = sum[0];
+                            prev[1] = sum[1];
+                        }
                     }
                 }
                 if (!SECOND) tmem::st_x16(tcol + 32 * q + 16 * hh, tv);

@@ -41,6 +41,15 @@ gspn_status generic_bwd(const Problem& p, const DeviceInfo& dev, const void* x, 
                         const void* lam, const void* dout, void* dx, void* dlogits, void* dlam, void* ws,
                         cudaStream_t s);
 
+// ---- planes of at most 64x64, any mode: one CTA per plane, one warp per direction ----
+bool small_eligible(const Problem& p, int backward);
+size_t small_bwd_workspace(const Problem& p);
+int small_bwd_launches(const Problem& p);
+gspn_status small_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                      void* out, cudaStream_t s);
+gspn_status small_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                      const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s);
+
 // ---- compact 64x64 bf16 forward (TMA-fed, packed fp32x2) ------------------------
 bool c64_eligible(const Problem& p);
 size_t c64_fwd_workspace(const Problem& p);

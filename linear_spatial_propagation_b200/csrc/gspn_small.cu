@@ -1,0 +1,436 @@
+// gspn_small.cu -- GSPN forward and backward for planes of at most 64x64, in
+// any dtype, direction set, local-group count and weight mode (per-channel
+// taps in particular: the tiny-backbone 56x56 and local 28x28 stages of
+// "Parallel Sequence Modeling via Generalized Spatial Propagation Network").
+//
+// One CTA per (b, c) plane, one warp per enabled direction: the four scans of
+// a plane (Key design 2) run side by side instead of one after the other, and
+// each keeps its own fp32 copy of the plane in shared memory, summed in
+// direction order at the end (the merge), so the result does not depend on
+// timing.  Lane l holds positions l (and l+32: P = 2) of a line; the previous line sits
+// in a shared line buffer with a zero halo, so tap k of position j reads slot
+// j+k.  The tap weights are recomputed from the logits where they are used:
+// s_k = sigmoid(logit_k) on the taps whose source lies in the line, w_k =
+// s_k / sum s (Key design 1).
+//
+// Inputs are read 8 lines at a time (4 with one position per lane): each lane
+// loads its positions' values of those lines in one go.  For a row scan the lanes of a warp read along a
+// row; for a column scan each lane reads the neighbouring pixels of its row,
+// with 8-byte loads where the pieces are aligned.
+//
+// Backward: per direction, the lines are recomputed into shared memory, then
+// the adjoint runs from the last line to the first with the transposed taps
+// ("GSPN-2: Efficient Parallel Sequence Modeling", Backward Benchmark):
+//   a_i[j] = G_i[j] + sum_k w_{i+1}[j-k+1][k] a_{i+1}[j-k+1]  (no carry into a
+//            line whose successor starts a group),
+//   dx += lambda a, dlambda = x a, dw_k = a h_{i-1}[j+k-1],
+//   dlogit_k = s_k (1 - s_k) / S (dw_k - sum_m w_m dw_m)  (valid taps; 0 else).
+// dx is summed over the directions in shared memory, in direction order.
+#include "gspn_internal.h"
+
+namespace gspn {
+
+namespace {
+
+constexpr int kLS = 66;    // line buffer: up to 64 positions + a zero halo at each end
+// lines whose inputs are loaded together: 8 with two positions per lane, 4 with
+// one (fewer registers, more CTAs per SM for the many small planes)
+template <int P>
+__host__ __device__ constexpr int chunk_of() { return P == 1 ? 4 : 8; }
+constexpr int kSmallSmemCap = 200 * 1024;
+
+struct SmallArgs {
+    Launch g;
+    const void* x;
+    const void* logits;
+    const void* lam;
+    const void* dout;
+    void* out;      // forward
+    void* dx;       // backward
+    void* dlogits;
+    void* dlam;
+    float* dlog_ws;  // backward, shared taps: fp32 sums over channels [D][B][3][HW]
+};
+
+// the normalised taps of position j (valid ones only) from the raw logits
+__device__ __forceinline__ void taps(float g0, float g1, float g2, int j, int N, float& s0, float& s1, float& s2) {
+    s0 = j > 0 ? sigmoidf(g0) : 0.f;
+    s1 = sigmoidf(g1);
+    s2 = j < N - 1 ? sigmoidf(g2) : 0.f;
+}
+
+// For a column scan the CH values of one position over lines i0, i0+1, ...
+// (DOWN: i0, i0-1, ...) are CH neighbouring pixels of one row.  This reads
+// them with 8-byte loads and returns true when the piece is whole and aligned.
+template <int CH, bool DOWN, typename T>
+__device__ __forceinline__ bool load_row_piece(const T* src, int d, int W, int L, int i0, int j, float (&v)[CH]) {
+    constexpr int kPer = 8 / (int)sizeof(T);  // elements per 8-byte load
+    static_assert(CH % kPer == 0, "whole 8-byte loads");
+    const int ilo = DOWN ? i0 - (CH - 1) : i0;  // the lowest line of the chunk
+    if (ilo < 0 || ilo + CH > L) return false;
+    // pixels of lines ilo..ilo+7: ascending columns for left->right, descending for right->left
+    const int first = d == L2R ? j * W + ilo : j * W + (W - CH - ilo);
+    if ((reinterpret_cast<uintptr_t>(src + first) & 7u) != 0) return false;
+    float t[CH];
+#pragma unroll
+    for (int u = 0; u < CH / kPer; ++u) {
+        const uint2 w = __ldg(reinterpret_cast<const uint2*>(src + first) + u);
+        if constexpr (sizeof(T) == 4) {
+            t[2 * u] = __uint_as_float(w.x);
+            t[2 * u + 1] = __uint_as_float(w.y);
+        } else {
+            t[4 * u] = __uint_as_float(w.x << 16);
+            t[4 * u + 1] = __uint_as_float(w.x & 0xffff0000u);
+            t[4 * u + 2] = __uint_as_float(w.y << 16);
+            t[4 * u + 3] = __uint_as_float(w.y & 0xffff0000u);
+        }
+    }
+    // t[m] is line ilo + m (left->right) or ilo + CH-1 - m (right->left); two
+    // branches keep every index a compile-time constant
+    if (d == L2R) {
+#pragma unroll
+        for (int e = 0; e < CH; ++e) v[e] = t[DOWN ? CH - 1 - e : e];
+    } else {
+#pragma unroll
+        for (int e = 0; e < CH; ++e) v[e] = t[DOWN ? e : CH - 1 - e];
+    }
+    return true;
+}
+
+// The chunk's inputs of lane positions j = lane + 32r: NT planes (x, lambda, the
+// three logits, and dout in the backward) at lines i0 +- e.  Column scans use the
+// row-piece loads when every plane's piece is aligned (the planes share the
+// row offsets, so one test decides); otherwise one pixel index per (r, e) serves
+// all planes.
+template <int CH, bool DOWN, int P, int NT, typename T>
+__device__ __forceinline__ void load_chunk(const T* const (&src)[NT], int d, int H, int W, int L, int N, int i0,
+                                           int lane, float (&v)[NT][P][CH]) {
+#pragma unroll
+    for (int r = 0; r < P; ++r) {
+        const int j = lane + 32 * r;
+        bool done = false;
+        if ((d == L2R || d == R2L) && j < N) {
+            done = true;
+#pragma unroll
+            for (int k = 0; k < NT; ++k) done = done && load_row_piece<CH, DOWN>(src[k], d, W, L, i0, j, v[k][r]);
+        }
+        if (!done) {
+#pragma unroll
+            for (int e = 0; e < CH; ++e) {
+                const int i = DOWN ? i0 - e : i0 + e;
+                const bool in = j < N && i >= 0 && i < L;
+                const int p = in ? pix(d, H, W, i, j) : 0;  // in bounds for idle lanes
+#pragma unroll
+                for (int k = 0; k < NT; ++k) v[k][r][e] = in ? load_elt(src[k], p) : 0.f;
+            }
+        }
+    }
+}
+
+template <typename T, int P>
+__global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
+    constexpr int CH = chunk_of<P>();
+    extern __shared__ float smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C, D = a.g.D;
+    const int64_t plane = blockIdx.x;
+    const int64_t b = plane / C, c = plane % C, cw = a.g.shared ? 0 : c;
+    const int Cw = a.g.shared ? 1 : C;
+    float* const acc = smem + (size_t)warp * HW;  // this direction's copy of the plane
+    float* hp = smem + (size_t)D * HW + (size_t)warp * 2 * kLS;
+    float* hc = hp + kLS;
+
+    // (a select, not an index, keeps the parameter block out of local memory)
+    const int slot = warp, d = slot == 0 ? a.g.dirs[0] : slot == 1 ? a.g.dirs[1] : slot == 2 ? a.g.dirs[2] : a.g.dirs[3];
+    const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
+    const T* x = static_cast<const T*>(a.x) + plane * HW;
+    const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
+    const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+    const T* const srcs[5] = {x, lam, lg, lg + HW, lg + 2 * HW};
+    if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
+    __syncwarp();
+
+    for (int i0 = 0; i0 < L; i0 += CH) {
+        float vin[5][P][CH];
+        load_chunk<CH, false, P, 5>(srcs, d, H, W, L, N, i0, lane, vin);
+        auto& vx = vin[0];
+        auto& vl = vin[1];
+        auto& v0 = vin[2];
+        auto& v1 = vin[3];
+        auto& v2 = vin[4];
+#pragma unroll
+        for (int e = 0; e < CH; ++e) {
+            const int i = i0 + e;
+            if (i >= L) break;
+            const bool carry = (i % seg) != 0;
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                const int j = lane + 32 * r;
+                if (j < N) {
+                    float v = vl[r][e] * vx[r][e];
+                    if (carry) {
+                        float s0, s1, s2;
+                        taps(v0[r][e], v1[r][e], v2[r][e], j, N, s0, s1, s2);
+                        v += (s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2]) / (s0 + s1 + s2);
+                    }
+                    hc[j + 1] = v;
+                    acc[pix(d, H, W, i, j)] = v;
+                }
+            }
+            __syncwarp();
+            float* t = hp;
+            hp = hc;
+            hc = t;
+        }
+    }
+    __syncthreads();
+    // the merge: the directions' planes summed in direction order, one store per pixel
+    T* out = static_cast<T*>(a.out) + plane * HW;
+    for (int q = threadIdx.x; q < HW; q += blockDim.x) {
+        float s = smem[q];
+        for (int k = 1; k < D; ++k) s += smem[(size_t)k * HW + q];
+        store_elt(out, q, s);
+    }
+}
+
+template <typename T, int P>
+__global__ void __launch_bounds__(128) small_bwd_kernel(SmallArgs a) {
+    constexpr int CH = chunk_of<P>();
+    extern __shared__ float smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C, D = a.g.D;
+    const int64_t plane = blockIdx.x;
+    const int64_t b = plane / C, c = plane % C, cw = a.g.shared ? 0 : c;
+    const int Cw = a.g.shared ? 1 : C;
+    float* const hst = smem + (size_t)warp * HW;                 // this direction's lines, scan coordinates
+    float* const dxacc = smem + (size_t)(D + warp) * HW;         // this direction's share of dx
+    float* const lb = smem + (size_t)2 * D * HW + (size_t)warp * 6 * kLS;  // line buffers
+
+    // (a select, not an index, keeps the parameter block out of local memory)
+    const int slot = warp, d = slot == 0 ? a.g.dirs[0] : slot == 1 ? a.g.dirs[1] : slot == 2 ? a.g.dirs[2] : a.g.dirs[3];
+    const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
+    const T* x = static_cast<const T*>(a.x) + plane * HW;
+    const T* g = static_cast<const T*>(a.dout) + plane * HW;
+    const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
+    const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+    T* dlam = static_cast<T*>(a.dlam) + ((slot * (int64_t)B + b) * C + c) * HW;
+    const T* const srcs[5] = {x, lam, lg, lg + HW, lg + 2 * HW};
+    const T* const srcs6[6] = {g, x, lam, lg, lg + HW, lg + 2 * HW};
+
+    // 1. recompute this direction's lines into shared memory
+    {
+        float* hp = lb;
+        float* hc = lb + kLS;
+        if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
+        __syncwarp();
+        for (int i0 = 0; i0 < L; i0 += CH) {
+            float vin[5][P][CH];
+            load_chunk<CH, false, P, 5>(srcs, d, H, W, L, N, i0, lane, vin);
+            auto& vx = vin[0];
+            auto& vl = vin[1];
+            auto& v0 = vin[2];
+            auto& v1 = vin[3];
+            auto& v2 = vin[4];
+#pragma unroll
+            for (int e = 0; e < CH; ++e) {
+                const int i = i0 + e;
+                if (i >= L) break;
+                const bool carry = (i % seg) != 0;
+#pragma unroll
+                for (int r = 0; r < P; ++r) {
+                    const int j = lane + 32 * r;
+                    if (j < N) {
+                        float v = vl[r][e] * vx[r][e];
+                        if (carry) {
+                            float s0, s1, s2;
+                            taps(v0[r][e], v1[r][e], v2[r][e], j, N, s0, s1, s2);
+                            v += (s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2]) / (s0 + s1 + s2);
+                        }
+                        hc[j + 1] = v;
+                        hst[i * N + j] = v;
+                    }
+                }
+                __syncwarp();
+                float* t = hp;
+                hp = hc;
+                hc = t;
+            }
+        }
+    }
+
+    // 2. the adjoint from the last line to the first; the products w_k a of the
+    //    line below wait in three line buffers (zero halos) for its predecessor
+    float* qn = lb;
+    float* qc = lb + 3 * kLS;
+    for (int q = lane; q < 6 * kLS; q += 32) lb[q] = 0.f;
+    __syncwarp();
+    for (int it = 0; it < L; it += CH) {
+        // lines i = L-1-it-e, e < CH
+        float vin[6][P][CH];
+        load_chunk<CH, true, P, 6>(srcs6, d, H, W, L, N, L - 1 - it, lane, vin);
+        auto& vg = vin[0];
+        auto& vx = vin[1];
+        auto& vl = vin[2];
+        auto& v0 = vin[3];
+        auto& v1 = vin[4];
+        auto& v2 = vin[5];
+#pragma unroll
+        for (int e = 0; e < CH; ++e) {
+            const int i = L - 1 - it - e;
+            if (i < 0) break;
+            const bool carry_out = (i % seg) != 0;                      // line i reads line i-1
+            const bool carry_in = (i + 1 < L) && ((i + 1) % seg != 0);  // line i+1 read line i
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                const int j = lane + 32 * r;
+                if (j < N) {
+                    const int p = pix(d, H, W, i, j);
+                    float av = vg[r][e];
+                    if (carry_in) av += qn[j + 2] + qn[kLS + j + 1] + qn[2 * kLS + j];
+                    dxacc[p] = vl[r][e] * av;
+                    store_elt(dlam, p, vx[r][e] * av);
+                    float dl0 = 0.f, dl1 = 0.f, dl2 = 0.f, q0 = 0.f, q1 = 0.f, q2 = 0.f;
+                    if (carry_out) {
+                        float s0, s1, s2;
+                        taps(v0[r][e], v1[r][e], v2[r][e], j, N, s0, s1, s2);
+                        const float rs = 1.f / (s0 + s1 + s2);
+                        const float* hprev = hst + (i - 1) * N;
+                        const float dw0 = j > 0 ? av * hprev[j - 1] : 0.f;
+                        const float dw1 = av * hprev[j];
+                        const float dw2 = j < N - 1 ? av * hprev[j + 1] : 0.f;
+                        // dw_k - sum_m w_m dw_m = sum_m w_m (dw_k - dw_m), since the w sum to 1
+                        const float r2 = rs * rs;
+                        dl0 = s0 * (1.f - s0) * r2 * (s1 * (dw0 - dw1) + s2 * (dw0 - dw2));
+                        dl1 = s1 * (1.f - s1) * r2 * (s0 * (dw1 - dw0) + s2 * (dw1 - dw2));
+                        dl2 = s2 * (1.f - s2) * r2 * (s0 * (dw2 - dw0) + s1 * (dw2 - dw1));
+                        q0 = s0 * rs * av;
+                        q1 = s1 * rs * av;
+                        q2 = s2 * rs * av;
+                    }
+                    qc[j + 1] = q0;
+                    qc[kLS + j + 1] = q1;
+                    qc[2 * kLS + j + 1] = q2;
+                    if (a.g.shared) {
+                        if (carry_out) {
+                            float* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
+                            if (j > 0) atomicAdd(dw + p, dl0);
+                            atomicAdd(dw + HW + p, dl1);
+                            if (j < N - 1) atomicAdd(dw + 2 * HW + p, dl2);
+                        }
+                    } else {
+                        T* dlg = static_cast<T*>(a.dlogits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+                        store_elt(dlg, p, dl0);
+                        store_elt(dlg, HW + p, dl1);
+                        store_elt(dlg, 2 * HW + p, dl2);
+                    }
+                }
+            }
+            __syncwarp();
+            float* t = qn;
+            qn = qc;
+            qc = t;
+        }
+    }
+    __syncthreads();
+    // dx: the directions' shares summed in direction order
+    T* dx = static_cast<T*>(a.dx) + plane * HW;
+    for (int q = threadIdx.x; q < HW; q += blockDim.x) {
+        float s = smem[(size_t)D * HW + q];
+        for (int k = 1; k < D; ++k) s += smem[(size_t)(D + k) * HW + q];
+        store_elt(dx, q, s);
+    }
+}
+
+__global__ void small_zero_kernel(float* p, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = 0.f;
+}
+
+template <typename T>
+__global__ void small_convert_kernel(const float* src, T* dst, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+        store_elt(dst, i, src[i]);
+}
+
+size_t fwd_smem(const Problem& p) { return ((size_t)p.g.D * p.HW + (size_t)p.g.D * 2 * kLS) * sizeof(float); }
+size_t bwd_smem(const Problem& p) { return ((size_t)2 * p.g.D * p.HW + (size_t)p.g.D * 6 * kLS) * sizeof(float); }
+unsigned grid_1d(int64_t n) {
+    const int64_t g = (n + 255) / 256;
+    return (unsigned)(g < 4096 ? (g > 0 ? g : 1) : 4096);
+}
+
+}  // namespace
+
+// (the shared-memory cap is below what every sm_100 device lets a block opt in to)
+bool small_eligible(const Problem& p, int backward) {
+    if (p.g.H > 64 || p.g.W > 64 || p.planes > 0x7fffffff) return false;
+    return (backward ? bwd_smem(p) : fwd_smem(p)) <= (size_t)kSmallSmemCap;
+}
+
+size_t small_bwd_workspace(const Problem& p) {
+    return p.g.shared ? align_up((size_t)p.g.D * p.g.B * 3 * p.HW * sizeof(float), kWsAlign) : 0;
+}
+
+int small_bwd_launches(const Problem& p) { return p.g.shared ? 3 : 1; }
+
+gspn_status small_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                      void* out, cudaStream_t s) {
+    (void)dev;
+    SmallArgs a{};
+    a.g = p.g;
+    a.x = x;
+    a.logits = logits;
+    a.lam = lam;
+    a.out = out;
+    const bool f32 = p.d.dtype == GSPN_F32, one = (p.g.H > p.g.W ? p.g.H : p.g.W) <= 32;
+    // one position per lane when every line fits in 32 lanes: half the registers
+    const void* fn = f32 ? (one ? (const void*)small_fwd_kernel<float, 1> : (const void*)small_fwd_kernel<float, 2>)
+                         : (one ? (const void*)small_fwd_kernel<__nv_bfloat16, 1>
+                                : (const void*)small_fwd_kernel<__nv_bfloat16, 2>);
+    const int smem = (int)fwd_smem(p);
+    if (ensure_smem_attr(fn, smem, (f32 ? 22 : 23) + (one ? 4 : 0)) != cudaSuccess) return GSPN_ERR_CUDA;
+    void* args[] = {&a};
+    if (cudaLaunchKernel(fn, dim3((unsigned)p.planes), dim3(32 * p.g.D), args, smem, s) != cudaSuccess)
+        return GSPN_ERR_CUDA;
+    return cudaGetLastError() == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+}
+
+gspn_status small_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                      const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s) {
+    (void)dev;
+    SmallArgs a{};
+    a.g = p.g;
+    a.x = x;
+    a.logits = logits;
+    a.lam = lam;
+    a.dout = dout;
+    a.dx = dx;
+    a.dlogits = dlogits;
+    a.dlam = dlam;
+    a.dlog_ws = static_cast<float*>(ws);
+    const int64_t nlog = (int64_t)p.g.D * p.g.B * 3 * p.HW;
+    if (p.g.shared) {
+        small_zero_kernel<<<grid_1d(nlog), 256, 0, s>>>(a.dlog_ws, nlog);
+        if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
+    }
+    const bool f32 = p.d.dtype == GSPN_F32, one = (p.g.H > p.g.W ? p.g.H : p.g.W) <= 32;
+    const void* fn = f32 ? (one ? (const void*)small_bwd_kernel<float, 1> : (const void*)small_bwd_kernel<float, 2>)
+                         : (one ? (const void*)small_bwd_kernel<__nv_bfloat16, 1>
+                                : (const void*)small_bwd_kernel<__nv_bfloat16, 2>);
+    const int smem = (int)bwd_smem(p);
+    if (ensure_smem_attr(fn, smem, (f32 ? 24 : 25) + (one ? 4 : 0)) != cudaSuccess) return GSPN_ERR_CUDA;
+    void* args[] = {&a};
+    if (cudaLaunchKernel(fn, dim3((unsigned)p.planes), dim3(32 * p.g.D), args, smem, s) != cudaSuccess)
+        return GSPN_ERR_CUDA;
+    if (p.g.shared) {
+        if (f32)
+            small_convert_kernel<float><<<grid_1d(nlog), 256, 0, s>>>(a.dlog_ws, static_cast<float*>(dlogits), nlog);
+        else
+            small_convert_kernel<__nv_bfloat16>
+                <<<grid_1d(nlog), 256, 0, s>>>(a.dlog_ws, static_cast<__nv_bfloat16*>(dlogits), nlog);
+        if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
+    }
+    return GSPN_OK;
+}
+
+}  // namespace gspn

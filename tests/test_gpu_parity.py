@@ -290,3 +290,42 @@ def test_compact128_backward_dispatch_and_guards():
     gu.assert_close(gu.from_dev(views[0]), rdx, w.dtype, "dx")
     gu.assert_close(gu.from_dev(views[1]), rdlg, w.dtype, "dlogits")
     gu.assert_close(gu.from_dev(views[2]), rdlam, w.dtype, "dlam")
+
+
+@pytest.mark.parametrize("case", [(1, 3, 56, 56, 15, 1, False, "f32"), (2, 5, 40, 24, 15, 4, True, "bf16"),
+                                  (1, 4, 28, 28, 5, 7, False, "bf16"), (1, 2, 64, 64, 10, 1, False, "f32")],
+                         ids=lambda c: "x".join(map(str, c)))
+def test_small_plane_dispatch_guards_and_parity(case):
+    """Planes of at most 64x64 run on the one-CTA-per-plane kernels: their
+    dispatch, canaries around every output, and the oracle's results (both
+    passes, per-channel and shared taps, local groups, partial direction sets,
+    aligned and unaligned rows)."""
+    import linear_spatial_propagation_b200 as lsp
+    t = gu.torch()
+    w = shape_workload(*case, seed=700 + sum(case[:4]))
+    d = lsp.make_desc(w.B, w.C, w.H, w.W, w.dir_mask, w.groups, w.shared, w.dtype)
+    assert lsp.gspn_variant_name(d, 0) == "small_plane_fwd"
+    assert lsp.gspn_variant_name(d, 1) == "small_plane_bwd"
+    inp = synth.make_inputs(w, with_dout=True)
+    dinp = gu.dev_inputs(w, inp)
+    tdt = dinp["x"].dtype
+    guard = 4096
+
+    def guarded(like):
+        buf = t.full((like.numel() + 2 * guard,), -3.0, dtype=tdt, device="cuda")
+        return buf, buf[guard:guard + like.numel()].view(like.shape)
+
+    ob, out = guarded(dinp["x"])
+    lsp.forward(dinp["x"], dinp["logits"], dinp["lam"], dir_mask=w.dir_mask, groups=w.groups, shared=w.shared,
+                out=out)
+    grads = [guarded(x) for x in (dinp["x"], dinp["logits"], dinp["lam"])]
+    lsp.backward(dinp["x"], dinp["logits"], dinp["lam"], dinp["dout"], dir_mask=w.dir_mask, groups=w.groups,
+                 shared=w.shared, grads=tuple(v for _, v in grads))
+    t.cuda.synchronize()
+    for b, v in [(ob, out)] + grads:
+        assert bool((b[:guard] == -3.0).all()) and bool((b[guard + v.numel():] == -3.0).all())
+    gu.assert_close(gu.from_dev(out), oracle.fwd_workload(w, inp), w.dtype, "small-plane forward")
+    rdx, rdlg, rdlam = oracle.bwd_workload(w, inp)
+    gu.assert_close(gu.from_dev(grads[0][1]), rdx, w.dtype, "dx")
+    gu.assert_close(gu.from_dev(grads[1][1]), rdlg, w.dtype, "dlogits")
+    gu.assert_close(gu.from_dev(grads[2][1]), rdlam, w.dtype, "dlam")
