@@ -104,3 +104,40 @@ def test_python_helpers_raise_on_error():
         st = fwd(lsp.make_desc(1, 1, 4, 4, dir_mask=0))
         raise lsp.GspnError(st, "gspn_fwd")
     assert e.value.status == 1
+
+
+@pytest.mark.parametrize("args, fwd, bwd", [
+    # planes of at most 64x64 in any mode: one CTA per plane, one warp per direction
+    ((8, 96, 56, 56, 15, 1, False, "f32"), ("small_plane_fwd", 1), ("small_plane_bwd", 1)),
+    ((1, 2, 64, 64, 5, 2, False, "bf16"), ("small_plane_fwd", 1), ("small_plane_bwd", 1)),
+    ((3, 9, 64, 64, 15, 1, True, "bf16"), ("small_plane_fwd", 1), ("small_plane_bwd", 3)),  # C % 8 != 0
+    ((1, 1, 16, 16, 1, 1, False, "f32"), ("small_plane_fwd", 1), ("small_plane_bwd", 1)),
+    # anything larger: the generic kernels
+    ((1, 2, 65, 64, 15, 1, False, "f32"), ("generic_fwd", 1), ("generic_bwd", 1)),
+    ((1, 2, 97, 41, 9, 1, False, "f32"), ("generic_fwd", 1), ("generic_bwd", 1)),
+    ((2, 6, 128, 128, 15, 1, True, "bf16"), ("generic_fwd", 1), ("generic_bwd", 3)),  # C % 4 != 0
+])
+def test_path_chooser(args, fwd, bwd):
+    d = lsp.make_desc(*args)
+    assert (lsp.gspn_variant_name(d, 0), lsp.gspn_launches_per_call(d, 0)) == fwd
+    assert (lsp.gspn_variant_name(d, 1), lsp.gspn_launches_per_call(d, 1)) == bwd
+
+
+@pytest.mark.parametrize("args, fast", [
+    ((32, 1152, 64, 64, 15, 1, True, "bf16"), "compact64_tma"),
+    ((2, 1152, 128, 128, 15, 1, True, "bf16"), "compact128_tma"),
+    ((1, 4, 128, 128, 15, 4, True, "bf16"), "compact128_tma"),
+])
+def test_compact_shapes_take_the_tma_kernels_when_the_encoder_is_there(args, fast):
+    """The compact shapes run on the TMA-fed kernels wherever the driver's
+    tensor-map encoder is available (a GPU host); without it the chooser falls
+    back to the small-plane or generic kernels, which also cover them."""
+    d = lsp.make_desc(*args)
+    small = max(args[2], args[3]) <= 64
+    for bwd, launches in ((0, 2), (1, 3)):
+        name = lsp.gspn_variant_name(d, bwd)
+        suffix = "_bwd" if bwd else "_fwd"
+        if name == fast + suffix:
+            assert lsp.gspn_launches_per_call(d, bwd) == launches
+        else:
+            assert name == ("small_plane" if small else "generic") + suffix
