@@ -38,8 +38,8 @@
 // * x / lambda are streamed by TMA into a per-warp ring of 4 KB stages (8
 //   scan steps each): column chunks (8 columns x 64 rows) for the row pass
 //   and row chunks (64 columns x 8 rows) for the column pass.  A column chunk
-//   is fetched as two boxes of every other row (row element stride 2), so
-//   rows 2t and 2t+1 of lane t sit in two 512-byte slices and the 16-byte
+//   is one box of a 4-D view of the planes (column, row / 2, row % 2, plane),
+//   so rows 2t and 2t+1 of lane t sit in two 512-byte slices and the 16-byte
 //   reads of 8 lanes cover 128 contiguous bytes.  (A 16-byte wide box with
 //   the 128-byte swizzle would put every row on its own 128-byte line, eight
 //   times the space.)  A stage is copied to registers at its start and
@@ -70,7 +70,7 @@ constexpr int NCW = 8;         // consumer warps per CTA (one plane each), one C
 constexpr int NST = 2;         // x/lambda ring stages per consumer warp
 constexpr int NWS = 4;         // tap-weight ring stages per CTA
 constexpr int BOX = 1024;      // bytes per TMA box (one plane)
-constexpr int SLICE = 512;     // one element-stride-2 column box
+constexpr int SLICE = 512;     // the even or odd rows of a column chunk
 constexpr int STAGE = 4 * BOX;
 constexpr int HACC = S * S * 4;
 constexpr int WCHUNK = 8 * S * 16;  // tap weights of 8 scan steps (8 table rows)
@@ -225,13 +225,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (local < 8) {
                         const int q = local;
                         // x and lambda(left->right) at columns 8q.., x and lambda(right->left) at
-                        // 8(7-q)..; rows r_lo, r_lo + 2, ... go to slice r_lo
-                        for (int r = 0; r < 2; ++r) {
-                            tma::load_3d(dst + 0 * BOX + r * SLICE, &tm_xc, 8 * q, r, plane, bar);
-                            tma::load_3d(dst + 1 * BOX + r * SLICE, &tm_lc, 8 * q, r, 2 * BC + plane, bar);
-                            tma::load_3d(dst + 2 * BOX + r * SLICE, &tm_xc, 8 * (7 - q), r, plane, bar);
-                            tma::load_3d(dst + 3 * BOX + r * SLICE, &tm_lc, 8 * (7 - q), r, 3 * BC + plane, bar);
-                        }
+                        // 8(7-q)..; all 64 rows through the (column, row/2, row%2) view, so row
+                        // 2t+p lands in slice p at t*16
+                        tma::load_4d(dst + 0 * BOX, &tm_xc, 8 * q, 0, 0, plane, bar);
+                        tma::load_4d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 0, 2 * BC + plane, bar);
+                        tma::load_4d(dst + 2 * BOX, &tm_xc, 8 * (7 - q), 0, 0, plane, bar);
+                        tma::load_4d(dst + 3 * BOX, &tm_lc, 8 * (7 - q), 0, 0, 3 * BC + plane, bar);
                     } else {
                         const int q = local - 8;
                         // x and lambda(top->bottom) at rows 8q.., x and lambda(bottom->top) at rows 56-8q..
@@ -528,6 +527,21 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c,
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Row-pass view of the same planes: (column, row / 2, row % 2, plane); one box =
+// 8 columns of all 64 rows, laid out [row % 2][row / 2][8 columns], so the
+// 16-byte reads of a warp (lane t: rows 2t, 2t+1) are conflict-free.
+bool make_map_cols(CUtensorMap* m, const void* base, uint64_t planes) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {S, S / 2, 2, planes};
+    const cuuint64_t strides[3] = {2 * S * 2, S * 2, (cuuint64_t)S * S * 2};
+    const cuuint32_t box[4] = {8, S / 2, 2, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <bool LOCAL>
 gspn_status launch_c64(const DeviceInfo& dev, const CUtensorMap& xc, const CUtensorMap& lc, const CUtensorMap& xr,
                        const CUtensorMap& lr, const C64Args& a, cudaStream_t s) {
@@ -555,8 +569,7 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     CUtensorMap xc, lc, xr, lr;
     const uint64_t BC = (uint64_t)p.planes;
     // column chunks: 8 columns x every other row (32 rows); row chunks: 64 columns x 8 rows
-    if (!make_map(&xc, x, BC, 8, 64, 2, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
-        !make_map(&lc, lam, 4 * BC, 8, 64, 2, CU_TENSOR_MAP_L2_PROMOTION_NONE) ||
+    if (!make_map_cols(&xc, x, BC) || !make_map_cols(&lc, lam, 4 * BC) ||
         !make_map(&xr, x, BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) ||
         !make_map(&lr, lam, 4 * BC, 64, 8, 1, CU_TENSOR_MAP_L2_PROMOTION_L2_128B))
         return GSPN_ERR_UNSUPPORTED;

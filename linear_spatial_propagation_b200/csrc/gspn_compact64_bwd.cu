@@ -76,7 +76,7 @@ constexpr int WRING = NCW * WARP_BYTES;
 constexpr int DSTG = WRING + NWS * WCHUNK;    // 2 sets x NCW slots
 constexpr int NSET = 3;                         // slot sets, one reducer warp each
 constexpr int DOUT = DSTG + NSET * NCW * DSLOT;  // a reduced half chunk per set: [dir*2 + value][step][position j]
-constexpr int DLS = DOUT + NSET * DSLOT;          // per warp: row-pass dlambda of a chunk, A then B, [row][8 columns]
+constexpr int DLS = DOUT + NSET * DSLOT;          // per warp: row-pass dlambda of a chunk, A then B, [row % 2][row / 2][8 columns]
 constexpr int BARS = DLS + NCW * 2 * BOX;
 constexpr int NBAR = NCW * NST + 2 * NWS + 2 * NSET + 1;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
@@ -381,8 +381,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
 
     // Data of chunk kk (lane 0): x, lambda_A, lambda_B (sweep 2 only), dout of
-    // the chunk's 8 columns (row pass: [64 rows][8 columns]) or rows (column
-    // pass: [8 rows][64 columns]).
+    // the chunk's 8 columns (row pass: [row % 2][row / 2][8 columns] through the
+    // 4-D view, conflict-free 16-byte reads) or rows (column pass: [8 rows][64
+    // columns]).
     auto issue = [&](int kk) {
         if (kk >= nchunks) return;
         const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
@@ -394,10 +395,10 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma::mbar_expect_tx(bar, sweep ? 4 * BOX : 3 * BOX);
         const int la = pass ? 0 : 2, lb = pass ? 1 : 3;  // lambda slots of A and B
         if (pass == 0) {
-            tma::load_3d(dst + 0 * BOX, &tm_xc, 8 * q, 0, plane, bar);
-            tma::load_3d(dst + 1 * BOX, &tm_lc, 8 * q, 0, la * BC + plane, bar);
-            if (sweep) tma::load_3d(dst + 2 * BOX, &tm_lc, 8 * q, 0, lb * BC + plane, bar);
-            tma::load_3d(dst + 3 * BOX, &tm_gc, 8 * q, 0, plane, bar);
+            tma::load_4d(dst + 0 * BOX, &tm_xc, 8 * q, 0, 0, plane, bar);
+            tma::load_4d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 0, la * BC + plane, bar);
+            if (sweep) tma::load_4d(dst + 2 * BOX, &tm_lc, 8 * q, 0, 0, lb * BC + plane, bar);
+            tma::load_4d(dst + 3 * BOX, &tm_gc, 8 * q, 0, 0, plane, bar);
         } else {
             tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
             tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, la * BC + plane, bar);
@@ -480,12 +481,12 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint4 X[2] = {}, LA[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, Gr[8] = {};
                 if constexpr (pass == 0) {
-                    const unsigned char* st = ringp + stage * STAGE + t * 32;  // rows 2t, 2t+1
+                    const unsigned char* st = ringp + stage * STAGE + t * 16;  // rows 2t, 2t+1: slices 0, 1
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        X[p] = lds128(st + 0 * BOX + p * 16);
-                        LA[p] = lds128(st + 1 * BOX + p * 16);
-                        G[p] = lds128(st + 3 * BOX + p * 16);
+                        X[p] = lds128(st + 0 * BOX + p * 512);
+                        LA[p] = lds128(st + 1 * BOX + p * 512);
+                        G[p] = lds128(st + 3 * BOX + p * 512);
                     }
                 } else {
                     const unsigned char* st = ringp + stage * STAGE + t * 4;
@@ -550,13 +551,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 uint4 X[2] = {}, LA[2] = {}, LB[2] = {}, G[2] = {};
                 uint32_t Xr[8] = {}, LAr[8] = {}, LBr[8] = {}, Gr[8] = {};
                 if constexpr (pass == 0) {
-                    const unsigned char* st = ringp + stage * STAGE + t * 32;  // rows 2t, 2t+1
+                    const unsigned char* st = ringp + stage * STAGE + t * 16;  // rows 2t, 2t+1: slices 0, 1
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        X[p] = lds128(st + 0 * BOX + p * 16);
-                        LA[p] = lds128(st + 1 * BOX + p * 16);
-                        LB[p] = lds128(st + 2 * BOX + p * 16);
-                        G[p] = lds128(st + 3 * BOX + p * 16);
+                        X[p] = lds128(st + 0 * BOX + p * 512);
+                        LA[p] = lds128(st + 1 * BOX + p * 512);
+                        LB[p] = lds128(st + 2 * BOX + p * 512);
+                        G[p] = lds128(st + 3 * BOX + p * 512);
                     }
                 } else {
                     const unsigned char* st = ringp + stage * STAGE + t * 4;
@@ -663,22 +664,22 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
                 if constexpr (pass == 0) {
-                    // dlambda of the chunk's 8 columns: staged [row][8 columns] and
+                    // dlambda of the chunk's 8 columns: staged [row % 2][row / 2][8 columns] and
                     // written by two tiled bulk stores
                     if (t == 0) tma::bulk_wait_read();  // the previous chunk's stores have read the stage
                     __syncwarp();
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
-                        *reinterpret_cast<uint4*>(dlst + t * 32 + p * 16) =
+                        *reinterpret_cast<uint4*>(dlst + t * 16 + p * 512) =
                             make_uint4(dlA[p][0], dlA[p][1], dlA[p][2], dlA[p][3]);
-                        *reinterpret_cast<uint4*>(dlst + BOX + t * 32 + p * 16) =
+                        *reinterpret_cast<uint4*>(dlst + BOX + t * 16 + p * 512) =
                             make_uint4(dlB[p][0], dlB[p][1], dlB[p][2], dlB[p][3]);
                     }
                     tma::fence_proxy_async();
                     __syncwarp();
                     if (t == 0) {
-                        tma::store_3d(&tm_dl, dlsa, 8 * q, 0, la * BC + plane);
-                        tma::store_3d(&tm_dl, dlsa + BOX, 8 * q, 0, lb * BC + plane);
+                        tma::store_4d(&tm_dl, dlsa, 8 * q, 0, 0, la * BC + plane);
+                        tma::store_4d(&tm_dl, dlsa + BOX, 8 * q, 0, 0, lb * BC + plane);
                         tma::bulk_commit();
                     }
                 } else if (q == 4 || q == 0) {
@@ -729,6 +730,18 @@ EncodeTiledFn encode_fn_b() {
     return fn;
 }
 
+bool make_map_cols_b(CUtensorMap* m, const void* base, uint64_t planes) {
+    EncodeTiledFn fn = encode_fn_b();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {S, S / 2, 2, planes};
+    const cuuint64_t strides[3] = {2 * S * 2, S * 2, (cuuint64_t)S * S * 2};
+    const cuuint32_t box[4] = {8, S / 2, 2, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 bool make_map_b(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r) {
     EncodeTiledFn fn = encode_fn_b();
     if (!fn) return false;
@@ -767,9 +780,9 @@ gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
                     const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s) {
     CUtensorMap xc, lc, gc, xr, lr, gr, dl;
     const uint64_t BC = (uint64_t)p.planes;
-    if (!make_map_b(&xc, x, BC, 8, 64) || !make_map_b(&lc, lam, 4 * BC, 8, 64) || !make_map_b(&gc, dout, BC, 8, 64) ||
+    if (!make_map_cols_b(&xc, x, BC) || !make_map_cols_b(&lc, lam, 4 * BC) || !make_map_cols_b(&gc, dout, BC) ||
         !make_map_b(&xr, x, BC, 64, 8) || !make_map_b(&lr, lam, 4 * BC, 64, 8) || !make_map_b(&gr, dout, BC, 64, 8) ||
-        !make_map_b(&dl, dlam, 4 * BC, 8, 64))
+        !make_map_cols_b(&dl, dlam, 4 * BC))
         return GSPN_ERR_UNSUPPORTED;
     char* w = static_cast<char*>(ws);
     C64BArgs a;
