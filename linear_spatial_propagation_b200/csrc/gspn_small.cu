@@ -52,11 +52,16 @@ struct SmallArgs {
     float* dlog_ws;  // backward, shared taps: fp32 sums over channels [D][B][3][HW]
 };
 
-// the normalised taps of position j (valid ones only) from the raw logits
+// The sigmoids of the valid taps of position j from the raw logits.  These
+// kernels compute the taps at every use, so the divisions take the fast
+// reciprocal path of __fdividef (a couple of ulp) instead of IEEE division;
+// its result is 0 once 1 + e^-z passes 2^126 (logits below about -87), where
+// the sigmoid is below 1e-38 anyway.
+__device__ __forceinline__ float fast_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 __device__ __forceinline__ void taps(float g0, float g1, float g2, int j, int N, float& s0, float& s1, float& s2) {
-    s0 = j > 0 ? sigmoidf(g0) : 0.f;
-    s1 = sigmoidf(g1);
-    s2 = j < N - 1 ? sigmoidf(g2) : 0.f;
+    s0 = j > 0 ? fast_sigmoid(g0) : 0.f;
+    s1 = fast_sigmoid(g1);
+    s2 = j < N - 1 ? fast_sigmoid(g2) : 0.f;
 }
 
 // For a column scan the CH values of one position over lines i0, i0+1, ...
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
                     if (carry) {
                         float s0, s1, s2;
                         taps(v0[r][e], v1[r][e], v2[r][e], j, N, s0, s1, s2);
-                        v += (s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2]) / (s0 + s1 + s2);
+                        v += __fdividef(s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2], s0 + s1 + s2);
                     }
                     hc[j + 1] = v;
                     acc[pix(d, H, W, i, j)] = v;
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(128) small_bwd_kernel(SmallArgs a) {
                         if (carry) {
                             float s0, s1, s2;
                             taps(v0[r][e], v1[r][e], v2[r][e], j, N, s0, s1, s2);
-                            v += (s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2]) / (s0 + s1 + s2);
+                            v += __fdividef(s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2], s0 + s1 + s2);
                         }
                         hc[j + 1] = v;
                         hst[i * N + j] = v;
@@ -293,7 +298,7 @@ __global__ void __launch_bounds__(128) small_bwd_kernel(SmallArgs a) {
                     if (carry_out) {
                         float s0, s1, s2;
                         taps(v0[r][e], v1[r][e], v2[r][e], j, N, s0, s1, s2);
-                        const float rs = 1.f / (s0 + s1 + s2);
+                        const float rs = __fdividef(1.f, s0 + s1 + s2);
                         const float* hprev = hst + (i - 1) * N;
                         const float dw0 = j > 0 ? av * hprev[j - 1] : 0.f;
                         const float dw1 = av * hprev[j];
