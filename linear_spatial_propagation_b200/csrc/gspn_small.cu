@@ -198,8 +198,9 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
     }
 }
 
+// (with one position per lane, at most 80 registers: 6 CTAs per SM)
 template <typename T, int P>
-__global__ void __launch_bounds__(128) small_bwd_kernel(SmallArgs a) {
+__global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArgs a) {
     constexpr int CH = chunk_of<P>();
     extern __shared__ float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
