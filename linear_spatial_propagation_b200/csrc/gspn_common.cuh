@@ -30,6 +30,15 @@ __host__ __device__ __forceinline__ int pix(int d, int H, int W, int i, int j) {
     }
 }
 
+// The same map as an offset o + i*si + j*sj, for loops that walk a direction
+// without a branch per access.
+struct Walk {
+    int o, si, sj;
+};
+__host__ __device__ __forceinline__ Walk walk_of(int d, int H, int W) {
+    return d == T2B ? Walk{0, W, 1} : d == B2T ? Walk{(H - 1) * W, -W, 1} : d == L2R ? Walk{0, 1, W} : Walk{W - 1, -1, W};
+}
+
 // ---- element access ---------------------------------------------------------
 // bf16 <-> fp32: a bf16 value is the top 16 bits of the fp32 with the same value.
 __device__ __forceinline__ float bf16_bits_to_float(uint16_t u) { return __uint_as_float(((uint32_t)u) << 16); }
@@ -54,5 +63,12 @@ struct Launch {
     int groups;
     int shared;       // 1: logits have one channel (Cw = 1)
 };
+
+// Direction of slot `slot` < 4.  A chain of selects, not an index: indexing the
+// array with a runtime value would copy the kernel's parameter block into
+// local memory.
+__device__ __forceinline__ int dir_of(const Launch& g, int slot) {
+    return slot == 0 ? g.dirs[0] : slot == 1 ? g.dirs[1] : slot == 2 ? g.dirs[2] : g.dirs[3];
+}
 
 }  // namespace gspn

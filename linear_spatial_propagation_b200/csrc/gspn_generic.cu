@@ -49,7 +49,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_kernel(FwdArgs a) 
     const T* x = static_cast<const T*>(a.x) + plane * HW;
 
     for (int slot = 0; slot < a.g.D; ++slot) {
-        const int d = a.g.dirs[slot];
+        const int d = dir_of(a.g, slot);
         const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
         const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
         const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
@@ -57,10 +57,11 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_kernel(FwdArgs a) 
         float* hc = wsm + a.lstride;
         if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
         __syncwarp();
-        for (int i = 0; i < L; ++i) {
-            const bool carry = (i % seg) != 0;
+        const Walk wk = walk_of(d, H, W);
+        for (int i = 0, gi = 0; i < L; ++i, gi = gi + 1 == seg ? 0 : gi + 1) {  // gi = i % seg
+            const bool carry = gi != 0;
             for (int j = lane; j < N; j += 32) {
-                const int p = pix(d, H, W, i, j);
+                const int p = wk.o + i * wk.si + j * wk.sj;
                 float v = load_elt(lam, p) * load_elt(x, p);
                 if (carry) {
                     const float s0 = j > 0 ? sigmoidf(load_elt(lg, p)) : 0.f;
@@ -99,7 +100,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_pipelined_kernel(F
     const T* x = static_cast<const T*>(a.x) + plane * HW;
 
     for (int slot = 0; slot < a.g.D; ++slot) {
-        const int d = a.g.dirs[slot];
+        const int d = dir_of(a.g, slot);
         const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
         const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
         const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
@@ -109,11 +110,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_pipelined_kernel(F
         __syncwarp();
         // inputs of the line in flight: lambda*x and the three raw tap logits
         float lx[P], g0[P], g1[P], g2[P];
+        const Walk wk = walk_of(d, H, W);
         auto fetch = [&](int i, float (&flx)[P], float (&f0)[P], float (&f1)[P], float (&f2)[P]) {
 #pragma unroll
             for (int r = 0; r < P; ++r) {
                 const int j = lane + 32 * r;
-                const int pp = j < N ? pix(d, H, W, i, j) : 0;  // in bounds for idle lanes
+                const int pp = j < N ? wk.o + i * wk.si + j * wk.sj : 0;  // in bounds for idle lanes
                 flx[r] = load_elt(lam, pp) * load_elt(x, pp);
                 f0[r] = load_elt(lg, pp);
                 f1[r] = load_elt(lg, HW + pp);
@@ -121,10 +123,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_pipelined_kernel(F
             }
         };
         fetch(0, lx, g0, g1, g2);
-        for (int i = 0; i < L; ++i) {
+        for (int i = 0, gi = 0; i < L; ++i, gi = gi + 1 == seg ? 0 : gi + 1) {  // gi = i % seg
             float nlx[P], n0[P], n1[P], n2[P];
             if (i + 1 < L) fetch(i + 1, nlx, n0, n1, n2);
-            const bool carry = (i % seg) != 0;
+            const bool carry = gi != 0;
 #pragma unroll
             for (int r = 0; r < P; ++r) {
                 const int j = lane + 32 * r;
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_fwd_pipelined_kernel(F
                         v += num / (s0 + s1 + s2);
                     }
                     hc[j + 1] = v;
-                    const int pp = pix(d, H, W, i, j);
+                    const int pp = wk.o + i * wk.si + j * wk.sj;
                     acc[pp] = slot == 0 ? v : acc[pp] + v;
                 }
             }
@@ -199,11 +201,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) 
     const T* g = static_cast<const T*>(a.dout) + plane * HW;
 
     for (int slot = 0; slot < a.g.D; ++slot) {
-        const int d = a.g.dirs[slot];
+        const int d = dir_of(a.g, slot);
         const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
         const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
         const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
         T* dlam = static_cast<T*>(a.dlam) + ((slot * (int64_t)B + b) * C + c) * HW;
+        const Walk wk = walk_of(d, H, W);
 
         // 1. recompute this direction's lines into hst (scan coordinates)
         {
@@ -211,10 +214,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) 
             float* hc = wsm + ls;
             if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
             __syncwarp();
-            for (int i = 0; i < L; ++i) {
-                const bool carry = (i % seg) != 0;
+            for (int i = 0, gi = 0; i < L; ++i, gi = gi + 1 == seg ? 0 : gi + 1) {  // gi = i % seg
+                const bool carry = gi != 0;
                 for (int j = lane; j < N; j += 32) {
-                    const int p = pix(d, H, W, i, j);
+                    const int p = wk.o + i * wk.si + j * wk.sj;
                     float v = load_elt(lam, p) * load_elt(x, p);
                     if (carry) {
                         const float s0 = j > 0 ? sigmoidf(load_elt(lg, p)) : 0.f;
@@ -234,11 +237,12 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) 
         float* qc = wsm + 3 * ls;  // 3 buffers: products of line i
         for (int q = lane; q < 6 * ls; q += 32) wsm[q] = 0.f;
         __syncwarp();
-        for (int i = L - 1; i >= 0; --i) {
-            const bool carry_out = (i % seg) != 0;                 // line i reads line i-1
-            const bool carry_in = (i + 1 < L) && ((i + 1) % seg != 0);  // line i+1 read line i
+        // gi = i % seg, counted down from L-1 (seg divides L)
+        for (int i = L - 1, gi = seg - 1; i >= 0; --i, gi = gi == 0 ? seg - 1 : gi - 1) {
+            const bool carry_out = gi != 0;                      // line i reads line i-1
+            const bool carry_in = (i + 1 < L) && gi != seg - 1;  // line i+1 read line i
             for (int j = lane; j < N; j += 32) {
-                const int p = pix(d, H, W, i, j);
+                const int p = wk.o + i * wk.si + j * wk.sj;
                 float av = load_elt(g, p);
                 if (carry_in) av += qn[j + 2] + qn[ls + j + 1] + qn[2 * ls + j];
                 const float lv = load_elt(lam, p), xv = load_elt(x, p);

@@ -34,9 +34,11 @@ namespace {
 
 constexpr int kLS = 66;    // line buffer: up to 64 positions + a zero halo at each end
 // lines whose inputs are loaded together: 8 with two positions per lane, 4 with
-// one (fewer registers, more CTAs per SM for the many small planes)
-template <int P>
-__host__ __device__ constexpr int chunk_of() { return P == 1 ? 4 : 8; }
+// one (fewer registers, more CTAs per SM for the many small planes); the bf16
+// backward with two positions per lane takes 4 as well, which keeps its six
+// input planes within the 168 registers of 3 CTAs per SM
+template <int P, bool BWD = false, int BYTES = 4>
+__host__ __device__ constexpr int chunk_of() { return P == 1 || (BWD && BYTES == 2) ? 4 : 8; }
 constexpr int kSmallSmemCap = 200 * 1024;
 
 struct SmallArgs {
@@ -108,8 +110,8 @@ __device__ __forceinline__ bool load_row_piece(const T* src, int d, int W, int L
 // row offsets, so one test decides); otherwise one pixel index per (r, e) serves
 // all planes.
 template <int CH, bool DOWN, int P, int NT, typename T>
-__device__ __forceinline__ void load_chunk(const T* const (&src)[NT], int d, int H, int W, int L, int N, int i0,
-                                           int lane, float (&v)[NT][P][CH]) {
+__device__ __forceinline__ void load_chunk(const T* const (&src)[NT], int d, const Walk& wk, int W, int L, int N,
+                                           int i0, int lane, float (&v)[NT][P][CH]) {
 #pragma unroll
     for (int r = 0; r < P; ++r) {
         const int j = lane + 32 * r;
@@ -124,7 +126,7 @@ __device__ __forceinline__ void load_chunk(const T* const (&src)[NT], int d, int
             for (int e = 0; e < CH; ++e) {
                 const int i = DOWN ? i0 - e : i0 + e;
                 const bool in = j < N && i >= 0 && i < L;
-                const int p = in ? pix(d, H, W, i, j) : 0;  // in bounds for idle lanes
+                const int p = in ? wk.o + i * wk.si + j * wk.sj : 0;  // in bounds for idle lanes
 #pragma unroll
                 for (int k = 0; k < NT; ++k) v[k][r][e] = in ? load_elt(src[k], p) : 0.f;
             }
@@ -145,8 +147,7 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
     float* hp = smem + (size_t)D * HW + (size_t)warp * 2 * kLS;
     float* hc = hp + kLS;
 
-    // (a select, not an index, keeps the parameter block out of local memory)
-    const int slot = warp, d = slot == 0 ? a.g.dirs[0] : slot == 1 ? a.g.dirs[1] : slot == 2 ? a.g.dirs[2] : a.g.dirs[3];
+    const int slot = warp, d = dir_of(a.g, slot);
     const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
     const T* x = static_cast<const T*>(a.x) + plane * HW;
     const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
@@ -154,10 +155,15 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
     const T* const srcs[5] = {x, lam, lg, lg + HW, lg + 2 * HW};
     if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
     __syncwarp();
+    const Walk wk = walk_of(d, H, W);
+    int pj[P];  // plane offset of this lane's positions on line 0
+#pragma unroll
+    for (int r = 0; r < P; ++r) pj[r] = wk.o + (lane + 32 * r) * wk.sj;
 
+    int gi = 0;  // the line's index within its local group (i % seg, kept by counting)
     for (int i0 = 0; i0 < L; i0 += CH) {
         float vin[5][P][CH];
-        load_chunk<CH, false, P, 5>(srcs, d, H, W, L, N, i0, lane, vin);
+        load_chunk<CH, false, P, 5>(srcs, d, wk, W, L, N, i0, lane, vin);
         auto& vx = vin[0];
         auto& vl = vin[1];
         auto& v0 = vin[2];
@@ -167,7 +173,9 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
         for (int e = 0; e < CH; ++e) {
             const int i = i0 + e;
             if (i >= L) break;
-            const bool carry = (i % seg) != 0;
+            const bool carry = gi != 0;
+            gi = gi + 1 == seg ? 0 : gi + 1;
+            const int pi = i * wk.si;
 #pragma unroll
             for (int r = 0; r < P; ++r) {
                 const int j = lane + 32 * r;
@@ -179,7 +187,7 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
                         v += __fdividef(s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2], s0 + s1 + s2);
                     }
                     hc[j + 1] = v;
-                    acc[pix(d, H, W, i, j)] = v;
+                    acc[pj[r] + pi] = v;
                 }
             }
             __syncwarp();
@@ -201,7 +209,7 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
 // (with one position per lane, at most 80 registers: 6 CTAs per SM)
 template <typename T, int P>
 __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArgs a) {
-    constexpr int CH = chunk_of<P>();
+    constexpr int CH = chunk_of<P, true, (int)sizeof(T)>();
     extern __shared__ float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C, D = a.g.D;
@@ -212,8 +220,7 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
     float* const dxacc = smem + (size_t)(D + warp) * HW;         // this direction's share of dx
     float* const lb = smem + (size_t)2 * D * HW + (size_t)warp * 6 * kLS;  // line buffers
 
-    // (a select, not an index, keeps the parameter block out of local memory)
-    const int slot = warp, d = slot == 0 ? a.g.dirs[0] : slot == 1 ? a.g.dirs[1] : slot == 2 ? a.g.dirs[2] : a.g.dirs[3];
+    const int slot = warp, d = dir_of(a.g, slot);
     const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
     const T* x = static_cast<const T*>(a.x) + plane * HW;
     const T* g = static_cast<const T*>(a.dout) + plane * HW;
@@ -223,15 +230,18 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
     const T* const srcs[5] = {x, lam, lg, lg + HW, lg + 2 * HW};
     const T* const srcs6[6] = {g, x, lam, lg, lg + HW, lg + 2 * HW};
 
+    const Walk wk = walk_of(d, H, W);
+
     // 1. recompute this direction's lines into shared memory
     {
         float* hp = lb;
         float* hc = lb + kLS;
         if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
         __syncwarp();
+        int gi = 0;  // i % seg, kept by counting
         for (int i0 = 0; i0 < L; i0 += CH) {
             float vin[5][P][CH];
-            load_chunk<CH, false, P, 5>(srcs, d, H, W, L, N, i0, lane, vin);
+            load_chunk<CH, false, P, 5>(srcs, d, wk, W, L, N, i0, lane, vin);
             auto& vx = vin[0];
             auto& vl = vin[1];
             auto& v0 = vin[2];
@@ -241,7 +251,8 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
             for (int e = 0; e < CH; ++e) {
                 const int i = i0 + e;
                 if (i >= L) break;
-                const bool carry = (i % seg) != 0;
+                const bool carry = gi != 0;
+                gi = gi + 1 == seg ? 0 : gi + 1;
 #pragma unroll
                 for (int r = 0; r < P; ++r) {
                     const int j = lane + 32 * r;
@@ -270,10 +281,11 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
     float* qc = lb + 3 * kLS;
     for (int q = lane; q < 6 * kLS; q += 32) lb[q] = 0.f;
     __syncwarp();
+    int gi = seg - 1;  // i % seg for i = L-1 (seg divides L), kept by counting down
     for (int it = 0; it < L; it += CH) {
         // lines i = L-1-it-e, e < CH
         float vin[6][P][CH];
-        load_chunk<CH, true, P, 6>(srcs6, d, H, W, L, N, L - 1 - it, lane, vin);
+        load_chunk<CH, true, P, 6>(srcs6, d, wk, W, L, N, L - 1 - it, lane, vin);
         auto& vg = vin[0];
         auto& vx = vin[1];
         auto& vl = vin[2];
@@ -284,13 +296,15 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
         for (int e = 0; e < CH; ++e) {
             const int i = L - 1 - it - e;
             if (i < 0) break;
-            const bool carry_out = (i % seg) != 0;                      // line i reads line i-1
-            const bool carry_in = (i + 1 < L) && ((i + 1) % seg != 0);  // line i+1 read line i
+            const bool carry_out = gi != 0;                   // line i reads line i-1
+            const bool carry_in = (i + 1 < L) && gi != seg - 1;  // line i+1 read line i
+            gi = gi == 0 ? seg - 1 : gi - 1;
+            const int pi = wk.o + i * wk.si;
 #pragma unroll
             for (int r = 0; r < P; ++r) {
                 const int j = lane + 32 * r;
                 if (j < N) {
-                    const int p = pix(d, H, W, i, j);
+                    const int p = pi + j * wk.sj;
                     float av = vg[r][e];
                     if (carry_in) av += qn[j + 2] + qn[kLS + j + 1] + qn[2 * kLS + j];
                     dxacc[p] = vl[r][e] * av;
