@@ -104,6 +104,46 @@ __device__ __forceinline__ bool load_row_piece(const T* src, int d, int W, int L
     return true;
 }
 
+// The reverse of load_row_piece for the bf16 backward's outputs of a column
+// scan.  Line itop - e (e < CH, lines below 0 absent) of position j in
+// direction d (left->right or right->left) is bf16 value e of v, two per word
+// (even e in the low half), so a tensor's CH values of one chunk are CH
+// neighbouring pixels of row j.  They leave as one 8-byte store per 4 when
+// the piece is whole and aligned, else one element at a time.
+template <int CH>
+__device__ __forceinline__ void put_bf16(uint32_t (&v)[CH / 2], int e, float x) {
+    const uint32_t b = __bfloat16_as_ushort(__float2bfloat16_rn(x));
+    v[e >> 1] = (e & 1) ? (v[e >> 1] | (b << 16)) : b;
+}
+template <int CH>
+__device__ __forceinline__ void store_row_piece(__nv_bfloat16* dst, int d, int W, int itop, int j,
+                                                const uint32_t (&v)[CH / 2]) {
+    static_assert(CH % 4 == 0, "whole 8-byte stores");
+    const int ilo = itop - (CH - 1);
+    // address order: left->right holds line ilo + m at element m (e = CH-1-m),
+    // right->left line itop - m (e = m)
+    const int first = d == L2R ? j * W + ilo : j * W + (W - 1 - itop);
+    if (ilo >= 0 && (reinterpret_cast<uintptr_t>(dst + first) & 7u) == 0) {
+        uint32_t w[CH / 2];
+        if (d == L2R) {
+#pragma unroll
+            for (int u = 0; u < CH / 2; ++u) w[u] = __byte_perm(v[CH / 2 - 1 - u], 0, 0x1032);  // halves swapped
+        } else {
+#pragma unroll
+            for (int u = 0; u < CH / 2; ++u) w[u] = v[u];
+        }
+#pragma unroll
+        for (int u = 0; u < CH / 4; ++u) reinterpret_cast<uint2*>(dst + first)[u] = make_uint2(w[2 * u], w[2 * u + 1]);
+    } else {
+        unsigned short* const o = reinterpret_cast<unsigned short*>(dst);
+#pragma unroll
+        for (int e = 0; e < CH; ++e) {
+            const int i = itop - e;
+            if (i >= 0) o[d == L2R ? j * W + i : j * W + (W - 1 - i)] = (unsigned short)(v[e >> 1] >> (16 * (e & 1)));
+        }
+    }
+}
+
 // The chunk's inputs of lane positions j = lane + 32r: NT planes (x, lambda, the
 // three logits, and dout in the backward) at lines i0 +- e.  Column scans use the
 // row-piece loads when every plane's piece is aligned (the planes share the
@@ -206,9 +246,10 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
     }
 }
 
-// (with one position per lane, at most 80 registers: 6 CTAs per SM)
+// (with one position per lane, at most 80 registers for fp32: 6 CTAs per SM;
+// bf16 holds the row pieces as well and takes 5)
 template <typename T, int P>
-__global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArgs a) {
+__global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) small_bwd_kernel(SmallArgs a) {
     constexpr int CH = chunk_of<P, true, (int)sizeof(T)>();
     extern __shared__ float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -227,8 +268,15 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
     const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
     const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
     T* dlam = static_cast<T*>(a.dlam) + ((slot * (int64_t)B + b) * C + c) * HW;
+    T* dlg = static_cast<T*>(a.dlogits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
     const T* const srcs[5] = {x, lam, lg, lg + HW, lg + 2 * HW};
     const T* const srcs6[6] = {g, x, lam, lg, lg + HW, lg + 2 * HW};
+    // A column scan's dlambda and dlogits of one position and chunk are
+    // neighbouring pixels of a row.  In bf16 they are gathered and written as
+    // 8-byte pieces (4 lines), instead of one scattered 2-byte element per
+    // lane and line; fp32 keeps the element stores (measured faster there).
+    constexpr bool kPieces = sizeof(T) == 2;
+    const bool col = d == L2R || d == R2L;
 
     const Walk wk = walk_of(d, H, W);
 
@@ -292,6 +340,8 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
         auto& v0 = vin[3];
         auto& v1 = vin[4];
         auto& v2 = vin[5];
+        // column scans in bf16: the chunk's dlambda and dlogits, written as row pieces at its end
+        uint32_t cl[P][CH / 2], cg0[P][CH / 2], cg1[P][CH / 2], cg2[P][CH / 2];
 #pragma unroll
         for (int e = 0; e < CH; ++e) {
             const int i = L - 1 - it - e;
@@ -308,7 +358,10 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
                     float av = vg[r][e];
                     if (carry_in) av += qn[j + 2] + qn[kLS + j + 1] + qn[2 * kLS + j];
                     dxacc[p] = vl[r][e] * av;
-                    store_elt(dlam, p, vx[r][e] * av);
+                    if (kPieces && col)
+                        put_bf16<CH>(cl[r], e, vx[r][e] * av);
+                    else
+                        store_elt(dlam, p, vx[r][e] * av);
                     float dl0 = 0.f, dl1 = 0.f, dl2 = 0.f, q0 = 0.f, q1 = 0.f, q2 = 0.f;
                     if (carry_out) {
                         float s0, s1, s2;
@@ -337,8 +390,11 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
                             atomicAdd(dw + HW + p, dl1);
                             if (j < N - 1) atomicAdd(dw + 2 * HW + p, dl2);
                         }
+                    } else if (kPieces && col) {
+                        put_bf16<CH>(cg0[r], e, dl0);
+                        put_bf16<CH>(cg1[r], e, dl1);
+                        put_bf16<CH>(cg2[r], e, dl2);
                     } else {
-                        T* dlg = static_cast<T*>(a.dlogits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
                         store_elt(dlg, p, dl0);
                         store_elt(dlg, HW + p, dl1);
                         store_elt(dlg, 2 * HW + p, dl2);
@@ -349,6 +405,24 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : 6) small_bwd_kernel(SmallArg
             float* t = qn;
             qn = qc;
             qc = t;
+        }
+        if constexpr (kPieces) {
+            if (col) {
+                __nv_bfloat16* const bl = reinterpret_cast<__nv_bfloat16*>(dlam);
+                __nv_bfloat16* const bg = reinterpret_cast<__nv_bfloat16*>(dlg);
+#pragma unroll
+                for (int r = 0; r < P; ++r) {
+                    const int j = lane + 32 * r;
+                    if (j < N) {
+                        store_row_piece<CH>(bl, d, W, L - 1 - it, j, cl[r]);
+                        if (!a.g.shared) {
+                            store_row_piece<CH>(bg, d, W, L - 1 - it, j, cg0[r]);
+                            store_row_piece<CH>(bg + HW, d, W, L - 1 - it, j, cg1[r]);
+                            store_row_piece<CH>(bg + 2 * HW, d, W, L - 1 - it, j, cg2[r]);
+                        }
+                    }
+                }
+            }
         }
     }
     __syncthreads();
