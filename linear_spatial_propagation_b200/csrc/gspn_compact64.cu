@@ -20,7 +20,8 @@
 //   positions per lane.  The 8 warps step through the same sequence of
 //   8-step chunks, so one producer warp streams each chunk's tap weights
 //   (8 table rows, 8 KB) with a single bulk copy into a 4-stage ring that all
-//   8 warps read; each warp copies the chunk to registers and releases it.
+//   8 warps read; each warp reads a step's weights one step ahead and releases
+//   the stage after its last step.
 // * The two directions of a pair (left->right with right->left, top->bottom
 //   with bottom->top) advance together: lane values are float2 (one
 //   direction per half) and the update is the packed fp32x2 FMA of sm_100;
@@ -269,24 +270,29 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_wait(wfull0 + 8 * (kk % NWS), (kk / NWS) & 1, 100000000ull);
     };
 
-    // Chunk start: wait for the data stage and the weight stage of chunk k, copy
-    // both to registers, hand both stages back (data: refill with chunk k + NST;
-    // weights: one arrival per warp on the stage's "consumed" barrier).
-    float4 wr[8][2];
-    auto weights_in = [&]() -> bool {
-        const int ws = k % NWS;
-        const bool ok = tma::mbar_wait(wfull0 + 8 * ws, (k / NWS) & 1);
-        if (!__all_sync(FULL, ok)) return false;
-        const unsigned char* wsrc = wring + ws * WCHUNK + t * 16;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            wr[e][0] = lds128f(wsrc + e * 1024);
-            wr[e][1] = lds128f(wsrc + e * 1024 + 512);
+    // Tap weights are read one step ahead: during step e of chunk c a warp loads
+    // the 2 x 16 bytes of step e+1 into registers.  At the chunk's last step it
+    // hands the weight stage back (every lane fences its reads of the stage
+    // before the async-proxy refill; one arrival per warp) and takes step 0 of
+    // chunk c+1.  Data stages are copied to registers whole at the chunk's start.
+    float4 wc[2];  // tap weights of the current step
+    auto wstep = [&](int c, int e, float4 (&wn)[2]) -> bool {
+        if (e < 7) {
+            const unsigned char* wsrc = wring + (c % NWS) * WCHUNK + t * 16 + (e + 1) * 1024;
+            wn[0] = lds128f(wsrc);
+            wn[1] = lds128f(wsrc + 512);
+            return true;
         }
-        // every lane's reads of the stage come before the async-proxy refill
         tma::fence_proxy_async();
         __syncwarp();
-        if (t == 0) tma::mbar_arrive(wempty0 + 8 * ws);
+        if (t == 0) tma::mbar_arrive(wempty0 + 8 * (c % NWS));
+        if (c + 1 < nchunks) {
+            const bool okw = tma::mbar_wait(wfull0 + 8 * ((c + 1) % NWS), ((c + 1) / NWS) & 1);
+            if (!__all_sync(FULL, okw)) return false;
+            const unsigned char* wsrc = wring + ((c + 1) % NWS) * WCHUNK + t * 16;
+            wn[0] = lds128f(wsrc);
+            wn[1] = lds128f(wsrc + 512);
+        }
         return true;
     };
     auto acquire = [&]() -> bool {
@@ -321,7 +327,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         constexpr bool SECOND = decltype(second)::value;
         for (int qq = 0; qq < 4; ++qq) {
             const int q = SECOND ? qq + 4 : qq;
-            if (!weights_in() || !acquire()) return false;
+            const int c = k;
+            if (!acquire()) return false;
             const unsigned char* st = ringp + stage * STAGE + t * 16;
             uint4 XA[2], LA[2], XB[2], LB[2];
 #pragma unroll
@@ -356,7 +363,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                         base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1),
                                            h[p].y);
                     }
-                    scan_core(h, base, wr[e]);
+                    float4 wn[2];
+                    if (!wstep(c, e, wn)) return false;
+                    scan_core(h, base, wc);
+                    wc[0] = wn[0];
+                    wc[1] = wn[1];
                     if constexpr (!SECOND) {
 #pragma unroll
                         for (int p = 0; p < 2; ++p) {
@@ -400,7 +411,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         constexpr bool SECOND = decltype(second)::value;
         for (int qq = 0; qq < 4; ++qq) {
             const int q = SECOND ? qq + 4 : qq;
-            if (!weights_in() || !acquire()) return false;
+            const int c = k;
+            if (!acquire()) return false;
             const unsigned char* st = ringp + stage * STAGE + t * 4;
             uint32_t XA[8], LA[8], XB[8], LB[8];
 #pragma unroll
@@ -434,7 +446,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                     base[1].x = fma_bf_hi(LA[e], XA[e], h[1].x);
                     base[0].y = fma_bf_lo(LB[e], XB[e], h[0].y);
                     base[1].y = fma_bf_hi(LB[e], XB[e], h[1].y);
-                    scan_core(h, base, wr[e]);
+                    float4 wn[2];
+                    if (!wstep(c, e, wn)) return false;
+                    scan_core(h, base, wc);
+                    wc[0] = wn[0];
+                    wc[1] = wn[1];
                     if (!SECOND) {
                         // first arrival of this pass: the row sum of the pixel plus this
                         // direction's value, parked in TMEM
@@ -465,6 +481,12 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
 
     bool ok = true;
+    if (nchunks > 0) {
+        const bool okw = tma::mbar_wait(wfull0, 0);
+        ok = __all_sync(FULL, okw);
+        wc[0] = lds128f(wring + t * 16);
+        wc[1] = lds128f(wring + t * 16 + 512);
+    }
     for (int group = blockIdx.x; ok && group < a.groups; group += gridDim.x) {
         outp = a.out + (size_t)(8 * group + warp) * S * S + 2 * t;
         h[0] = h[1] = make_float2(0.f, 0.f);
