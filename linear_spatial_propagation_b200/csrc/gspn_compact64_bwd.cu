@@ -575,17 +575,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                 auto lbv = [&](int e) { return pass == 0 ? make_float2(bfv(LB[0], e), bfv(LB[1], e)) : bf2(LBr[e]); };
                 auto gv = [&](int e) { return pass == 0 ? make_float2(bfv(G[0], e), bfv(G[1], e)) : bf2(Gr[e]); };
 
-                // h_A(s-1) (the state line s reads) and a_B(s) of the chunk, from sweep 1
+                // h_A(s-1) (the state line s reads) and a_B(s) of the chunk, from sweep 1,
+                // half a chunk at a time (steps 7..4 first)
                 float2 hAp[8], aBs[8];
-                {
-                    uint32_t sv[32];
-                    tmem::ld_x32(tstate + 32 * q, sv);
-                    tmem::wait_ld(sv);
+                uint32_t svh[16];
+                tmem::ld_x16(tstate + 32 * q + 16, svh);
+                tmem::wait_ld16(svh);
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        hAp[e] = make_float2(__uint_as_float(sv[4 * e]), __uint_as_float(sv[4 * e + 1]));
-                        aBs[e] = make_float2(__uint_as_float(sv[4 * e + 2]), __uint_as_float(sv[4 * e + 3]));
-                    }
+                for (int e = 4; e < 8; ++e) {
+                    hAp[e] = make_float2(__uint_as_float(svh[4 * (e - 4)]), __uint_as_float(svh[4 * (e - 4) + 1]));
+                    aBs[e] = make_float2(__uint_as_float(svh[4 * (e - 4) + 2]), __uint_as_float(svh[4 * (e - 4) + 3]));
                 }
                 uint32_t dlA[2][4], dlB[2][4];  // row pass: dlambda of rows 2t+p, 8 columns (bf16 pairs)
                 float2 dlAo, dlBo;               // row pass: dlambda of the odd column of a pair
@@ -599,7 +598,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int ee = 0; ee < 8; ++ee) {
                     const int e = 7 - ee;
                     const int s = 8 * q + e;
+                    if (ee == 2) tmem::ld_x16(tstate + 32 * q, svh);  // steps 3..0, in flight for two steps
                     if (ee == 4) {
+                        tmem::wait_ld16(svh);
+#pragma unroll
+                        for (int e2 = 0; e2 < 4; ++e2) {
+                            hAp[e2] = make_float2(__uint_as_float(svh[4 * e2]), __uint_as_float(svh[4 * e2 + 1]));
+                            aBs[e2] = make_float2(__uint_as_float(svh[4 * e2 + 2]), __uint_as_float(svh[4 * e2 + 3]));
+                        }
                         dpublish();
                         ds = dslot();
                         if (ds == nullptr) {
