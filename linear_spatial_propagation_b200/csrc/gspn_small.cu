@@ -13,7 +13,7 @@
 // s_k = sigmoid(logit_k) on the taps whose source lies in the line, w_k =
 // s_k / sum s (Key design 1).
 //
-// Inputs are read 8 lines at a time (4 with one position per lane): each lane
+// Inputs are read 4 lines at a time (8 for fp32 with two positions per lane): each lane
 // loads its positions' values of those lines in one go.  For a row scan the lanes of a warp read along a
 // row; for a column scan each lane reads the neighbouring pixels of its row,
 // with 8-byte loads where the pieces are aligned.
@@ -33,12 +33,14 @@ namespace gspn {
 namespace {
 
 constexpr int kLS = 66;    // line buffer: up to 64 positions + a zero halo at each end
-// lines whose inputs are loaded together: 8 with two positions per lane, 4 with
-// one (fewer registers, more CTAs per SM for the many small planes); the bf16
-// backward with two positions per lane takes 4 as well, which keeps its six
-// input planes within the 168 registers of 3 CTAs per SM
-template <int P, bool BWD = false, int BYTES = 4>
-__host__ __device__ constexpr int chunk_of() { return P == 1 || (BWD && BYTES == 2) ? 4 : 8; }
+// lines whose inputs are loaded together: 8 for fp32 with two positions per
+// lane, 4 otherwise.  With one position per lane that means fewer registers and
+// more CTAs per SM for the many small planes; for bf16 with two positions it
+// was measured faster in the forward (64x64: 145 -> 119 us) and keeps the
+// backward's six input planes within the 168 registers of 3 CTAs per SM.  fp32
+// with two positions is faster with 8 (56x56 forward: 93 against 159 us).
+template <int P, int BYTES>
+__host__ __device__ constexpr int chunk_of() { return P == 2 && BYTES == 4 ? 8 : 4; }
 constexpr int kSmallSmemCap = 200 * 1024;
 
 struct SmallArgs {
@@ -176,7 +178,7 @@ __device__ __forceinline__ void load_chunk(const T* const (&src)[NT], int d, con
 
 template <typename T, int P>
 __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
-    constexpr int CH = chunk_of<P>();
+    constexpr int CH = chunk_of<P, (int)sizeof(T)>();
     extern __shared__ float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C, D = a.g.D;
@@ -250,7 +252,7 @@ __global__ void __launch_bounds__(128) small_fwd_kernel(SmallArgs a) {
 // bf16 holds the row pieces as well and takes 5)
 template <typename T, int P>
 __global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) small_bwd_kernel(SmallArgs a) {
-    constexpr int CH = chunk_of<P, true, (int)sizeof(T)>();
+    constexpr int CH = chunk_of<P, (int)sizeof(T)>();
     extern __shared__ float smem[];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C, D = a.g.D;
