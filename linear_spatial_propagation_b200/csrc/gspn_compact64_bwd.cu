@@ -224,6 +224,18 @@ __device__ __forceinline__ float2 adjoint(float2 a, float2 g, const Taps& w, int
     return add2(n, make_float2(p2l, p0r));
 }
 
+// The same adjoint step with g + a already formed (from the bf16 g by one
+// mixed-precision FMA per position: g * 1 + a, the same single rounding).
+__device__ __forceinline__ float2 adjoint_ga(float2 a, float2 ga, const Taps& w, int t) {
+    const float2 p0 = mul2(w.w0, a), p2 = mul2(w.w2, a);
+    const float p0r = __shfl_sync(FULL, p0.x, (t + 1) & 31);
+    const float p2l = __shfl_sync(FULL, p2.y, (t + 31) & 31);
+    const float2 n = add2(fma2(make_float2(-1.f, -1.f), p2, fma2(make_float2(-1.f, -1.f), p0, ga)),
+                          make_float2(p0.y, p2.x));
+    return add2(n, make_float2(p2l, p0r));
+}
+constexpr uint32_t kOneBf2 = 0x3F803F80u;  // bf16 1.0 in both halves
+
 // 12 warps put 3 on each of the SM's four schedulers, each with a quarter of
 // the register file: at most 16384 / (3 * 32) -> 168 registers per thread
 template <bool LOCAL>
@@ -502,15 +514,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 for (int e = 0; e < 8; ++e) {
                     Taps WA, WB;
                     wrow(e, WA, WB);
-                    float2 x, lam, g;
+                    // lambda x and g + a_B from the bf16 words by mixed-precision FMAs
+                    float2 lx, ga;
                     if constexpr (pass == 0) {
-                        x = make_float2(bfv(X[0], e), bfv(X[1], e));
-                        lam = make_float2(bfv(LA[0], e), bfv(LA[1], e));
-                        g = make_float2(bfv(G[0], e), bfv(G[1], e));
+                        lx = make_float2(fma_bf(e & 1, word_of(LA[0], e >> 1), word_of(X[0], e >> 1), 0.f),
+                                         fma_bf(e & 1, word_of(LA[1], e >> 1), word_of(X[1], e >> 1), 0.f));
                     } else {
-                        x = bf2(Xr[e]);
-                        lam = bf2(LAr[e]);
-                        g = bf2(Gr[e]);
+                        lx = make_float2(fma_bf_lo(LAr[e], Xr[e], 0.f), fma_bf_hi(LAr[e], Xr[e], 0.f));
                     }
                     float2 hL, hR;
                     // local groups: line s of A starts a group, and line s-1 of B (the
@@ -522,8 +532,14 @@ __global__ void __launch_bounds__(THREADS, 1)
                     sv[4 * e] = __float_as_uint(hA.x);
                     sv[4 * e + 1] = __float_as_uint(hA.y);
                     float2 mA_;
-                    hA = fwd_step(hA, mul2(lam, x), WA, t, hL, hR, mA_);
-                    aB = adjoint(aB, g, WBp, t);
+                    hA = fwd_step(hA, lx, WA, t, hL, hR, mA_);
+                    if constexpr (pass == 0) {
+                        ga = make_float2(fma_bf(e & 1, word_of(G[0], e >> 1), kOneBf2, aB.x),
+                                         fma_bf(e & 1, word_of(G[1], e >> 1), kOneBf2, aB.y));
+                    } else {
+                        ga = make_float2(fma_bf_lo(Gr[e], kOneBf2, aB.x), fma_bf_hi(Gr[e], kOneBf2, aB.y));
+                    }
+                    aB = adjoint_ga(aB, ga, WBp, t);
                     sv[4 * e + 2] = __float_as_uint(aB.x);
                     sv[4 * e + 3] = __float_as_uint(aB.y);
                     WBp = WB;
@@ -624,7 +640,16 @@ __global__ void __launch_bounds__(THREADS, 1)
                         hB = make_float2(0.f, 0.f);
                     }
                     // adjoint of A at s from s+1 (taps of line s+1)
-                    aA = adjoint(aA, gv(e), WAn, t);
+                    {
+                        float2 gaA;
+                        if constexpr (pass == 0) {
+                            gaA = make_float2(fma_bf(e & 1, word_of(G[0], e >> 1), kOneBf2, aA.x),
+                                              fma_bf(e & 1, word_of(G[1], e >> 1), kOneBf2, aA.y));
+                        } else {
+                            gaA = make_float2(fma_bf_lo(Gr[e], kOneBf2, aA.x), fma_bf_hi(Gr[e], kOneBf2, aA.y));
+                        }
+                        aA = adjoint_ga(aA, gaA, WAn, t);
+                    }
                     WAn = WA;
                     // forward of B at s from s+1 (taps of B's line at s) and B's tap values
                     float2 hL, hR, m;
