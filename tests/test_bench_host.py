@@ -1,6 +1,7 @@
 """Host-side logic of bench.py, on CPU: the reference arm's JSON line, the
 silent non-zero ranks, and the max-over-ranks / whole-job aggregation of the
-multi-GPU replicas exercised over a world-size-2 gloo group."""
+multi-GPU replicas exercised over a world-size-2 gloo group, and the rule that
+roofline.traffic is reported only for the sources it was captured on."""
 import json
 import os
 import socket
@@ -87,3 +88,23 @@ def test_max_over_ranks_with_two_gloo_ranks():
     for rank, ms, gbs in res:
         assert ms == 11.0                       # every rank sees the slowest rank's time
         assert gbs == pytest.approx(2 * 1_000_000_000 / 11e-3 / 1e9)  # both ranks' bytes
+
+
+def test_roofline_traffic_only_for_the_sources_it_was_captured_on(monkeypatch):
+    """roofline.traffic comes from the committed ncu capture only while the
+    dominant kernel's sources hash to the value stored with it; any source
+    change turns it into null until a new capture is committed."""
+    import bench
+    import synth
+    w = synth.WORKLOADS["compact_4dir_bf16_b32c1152_64x64"]
+    with open(os.path.join(ROOT, "profiles", "ncu_traffic.json")) as f:
+        stored = json.load(f)[w.name]
+    for kernel_pass in ("fwd", "bwd"):
+        ent = stored[kernel_pass]
+        assert ent["dram_bytes_per_launch"] > 0
+        monkeypatch.setattr(bench, "csrc_hash", lambda p, h=ent["csrc_hash"]: h)
+        assert bench.ncu_traffic(kernel_pass, w) == ent["dram_bytes_per_launch"]
+        monkeypatch.setattr(bench, "csrc_hash", lambda p: "0" * 16)
+        assert bench.ncu_traffic(kernel_pass, w) is None
+    # a workload without a capture has no traffic either
+    assert bench.ncu_traffic("bwd", synth.WORKLOADS["t2b_f32_b1c4_16x16"]) is None
