@@ -9,10 +9,17 @@ module compiles it with gcc on first use, widens the stored inputs to double
 and calls it through ctypes.  See ``gspn_ref.c`` for what is computed and which
 passage of the GSPN / GSPN-2 pages each step follows.
 
+``block_fwd`` adds the compressed propagation block around the scan: the
+projection of the C input channels onto C_proxy channels, the four
+single-direction scans of those planes, a learnable per-(direction, channel)
+merger, an RMS normalisation over the proxy channels of each pixel, and the
+projection back to C channels.  Its matrix products are numpy ``einsum`` in
+float64; its scans are the C oracle's, one direction at a time.
+
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
-against closed forms, invariants, brute force and hand-derived values.  The
-pages print no worked numeric example, so absolute values are pinned only
-through those derivations.
+and ``tests/test_oracle_block_pins.py`` against closed forms, invariants,
+brute force and hand-derived values.  The pages print no worked numeric
+example, so absolute values are pinned only through those derivations.
 """
 from __future__ import annotations
 
@@ -143,3 +150,68 @@ def fwd_workload(w, inp: Dict[str, np.ndarray], nthreads: int = 1) -> np.ndarray
 def bwd_workload(w, inp: Dict[str, np.ndarray], nthreads: int = 1):
     return bwd(inp["x"], inp["logits"], inp["lam"], inp["dout"], dir_mask=w.dir_mask, groups=w.groups,
                shared=w.shared, dtype=w.dtype, nthreads=nthreads)
+
+
+# ---------------------------------------------------------------------------
+# Compressed propagation block
+# ---------------------------------------------------------------------------
+_DIR_BITS = (1, 2, 4, 8)  # T2B, B2T, L2R, R2L: the D axis order of lambda, logits and alpha
+
+
+def block_fwd(x, v_proj, logits, lam, alpha, gamma, u_proj, *, groups: int = 1, norm: bool = True,
+              eps: float = 1e-6, dtype: str = "f64", nthreads: int = 1, return_parts: bool = False):
+    """y[B,C,H,W] (float64) of the compressed propagation block.
+
+    Steps, each in float64:
+
+    1. proxy projection ("GSPN-2: Efficient Parallel Sequence Modeling",
+       OpenReview response, "Relate Compressive Proxy Dimension to Low-rank
+       Approximation": x in R^{N x C x H x W} is projected by a linear layer to
+       C_proxy channels): xp[b,k] = sum_c v_proj[k,c] x[b,c];
+    2. the GSPN line scan of the proxy planes in each of the four directions
+       separately ("Parallel Sequence Modeling via Generalized Spatial
+       Propagation Network", Key design 2), with channel-shared taps
+       (compact mode) and per-channel lambda;
+    3. the learnable merger of the four directions (same page, Key design 2:
+       "aggregated by a learnable merger"), read as one weight per direction
+       and proxy channel: m[b,k] = sum_d alpha[d,k] h_d[b,k];
+    4. the fused normalisation ("Scaling Parallel Sequence Models to Vision
+       Foundation Models", abstract: a compressed latent-space propagation
+       block with fused normalisation), read as an RMS normalisation over the
+       proxy channels of each pixel with a per-channel gain:
+       n[b,k] = gamma[k] m[b,k] / sqrt(mean_k m[b,k]^2 + eps)  (skipped when
+       ``norm`` is false);
+    5. the projection back to C channels (the same OpenReview passage):
+       y[b,c] = sum_k u_proj[c,k] n[b,k].
+
+    Shapes: x [B,C,H,W]; v_proj [Cp,C]; logits [4,B,1,3,H,W]; lam
+    [4,B,Cp,H,W]; alpha [4,Cp]; gamma [Cp]; u_proj [C,Cp].  ``dtype`` names
+    how x, v_proj, logits, lam and u_proj are stored ("f64", "f32", "bf16");
+    alpha and gamma are float arrays.  With ``return_parts`` the function also
+    returns the intermediates (xp, the four h_d, m, n).
+    """
+    conv = (lambda a: widen(a, dtype)) if dtype != "f64" else (lambda a: np.ascontiguousarray(a, dtype=np.float64))
+    xs, vs, ls, ms, us = conv(x), conv(v_proj), conv(logits), conv(lam), conv(u_proj)
+    al = np.asarray(alpha, dtype=np.float64)
+    ga = np.asarray(gamma, dtype=np.float64)
+    B, C, H, W = xs.shape
+    Cp = vs.shape[0]
+    if vs.shape != (Cp, C) or us.shape != (C, Cp) or ls.shape != (4, B, 1, 3, H, W) or \
+            ms.shape != (4, B, Cp, H, W) or al.shape != (4, Cp) or ga.shape != (Cp,):
+        raise ValueError("bad block shapes")
+    xp = np.einsum("kc,bchw->bkhw", vs, xs)
+    hs = []
+    for d, bit in enumerate(_DIR_BITS):
+        hs.append(fwd(xp, ls[d:d + 1], ms[d:d + 1], dir_mask=bit, groups=groups, shared=True, nthreads=nthreads))
+    m = np.zeros_like(xp)
+    for d in range(4):
+        m += al[d][None, :, None, None] * hs[d]
+    if norm:
+        r = np.sqrt(np.mean(m * m, axis=1, keepdims=True) + eps)
+        n = m / r * ga[None, :, None, None]
+    else:
+        n = m
+    y = np.einsum("ck,bkhw->bchw", us, n)
+    if return_parts:
+        return y, {"xp": xp, "h": hs, "m": m, "n": n}
+    return y
