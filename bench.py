@@ -433,6 +433,12 @@ def run_gpu(args, w):
                        "kind": "oracle",
                        "sample": f"fwd+bwd of {s['images']} batch image(s) x C={s['channels']} planes of "
                                  f"{w.name}, B=1 each ({s['seconds']:.1f} s)"}
+                # the same oracle on one thread, on a smaller sample of the same workload
+                s1 = oracle_sample(w, args.cpu_seconds / 3.0, 1)
+                cpu["single_thread"] = {
+                    "value": s1["bytes"] / s1["seconds"] / 1e9, "unit": "GB/s", "cores": 1,
+                    "sample": f"fwd+bwd of {s1['images']} batch image(s) x C={s1['channels']} planes of "
+                              f"{w.name}, B=1 each ({s1['seconds']:.1f} s)"}
             except Exception as ex:  # the baseline must not sink the GPU line
                 cpu = {"value": None, "unit": "GB/s", "cores": os.cpu_count() or 1, "kind": "oracle",
                        "sample": f"failed: {ex!r}"[:200]}

@@ -46,9 +46,13 @@
  * rounded to nearest-even once, at the store.
  *
  * Ownership and streams.  Every pointer is a device pointer owned by the
- * caller, including the workspace.  The library allocates no memory, keeps
- * no state between calls and never synchronises the stream; calls are
- * asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ * caller, including the workspace.  gspn_fwd and gspn_bwd allocate no memory,
+ * keep no state between calls and never synchronise the stream (unless
+ * gspn_set_sync_check is on); calls are asynchronous on `stream` (a
+ * cudaStream_t; NULL = legacy default stream).  The one exception is
+ * gspn_fwd_noalloc, whose scratch is a fixed device array of the library
+ * itself (see there).  Process-wide settings: the device wait limit, the
+ * synchronous check and the stall test hook below.
  * Outputs are overwritten, never accumulated into.  Inputs and outputs must
  * not alias.  Concurrent calls on different streams may not share a
  * workspace.
@@ -67,6 +71,20 @@
  *                         runtime's own error is left for cudaGetLastError);
  *   GSPN_ERR_SCRATCH_LIMIT  (gspn_fwd_noalloc only) the problem does not fit
  *                         the library's fixed scratch.
+ * Device-side timeouts.  The TMA-fed kernels (the compact 64x64 and 128x128
+ * paths; gspn_variant_name names them "compact*_tma_*") hand data between
+ * warps through shared-memory barriers.  Every such wait is bounded (2 s by
+ * default, gspn_set_wait_limit_ns); when one runs out, the kernel records an
+ * error word in its workspace, waits for its own copies in flight, frees its
+ * tensor memory and returns, so the GPU stays usable but the outputs are not
+ * valid.  The launching call has already returned GSPN_OK by then; the caller
+ * learns of the timeout with gspn_device_status (or gspn_noalloc_status),
+ * which synchronises the stream and returns
+ *   GSPN_ERR_TIMEOUT      a bounded device wait of the last call that used
+ *                         this workspace ran out.
+ * With gspn_set_sync_check(1) every gspn_fwd / gspn_bwd / gspn_fwd_noalloc
+ * synchronises its stream itself and returns GSPN_ERR_TIMEOUT directly (a
+ * debugging mode: it serialises the host with the GPU).
  * No exception or signal crosses the ABI.
  */
 #ifndef GSPN_H_
@@ -149,15 +167,105 @@ gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, c
  * return GSPN_ERR_SCRATCH_LIMIT and other descriptors GSPN_ERR_UNSUPPORTED,
  * both before any launch; argument errors are reported as by gspn_fwd.
  *
- * The first call on a device looks up the array's device address for that
- * device (cudaGetSymbolAddress) and caches it; make that first call before
- * any stream capture begins.  All calls share the one array and each call
- * rewrites what it reads, so results never depend on an earlier call, but
- * calls whose execution overlaps on the GPU (different streams, or graphs
- * replayed concurrently) race on it: serialise them.  Nothing is allocated
- * or freed, here or in any library routine this calls. */
+ * Every call looks up the array's device address in the current context
+ * (cudaGetSymbolAddress; in host code the array's name is not a device
+ * address), so a context torn down and recreated (cudaDeviceReset) gets the
+ * new address.  With lazy module loading (the CUDA 12 default) the first call
+ * on a device also makes the runtime load the module, which places the array:
+ * make that first call before any stream capture begins.  All calls share the
+ * one array and each call rewrites what it reads, so results never depend on
+ * an earlier call, but calls whose execution overlaps on the GPU (different
+ * streams, or graphs replayed concurrently) race on it: serialise them.
+ * Beyond that first module load, nothing is allocated or freed, here or in
+ * any library routine this calls.  gspn_noalloc_status reads the array's
+ * error word. */
 gspn_status gspn_fwd_noalloc(const gspn_desc* desc, const void* x, const void* logits, const void* lambda,
                              void* out, void* stream);
+
+/* Synchronises `stream`, then reports how the last gspn_fwd (backward = 0)
+ * or gspn_bwd (backward = 1) call with this descriptor and this workspace
+ * ended on the device: GSPN_ERR_TIMEOUT if one of its bounded waits ran out
+ * (its outputs are then invalid), GSPN_ERR_CUDA if the stream reports a CUDA
+ * error, else GSPN_OK.  Kernel families without device-side waits always
+ * give GSPN_OK after the synchronisation.  workspace: the one that call
+ * used (may be NULL only for those families).  No counterpart in the GSPN
+ * pages: it is how a caller learns of a timeout (see "Device-side timeouts"
+ * above). */
+gspn_status gspn_device_status(const gspn_desc* desc, int backward, const void* workspace, void* stream);
+
+/* The same for the last gspn_fwd_noalloc call: synchronises `stream` and reads
+ * the error word of the library's fixed scratch. */
+gspn_status gspn_noalloc_status(void* stream);
+
+/* Sets the limit, in nanoseconds, of every device-side wait of the TMA-fed
+ * kernels on data, a pipeline stage or another warp, for launches made after
+ * the call, process-wide; 0 restores the default of 2 s.  Returns the
+ * previous limit.  Waits that only drain a kernel's own copies or release its
+ * tensor memory keep fixed bounds (0.1 s and 20 s).  Thread-safe. */
+uint64_t gspn_set_wait_limit_ns(uint64_t limit_ns);
+
+/* on != 0: every later gspn_fwd, gspn_bwd and gspn_fwd_noalloc call
+ * synchronises its stream and returns GSPN_ERR_TIMEOUT itself when a wait ran
+ * out (a debugging mode).  Returns the previous setting.  Process-wide. */
+int gspn_set_sync_check(int on);
+
+/* Test hook for the timeout path.  on != 0: in every later launch of a
+ * TMA-fed kernel, one warp of the first CTA begins with a wait on a barrier
+ * that only its own final arrival can complete, so that wait runs out after
+ * the wait limit and the kernel ends through its error path (the other warps'
+ * waits then run out in turn).  No fault, trap or unbounded wait is involved.
+ * Returns the previous setting.  Process-wide; off by default. */
+int gspn_set_stall_test(int on);
+
+/* ---- Compressed propagation block --------------------------------------------
+ *
+ * y = U . RMSNorm_k( sum_d alpha[d,k] scan_d(V . x) ) . gamma, per pixel:
+ *   xp[b,k]  = sum_c V[k,c] x[b,c]                  proxy projection to Cp channels
+ *   h_d[b,k] = the GSPN scan of xp[b,k] in direction d (channel-shared taps,
+ *              per-channel lambda, local groups as in gspn_fwd)
+ *   m[b,k]   = sum_d alpha[d,k] h_d[b,k]             learnable merger
+ *   n[b,k]   = gamma[k] m[b,k] / sqrt(mean_k m[b,k]^2 + eps)   (norm = 1; n = m if 0)
+ *   y[b,c]   = sum_k U[c,k] n[b,k]                   projection back to C channels
+ * Sources: "GSPN-2: Efficient Parallel Sequence Modeling" (OpenReview response,
+ * "Relate Compressive Proxy Dimension to Low-rank Approximation": a linear
+ * layer to C_proxy channels, the recurrence there, the projection back);
+ * "Parallel Sequence Modeling via Generalized Spatial Propagation Network",
+ * Key design 2 (the four directions aggregated by a learnable merger);
+ * "Scaling Parallel Sequence Models to Vision Foundation Models", abstract (a
+ * compressed latent-space propagation block with fused normalisation).  The
+ * pages give neither the merger's nor the normalisation's formula: this
+ * library reads them as one weight per (direction, proxy channel) and as an
+ * RMS normalisation over the proxy channels of each pixel with a per-channel
+ * gain (a LayerNorm over 2 proxy channels would collapse to +-1).
+ *
+ * Layouts (dense, row-major): x, y [B,C,H,W] bf16; v_proj [Cp,C] bf16;
+ * u_proj [C,Cp] bf16; lambda [4,B,Cp,H,W] bf16; logits [4,B,1,3,H,W] bf16
+ * (one tap set per pixel and direction for all proxy channels); alpha [4,Cp]
+ * fp32; gamma [Cp] fp32.  The 4 axis is T2B, B2T, L2R, R2L.  Arithmetic is
+ * fp32 (the projections on the tensor cores with bf16 operands: x, V and U as
+ * stored, n rounded to bf16 once); y is rounded to bf16 once.
+ * Limits (else GSPN_ERR_UNSUPPORTED): 1 <= Cp <= 32, H and W <= 128, C and H*W
+ * multiples of 8, C <= 3072 (Cp <= 16) or 1536 (Cp <= 32).
+ * Errors and ownership as for gspn_fwd; a bounded device wait that runs out
+ * is reported by gspn_block_device_status. */
+typedef struct {
+    int64_t B, C, H, W;  /* batch, channels, rows, columns; each >= 1 */
+    int32_t Cp;          /* proxy channels */
+    int32_t groups;      /* local groups along each scan axis; 1 = global scan */
+    int32_t norm;        /* 1: RMS normalisation over the proxy channels */
+    float eps;           /* 0 <= eps <= 1, added to the mean square */
+} gspn_block_desc;
+
+/* Bytes of device workspace (256-byte aligned) gspn_block_fwd needs; 0 for a
+ * descriptor it would reject. */
+size_t gspn_block_workspace_size(const gspn_block_desc* desc);
+
+gspn_status gspn_block_fwd(const gspn_block_desc* desc, const void* x, const void* v_proj, const void* logits,
+                           const void* lambda, const float* alpha, const float* gamma, const void* u_proj, void* y,
+                           void* workspace, size_t ws_bytes, void* stream);
+
+/* As gspn_device_status, for the last gspn_block_fwd with this workspace. */
+gspn_status gspn_block_device_status(const gspn_block_desc* desc, const void* workspace, void* stream);
 
 /* Number of kernel launches one gspn_fwd (backward = 0) / gspn_bwd
  * (backward = 1) call with this descriptor issues; 0 for a descriptor the

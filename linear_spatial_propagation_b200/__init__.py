@@ -25,14 +25,23 @@ STATUS = {
 }
 
 # every symbol include/gspn.h declares
-EXPORTS = ("gspn_workspace_size", "gspn_fwd", "gspn_bwd", "gspn_fwd_noalloc", "gspn_launches_per_call",
-           "gspn_variant_name", "gspn_status_string", "gspn_version")
+EXPORTS = ("gspn_workspace_size", "gspn_fwd", "gspn_bwd", "gspn_fwd_noalloc", "gspn_device_status",
+           "gspn_noalloc_status", "gspn_set_wait_limit_ns", "gspn_set_sync_check", "gspn_set_stall_test",
+           "gspn_block_workspace_size", "gspn_block_fwd", "gspn_block_device_status",
+           "gspn_launches_per_call", "gspn_variant_name", "gspn_status_string", "gspn_version")
 
 
 class GspnError(RuntimeError):
     def __init__(self, status: int, what: str):
         super().__init__(f"{what}: {STATUS.get(status, status)} ({gspn_status_string(status)})")
         self.status = status
+
+
+class gspn_block_desc(ctypes.Structure):
+    _fields_ = [
+        ("B", ctypes.c_int64), ("C", ctypes.c_int64), ("H", ctypes.c_int64), ("W", ctypes.c_int64),
+        ("Cp", ctypes.c_int32), ("groups", ctypes.c_int32), ("norm", ctypes.c_int32), ("eps", ctypes.c_float),
+    ]
 
 
 class gspn_desc(ctypes.Structure):
@@ -69,6 +78,23 @@ def load(build_if_missing: bool = True) -> ctypes.CDLL:
     lib.gspn_bwd.restype = ctypes.c_int
     lib.gspn_fwd_noalloc.argtypes = [dp, vp, vp, vp, vp, vp]
     lib.gspn_fwd_noalloc.restype = ctypes.c_int
+    lib.gspn_device_status.argtypes = [dp, ctypes.c_int, vp, vp]
+    lib.gspn_device_status.restype = ctypes.c_int
+    lib.gspn_noalloc_status.argtypes = [vp]
+    lib.gspn_noalloc_status.restype = ctypes.c_int
+    lib.gspn_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+    lib.gspn_set_wait_limit_ns.restype = ctypes.c_uint64
+    lib.gspn_set_sync_check.argtypes = [ctypes.c_int]
+    lib.gspn_set_sync_check.restype = ctypes.c_int
+    lib.gspn_set_stall_test.argtypes = [ctypes.c_int]
+    lib.gspn_set_stall_test.restype = ctypes.c_int
+    bdp = ctypes.POINTER(gspn_block_desc)
+    lib.gspn_block_workspace_size.argtypes = [bdp]
+    lib.gspn_block_workspace_size.restype = sz
+    lib.gspn_block_fwd.argtypes = [bdp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.gspn_block_fwd.restype = ctypes.c_int
+    lib.gspn_block_device_status.argtypes = [bdp, vp, vp]
+    lib.gspn_block_device_status.restype = ctypes.c_int
     lib.gspn_launches_per_call.argtypes = [dp, ctypes.c_int]
     lib.gspn_launches_per_call.restype = ctypes.c_int
     lib.gspn_variant_name.argtypes = [dp, ctypes.c_int]
@@ -106,6 +132,46 @@ def gspn_fwd_noalloc(desc: gspn_desc, x: int, logits: int, lam: int, out: int, s
     """Forward on the library's fixed device scratch: for callers that cannot
     allocate device memory (no workspace argument).  See include/gspn.h."""
     return int(load().gspn_fwd_noalloc(ctypes.byref(desc), x, logits, lam, out, stream or None))
+
+
+def gspn_device_status(desc: gspn_desc, backward: int, workspace: int, stream: int) -> int:
+    """Synchronise `stream`; GSPN_ERR_TIMEOUT if a bounded device wait of the
+    last call with this workspace ran out (see include/gspn.h)."""
+    return int(load().gspn_device_status(ctypes.byref(desc), int(backward), workspace or None, stream or None))
+
+
+def gspn_noalloc_status(stream: int) -> int:
+    return int(load().gspn_noalloc_status(stream or None))
+
+
+def gspn_set_wait_limit_ns(limit_ns: int) -> int:
+    return int(load().gspn_set_wait_limit_ns(int(limit_ns)))
+
+
+def gspn_set_sync_check(on: int) -> int:
+    return int(load().gspn_set_sync_check(int(on)))
+
+
+def gspn_set_stall_test(on: int) -> int:
+    return int(load().gspn_set_stall_test(int(on)))
+
+
+def make_block_desc(B, C, H, W, Cp, groups=1, norm=True, eps=1e-6) -> gspn_block_desc:
+    return gspn_block_desc(int(B), int(C), int(H), int(W), int(Cp), int(groups), int(bool(norm)), float(eps))
+
+
+def gspn_block_workspace_size(desc: gspn_block_desc) -> int:
+    return int(load().gspn_block_workspace_size(ctypes.byref(desc)))
+
+
+def gspn_block_fwd(desc: gspn_block_desc, x: int, v_proj: int, logits: int, lam: int, alpha: int, gamma: int,
+                   u_proj: int, y: int, workspace: int, ws_bytes: int, stream: int) -> int:
+    return int(load().gspn_block_fwd(ctypes.byref(desc), x, v_proj, logits, lam, alpha, gamma, u_proj, y,
+                                     workspace or None, int(ws_bytes), stream or None))
+
+
+def gspn_block_device_status(desc: gspn_block_desc, workspace: int, stream: int) -> int:
+    return int(load().gspn_block_device_status(ctypes.byref(desc), workspace or None, stream or None))
 
 
 def gspn_launches_per_call(desc: gspn_desc, backward: int = 0) -> int:
@@ -209,3 +275,33 @@ def backward(x, logits, lam, dout, dir_mask=ALL_DIRS, groups=1, shared=False, gr
     if st != 0:
         raise GspnError(st, "gspn_bwd")
     return dx, dlg, dlam
+
+
+def block_forward(x, v_proj, logits, lam, alpha, gamma, u_proj, groups=1, norm=True, eps=1e-6, y=None, ws=None,
+                  stream=None):
+    """y of the compressed propagation block (layouts as in include/gspn.h):
+    x [B,C,H,W], v_proj [Cp,C], u_proj [C,Cp], logits [4,B,1,3,H,W],
+    lam [4,B,Cp,H,W] (all bf16); alpha [4,Cp], gamma [Cp] (fp32)."""
+    torch = _torch()
+    B, C, H, W = x.shape
+    Cp = v_proj.shape[0]
+    desc = make_block_desc(B, C, H, W, Cp, groups, norm, eps)
+    bf, f32 = torch.bfloat16, torch.float32
+    for t, shp, n, dt in ((x, (B, C, H, W), "x", bf), (v_proj, (Cp, C), "v_proj", bf), (u_proj, (C, Cp), "u_proj", bf),
+                          (logits, (4, B, 1, 3, H, W), "logits", bf), (lam, (4, B, Cp, H, W), "lam", bf),
+                          (alpha, (4, Cp), "alpha", f32), (gamma, (Cp,), "gamma", f32)):
+        _check(t, shp, n, dt, x.device)
+    if y is None:
+        y = torch.empty_like(x)
+    _check(y, (B, C, H, W), "y", bf, x.device)
+    if ws is None:
+        n = gspn_block_workspace_size(desc)
+        if n == 0:
+            raise GspnError(2, "gspn_block_workspace_size")
+        ws = torch.empty(n, dtype=torch.uint8, device=x.device)
+    s = stream if stream is not None else torch.cuda.current_stream(x.device).cuda_stream
+    st = gspn_block_fwd(desc, x.data_ptr(), v_proj.data_ptr(), logits.data_ptr(), lam.data_ptr(), alpha.data_ptr(),
+                        gamma.data_ptr(), u_proj.data_ptr(), y.data_ptr(), ws.data_ptr(), ws.numel(), s)
+    if st != 0:
+        raise GspnError(st, "gspn_block_fwd")
+    return y

@@ -12,7 +12,8 @@ namespace gspn {
 namespace {
 
 constexpr int kMaxDevices = 64;
-constexpr int kMaxAttrSlots = 32;
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;  // 2 s
+constexpr int kMaxAttrSlots = 48;
 
 struct DevCache {
     std::atomic<int> ready{0};
@@ -75,15 +76,51 @@ gspn_status check_ws(void* ws, size_t have, size_t need) {
 // The kernel family a descriptor runs on: the TMA-fed compact kernels for their
 // shapes, the one-CTA-per-plane kernels for planes of at most 64x64, the generic
 // kernels for everything else.
-enum class Path { kC64, kC128, kSmall, kGeneric };
+enum class Path { kC64, kC128, kSmall, kLarge, kGeneric };
 Path pick(const Problem& p, int backward) {
     if (backward ? c64_bwd_eligible(p) : c64_eligible(p)) return Path::kC64;
     if (backward ? c128_bwd_eligible(p) : c128_eligible(p)) return Path::kC128;
     if (small_eligible(p, backward)) return Path::kSmall;
+    if (!backward && large_eligible(p)) return Path::kLarge;
     return Path::kGeneric;
 }
 
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int> g_stall_test{0};
+std::atomic<int> g_sync_check{0};
+
+// The error word a TMA-fed kernel family sets when a bounded wait expires sits
+// at offset 0 of its workspace; the other families have no device-side waits.
+bool has_status_word(Path path) { return path == Path::kC64 || path == Path::kC128; }
+
+// Synchronises `s` and maps the call's outcome to a status: a CUDA error, an
+// expired wait recorded in the error word at `word` (null: none), or OK.
+gspn_status sync_status(const void* word, cudaStream_t s) {
+    int v = 0;
+    if (word && cudaMemcpyAsync(&v, word, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GSPN_ERR_CUDA;
+    return v ? GSPN_ERR_TIMEOUT : GSPN_OK;
+}
+
 }  // namespace
+
+EncodeTiledFn encode_tiled() {
+    // a function-local static: initialised exactly once, even under concurrent first calls
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return reinterpret_cast<EncodeTiledFn>(p);
+    }();
+    return fn;
+}
+
+WaitCfg wait_cfg() {
+    return WaitCfg{g_wait_limit_ns.load(std::memory_order_relaxed), g_stall_test.load(std::memory_order_relaxed)};
+}
 
 cudaError_t device_info(DeviceInfo* out) {
     int dev = 0;
@@ -154,6 +191,7 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     case Path::kC64: return backward ? c64_bwd_workspace(p, dev) : c64_fwd_workspace(p);
     case Path::kC128: return backward ? c128_bwd_workspace(p, dev) : c128_fwd_workspace(p, dev);
     case Path::kSmall: return backward ? small_bwd_workspace(p) : 0;
+    case Path::kLarge: return large_fwd_workspace(p);
     default: return backward ? generic_bwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
     }
 }
@@ -165,6 +203,7 @@ int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     case Path::kC64:
     case Path::kC128: return backward ? 3 : 2;
     case Path::kSmall: return backward ? small_bwd_launches(p) : 1;
+    case Path::kLarge: return 1;
     default: return backward ? generic_bwd_launches(p) : 1;
     }
 }
@@ -176,6 +215,7 @@ const char* gspn_variant_name(const gspn_desc* desc, int backward) {
     case Path::kC64: return backward ? "compact64_tma_bwd" : "compact64_tma_fwd";
     case Path::kC128: return backward ? "compact128_tma_bwd" : "compact128_tma_fwd";
     case Path::kSmall: return backward ? "small_plane_bwd" : "small_plane_fwd";
+    case Path::kLarge: return "large_plane_fwd";
     default: return backward ? "generic_bwd" : "generic_fwd";
     }
 }
@@ -194,13 +234,17 @@ gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, c
                   path == Path::kC64    ? c64_fwd_workspace(p)
                   : path == Path::kC128 ? c128_fwd_workspace(p, dev)
                   : path == Path::kSmall ? 0
+                  : path == Path::kLarge ? large_fwd_workspace(p)
                                          : generic_fwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (path == Path::kC64) return c64_fwd(p, dev, x, logits, lambda, out, workspace, cs);
-    if (path == Path::kC128) return c128_fwd(p, dev, x, logits, lambda, out, workspace, cs);
-    if (path == Path::kSmall) return small_fwd(p, dev, x, logits, lambda, out, cs);
-    return generic_fwd(p, dev, x, logits, lambda, out, workspace, static_cast<cudaStream_t>(stream));
+    st = path == Path::kC64    ? c64_fwd(p, dev, x, logits, lambda, out, workspace, cs)
+         : path == Path::kC128 ? c128_fwd(p, dev, x, logits, lambda, out, workspace, cs)
+         : path == Path::kSmall ? small_fwd(p, dev, x, logits, lambda, out, cs)
+         : path == Path::kLarge ? large_fwd(p, x, logits, lambda, out, workspace, cs)
+                                : generic_fwd(p, dev, x, logits, lambda, out, workspace, cs);
+    if (st != GSPN_OK || !g_sync_check.load(std::memory_order_relaxed)) return st;
+    return sync_status(has_status_word(path) ? workspace : nullptr, cs);
 }
 
 gspn_status gspn_fwd_noalloc(const gspn_desc* desc, const void* x, const void* logits, const void* lambda, void* out,
@@ -212,8 +256,47 @@ gspn_status gspn_fwd_noalloc(const gspn_desc* desc, const void* x, const void* l
     if (st != GSPN_OK) return st;
     DeviceInfo dev;
     if (device_info(&dev) != cudaSuccess) return GSPN_ERR_CUDA;
-    return c64_fwd_noalloc(p, dev, x, logits, lambda, out, static_cast<cudaStream_t>(stream));
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    st = c64_fwd_noalloc(p, dev, x, logits, lambda, out, cs);
+    if (st != GSPN_OK || !g_sync_check.load(std::memory_order_relaxed)) return st;
+    return c64_noalloc_status(cs);
 }
+
+gspn_status gspn_noalloc_status(void* stream) { return c64_noalloc_status(static_cast<cudaStream_t>(stream)); }
+
+gspn_status gspn_device_status(const gspn_desc* desc, int backward, const void* workspace, void* stream) {
+    Problem p;
+    gspn_status st = validate(desc, &p);
+    if (st != GSPN_OK) return st;
+    const bool word = has_status_word(pick(p, backward));
+    if (word && !workspace) return GSPN_ERR_INVALID_ARG;
+    return sync_status(word ? workspace : nullptr, static_cast<cudaStream_t>(stream));
+}
+
+size_t gspn_block_workspace_size(const gspn_block_desc* desc) { return block_workspace(desc); }
+
+gspn_status gspn_block_fwd(const gspn_block_desc* desc, const void* x, const void* v_proj, const void* logits,
+                           const void* lambda, const float* alpha, const float* gamma, const void* u_proj, void* y,
+                           void* workspace, size_t ws_bytes, void* stream) {
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    gspn_status st = block_fwd(desc, x, v_proj, logits, lambda, alpha, gamma, u_proj, y, workspace, ws_bytes, cs);
+    if (st != GSPN_OK || !g_sync_check.load(std::memory_order_relaxed)) return st;
+    return sync_status(workspace, cs);
+}
+
+gspn_status gspn_block_device_status(const gspn_block_desc* desc, const void* workspace, void* stream) {
+    if (block_workspace(desc) == 0) return GSPN_ERR_INVALID_ARG;
+    if (!workspace) return GSPN_ERR_INVALID_ARG;
+    return sync_status(workspace, static_cast<cudaStream_t>(stream));
+}
+
+uint64_t gspn_set_wait_limit_ns(uint64_t limit_ns) {
+    return g_wait_limit_ns.exchange(limit_ns ? limit_ns : kDefaultWaitLimitNs);
+}
+
+int gspn_set_sync_check(int on) { return g_sync_check.exchange(on ? 1 : 0); }
+
+int gspn_set_stall_test(int on) { return g_stall_test.exchange(on ? 1 : 0); }
 
 gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, const void* lambda,
                      const void* dout, void* dx, void* dlogits, void* dlambda, void* workspace, size_t ws_bytes,
@@ -233,11 +316,12 @@ gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, c
                                          : generic_bwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
-    if (path == Path::kC64) return c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
-    if (path == Path::kC128) return c128_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
-    if (path == Path::kSmall) return small_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
-    return generic_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace,
-                       static_cast<cudaStream_t>(stream));
+    st = path == Path::kC64     ? c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs)
+         : path == Path::kC128  ? c128_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs)
+         : path == Path::kSmall ? small_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs)
+                                : generic_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
+    if (st != GSPN_OK || !g_sync_check.load(std::memory_order_relaxed)) return st;
+    return sync_status(has_status_word(path) ? workspace : nullptr, cs);
 }
 
 }  // extern "C"

@@ -158,6 +158,8 @@ struct C128Args {
     int* err;
     int B, C, segmask;
     int groups;  // B * C / 4 groups of 4 consecutive planes (one batch image each)
+    uint64_t limit;  // bound of every wait on data, a stage or another warp (ns)
+    int stall;       // test hook: consumer warp 0 of CTA 0 first waits on a barrier nothing completes
 };
 
 template <bool LOCAL>
@@ -224,7 +226,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int local = kk % CHUNKS_PER_GROUP, pass = local >> 4, q = local & 15;
                 if (pw == 0) {
                     const int ws = kk % NWS;
-                    if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kk / NWS) & 1) ^ 1, 32)) {
+                    if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kk / NWS) & 1) ^ 1, 32, a.limit)) {
                         ok = false;
                         break;
                     }
@@ -234,7 +236,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
                 }
                 const int st = kk % NST;
-                if (!tma::mbar_wait_sleep(xempty0 + 8 * (pw * NST + st), ((kk / NST) & 1) ^ 1, 32)) {
+                if (!tma::mbar_wait_sleep(xempty0 + 8 * (pw * NST + st), ((kk / NST) & 1) ^ 1, 32, a.limit)) {
                     ok = false;
                     break;
                 }
@@ -291,7 +293,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_wait(rbar0 + 8 * (i % NRS), (i / NRS) & 1, 100000000ull);
     };
     auto taps_in = [&](int kc) -> bool {
-        const bool ok = tma::mbar_wait(wfull0 + 8 * (kc % NWS), (kc / NWS) & 1);
+        const bool ok = tma::mbar_wait(wfull0 + 8 * (kc % NWS), (kc / NWS) & 1, a.limit);
         return __all_sync(FULL, ok);
     };
     // Stages are handed back by every lane: its generic-proxy reads of the stage
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         tma::mbar_arrive(wempty0 + 8 * (kc % NWS));
     };
     auto acquire = [&]() -> bool {
-        const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
+        const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u, a.limit);
         return __all_sync(FULL, ok);
     };
     // the stage is in registers: hand it back to its producer
@@ -425,7 +427,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         release();
         const unsigned char* rs = nullptr;
         if (q < 8) {
-            if (!__all_sync(FULL, tma::mbar_wait(rbar0 + 8 * (q % NRS), (q / NRS) & 1))) return false;
+            if (!__all_sync(FULL, tma::mbar_wait(rbar0 + 8 * (q % NRS), (q / NRS) & 1, a.limit))) return false;
             ++rs_done;
             rs = rsp + (q % NRS) * RSTAGE + t * 16;
         }
@@ -490,6 +492,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
 
     bool ok = true;
+    if (a.stall && blockIdx.x == 0 && warp == 0) {
+        // test hook: phase 0 of done0 needs this warp's own final arrival, so
+        // this wait can only run out; the kernel then takes its error path
+        ok = __all_sync(FULL, tma::mbar_wait(done0, 0, a.limit));
+    }
     for (int group = blockIdx.x; ok && group < a.groups; group += gridDim.x) {
         const int plane = NCW * group + warp;
         outp = a.out + (size_t)plane * S * S + 4 * t;
@@ -526,29 +533,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---- host side ----------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn128() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 // Row-pass view of a stack of 128x128 bf16 planes: (column, row / 4, row % 4,
 // plane), one box = 8 columns of all 128 rows, laid out [row % 4][row / 4][8 columns].
 bool make_map_cols(CUtensorMap* m, const void* base, uint64_t planes) {
-    EncodeTiledFn fn = encode_fn128();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[4] = {S, S / 4, 4, planes};
     const cuuint64_t strides[3] = {4 * S * 2, S * 2, (cuuint64_t)S * S * 2};
@@ -561,7 +549,7 @@ bool make_map_cols(CUtensorMap* m, const void* base, uint64_t planes) {
 
 // Column-pass view: (column, row, plane), one box = all 128 columns of 8 rows.
 bool make_map_rows(CUtensorMap* m, const void* base, uint64_t planes) {
-    EncodeTiledFn fn = encode_fn128();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, (cuuint64_t)S * S * 2};
@@ -582,7 +570,7 @@ size_t c128_tab_bytes(const Problem& p) { return align_up((size_t)p.g.B * 2 * S 
 
 bool c128_eligible(const Problem& p) {
     return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
-           S % p.g.groups == 0 && p.g.C % NCW == 0 && p.planes <= 0x7fffffff / 4 && encode_fn128() != nullptr;
+           S % p.g.groups == 0 && p.g.C % NCW == 0 && p.planes <= 0x7fffffff / 4 && encode_tiled() != nullptr;
 }
 
 size_t c128_fwd_workspace(const Problem& p, const DeviceInfo& dev) {
@@ -601,6 +589,9 @@ gspn_status c128_fwd(const Problem& p, const DeviceInfo& dev, const void* x, con
     char* w = static_cast<char*>(ws);
     C128Args a;
     a.err = reinterpret_cast<int*>(w);
+    const WaitCfg wc = wait_cfg();
+    a.limit = wc.limit_ns;
+    a.stall = wc.stall;
     a.wtab = reinterpret_cast<const float4*>(w + kWsAlign);
     a.rsum = reinterpret_cast<float*>(w + kWsAlign + c128_tab_bytes(p));
     a.out = static_cast<__nv_bfloat16*>(out);

@@ -163,6 +163,8 @@ struct C128BArgs {
     int B, C;
     int groups;   // B * C / 4
     int segmask;  // local groups: lines per group - 1 (127 = global)
+    uint64_t limit;  // bound of every wait on data, a stage or another warp (ns)
+    int stall;       // test hook: compute warp 0 of CTA 0 first waits on a barrier nothing completes
 };
 
 // bf16 element e of 8 packed in a uint4, widened
@@ -301,7 +303,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (t == 0) {
             for (int kc = 0; kc < nchunks; ++kc) {
                 const int ws = kc % NWS;
-                if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1, 200)) {
+                if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1, 200, a.limit)) {
                     atomicExch(a.err, 1);
                     break;
                 }
@@ -335,7 +337,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int pass = l >> 5, q = 15 - ((l >> 1) & 15), h = 1 - (l & 1), set = n % NSET;
                 if (set != rid) continue;
                 float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S + (8 * q + 4 * h) * S;
-                if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n / NSET) & 1, 128))) {
+                if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n / NSET) & 1, 128, a.limit))) {
                     ok = false;
                     break;
                 }
@@ -444,8 +446,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (t == 0) tma::bulk_wait_all();
     };
     auto acquire = [&]() -> bool {
-        const bool ok1 = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
-        const bool ok2 = tma::mbar_wait(wfull0 + 8 * (k % NWS), (k / NWS) & 1);
+        const bool ok1 = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u, a.limit);
+        const bool ok2 = tma::mbar_wait(wfull0 + 8 * (k % NWS), (k / NWS) & 1, a.limit);
         return __all_sync(FULL, ok1 && ok2);
     };
     // the data stage is in registers: refill it (every lane orders its reads of
@@ -492,7 +494,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // dchunk % NSET, free once the reducer has handed the set back
     int dchunk = 0;
     auto dslot = [&]() -> float* {
-        const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk % NSET), ((dchunk / NSET) & 1) ^ 1);
+        const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk % NSET), ((dchunk / NSET) & 1) ^ 1, a.limit);
         if (!__all_sync(FULL, ok)) return nullptr;
         return reinterpret_cast<float*>(smem + DSTG + ((dchunk % NSET) * NCW + warp) * DSLOT);
     };
@@ -502,7 +504,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
 
     const Taps4 zero_taps = {{make_float2(0.f, 0.f), make_float2(0.f, 0.f)}, {make_float2(0.f, 0.f), make_float2(0.f, 0.f)}};
-    for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
+    bool stalled = false;
+    if (a.stall && blockIdx.x == 0 && warp == 0 &&
+        !__all_sync(FULL, tma::mbar_wait(done0, 0, a.limit))) {
+        // test hook: phase 0 of done0 needs this warp's own final arrival, so the
+        // wait above can only run out; take the error path
+        fail();
+        stalled = true;
+    }
+    for (int group = blockIdx.x; !stalled && group < a.groups; group += gridDim.x) {
         const int plane = NCW * group + warp;
 
         auto run_pass = [&](auto pass_c) -> bool {
@@ -621,7 +631,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                 }
                 release_data();
-                if (!__all_sync(FULL, tma::mbar_wait(abar0 + 8 * (qq % NAS), (qq / NAS) & 1))) {
+                if (!__all_sync(FULL, tma::mbar_wait(abar0 + 8 * (qq % NAS), (qq / NAS) & 1, a.limit))) {
                     ++k;  // the data stage of this chunk was consumed
                     fail();
                     return false;
@@ -795,29 +805,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---- host side ----------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn128b() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 // Row-pass view of a stack of 128x128 bf16 planes: (column, row / 4, row % 4,
 // plane); one box = 8 columns of all 128 rows, laid out [row % 4][row / 4][8 columns].
 bool make_map_cols_b(CUtensorMap* m, const void* base, uint64_t planes) {
-    EncodeTiledFn fn = encode_fn128b();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[4] = {S, S / 4, 4, planes};
     const cuuint64_t strides[3] = {4 * S * 2, S * 2, (cuuint64_t)S * S * 2};
@@ -830,7 +821,7 @@ bool make_map_cols_b(CUtensorMap* m, const void* base, uint64_t planes) {
 
 // Column-pass view: (column, row, plane); one box = all 128 columns of 8 rows.
 bool make_map_rows_b(CUtensorMap* m, const void* base, uint64_t planes) {
-    EncodeTiledFn fn = encode_fn128b();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, (cuuint64_t)S * S * 2};
@@ -852,7 +843,7 @@ size_t c128b_sum_bytes(const Problem& p) { return align_up((size_t)p.g.B * 2 * 4
 
 bool c128_bwd_eligible(const Problem& p) {
     return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
-           S % p.g.groups == 0 && p.g.C % NCW == 0 && p.planes <= 0x7fffffff / 4 && encode_fn128b() != nullptr;
+           S % p.g.groups == 0 && p.g.C % NCW == 0 && p.planes <= 0x7fffffff / 4 && encode_tiled() != nullptr;
 }
 
 size_t c128_bwd_workspace(const Problem& p, const DeviceInfo& dev) {
@@ -874,6 +865,9 @@ gspn_status c128_bwd(const Problem& p, const DeviceInfo& dev, const void* x, con
     char* w = static_cast<char*>(ws);
     C128BArgs a;
     a.err = reinterpret_cast<int*>(w);
+    const WaitCfg wc = wait_cfg();
+    a.limit = wc.limit_ns;
+    a.stall = wc.stall;
     a.btab = reinterpret_cast<const float4*>(w + kWsAlign);
     a.dsum = reinterpret_cast<float*>(w + kWsAlign + c128b_tab_bytes(p));
     a.dxh = reinterpret_cast<float*>(w + kWsAlign + c128b_tab_bytes(p) + c128b_sum_bytes(p));

@@ -50,7 +50,6 @@
 //   pass (each lane reads columns 2t, 2t+1 of one row).
 // * Every mbarrier wait is bounded (2 s); on expiry the warp records an
 //   error word in the workspace, drains its outstanding copies and returns.
-#include <atomic>
 #include <type_traits>
 
 #include "gspn_internal.h"
@@ -139,6 +138,8 @@ struct C64Args {
     int* err;
     int B, C, seg;
     int groups;  // B * C / 8 groups of 8 consecutive planes (one batch image each)
+    uint64_t limit;  // bound of every wait on data, a stage or another warp (ns)
+    int stall;       // test hook: consumer warp 0 of CTA 0 first waits on a barrier nothing completes
 };
 
 template <bool LOCAL>
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int local = kk % CHUNKS_PER_GROUP, st = kk % NST;
                 if (pw == 0) {
                     const int ws = kk % NWS;
-                    if (!tma::mbar_wait(wempty0 + 8 * ws, ((kk / NWS) & 1) ^ 1)) {
+                    if (!tma::mbar_wait(wempty0 + 8 * ws, ((kk / NWS) & 1) ^ 1, a.limit)) {
                         ok = false;
                         break;
                     }
@@ -216,7 +217,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
                 }
                 for (int w = 2 * pw; w < 2 * pw + 2; ++w) {
-                    if (!tma::mbar_wait(xempty0 + 8 * (w * NST + st), ((kk / NST) & 1) ^ 1)) {
+                    if (!tma::mbar_wait(xempty0 + 8 * (w * NST + st), ((kk / NST) & 1) ^ 1, a.limit)) {
                         ok = false;
                         break;
                     }
@@ -287,7 +288,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         __syncwarp();
         if (t == 0) tma::mbar_arrive(wempty0 + 8 * (c % NWS));
         if (c + 1 < nchunks) {
-            const bool okw = tma::mbar_wait(wfull0 + 8 * ((c + 1) % NWS), ((c + 1) / NWS) & 1);
+            const bool okw = tma::mbar_wait(wfull0 + 8 * ((c + 1) % NWS), ((c + 1) / NWS) & 1, a.limit);
             if (!__all_sync(FULL, okw)) return false;
             const unsigned char* wsrc = wring + ((c + 1) % NWS) * WCHUNK + t * 16;
             wn[0] = lds128f(wsrc);
@@ -296,7 +297,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         return true;
     };
     auto acquire = [&]() -> bool {
-        const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
+        const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u, a.limit);
         return __all_sync(FULL, ok);
     };
     // the stage is in registers: hand it back to its producer
@@ -481,8 +482,13 @@ __global__ void __launch_bounds__(THREADS, 1)
     };
 
     bool ok = true;
-    if (nchunks > 0) {
-        const bool okw = tma::mbar_wait(wfull0, 0);
+    if (a.stall && blockIdx.x == 0 && warp == 0) {
+        // test hook: phase 0 of done0 needs this warp's own final arrival, so
+        // this wait can only run out; the kernel then takes its error path
+        ok = __all_sync(FULL, tma::mbar_wait(done0, 0, a.limit));
+    }
+    if (ok && nchunks > 0) {
+        const bool okw = tma::mbar_wait(wfull0, 0, a.limit);
         ok = __all_sync(FULL, okw);
         wc[0] = lds128f(wring + t * 16);
         wc[1] = lds128f(wring + t * 16 + 512);
@@ -515,30 +521,11 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---- host side ----------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 // 3-D view (column, row, plane) of a stack of 64x64 bf16 planes; one plane per
 // box of box_c columns x box_r rows (every row_step-th row).
 bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r, uint32_t row_step,
               CUtensorMapL2promotion promo) {
-    EncodeTiledFn fn = encode_fn();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, S * S * 2};
@@ -553,7 +540,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c,
 // 8 columns of all 64 rows, laid out [row % 2][row / 2][8 columns], so the
 // 16-byte reads of a warp (lane t: rows 2t, 2t+1) are conflict-free.
 bool make_map_cols(CUtensorMap* m, const void* base, uint64_t planes) {
-    EncodeTiledFn fn = encode_fn();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[4] = {S, S / 2, 2, planes};
     const cuuint64_t strides[3] = {2 * S * 2, S * 2, (cuuint64_t)S * S * 2};
@@ -579,7 +566,7 @@ gspn_status launch_c64(const DeviceInfo& dev, const CUtensorMap& xc, const CUten
 
 bool c64_eligible(const Problem& p) {
     return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
-           p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_fn() != nullptr;
+           p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_tiled() != nullptr;
 }
 
 size_t c64_fwd_workspace(const Problem& p) {
@@ -604,6 +591,9 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     a.C = p.g.C;
     a.seg = S / p.g.groups;
     a.groups = (int)(p.planes / 8);
+    const WaitCfg wc = wait_cfg();
+    a.limit = wc.limit_ns;
+    a.stall = wc.stall;
     const int nw = p.g.B * 2 * S * S;
     c64_weights_kernel<__nv_bfloat16><<<(nw + 255) / 256, 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(logits), const_cast<float4*>(a.wtab), a.err, p.g.B);
@@ -621,24 +611,37 @@ namespace {
 constexpr int kNoAllocMaxBatch = 32;
 constexpr size_t kNoAllocBytes = kWsAlign + (size_t)kNoAllocMaxBatch * 2 * S * S * sizeof(float4);
 __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocBytes];
-constexpr int kMaxNoAllocDevices = 64;
-std::atomic<void*> g_noalloc_ptr[kMaxNoAllocDevices];
+
+// Device address of the array in the current context.  In host code the
+// array's name is only a host-side stand-in.  The address is looked up on
+// every call (a host-side table lookup once the module is loaded), so a
+// context that was torn down and recreated -- cudaDeviceReset, or a primary
+// context released and retained again -- never sees a stale address.  With
+// lazy module loading the first call on a device also loads the module, which
+// places the array: make that first call before any stream capture begins.
+void* noalloc_scratch() {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+    return ptr;
+}
 }  // namespace
 
 gspn_status c64_fwd_noalloc(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
                             const void* lam, void* out, cudaStream_t s) {
     if (!c64_eligible(p)) return GSPN_ERR_UNSUPPORTED;
     if (p.g.B > kNoAllocMaxBatch || c64_fwd_workspace(p) > kNoAllocBytes) return GSPN_ERR_SCRATCH_LIMIT;
-    int d = 0;
-    if (cudaGetDevice(&d) != cudaSuccess || d < 0 || d >= kMaxNoAllocDevices) return GSPN_ERR_CUDA;
-    // set-up, once per device with that device current: the device address of
-    // the array (in host code its name is only a host-side stand-in)
-    void* ptr = g_noalloc_ptr[d].load(std::memory_order_acquire);
-    if (!ptr) {
-        if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || !ptr) return GSPN_ERR_CUDA;
-        g_noalloc_ptr[d].store(ptr, std::memory_order_release);
-    }
+    void* ptr = noalloc_scratch();
+    if (!ptr) return GSPN_ERR_CUDA;
     return c64_fwd(p, dev, x, logits, lam, out, ptr, s);
+}
+
+gspn_status c64_noalloc_status(cudaStream_t s) {
+    void* ptr = noalloc_scratch();
+    if (!ptr) return GSPN_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyAsync(&v, ptr, sizeof(v), cudaMemcpyDeviceToHost, s) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return GSPN_ERR_CUDA;
+    return v ? GSPN_ERR_TIMEOUT : GSPN_OK;
 }
 
 }  // namespace gspn

@@ -164,6 +164,8 @@ struct C64BArgs {
     int B, C;
     int groups;   // B * C / 8
     int segmask;  // local groups: lines per group - 1 (a power of two minus one; 63 = global)
+    uint64_t limit;  // bound of every wait on data, a stage or another warp (ns)
+    int stall;       // test hook: compute warp 0 of CTA 0 first waits on a barrier nothing completes
 };
 
 // bf16 element e of 8 packed in a uint4, widened
@@ -214,18 +216,9 @@ __device__ __forceinline__ float2 fwd_step(float2 h, float2 lx, const Taps& w, i
 // Adjoint step: a(line i) = g + W_{i+1}^T a(line i+1), with w the taps of
 // line i+1: a'[j] = g[j] + w1[j] a[j] + w0[j+1] a[j+1] + w2[j-1] a[j-1].  The
 // rotated shuffles bring in w0 a at j = 0 and w2 a at j = 63, both zero.
-__device__ __forceinline__ float2 adjoint(float2 a, float2 g, const Taps& w, int t) {
-    const float2 p0 = mul2(w.w0, a), p2 = mul2(w.w2, a);
-    const float p0r = __shfl_sync(FULL, p0.x, (t + 1) & 31);  // w0 a at j = 2t+2
-    const float p2l = __shfl_sync(FULL, p2.y, (t + 31) & 31); // w2 a at j = 2t-1
-    // the in-lane terms are summed while the shuffles are in flight
-    const float2 n = add2(fma2(make_float2(-1.f, -1.f), p2, fma2(make_float2(-1.f, -1.f), p0, add2(g, a))),
-                          make_float2(p0.y, p2.x));
-    return add2(n, make_float2(p2l, p0r));
-}
-
-// The same adjoint step with g + a already formed (from the bf16 g by one
-// mixed-precision FMA per position: g * 1 + a, the same single rounding).
+// g + a arrives already formed (from the bf16 g by one mixed-precision FMA per
+// position: g * 1 + a, a single rounding); the in-lane terms are summed while
+// the shuffles are in flight.
 __device__ __forceinline__ float2 adjoint_ga(float2 a, float2 ga, const Taps& w, int t) {
     const float2 p0 = mul2(w.w0, a), p2 = mul2(w.w2, a);
     const float p0r = __shfl_sync(FULL, p0.x, (t + 1) & 31);
@@ -295,7 +288,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (t == 0) {
             for (int kc = 0; kc < nchunks; ++kc) {
                 const int ws = kc % NWS;
-                if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1, 200)) {
+                if (!tma::mbar_wait_sleep(wempty0 + 8 * ws, ((kc / NWS) & 1) ^ 1, 200, a.limit)) {
                     atomicExch(a.err, 1);
                     break;
                 }
@@ -329,7 +322,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int pass = l >> 4, q = 7 - ((l >> 1) & 7), h = 1 - (l & 1), set = n % NSET;
                 if (set != rid) continue;
                 float* const dsum = a.dsum + (size_t)(b * 2 + pass) * 4 * S * S + (8 * q + 4 * h) * S;
-                if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n / NSET) & 1, 128))) {
+                if (!__all_sync(FULL, tma::mbar_wait_sleep(dfull0 + 8 * set, (n / NSET) & 1, 128, a.limit))) {
                     ok = false;
                     break;
                 }
@@ -432,8 +425,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_wait(wfull0 + 8 * (kk % NWS), (kk / NWS) & 1, 100000000ull);
     };
     auto acquire = [&]() -> bool {
-        const bool ok1 = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u);
-        const bool ok2 = tma::mbar_wait(wfull0 + 8 * (k % NWS), (k / NWS) & 1);
+        const bool ok1 = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u, a.limit);
+        const bool ok2 = tma::mbar_wait(wfull0 + 8 * (k % NWS), (k / NWS) & 1, a.limit);
         return __all_sync(FULL, ok1 && ok2);
     };
     // the data stage is in registers: refill it (every lane orders its reads of
@@ -465,7 +458,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // dchunk % NSET, free once the reducer has handed the set back
     int dchunk = 0;
     auto dslot = [&]() -> float* {
-        const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk % NSET), ((dchunk / NSET) & 1) ^ 1);
+        const bool ok = tma::mbar_wait(dempty0 + 8 * (dchunk % NSET), ((dchunk / NSET) & 1) ^ 1, a.limit);
         if (!__all_sync(FULL, ok)) return nullptr;
         return reinterpret_cast<float*>(smem + DSTG + ((dchunk % NSET) * NCW + warp) * DSLOT);
     };
@@ -474,7 +467,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         ++dchunk;
     };
 
-    for (int group = blockIdx.x; group < a.groups; group += gridDim.x) {
+    bool stalled = false;
+    if (a.stall && blockIdx.x == 0 && warp == 0 &&
+        !__all_sync(FULL, tma::mbar_wait(done0, 0, a.limit))) {
+        // test hook: phase 0 of done0 needs this warp's own final arrival, so the
+        // wait above can only run out; take the error path
+        fail();
+        stalled = true;
+    }
+    for (int group = blockIdx.x; !stalled && group < a.groups; group += gridDim.x) {
         const int plane = 8 * group + warp;
 
         auto run_pass = [&](auto pass_c) -> bool {
@@ -589,7 +590,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                 auto xv = [&](int e) { return pass == 0 ? make_float2(bfv(X[0], e), bfv(X[1], e)) : bf2(Xr[e]); };
                 auto lav = [&](int e) { return pass == 0 ? make_float2(bfv(LA[0], e), bfv(LA[1], e)) : bf2(LAr[e]); };
                 auto lbv = [&](int e) { return pass == 0 ? make_float2(bfv(LB[0], e), bfv(LB[1], e)) : bf2(LBr[e]); };
-                auto gv = [&](int e) { return pass == 0 ? make_float2(bfv(G[0], e), bfv(G[1], e)) : bf2(Gr[e]); };
 
                 // h_A(s-1) (the state line s reads) and a_B(s) of the chunk, from sweep 1,
                 // half a chunk at a time (steps 7..4 first)
@@ -742,27 +742,8 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // ---- host side ----------------------------------------------------------------------
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn_b() {
-    static EncodeTiledFn fn = nullptr;
-    static bool tried = false;
-    if (!tried) {
-        tried = true;
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 bool make_map_cols_b(CUtensorMap* m, const void* base, uint64_t planes) {
-    EncodeTiledFn fn = encode_fn_b();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[4] = {S, S / 2, 2, planes};
     const cuuint64_t strides[3] = {2 * S * 2, S * 2, (cuuint64_t)S * S * 2};
@@ -774,7 +755,7 @@ bool make_map_cols_b(CUtensorMap* m, const void* base, uint64_t planes) {
 }
 
 bool make_map_b(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_c, uint32_t box_r) {
-    EncodeTiledFn fn = encode_fn_b();
+    EncodeTiledFn fn = encode_tiled();
     if (!fn) return false;
     const cuuint64_t dims[3] = {S, S, planes};
     const cuuint64_t strides[2] = {S * 2, S * S * 2};
@@ -789,7 +770,7 @@ bool make_map_b(CUtensorMap* m, const void* base, uint64_t planes, uint32_t box_
 
 bool c64_bwd_eligible(const Problem& p) {
     return p.d.dtype == GSPN_BF16 && p.g.shared && p.d.dir_mask == 15u && p.g.H == S && p.g.W == S &&
-           S % p.g.groups == 0 && p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_fn_b() != nullptr;
+           S % p.g.groups == 0 && p.g.C % 8 == 0 && p.planes <= 0x7fffffff / 4 && encode_tiled() != nullptr;
 }
 
 namespace {
@@ -818,6 +799,9 @@ gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
     char* w = static_cast<char*>(ws);
     C64BArgs a;
     a.err = reinterpret_cast<int*>(w);
+    const WaitCfg wc = wait_cfg();
+    a.limit = wc.limit_ns;
+    a.stall = wc.stall;
     a.btab = reinterpret_cast<const float4*>(w + kWsAlign);
     a.dsum = reinterpret_cast<float*>(w + kWsAlign + tab_bytes(p));
     a.dxh = reinterpret_cast<float*>(w + kWsAlign + tab_bytes(p) + sum_bytes(p));

@@ -2,6 +2,7 @@
 // the kernel families.  Not part of the public ABI.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 
 #include "../../include/gspn.h"
@@ -31,6 +32,24 @@ cudaError_t device_info(DeviceInfo* out);
 // Sets the max-dynamic-smem attribute of `fn` once per device.
 cudaError_t ensure_smem_attr(const void* fn, int bytes, int slot);
 
+// cuTensorMapEncodeTiled from the driver, looked up once (thread-safe); null
+// when the driver does not provide it.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled();
+
+// Device-side waits of the TMA-fed kernels, process-wide: the limit of every
+// wait on data, a stage or a peer warp (gspn_set_wait_limit_ns), and the test
+// hook of gspn_set_stall_test (one wait per call on a barrier that nothing
+// completes).  Waits that drain copies or release tensor memory keep fixed
+// bounds of their own.
+struct WaitCfg {
+    uint64_t limit_ns;
+    int stall;
+};
+WaitCfg wait_cfg();
+
 // ---- generic kernels (any shape, dtype, mode) ---------------------------------
 size_t generic_fwd_workspace(const Problem& p, const DeviceInfo& dev);
 gspn_status generic_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
@@ -50,6 +69,12 @@ gspn_status small_fwd(const Problem& p, const DeviceInfo& dev, const void* x, co
 gspn_status small_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
                       const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s);
 
+// ---- planes with lines of 65..512 positions: one CTA streams a plane line by line (forward) ----
+bool large_eligible(const Problem& p);
+size_t large_fwd_workspace(const Problem& p);
+gspn_status large_fwd(const Problem& p, const void* x, const void* logits, const void* lam, void* out, void* ws,
+                      cudaStream_t s);
+
 // ---- compact 64x64 bf16 forward (TMA-fed, packed fp32x2) ------------------------
 bool c64_eligible(const Problem& p);
 size_t c64_fwd_workspace(const Problem& p);
@@ -58,6 +83,8 @@ gspn_status c64_fwd(const Problem& p, const DeviceInfo& dev, const void* x, cons
 // the same forward on the library's fixed device scratch (no workspace argument)
 gspn_status c64_fwd_noalloc(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits,
                             const void* lam, void* out, cudaStream_t s);
+// synchronises `s`, then reads the error word of the fixed scratch
+gspn_status c64_noalloc_status(cudaStream_t s);
 
 // ---- compact 128x128 bf16 forward (TMA-fed, first arrivals in TMEM) ------------------
 bool c128_eligible(const Problem& p);
@@ -76,5 +103,11 @@ bool c64_bwd_eligible(const Problem& p);
 size_t c64_bwd_workspace(const Problem& p, const DeviceInfo& dev);
 gspn_status c64_bwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
                     const void* dout, void* dx, void* dlogits, void* dlam, void* ws, cudaStream_t s);
+
+// ---- compressed propagation block (proxy projection, scan, merger, norm, back-projection) ----
+size_t block_workspace(const gspn_block_desc* d);
+gspn_status block_fwd(const gspn_block_desc* d, const void* x, const void* v, const void* logits, const void* lam,
+                      const float* alpha, const float* gamma, const void* u, void* y, void* ws, size_t ws_bytes,
+                      cudaStream_t s);
 
 }  // namespace gspn

@@ -174,3 +174,55 @@ def plane_slice(w: Workload, inp: Dict[str, np.ndarray], b: int, c: int) -> Dict
     if "dout" in inp:
         sl["dout"] = inp["dout"][b:b + 1, c:c + 1]
     return {k: np.ascontiguousarray(v) for k, v in sl.items()}
+
+
+# ---------------------------------------------------------------------------
+# Compressed propagation block inputs
+# ---------------------------------------------------------------------------
+@dataclasses.dataclass(frozen=True)
+class BlockWorkload:
+    """Shape and seed of one compressed-propagation-block invocation (all four
+    directions, channel-shared taps over the Cp proxy planes)."""
+
+    name: str
+    B: int
+    C: int
+    H: int
+    W: int
+    Cp: int
+    groups: int
+    seed: int
+    norm: bool = True
+    eps: float = 1e-6
+
+    def replace(self, **kw) -> "BlockWorkload":
+        return dataclasses.replace(self, **kw)
+
+
+# The block at the 1K foundation shape with the proxy width the GSPN-2
+# response selects (C_proxy = 2), and at its widest ablation point (32).
+BLOCK_WORKLOADS: Dict[str, BlockWorkload] = {
+    w.name: w
+    for w in (
+        BlockWorkload("block_cp2_bf16_b32c1152_64x64", 32, 1152, 64, 64, 2, 1, 20),
+        BlockWorkload("block_cp32_bf16_b32c1152_64x64", 32, 1152, 64, 64, 32, 1, 21),
+    )
+}
+
+
+def make_block_inputs(w: BlockWorkload) -> Dict[str, np.ndarray]:
+    """Seeded inputs of a block workload.  bf16 bit patterns (uint16) for x
+    [B,C,H,W] ~ N(0,1), v_proj [Cp,C] ~ N(0, 1/C), u_proj [C,Cp] ~ N(0, 1/Cp),
+    lam [4,B,Cp,H,W] ~ U(0,1), logits [4,B,1,3,H,W] ~ N(0,1); float32 alpha
+    [4,Cp] ~ N(0,1) and gamma [Cp] ~ 0.5 + U(0,1).  Every tensor has its own
+    child of SeedSequence(seed), in the order listed."""
+    kids = np.random.SeedSequence(w.seed).spawn(7)
+    return {
+        "x": _fill(kids[0], "normal", (w.B, w.C, w.H, w.W), 1.0, True),
+        "v_proj": _fill(kids[1], "normal", (w.Cp, w.C), float(1.0 / np.sqrt(w.C)), True),
+        "u_proj": _fill(kids[2], "normal", (w.C, w.Cp), float(1.0 / np.sqrt(w.Cp)), True),
+        "lam": _fill(kids[3], "uniform", (4, w.B, w.Cp, w.H, w.W), 1.0, True),
+        "logits": _fill(kids[4], "normal", (4, w.B, 1, 3, w.H, w.W), 1.0, True),
+        "alpha": _fill(kids[5], "normal", (4, w.Cp), 1.0, False),
+        "gamma": (0.5 + _fill(kids[6], "uniform", (w.Cp,), 1.0, False)).astype(np.float32),
+    }

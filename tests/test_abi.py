@@ -33,9 +33,27 @@ def test_library_loads_and_exports_every_declared_symbol():
 def test_version_and_status_strings():
     assert lsp.gspn_version() >= 100
     assert lsp.gspn_status_string(0) == "ok"
-    for s in range(1, 7):
+    for s in range(1, 8):
         assert lsp.gspn_status_string(s) and lsp.gspn_status_string(s) != "unknown status"
+    assert "timed out" in lsp.gspn_status_string(6)
     assert lsp.gspn_status_string(99) == "unknown status"
+
+
+def test_wait_settings_round_trip():
+    """The process-wide wait limit, stall hook and sync-check switch return
+    their previous values; a limit of 0 restores the 2 s default."""
+    assert lsp.gspn_set_wait_limit_ns(12345) == 2_000_000_000
+    assert lsp.gspn_set_wait_limit_ns(0) == 12345
+    assert lsp.gspn_set_wait_limit_ns(0) == 2_000_000_000
+    assert lsp.gspn_set_stall_test(1) == 0
+    assert lsp.gspn_set_stall_test(0) == 1
+    assert lsp.gspn_set_sync_check(7) == 0
+    assert lsp.gspn_set_sync_check(0) == 1
+
+
+def test_device_status_rejects_a_bad_descriptor():
+    assert lsp.gspn_device_status(lsp.make_desc(0, 1, 8, 8), 0, 0, 0) == 1
+    assert lsp.gspn_device_status(lsp.make_desc(1, 1, 8, 8, dir_mask=0), 1, 0, 0) == 1
 
 
 A = 1 << 20  # a 16-byte aligned fake device address: never dereferenced on rejected calls
@@ -112,10 +130,14 @@ def test_python_helpers_raise_on_error():
     ((1, 2, 64, 64, 5, 2, False, "bf16"), ("small_plane_fwd", 1), ("small_plane_bwd", 1)),
     ((3, 9, 64, 64, 15, 1, True, "bf16"), ("small_plane_fwd", 1), ("small_plane_bwd", 3)),  # C % 8 != 0
     ((1, 1, 16, 16, 1, 1, False, "f32"), ("small_plane_fwd", 1), ("small_plane_bwd", 1)),
-    # anything larger: the generic kernels
+    # longer lines with H, W multiples of 8 (up to 512): the large-plane forward
+    ((2, 6, 128, 128, 15, 1, True, "bf16"), ("large_plane_fwd", 1), ("generic_bwd", 3)),  # C % 4 != 0
+    ((1, 4, 512, 256, 15, 1, True, "bf16"), ("large_plane_fwd", 1), ("generic_bwd", 3)),
+    ((1, 2, 72, 320, 5, 1, False, "f32"), ("large_plane_fwd", 1), ("generic_bwd", 1)),
+    # anything else: the generic kernels
     ((1, 2, 65, 64, 15, 1, False, "f32"), ("generic_fwd", 1), ("generic_bwd", 1)),
     ((1, 2, 97, 41, 9, 1, False, "f32"), ("generic_fwd", 1), ("generic_bwd", 1)),
-    ((2, 6, 128, 128, 15, 1, True, "bf16"), ("generic_fwd", 1), ("generic_bwd", 3)),  # C % 4 != 0
+    ((1, 2, 1024, 8, 15, 1, True, "bf16"), ("generic_fwd", 1), ("generic_bwd", 3)),  # lines above 512
 ])
 def test_path_chooser(args, fwd, bwd):
     d = lsp.make_desc(*args)
@@ -131,7 +153,8 @@ def test_path_chooser(args, fwd, bwd):
 def test_compact_shapes_take_the_tma_kernels_when_the_encoder_is_there(args, fast):
     """The compact shapes run on the TMA-fed kernels wherever the driver's
     tensor-map encoder is available (a GPU host); without it the chooser falls
-    back to the small-plane or generic kernels, which also cover them."""
+    back to the small-plane, large-plane (forward) or generic kernels, which
+    also cover them."""
     d = lsp.make_desc(*args)
     small = max(args[2], args[3]) <= 64
     for bwd, launches in ((0, 2), (1, 3)):
@@ -140,4 +163,5 @@ def test_compact_shapes_take_the_tma_kernels_when_the_encoder_is_there(args, fas
         if name == fast + suffix:
             assert lsp.gspn_launches_per_call(d, bwd) == launches
         else:
-            assert name == ("small_plane" if small else "generic") + suffix
+            fallback = "small_plane" if small else ("generic" if bwd else "large_plane")
+            assert name == fallback + suffix

@@ -1,0 +1,57 @@
+"""GPU parity of the large-plane forward (lines of 65..512 positions, one CTA
+streaming a plane line by line) against the oracle.
+
+Shapes: 256x256 and 512x512 compact bf16 (the planes beyond the on-chip
+kernels), rectangular planes whose two scan directions use different warp
+counts, per-channel fp32 taps, local groups and partial direction sets.
+Canaries around the output catch stores outside it.  Tolerances as
+everywhere: 1e-5 (fp32) and 1e-2 (bf16) of max|reference|.
+"""
+import pytest
+
+import oracle
+import synth
+
+pytestmark = pytest.mark.gpu
+
+gu = pytest.importorskip("gpu_util")
+
+CASES = [
+    # B, C, H, W, dir_mask, groups, shared, dtype
+    (1, 4, 256, 256, 15, 1, True, "bf16"),
+    (1, 2, 512, 512, 15, 1, True, "bf16"),
+    (2, 3, 200, 136, 15, 1, False, "bf16"),   # 4 warps for column lines, 3 for row lines
+    (1, 3, 128, 96, 15, 4, False, "f32"),     # per-channel fp32, local groups
+    (1, 2, 72, 320, 5, 1, True, "f32"),       # T2B + L2R only
+    (1, 2, 264, 80, 10, 2, True, "bf16"),     # B2T + R2L, groups of 132 / 40 lines
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(map(str, c)))
+def test_large_plane_forward_matches_oracle(case):
+    import linear_spatial_propagation_b200 as lsp
+    t = gu.torch()
+    B, C, H, W, mask, g, shared, dtype = case
+    w = synth.Workload(f"large_{'x'.join(map(str, case))}", B, C, H, W, mask, g, shared, dtype, 1.0,
+                       4000 + H + W + C)
+    d = lsp.make_desc(B, C, H, W, mask, g, shared, dtype)
+    assert lsp.gspn_variant_name(d, 0) == "large_plane_fwd"
+    inp = synth.make_inputs(w, with_dout=False)
+    dinp = gu.dev_inputs(w, inp)
+    guard = 4096
+    buf = t.full((dinp["x"].numel() + 2 * guard,), -3.0, dtype=dinp["x"].dtype, device="cuda")
+    out = buf[guard:guard + dinp["x"].numel()].view(dinp["x"].shape)
+    gu.run_fwd(w, dinp, out=out)
+    t.cuda.synchronize()
+    assert bool((buf[:guard] == -3.0).all()) and bool((buf[guard + out.numel():] == -3.0).all())
+    gu.assert_close(gu.from_dev(out), oracle.fwd_workload(w, inp, nthreads=8), dtype, w.name)
+
+
+def test_large_plane_forward_is_deterministic():
+    t = gu.torch()
+    w = synth.Workload("large_det", 1, 4, 256, 256, 15, 1, True, "bf16", 1.0, 4100)
+    dinp = gu.dev_inputs(w, synth.make_inputs(w, with_dout=False))
+    o1 = gu.run_fwd(w, dinp)
+    o2 = gu.run_fwd(w, dinp)
+    t.cuda.synchronize()
+    assert bool(t.equal(o1, o2))
