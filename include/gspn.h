@@ -244,8 +244,8 @@ int gspn_set_stall_test(int on);
  * fp32; gamma [Cp] fp32.  The 4 axis is T2B, B2T, L2R, R2L.  Arithmetic is
  * fp32 (the projections on the tensor cores with bf16 operands: x, V and U as
  * stored, n rounded to bf16 once); y is rounded to bf16 once.
- * Limits (else GSPN_ERR_UNSUPPORTED): 1 <= Cp <= 32, H and W <= 128, C and H*W
- * multiples of 8, C <= 3072 (Cp <= 16) or 1536 (Cp <= 32).
+ * Limits (else GSPN_ERR_UNSUPPORTED): 1 <= Cp <= 32, H and W <= 128, C, H and
+ * W multiples of 8, C <= 3072 (Cp <= 16) or 1536 (Cp <= 32).
  * Errors and ownership as for gspn_fwd; a bounded device wait that runs out
  * is reported by gspn_block_device_status. */
 typedef struct {

@@ -27,7 +27,8 @@
 //   warp walks its lines, lane t holding P adjacent positions, the taps
 //   normalised from the logits where they are used.  It writes h_d in fp32.
 //   The proxy workload is a few planes per image, so this kernel is short and
-//   latency bound: it loads the next line while it computes the current one.
+//   latency bound: each warp stages its inputs in shared memory 8 lines at a
+//   time with cp.async, two chunks in flight, so no line waits on memory.
 // * block_out_kernel: per 128-pixel tile its prologue merges the four h_d with
 //   alpha, normalises over k and writes the bf16 operand n^T (K-major, K =
 //   C_proxy padded to 16 or 32) to shared memory; then one tcgen05 MMA per
@@ -267,13 +268,34 @@ struct ScanArgs {
 
 __device__ __forceinline__ float sigm(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
+// Inputs of the proxy scans are staged in shared memory a chunk of SC_CH lines
+// at a time with cp.async, two chunks per warp in flight, so a line never
+// waits for global memory.  Row scans (top->bottom, bottom->top) stage each
+// line as a contiguous row [line][position]; column scans (left->right,
+// right->left) stage, for every row, the chunk's SC_CH adjacent columns
+// [position][column].
+constexpr int SC_CH = 8;
+constexpr int SC_NMAX = 128;
+// per warp and buffer: xp (fp32), lambda and three logit taps (bf16)
+constexpr int SC_BUF = SC_CH * SC_NMAX * (4 + 2 + 3 * 2);
+constexpr int SC_SMEM = 4 * 2 * SC_BUF;
+
+__device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tma::smem_u32(sdst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 template <int P>
 __global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
+    extern __shared__ __align__(16) unsigned char sc_smem[];
     const int d = threadIdx.x >> 5, t = threadIdx.x & 31;
     const int plane = blockIdx.x;  // b * Cp + k
     const int b = plane / a.Cp;
     const int HW = a.H * a.W;
-    const int L = d < 2 ? a.H : a.W, N = d < 2 ? a.W : a.H;
+    const bool rows = d < 2;
+    const int L = rows ? a.H : a.W, N = rows ? a.W : a.H;
     const int seg = L / a.groups;
     const Walk wk = walk_of(d, a.H, a.W);
     const float* const xp = a.xp + (size_t)plane * HW;
@@ -281,61 +303,104 @@ __global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
         reinterpret_cast<const unsigned short*>(a.lam) + ((size_t)d * a.B * a.Cp + plane) * HW;
     const unsigned short* const lg = reinterpret_cast<const unsigned short*>(a.logits) + ((size_t)d * a.B + b) * 3 * HW;
     float* const out = a.h + ((size_t)d * a.B * a.Cp + plane) * HW;
+    unsigned char* const wbuf = sc_smem + d * 2 * SC_BUF;
+    // buffer layout: xp [SC_CH * N] fp32, then lambda, logit 0, 1, 2 [SC_CH * N] bf16 each
+    const int nch = SC_CH * N;
 
-    // lane t holds positions j = P t .. P t + P - 1 of a line
-    float h[P], u[P], g0[P], g1[P], g2[P];
-    float nu[P], n0[P], n1[P], n2[P];
-    auto load_line = [&](int i, float (&uu)[P], float (&l0)[P], float (&l1)[P], float (&l2)[P]) {
-#pragma unroll
-        for (int p = 0; p < P; ++p) {
-            const int j = P * t + p;
-            if (i < L && j < N) {
-                const int pix = wk.o + i * wk.si + j * wk.sj;
-                uu[p] = bf16_bits_to_float(__ldg(lam + pix)) * __ldg(xp + pix);
-                l0[p] = bf16_bits_to_float(__ldg(lg + pix));
-                l1[p] = bf16_bits_to_float(__ldg(lg + HW + pix));
-                l2[p] = bf16_bits_to_float(__ldg(lg + 2 * HW + pix));
-            } else {
-                uu[p] = l0[p] = l1[p] = l2[p] = 0.f;
+    // stage chunk c (lines c*SC_CH ..) into buffer c & 1
+    auto stage = [&](int c) {
+        unsigned char* const bx = wbuf + (c & 1) * SC_BUF;
+        unsigned char* const bl = bx + nch * 4;
+        const int i0 = c * SC_CH;
+        if (rows) {
+            // line i0 + e is row r: xp N*4 bytes, each bf16 tensor N*2 bytes, in 16-byte pieces
+            const int fx = N / 4, fb = N / 8, per_line = fx + 4 * fb;
+            for (int u = t; u < SC_CH * per_line; u += 32) {
+                const int e = u / per_line, v = u % per_line;
+                if (i0 + e >= L) continue;
+                const int row0 = wk.o + (i0 + e) * wk.si;  // pixel of position 0 of the line
+                if (v < fx) {
+                    cp_async16(bx + (e * N + 4 * v) * 4, xp + row0 + 4 * v);
+                } else {
+                    const int g = (v - fx) / fb, q = (v - fx) % fb;
+                    const unsigned short* src = g == 0 ? lam : lg + (g - 1) * HW;
+                    cp_async16(bl + ((size_t)g * nch + e * N + 8 * q) * 2, src + row0 + 8 * q);
+                }
+            }
+        } else {
+            // for every row j: the chunk's SC_CH adjacent columns, ascending in the image
+            const int c0 = wk.si > 0 ? i0 : a.W - SC_CH - i0;
+            for (int u = t; u < N * 6; u += 32) {
+                const int j = u / 6, v = u % 6;
+                const int pix = j * a.W + c0;
+                if (v < 2) {
+                    cp_async16(bx + (j * SC_CH + 4 * v) * 4, xp + pix + 4 * v);
+                } else {
+                    const int g = v - 2;
+                    const unsigned short* src = g == 0 ? lam : lg + (g - 1) * HW;
+                    cp_async16(bl + ((size_t)g * nch + j * SC_CH) * 2, src + pix);
+                }
             }
         }
+        cp_async_commit();
     };
-    load_line(0, u, g0, g1, g2);
+    // value of tensor g (0: xp, 1: lambda, 2..4: logit taps) at line e of the chunk, position j
+    auto val = [&](const unsigned char* bx, int g, int e, int j) -> float {
+        const int idx = rows ? e * N + j : j * SC_CH + (wk.si > 0 ? e : SC_CH - 1 - e);
+        if (g == 0) return reinterpret_cast<const float*>(bx)[idx];
+        const unsigned short* bl = reinterpret_cast<const unsigned short*>(bx + nch * 4) + (size_t)(g - 1) * nch;
+        return bf16_bits_to_float(bl[idx]);
+    };
+
+    const int nchunks = (L + SC_CH - 1) / SC_CH;
+    stage(0);
+    if (nchunks > 1) stage(1);
+    float h[P];
 #pragma unroll
     for (int p = 0; p < P; ++p) h[p] = 0.f;
-    int gpos = 0;  // position of line i within its local group
-    for (int i = 0; i < L; ++i) {
-        load_line(i + 1, nu, n0, n1, n2);  // in flight while line i is computed
-        // neighbours across lanes: the last position of lane t-1, the first of lane t+1
-        const float left = __shfl_up_sync(FULL, h[P - 1], 1);
-        const float right = __shfl_down_sync(FULL, h[0], 1);
-        float hn[P];
+    int gpos = 0;  // position of the line within its local group
+    for (int c = 0; c < nchunks; ++c) {
+        if (c + 1 < nchunks)
+            cp_async_wait<1>();
+        else
+            cp_async_wait<0>();
+        __syncwarp();  // every lane's pieces of chunk c are in shared memory
+        const unsigned char* const bx = wbuf + (c & 1) * SC_BUF;
+        for (int e = 0; e < SC_CH && c * SC_CH + e < L; ++e) {
+            const int i = c * SC_CH + e;
+            const float left = __shfl_up_sync(FULL, h[P - 1], 1);
+            const float right = __shfl_down_sync(FULL, h[0], 1);
+            float hn[P];
 #pragma unroll
-        for (int p = 0; p < P; ++p) {
-            const int j = P * t + p;
-            if (gpos == 0) {
-                hn[p] = u[p];  // h_{-1} = 0 at the start of a scan or of a local group
-            } else {
-                const float hl = p == 0 ? left : h[p - 1];
-                const float hr = p == P - 1 ? right : h[p + 1];
-                const float s0 = j > 0 ? sigm(g0[p]) : 0.f;
-                const float s1 = sigm(g1[p]);
-                const float s2 = j < N - 1 ? sigm(g2[p]) : 0.f;
-                const float r = __fdividef(1.f, s0 + s1 + s2);
-                hn[p] = fmaf(s0 * r, hl, fmaf(s1 * r, h[p], fmaf(s2 * r, hr, u[p])));
+            for (int p = 0; p < P; ++p) {
+                const int j = P * t + p;
+                if (j >= N) {
+                    hn[p] = 0.f;
+                    continue;
+                }
+                const float u = val(bx, 1, e, j) * val(bx, 0, e, j);
+                if (gpos == 0) {
+                    hn[p] = u;  // h_{-1} = 0 at the start of a scan or of a local group
+                } else {
+                    const float hl = p == 0 ? left : h[p - 1];
+                    const float hr = p == P - 1 ? right : h[p + 1];
+                    const float s0 = j > 0 ? sigm(val(bx, 2, e, j)) : 0.f;
+                    const float s1 = sigm(val(bx, 3, e, j));
+                    const float s2 = j < N - 1 ? sigm(val(bx, 4, e, j)) : 0.f;
+                    const float r = __fdividef(1.f, s0 + s1 + s2);
+                    hn[p] = fmaf(s0 * r, hl, fmaf(s1 * r, h[p], fmaf(s2 * r, hr, u)));
+                }
             }
-        }
 #pragma unroll
-        for (int p = 0; p < P; ++p) {
-            const int j = P * t + p;
-            h[p] = j < N ? hn[p] : 0.f;
-            if (j < N) out[wk.o + i * wk.si + j * wk.sj] = h[p];
-            u[p] = nu[p];
-            g0[p] = n0[p];
-            g1[p] = n1[p];
-            g2[p] = n2[p];
+            for (int p = 0; p < P; ++p) {
+                const int j = P * t + p;
+                h[p] = hn[p];
+                if (j < N) out[wk.o + i * wk.si + j * wk.sj] = h[p];
+            }
+            gpos = gpos + 1 == seg ? 0 : gpos + 1;
         }
-        gpos = gpos + 1 == seg ? 0 : gpos + 1;
+        __syncwarp();  // every lane is done with buffer c & 1 before it is refilled
+        if (c + 2 < nchunks) stage(c + 2);
     }
 }
 
@@ -390,7 +455,7 @@ __host__ __device__ constexpr int ob_smem_bytes(int C) {
 }
 
 template <int KPAD>
-__global__ void __launch_bounds__(OB_THREADS, 1)
+__global__ void __launch_bounds__(OB_THREADS, 2)
     block_out_kernel(const __grid_constant__ CUtensorMap tm_y, const OutArgs a) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     unsigned char* const smem = smem_raw + ((1024u - (tma::smem_u32(smem_raw) & 1023u)) & 1023u);
@@ -607,7 +672,7 @@ gspn_status block_validate(const gspn_block_desc* d) {
     if (d->B > (1 << 20) || d->C > (1 << 20)) return GSPN_ERR_INVALID_ARG;
     // kernel limits: proxy channels, line lengths, 16-byte TMA strides, U in shared memory
     if (d->Cp > 32 || d->H > 128 || d->W > 128) return GSPN_ERR_UNSUPPORTED;
-    if (d->C % 8 || (d->H * d->W) % 8) return GSPN_ERR_UNSUPPORTED;
+    if (d->C % 8 || d->H % 8 || d->W % 8) return GSPN_ERR_UNSUPPORTED;
     if (d->C > (d->Cp <= 16 ? 3072 : 1536)) return GSPN_ERR_UNSUPPORTED;
     if ((int64_t)d->B * d->C * d->H * d->W > ((int64_t)1 << 40)) return GSPN_ERR_INVALID_ARG;
     if (!encode_tiled()) return GSPN_ERR_UNSUPPORTED;
@@ -675,7 +740,9 @@ gspn_status launch_out(const DeviceInfo& dev, const gspn_block_desc& d, const fl
     const int smem = ob_smem_bytes<KPAD>((int)d.C);
     if (smem > dev.max_smem_optin) return GSPN_ERR_UNSUPPORTED;
     if (ensure_smem_attr(fn, smem, KPAD == 16 ? 34 : 35) != cudaSuccess) return GSPN_ERR_CUDA;
-    const int grid = a.ntiles < dev.sm_count ? a.ntiles : dev.sm_count;
+    // two CTAs per SM where shared memory allows (tensor memory: 2 x 256 columns)
+    const int per_sm = 2 * smem <= dev.max_smem_optin ? 2 : 1;
+    const int grid = a.ntiles < per_sm * dev.sm_count ? a.ntiles : per_sm * dev.sm_count;
     block_out_kernel<KPAD><<<grid, OB_THREADS, smem, s>>>(my, a);
     return cudaGetLastError() == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
 }
@@ -720,12 +787,12 @@ gspn_status block_fwd(const gspn_block_desc* d, const void* x, const void* v, co
     sa.groups = d->groups;
     const int nmax = (int)(d->H > d->W ? d->H : d->W);
     const int grid = (int)d->B * d->Cp;
-    if (nmax <= 32)
-        block_scan_kernel<1><<<grid, 128, 0, s>>>(sa);
-    else if (nmax <= 64)
-        block_scan_kernel<2><<<grid, 128, 0, s>>>(sa);
-    else
-        block_scan_kernel<4><<<grid, 128, 0, s>>>(sa);
+    const void* sfn = nmax <= 32   ? (const void*)block_scan_kernel<1>
+                      : nmax <= 64 ? (const void*)block_scan_kernel<2>
+                                   : (const void*)block_scan_kernel<4>;
+    if (ensure_smem_attr(sfn, SC_SMEM, nmax <= 32 ? 36 : nmax <= 64 ? 37 : 38) != cudaSuccess) return GSPN_ERR_CUDA;
+    void* sargs[] = {&sa};
+    if (cudaLaunchKernel(sfn, dim3(grid), dim3(128), sargs, SC_SMEM, s) != cudaSuccess) return GSPN_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
     return d->Cp <= 16 ? launch_out<16>(dev, *d, h, alpha, gamma, u, y, err, s)
                        : launch_out<32>(dev, *d, h, alpha, gamma, u, y, err, s);

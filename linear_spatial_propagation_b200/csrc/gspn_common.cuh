@@ -56,6 +56,20 @@ __device__ __forceinline__ void store_elt(__nv_bfloat16* p, int64_t i, float v) 
 // result is exact 0 for logits below about -88.
 __device__ __forceinline__ float sigmoidf(float z) { return 1.0f / (1.0f + __expf(-z)); }
 
+// ---- deterministic channel sums --------------------------------------------
+// Tap gradients summed over channels (channel-shared taps) accumulate as 64-bit
+// fixed-point integers with a resolution of 2^-32: integer addition is
+// associative, so the sums do not depend on the order in which planes arrive.
+// A value v adds round(v * 2^32); |v| and every partial sum must stay below
+// 2^31.  The quantisation (2^-33 per term at most) is far below fp32 rounding
+// for values above 2^-8.
+__device__ __forceinline__ void fix_add(unsigned long long* p, float v) {
+    atomicAdd(p, (unsigned long long)__float2ll_rn(v * 4294967296.0f));
+}
+__device__ __forceinline__ float fix_value(unsigned long long s) {
+    return (float)((double)(long long)s * (1.0 / 4294967296.0));
+}
+
 struct Launch {
     int B, C, H, W;
     int D;            // number of enabled directions

@@ -171,7 +171,7 @@ struct BwdArgs {
     void* dlam;
     float* hstore;   // [B*C][HW]: the current direction's lines, scan coordinates
     float* dx_ws;    // [B*C][HW] when the dx accumulator does not fit in smem
-    float* dlog_ws;  // [D][B][3][HW] fp32 sums over channels (shared mode)
+    unsigned long long* dlog_ws;  // [D][B][3][HW] fixed-point sums over channels (shared mode)
     int acc_in_smem;
     int warps_per_cta;
     int lstride;
@@ -272,10 +272,10 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) 
                 qc[2 * ls + j + 1] = q2;
                 if (a.g.shared) {
                     if (carry_out) {
-                        float* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
-                        if (j > 0) atomicAdd(dw + p, dl0);
-                        atomicAdd(dw + HW + p, dl1);
-                        if (j < N - 1) atomicAdd(dw + 2 * HW + p, dl2);
+                        unsigned long long* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
+                        if (j > 0) fix_add(dw + p, dl0);
+                        fix_add(dw + HW + p, dl1);
+                        if (j < N - 1) fix_add(dw + 2 * HW + p, dl2);
                     }
                 } else {
                     T* dlg = static_cast<T*>(a.dlogits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
@@ -293,15 +293,15 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) 
     for (int q = lane; q < HW; q += 32) store_elt(dx, q, dxacc[q]);
 }
 
-__global__ void zero_f32_kernel(float* p, int64_t n) {
+__global__ void zero_fix_kernel(unsigned long long* p, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        p[i] = 0.f;
+        p[i] = 0ull;
 }
 
 template <typename T>
-__global__ void convert_f32_kernel(const float* src, T* dst, int64_t n) {
+__global__ void convert_fix_kernel(const unsigned long long* src, T* dst, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        store_elt(dst, i, src[i]);
+        store_elt(dst, i, fix_value(src[i]));
 }
 
 struct Plan {
@@ -404,7 +404,7 @@ BwdWs bwd_ws_layout(const Problem& p, const DeviceInfo& dev) {
     w.dx_ws = off;
     if (!pl.acc_in_smem) off += align_up(plane_f, kWsAlign);
     w.dlog_ws = off;
-    if (p.g.shared) off += align_up((size_t)p.g.D * p.g.B * 3 * p.HW * sizeof(float), kWsAlign);
+    if (p.g.shared) off += align_up((size_t)p.g.D * p.g.B * 3 * p.HW * sizeof(unsigned long long), kWsAlign);
     w.total = off;
     return w;
 }
@@ -426,11 +426,11 @@ gspn_status generic_bwd(const Problem& p, const DeviceInfo& dev, const void* x, 
     a.dx = dx; a.dlogits = dlogits; a.dlam = dlam;
     a.hstore = reinterpret_cast<float*>(w + lay.hstore);
     a.dx_ws = reinterpret_cast<float*>(w + lay.dx_ws);
-    a.dlog_ws = reinterpret_cast<float*>(w + lay.dlog_ws);
+    a.dlog_ws = reinterpret_cast<unsigned long long*>(w + lay.dlog_ws);
     a.acc_in_smem = pl.acc_in_smem; a.warps_per_cta = pl.wpc; a.lstride = pl.lstride;
     const int64_t nlog = (int64_t)p.g.D * p.g.B * 3 * p.HW;
     if (p.g.shared) {
-        zero_f32_kernel<<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(a.dlog_ws, nlog);
+        zero_fix_kernel<<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(a.dlog_ws, nlog);
         cudaError_t e0 = cudaGetLastError();
         if (e0 != cudaSuccess) return GSPN_ERR_CUDA;
     }
@@ -448,10 +448,10 @@ gspn_status generic_bwd(const Problem& p, const DeviceInfo& dev, const void* x, 
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
     if (p.g.shared) {
         if (p.d.dtype == GSPN_F32)
-            convert_f32_kernel<float><<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(
+            convert_fix_kernel<float><<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(
                 a.dlog_ws, static_cast<float*>(dlogits), nlog);
         else
-            convert_f32_kernel<__nv_bfloat16><<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(
+            convert_fix_kernel<__nv_bfloat16><<<(unsigned)grid_for(nlog, 256), 256, 0, s>>>(
                 a.dlog_ws, static_cast<__nv_bfloat16*>(dlogits), nlog);
         e = cudaGetLastError();
         if (e != cudaSuccess) return GSPN_ERR_CUDA;

@@ -67,11 +67,15 @@ struct Chunk {
     static constexpr int CH = Elt<T>::CH;
     static constexpr int WPP = CH * (int)sizeof(T) / 4;  // words per position and tensor
     uint32_t v[5][2][WPP];
+    float acc[2][CH];  // the accumulator at the chunk's pixels (not the first direction)
 };
 
+// The chunk of lines i0 .. i0 + CH - 1 at positions j0, j0 + 1, and, when
+// `with_acc`, the accumulator values there.  The accumulator was written by
+// this CTA's previous direction, so it is read through the coherent path.
 template <typename T>
-__device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5], bool rowscan, const Walk& wk,
-                                           int W, int i0, int j0, int N) {
+__device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5], const float* acc, bool with_acc,
+                                           bool rowscan, const Walk& wk, int W, int i0, int j0, int N) {
     constexpr int CH = Elt<T>::CH;
     constexpr int WPP = Chunk<T>::WPP;
     if (rowscan) {
@@ -79,6 +83,10 @@ __device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5
 #pragma unroll
         for (int e = 0; e < CH; ++e) {
             const int pix = wk.o + (i0 + e) * wk.si + j0;
+            float2 av = make_float2(0.f, 0.f);
+            if (with_acc && j0 < N) av = *reinterpret_cast<const float2*>(acc + pix);  // j0 + 1 < N too: N is even
+            ck.acc[0][e] = av.x;
+            ck.acc[1][e] = av.y;
 #pragma unroll
             for (int s = 0; s < 5; ++s) {
                 const uint16_t* b16 = reinterpret_cast<const uint16_t*>(src[s] + pix);
@@ -108,6 +116,24 @@ __device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5
         for (int p = 0; p < 2; ++p) {
             const int j = j0 + p;
             const int first = wk.si > 0 ? wk.o + i0 + j * wk.sj : wk.o - (i0 + CH - 1) + j * wk.sj;
+            // the accumulator of these CTA pixels, in line order
+            float av[CH];
+#pragma unroll
+            for (int m = 0; m < CH; m += 4) {
+                float4 q = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (with_acc && j < N) q = *reinterpret_cast<const float4*>(acc + first + m);
+                av[m] = q.x;
+                av[m + 1] = q.y;
+                av[m + 2] = q.z;
+                av[m + 3] = q.w;
+            }
+            if (wk.si > 0) {
+#pragma unroll
+                for (int m = 0; m < CH; ++m) ck.acc[p][m] = av[m];
+            } else {
+#pragma unroll
+                for (int m = 0; m < CH; ++m) ck.acc[p][m] = av[CH - 1 - m];
+            }
 #pragma unroll
             for (int s = 0; s < 5; ++s) {
                 uint4 q = make_uint4(0u, 0u, 0u, 0u);
@@ -155,10 +181,10 @@ __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const La
         float h0 = 0.f, h1 = 0.f;
         int gpos = 0;
         Chunk<T> cur, nxt;
-        load_chunk<T>(cur, src, rowscan, wk, W, 0, j0, N);
+        load_chunk<T>(cur, src, acc, !first_dir, rowscan, wk, W, 0, j0, N);
         float colbuf[2][CH];  // column scans: a chunk of outputs per row, stored at the chunk's end
         for (int i0 = 0; i0 < L; i0 += CH) {
-            if (i0 + CH < L) load_chunk<T>(nxt, src, rowscan, wk, W, i0 + CH, j0, N);
+            if (i0 + CH < L) load_chunk<T>(nxt, src, acc, !first_dir, rowscan, wk, W, i0 + CH, j0, N);
 #pragma unroll
             for (int e = 0; e < CH; ++e) {
                 const int i = i0 + e;
@@ -200,16 +226,15 @@ __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const La
 #pragma unroll
                     for (int p = 0; p < 2; ++p) {
                         if (j0 + p >= N) continue;
-                        float v = hn[p];
-                        if (!first_dir) v += acc[pix + p];
+                        const float v = hn[p] + cur.acc[p][e];  // 0 for the first direction
                         if (last_dir)
                             store_elt(out, pix + p, v);
                         else
                             acc[pix + p] = v;
                     }
                 } else {
-                    colbuf[0][e] = h0;
-                    colbuf[1][e] = h1;
+                    colbuf[0][e] = h0 + cur.acc[0][e];
+                    colbuf[1][e] = h1 + cur.acc[1][e];
                 }
             }
             if (!rowscan) {
@@ -226,16 +251,6 @@ __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const La
                     } else {
 #pragma unroll
                         for (int m = 0; m < CH; ++m) v[m] = colbuf[p][CH - 1 - m];
-                    }
-                    if (!first_dir) {
-#pragma unroll
-                        for (int m = 0; m < CH; m += 4) {
-                            const float4 q = *reinterpret_cast<const float4*>(acc + first + m);
-                            v[m] += q.x;
-                            v[m + 1] += q.y;
-                            v[m + 2] += q.z;
-                            v[m + 3] += q.w;
-                        }
                     }
                     if (last_dir) {
 #pragma unroll

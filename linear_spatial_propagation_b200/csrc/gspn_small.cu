@@ -53,7 +53,7 @@ struct SmallArgs {
     void* dx;       // backward
     void* dlogits;
     void* dlam;
-    float* dlog_ws;  // backward, shared taps: fp32 sums over channels [D][B][3][HW]
+    unsigned long long* dlog_ws;  // backward, shared taps: fixed-point sums over channels [D][B][3][HW]
 };
 
 // The sigmoids of the valid taps of position j from the raw logits.  These
@@ -387,10 +387,10 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) smal
                     qc[2 * kLS + j + 1] = q2;
                     if (a.g.shared) {
                         if (carry_out) {
-                            float* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
-                            if (j > 0) atomicAdd(dw + p, dl0);
-                            atomicAdd(dw + HW + p, dl1);
-                            if (j < N - 1) atomicAdd(dw + 2 * HW + p, dl2);
+                            unsigned long long* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
+                            if (j > 0) fix_add(dw + p, dl0);
+                            fix_add(dw + HW + p, dl1);
+                            if (j < N - 1) fix_add(dw + 2 * HW + p, dl2);
                         }
                     } else if (kPieces && col) {
                         put_bf16<CH>(cg0[r], e, dl0);
@@ -437,15 +437,15 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) smal
     }
 }
 
-__global__ void small_zero_kernel(float* p, int64_t n) {
+__global__ void small_zero_kernel(unsigned long long* p, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        p[i] = 0.f;
+        p[i] = 0ull;
 }
 
 template <typename T>
-__global__ void small_convert_kernel(const float* src, T* dst, int64_t n) {
+__global__ void small_convert_kernel(const unsigned long long* src, T* dst, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
-        store_elt(dst, i, src[i]);
+        store_elt(dst, i, fix_value(src[i]));
 }
 
 size_t fwd_smem(const Problem& p) { return ((size_t)p.g.D * p.HW + (size_t)p.g.D * 2 * kLS) * sizeof(float); }
@@ -464,7 +464,7 @@ bool small_eligible(const Problem& p, int backward) {
 }
 
 size_t small_bwd_workspace(const Problem& p) {
-    return p.g.shared ? align_up((size_t)p.g.D * p.g.B * 3 * p.HW * sizeof(float), kWsAlign) : 0;
+    return p.g.shared ? align_up((size_t)p.g.D * p.g.B * 3 * p.HW * sizeof(unsigned long long), kWsAlign) : 0;
 }
 
 int small_bwd_launches(const Problem& p) { return p.g.shared ? 3 : 1; }
@@ -503,7 +503,7 @@ gspn_status small_bwd(const Problem& p, const DeviceInfo& dev, const void* x, co
     a.dx = dx;
     a.dlogits = dlogits;
     a.dlam = dlam;
-    a.dlog_ws = static_cast<float*>(ws);
+    a.dlog_ws = static_cast<unsigned long long*>(ws);
     const int64_t nlog = (int64_t)p.g.D * p.g.B * 3 * p.HW;
     if (p.g.shared) {
         small_zero_kernel<<<grid_1d(nlog), 256, 0, s>>>(a.dlog_ws, nlog);
