@@ -50,7 +50,8 @@ def parse():
     ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libgspn", choices=["libgspn", "reference"])
-    ap.add_argument("--workload", default=synth.HEADLINE, choices=list(synth.WORKLOADS))
+    ap.add_argument("--workload", default=synth.HEADLINE,
+                    choices=list(synth.WORKLOADS) + list(synth.BLOCK_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target length of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -234,6 +235,36 @@ def run_reference(args, w):
         "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
         "config": config_of(w, args.gpus),
         "cpu_baseline": {"value": val, "unit": "GB/s", "cores": nthreads, "kind": "oracle", "sample": sample},
+        "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_block_reference(args, w):
+    """The block oracle as the reference arm, on whole batch images."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    nthreads = os.cpu_count() or 1
+    steps, warm = max(1, args.steps), max(0, args.warmup)
+    per_step = max(0.5, min(args.cpu_seconds, 150.0 / (steps + warm)))
+    for _ in range(warm):
+        block_oracle_sample(w, per_step, nthreads)
+    tot_b, tot_s, imgs = 0, 0.0, 0
+    for _ in range(steps):
+        smp = block_oracle_sample(w, per_step, nthreads)
+        tot_b += smp["bytes"]
+        tot_s += smp["seconds"]
+        imgs = smp["images"]
+    val = tot_b / tot_s / 1e9
+    line = {
+        "impl": "reference", "metric": BLOCK_METRIC, "value": val, "unit": "GB/s", "n_gpus": args.gpus,
+        "steps": steps, "warmup": warm, "ms_per_step": tot_s / steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded numpy PCG64)",
+        "config": block_config(w, args.gpus),
+        "cpu_baseline": {"value": val, "unit": "GB/s", "cores": nthreads, "kind": "oracle",
+                         "sample": f"{imgs} batch image(s) of {w.name} per step, B=1 each"},
         "e2e": {"value": val, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -473,8 +504,164 @@ def run_gpu(args, w):
     return 0
 
 
+# ------------------------------------------------------------------------------
+# Compressed propagation block (gspn_block_fwd)
+# ------------------------------------------------------------------------------
+BLOCK_METRIC = "GSPN compressed block forward: achieved HBM GB/s (x, y, lambda and logits at the proxy width)"
+
+
+def block_bytes(w) -> int:
+    """Compulsory bytes of one block forward: x read and y written once,
+    lambda and the tap logits at the proxy width read once, the projection
+    matrices and the merger and norm weights read once."""
+    n = w.B * w.C * w.H * w.W
+    return (2 * n * 2 + 4 * w.B * w.Cp * w.H * w.W * 2 + 4 * w.B * 3 * w.H * w.W * 2 + 2 * w.C * w.Cp * 2
+            + 5 * w.Cp * 4)
+
+
+def block_config(w, n):
+    return {"workload": w.name, "B": w.B, "C": w.C, "H": w.H, "W": w.W, "C_proxy": w.Cp, "groups": w.groups,
+            "norm": "rms" if w.norm else "none", "io_dtype": "bf16", "pass": "fwd",
+            "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"}
+
+
+def block_oracle_sample(w, target_s: float, nthreads: int):
+    """The block oracle on as many whole batch images (each a B = 1 problem
+    drawn before its timing) as fit in about target_s seconds."""
+    import oracle
+    imgs, t = 0, 0.0
+    while imgs < w.B and (imgs == 0 or t < target_s):
+        sw = w.replace(B=1, seed=w.seed + 7 + imgs)
+        inp = synth.make_block_inputs(sw)
+        t0 = time.perf_counter()
+        oracle.block_fwd(inp["x"], inp["v_proj"], inp["logits"], inp["lam"], inp["alpha"], inp["gamma"],
+                         inp["u_proj"], groups=sw.groups, norm=sw.norm, eps=sw.eps, dtype="bf16", nthreads=nthreads)
+        t += time.perf_counter() - t0
+        imgs += 1
+    return {"seconds": t, "bytes": block_bytes(w.replace(B=1)) * imgs, "images": imgs}
+
+
+def run_block(args, w):
+    import torch
+
+    import linear_spatial_propagation_b200 as lsp
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    lsp.load(build_if_missing=False)
+    inp = synth.make_block_inputs(w.replace(seed=w.seed + 1000 * rank))
+
+    def pinned(a):
+        t = torch.from_numpy(a)
+        return (t.view(torch.bfloat16) if a.dtype == np.uint16 else t).pin_memory()
+
+    h = {k: pinned(v) for k, v in inp.items()}
+    d = {k: v.to(dev) for k, v in h.items()}
+    y = torch.empty_like(d["x"])
+    desc = lsp.make_block_desc(w.B, w.C, w.H, w.W, w.Cp, w.groups, w.norm, w.eps)
+    ws = torch.empty(lsp.gspn_block_workspace_size(desc), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(din=d, yo=None):
+        yo = y if yo is None else yo
+        st = lsp.gspn_block_fwd(desc, din["x"].data_ptr(), din["v_proj"].data_ptr(), din["logits"].data_ptr(),
+                                din["lam"].data_ptr(), din["alpha"].data_ptr(), din["gamma"].data_ptr(),
+                                din["u_proj"].data_ptr(), yo.data_ptr(), ws.data_ptr(), ws.numel(),
+                                stream.cuda_stream)
+        if st:
+            raise lsp.GspnError(st, "gspn_block_fwd")
+
+    def barrier():
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    barrier()
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    barrier()
+    clk = clocks.stop()
+    ms = max_over_ranks(dist, e0.elapsed_time(e1) / K, dev)
+    # end to end through the same entry point: every step copies its inputs up
+    # from pinned host memory and y back down (serialised on the stream)
+    E = args.e2e_steps
+    e2e_ms = None
+    h2d = sum(t.numel() * t.element_size() for t in h.values())
+    d2h = y.numel() * y.element_size()
+    if E > 0:
+        hy = torch.empty(y.shape, dtype=y.dtype).pin_memory()
+        barrier()
+        e2 = [torch.cuda.Event(enable_timing=True) for _ in range(2)]
+        e2[0].record(stream)
+        for _ in range(E):
+            for k in d:
+                d[k].copy_(h[k], non_blocking=True)
+            step()
+            hy.copy_(y, non_blocking=True)
+        e2[1].record(stream)
+        barrier()
+        e2e_ms = max_over_ranks(dist, e2[0].elapsed_time(e2[1]) / E, dev)
+    nb = block_bytes(w)
+    peak, peak_src = measured_peaks()
+    if rank == 0:
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            try:
+                smp = block_oracle_sample(w, args.cpu_seconds, os.cpu_count() or 1)
+                cpu = {"value": smp["bytes"] / smp["seconds"] / 1e9, "unit": "GB/s", "cores": os.cpu_count() or 1,
+                       "kind": "oracle", "sample": f"{smp['images']} batch image(s) of {w.name}, B=1 each "
+                                                   f"({smp['seconds']:.1f} s)"}
+            except Exception as ex:
+                cpu = {"value": None, "unit": "GB/s", "cores": os.cpu_count() or 1, "kind": "oracle",
+                       "sample": f"failed: {ex!r}"[:200]}
+        gbs = nb / (ms * 1e-3) / 1e9
+        line = {
+            "metric": BLOCK_METRIC, "value": job_gbs(nb, world, ms), "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded numpy PCG64, per-rank seed)",
+            "config": block_config(w, world), "bytes_per_step": nb,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                         "peak_source": f"{peak_src} copy bandwidth", "kernel": "gspn_block_fwd (3 launches)",
+                         "traffic": None},
+            "e2e": ({"value": job_gbs(nb, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                     "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms} if e2e_ms else None),
+            "gpu_launches": 3 * K, "clocks": clk, "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     args = parse()
+    if args.workload in synth.BLOCK_WORKLOADS:
+        bw = synth.BLOCK_WORKLOADS[args.workload]
+        if args.batch:
+            bw = bw.replace(B=args.batch, name=f"{bw.name}@B{args.batch}")
+        if args.impl == "reference":
+            return run_block_reference(args, bw)
+        return run_block(args, bw)
     w = synth.WORKLOADS[args.workload]
     if not w.backward:
         w = w.replace(backward=True)

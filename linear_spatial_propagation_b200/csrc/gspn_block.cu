@@ -366,41 +366,50 @@ __global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
             cp_async_wait<0>();
         __syncwarp();  // every lane's pieces of chunk c are in shared memory
         const unsigned char* const bx = wbuf + (c & 1) * SC_BUF;
-        for (int e = 0; e < SC_CH && c * SC_CH + e < L; ++e) {
+        // the chunk's taps and lambda * x first (they do not depend on the
+        // state): the sigmoids of all its lines overlap, and the buffer is free
+        // to refill before the lines are walked
+        float w0c[SC_CH][P], w2c[SC_CH][P], uc[SC_CH][P];
+#pragma unroll
+        for (int e = 0; e < SC_CH; ++e)
+#pragma unroll
+            for (int p = 0; p < P; ++p) {
+                const int j = P * t + p;
+                w0c[e][p] = w2c[e][p] = uc[e][p] = 0.f;
+                if (j < N) {
+                    uc[e][p] = val(bx, 1, e, j) * val(bx, 0, e, j);
+                    const float s0 = j > 0 ? sigm(val(bx, 2, e, j)) : 0.f;
+                    const float s1 = sigm(val(bx, 3, e, j));
+                    const float s2 = j < N - 1 ? sigm(val(bx, 4, e, j)) : 0.f;
+                    const float r = __fdividef(1.f, s0 + s1 + s2);
+                    w0c[e][p] = s0 * r;
+                    w2c[e][p] = s2 * r;
+                }
+            }
+        __syncwarp();  // every lane is done with buffer c & 1 before it is refilled
+        if (c + 2 < nchunks) stage(c + 2);
+#pragma unroll
+        for (int e = 0; e < SC_CH; ++e) {
             const int i = c * SC_CH + e;
             const float left = __shfl_up_sync(FULL, h[P - 1], 1);
             const float right = __shfl_down_sync(FULL, h[0], 1);
             float hn[P];
 #pragma unroll
             for (int p = 0; p < P; ++p) {
-                const int j = P * t + p;
-                if (j >= N) {
-                    hn[p] = 0.f;
-                    continue;
-                }
-                const float u = val(bx, 1, e, j) * val(bx, 0, e, j);
-                if (gpos == 0) {
-                    hn[p] = u;  // h_{-1} = 0 at the start of a scan or of a local group
-                } else {
-                    const float hl = p == 0 ? left : h[p - 1];
-                    const float hr = p == P - 1 ? right : h[p + 1];
-                    const float s0 = j > 0 ? sigm(val(bx, 2, e, j)) : 0.f;
-                    const float s1 = sigm(val(bx, 3, e, j));
-                    const float s2 = j < N - 1 ? sigm(val(bx, 4, e, j)) : 0.f;
-                    const float r = __fdividef(1.f, s0 + s1 + s2);
-                    hn[p] = fmaf(s0 * r, hl, fmaf(s1 * r, h[p], fmaf(s2 * r, hr, u)));
-                }
+                // h' = u + w0 h[j-1] + (1 - w0 - w2) h[j] + w2 h[j+1]; h_{-1} = 0 at
+                // the start of a scan or of a local group
+                const float hl = p == 0 ? left : h[p - 1];
+                const float hr = p == P - 1 ? right : h[p + 1];
+                hn[p] = gpos == 0 ? uc[e][p] : uc[e][p] + h[p] + w0c[e][p] * (hl - h[p]) + w2c[e][p] * (hr - h[p]);
             }
 #pragma unroll
             for (int p = 0; p < P; ++p) {
                 const int j = P * t + p;
-                h[p] = hn[p];
+                h[p] = j < N ? hn[p] : 0.f;
                 if (j < N) out[wk.o + i * wk.si + j * wk.sj] = h[p];
             }
             gpos = gpos + 1 == seg ? 0 : gpos + 1;
         }
-        __syncwarp();  // every lane is done with buffer c & 1 before it is refilled
-        if (c + 2 < nchunks) stage(c + 2);
     }
 }
 

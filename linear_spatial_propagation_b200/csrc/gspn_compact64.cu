@@ -18,10 +18,12 @@
 // * A CTA (one per SM) scans groups of 8 consecutive planes of one batch
 //   image, one plane per consumer warp, 32 lanes per 64-wide line and 2
 //   positions per lane.  The 8 warps step through the same sequence of
-//   8-step chunks, so one producer warp streams each chunk's tap weights
-//   (8 table rows, 8 KB) with a single bulk copy into a 4-stage ring that all
-//   8 warps read; each warp reads a step's weights one step ahead and releases
-//   the stage after its last step.
+//   8-step chunks, so each chunk's tap weights (8 table rows, 8 KB) arrive
+//   with a single bulk copy into a 4-stage ring that all 8 warps read; the
+//   four producer warps take the chunks in turn (producer p fills stage p),
+//   so the producer that also feeds two warps' data is not the only one
+//   streaming weights.  Each warp reads a step's weights one step ahead and
+//   releases the stage after its last step.
 // * The two directions of a pair (left->right with right->left, top->bottom
 //   with bottom->top) advance together: lane values are float2 (one
 //   direction per half) and the update is the packed fp32x2 FMA of sm_100;
@@ -82,6 +84,7 @@ constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
 constexpr int CHUNKS_PER_GROUP = 16;  // 8 column chunks + 8 row chunks
 constexpr int NPW = NCW / 2;  // producer warps, each feeding two consumer warps
 constexpr int THREADS = (NCW + NPW) * 32;
+static_assert(NWS == NPW, "producer p fills weight stage p");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(WARP_BYTES % 1024 == 0 && WCHUNK % 1024 == 0, "TMA destinations stay 1024-byte aligned");
 
@@ -190,8 +193,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     // 2p and 2p+1: chunk kk of warp w (plane 8*group + w of group blockIdx.x +
     // (kk/16)*gridDim.x; chunk kk%16: 0..7 column chunks, 8..15 row chunks;
     // lambda plane (slot, b, c) at slot*B*C + plane) goes to stage kk % NST of the
-    // warp's ring once the warp has read what the stage held.  Producer 0 also
-    // streams the tap-weight chunks, each one into the ring shared by the CTA.
+    // warp's ring once the warp has read what the stage held.  It also streams
+    // the tap-weight chunks kk with kk % 4 == p, into stage p of the ring
+    // shared by the CTA.
     if (warp >= NCW) {
         if (t == 0) {
             const int pw = warp - NCW;
@@ -205,7 +209,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int kk = 0; ok && kk < nchunks; ++kk) {
                 const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
                 const int local = kk % CHUNKS_PER_GROUP, st = kk % NST;
-                if (pw == 0) {
+                // the tap-weight chunks are spread over the producers: chunk kk goes
+                // to producer kk % NPW, which (NWS == NPW) always fills ring stage pw
+                if (kk % NPW == pw) {
                     const int ws = kk % NWS;
                     if (!tma::mbar_wait(wempty0 + 8 * ws, ((kk / NWS) & 1) ^ 1, a.limit)) {
                         ok = false;

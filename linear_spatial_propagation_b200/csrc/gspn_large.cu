@@ -19,7 +19,9 @@
 // fp32 accumulator plane in the workspace (first direction stores, the next
 // ones add, the last one adds and writes the output in the I/O dtype), so the
 // sum is taken in direction order and does not depend on timing.  Tap weights
-// are normalised from the logits where they are used (Key design 1).
+// are normalised from the logits (Key design 1) for a whole chunk before its
+// lines are walked, so the sigmoids overlap and the line loop carries only
+// the dependent update.
 #include "gspn_internal.h"
 
 namespace gspn {
@@ -185,6 +187,23 @@ __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const La
         float colbuf[2][CH];  // column scans: a chunk of outputs per row, stored at the chunk's end
         for (int i0 = 0; i0 < L; i0 += CH) {
             if (i0 + CH < L) load_chunk<T>(nxt, src, acc, !first_dir, rowscan, wk, W, i0 + CH, j0, N);
+            // the chunk's taps and lambda * x first: they do not depend on the
+            // state, so the sigmoids of all its lines and positions overlap, and
+            // the line loop below is only the dependent update
+            float w0c[CH][2], w2c[CH][2], uc[CH][2];
+#pragma unroll
+            for (int e = 0; e < CH; ++e)
+#pragma unroll
+                for (int p = 0; p < 2; ++p) {
+                    const int j = j0 + p;
+                    uc[e][p] = Elt<T>::get(cur.v[1][p], e) * Elt<T>::get(cur.v[0][p], e);
+                    const float s0 = j > 0 ? lg_sigmoid(Elt<T>::get(cur.v[2][p], e)) : 0.f;
+                    const float s1 = lg_sigmoid(Elt<T>::get(cur.v[3][p], e));
+                    const float s2 = j < N - 1 ? lg_sigmoid(Elt<T>::get(cur.v[4][p], e)) : 0.f;
+                    const float r = __fdividef(1.f, s0 + s1 + s2);
+                    w0c[e][p] = s0 * r;
+                    w2c[e][p] = s2 * r;
+                }
 #pragma unroll
             for (int e = 0; e < CH; ++e) {
                 const int i = i0 + e;
@@ -196,24 +215,20 @@ __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const La
                     if (t == 0) hl = warp > 0 ? edge[par ^ 1][warp - 1][1] : 0.f;
                     if (t == 31) hr = warp + 1 < a.nw ? edge[par ^ 1][warp + 1][0] : 0.f;
                 }
+                // h' = u + w0 h[j-1] + (1 - w0 - w2) h[j] + w2 h[j+1]; h_{-1} = 0 at a
+                // scan or group start; positions beyond the line stay 0
                 float hn[2];
-#pragma unroll
-                for (int p = 0; p < 2; ++p) {
-                    const int j = j0 + p;
-                    const float u = Elt<T>::get(cur.v[1][p], e) * Elt<T>::get(cur.v[0][p], e);
-                    if (gpos == 0 || j >= N) {
-                        hn[p] = j < N ? u : 0.f;  // h_{-1} = 0 at a scan or group start
-                    } else {
-                        const float s0 = j > 0 ? lg_sigmoid(Elt<T>::get(cur.v[2][p], e)) : 0.f;
-                        const float s1 = lg_sigmoid(Elt<T>::get(cur.v[3][p], e));
-                        const float s2 = j < N - 1 ? lg_sigmoid(Elt<T>::get(cur.v[4][p], e)) : 0.f;
-                        const float r = __fdividef(1.f, s0 + s1 + s2);
-                        const float left = p == 0 ? hl : h0, mid = p == 0 ? h0 : h1, right = p == 0 ? h1 : hr;
-                        hn[p] = fmaf(s0 * r, left, fmaf(s1 * r, mid, fmaf(s2 * r, right, u)));
-                    }
+                if (gpos == 0) {
+                    hn[0] = uc[e][0];
+                    hn[1] = uc[e][1];
+                } else {
+                    hn[0] = uc[e][0] + h0 + w0c[e][0] * (hl - h0) + w2c[e][0] * (h1 - h0);
+                    hn[1] = uc[e][1] + h1 + w0c[e][1] * (h0 - h1) + w2c[e][1] * (hr - h1);
                 }
-                h0 = hn[0];
-                h1 = hn[1];
+                h0 = j0 < N ? hn[0] : 0.f;
+                h1 = j0 + 1 < N ? hn[1] : 0.f;
+                hn[0] = h0;
+                hn[1] = h1;
                 if (a.nw > 1) {
                     if (t == 0) edge[par][warp][0] = h0;
                     if (t == 31) edge[par][warp][1] = h1;

@@ -37,6 +37,26 @@ def test_reference_arm_prints_the_contract_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
 
 
+def test_block_reference_arm_prints_the_contract_line():
+    r = _bench(["--impl", "reference", "--workload", "block_cp2_bf16_b32c1152_64x64", "--batch", "1", "--steps",
+                "1", "--warmup", "0", "--cpu-seconds", "0.2"])
+    assert r.returncode == 0, r.stderr
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["config"]["C_proxy"] == 2 and d["value"] > 0
+    assert d["cpu_baseline"]["value"] == d["value"]
+
+
+def test_block_bytes_count_x_y_and_the_proxy_inputs():
+    import bench
+    import synth
+    w = synth.BlockWorkload("b", 2, 16, 8, 8, 4, 1, 0)
+    n = 2 * 16 * 64
+    want = 2 * n * 2 + 4 * 2 * 4 * 64 * 2 + 4 * 2 * 3 * 64 * 2 + 2 * 16 * 4 * 2 + 5 * 4 * 4
+    assert bench.block_bytes(w) == want
+
+
 def test_reference_arm_other_ranks_exit_without_work():
     r = _bench(["--impl", "reference", "--workload", "t2b_f32_b1c4_16x16", "--steps", "1"],
                {"RANK": "1", "WORLD_SIZE": "2"})

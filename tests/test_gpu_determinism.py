@@ -1,7 +1,12 @@
 """Repeat-determinism of the backward: two calls on the same inputs give
-bit-identical dx, dlogits and dlambda on every path, including the
-channel-shared tap gradients of the small-plane and generic kernels, which
-sum over channels with order-independent fixed-point atomics."""
+bit-identical dx, dlogits and dlambda.
+
+dx and dlambda never depend on timing.  The channel-shared tap gradients of
+the small-plane and generic kernels sum over channels with order-independent
+fixed-point atomics, so they repeat bit for bit at any size.  The compact
+TMA kernels sum each CTA's share in a fixed order and then add the CTAs'
+shares into global fp32 sums; the cases here have two CTAs per batch image,
+where fp32 addition (commutative) still gives one result."""
 import pytest
 
 import synth
@@ -17,8 +22,8 @@ CASES = [
     ((1, 6, 96, 72, 15, 1, True, "bf16"), "generic_bwd"),
     ((1, 3, 80, 40, 15, 2, True, "f32"), "generic_bwd"),
     ((2, 8, 64, 64, 15, 1, False, "bf16"), "small_plane_bwd"),
-    ((2, 16, 64, 64, 15, 1, True, "bf16"), "compact64_tma_bwd"),
-    ((1, 8, 128, 128, 15, 1, True, "bf16"), "compact128_tma_bwd"),
+    ((2, 16, 64, 64, 15, 1, True, "bf16"), "compact64_tma_bwd"),    # 2 CTAs per image
+    ((1, 8, 128, 128, 15, 1, True, "bf16"), "compact128_tma_bwd"),  # 2 CTAs per image
 ]
 
 
