@@ -42,10 +42,15 @@
 //   shared->global fp32 reduce-adds to L2-resident sums.  Half chunks rotate
 //   over three slot sets, each with its own reducer warp, so the reductions
 //   overlap and a compute warp rarely waits for a set.
-// * x, lambda and dout are streamed by TMA exactly as in the compact forward
-//   (per-warp ring of 8-step chunks); the normalised tap weights (a table
+// * x, lambda and dout are streamed by TMA into a per-warp ring of 8-step
+//   chunks by four data-producer warps (two compute warps each), so the
+//   compute warps issue no copies; the normalised tap weights (a table
 //   written by a pre-kernel, one row per scan step with both directions at
 //   the same column) by a producer warp into a ring shared by the CTA.
+// * 16 warps in four warpgroups: compute (two), then the tap-table producer
+//   with the three reducers, then the four data producers.  The helper
+//   warpgroups hand registers to the compute ones with setmaxnreg (192 per
+//   compute thread, 64 per helper thread).
 // * Every wait is bounded (2 s); on expiry the warp records an error word,
 //   drains its copies and returns.
 #include <atomic>
@@ -78,10 +83,20 @@ constexpr int NSET = 3;                         // slot sets, one reducer warp e
 constexpr int DOUT = DSTG + NSET * NCW * DSLOT;  // a reduced half chunk per set: [dir*2 + value][step][position j]
 constexpr int DLS = DOUT + NSET * DSLOT;          // per warp: row-pass dlambda of a chunk, A then B, [row % 2][row / 2][8 columns]
 constexpr int BARS = DLS + NCW * 2 * BOX;
-constexpr int NBAR = NCW * NST + 2 * NWS + 2 * NSET + 1;
+constexpr int NBAR = 2 * NCW * NST + 2 * NWS + 2 * NSET + 1;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
 constexpr int CHUNKS_PER_GROUP = 32;  // row pass sweeps 1, 2; column pass sweeps 1, 2 (8 chunks each)
-constexpr int THREADS = (NCW + 1 + NSET) * 32;  // compute warps, tap-table producer, tap-value reducers
+constexpr int NDP = NCW / 2;                     // data producers, two compute warps each
+// warpgroups 0, 1: compute warps; warpgroup 2: tap-table producer and the
+// tap-value reducers; warpgroup 3: the data producers
+constexpr int THREADS = (NCW + 1 + NSET + NDP) * 32;
+static_assert(THREADS == 512, "four warpgroups");
+// Launched at 128 registers per thread (65536 / 512).  The helper warpgroups
+// give registers up and the compute warpgroups take them: on each scheduler
+// (warps k, k+4, k+8, k+12) 2 x 32 x kComputeRegs + 2 x 32 x kHelperRegs
+// must equal its 16384, or a setmaxnreg.inc would wait forever.
+constexpr int kComputeRegs = 192, kHelperRegs = 64;
+static_assert(2 * 32 * kComputeRegs + 2 * 32 * kHelperRegs == 16384, "register split");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 // ---- backward tap table ---------------------------------------------------------------
@@ -229,8 +244,7 @@ __device__ __forceinline__ float2 adjoint_ga(float2 a, float2 ga, const Taps& w,
 }
 constexpr uint32_t kOneBf2 = 0x3F803F80u;  // bf16 1.0 in both halves
 
-// 12 warps put 3 on each of the SM's four schedulers, each with a quarter of
-// the register file: at most 16384 / (3 * 32) -> 168 registers per thread
+// 16 warps, 4 per scheduler; see kComputeRegs for the register split
 template <bool LOCAL>
 __global__ void __launch_bounds__(THREADS, 1)
     c64b_kernel(const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
@@ -246,6 +260,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t dfull0 = wempty0 + 8 * NWS;  // [set]: the compute warps' slots of a chunk are written
     const uint32_t dempty0 = dfull0 + 8 * NSET;  // [set]: the reducer has read the set
     const uint32_t done0 = dempty0 + 8 * NSET;   // every compute warp is done with the tensor memory
+    const uint32_t xempty0 = done0 + 8;          // [warp][stage]: the compute warp has read its data stage
     uint32_t* const tslot = reinterpret_cast<uint32_t*>(smem + BARS + 8 * NBAR);
     if ((int)blockIdx.x >= a.groups) return;
 
@@ -260,6 +275,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma::mbar_init(dempty0 + 8 * s, 1);
         }
         tma::mbar_init(done0, NCW);
+        for (int s = 0; s < NCW * NST; ++s) tma::mbar_init(xempty0 + 8 * s, 32);
         tma::fence_barrier_init();
     }
     if (warp == 0) {  // compute warp 0 owns the CTA's tensor memory: all 512 columns
@@ -283,6 +299,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         q = sweep ? 7 - (l & 7) : (l & 7);
     };
 
+    // ---------------- helper warpgroups 2 and 3 ----------------
+    // Every helper warp executes the one register release below (a warpgroup
+    // must execute the same setmaxnreg), then takes its role.
+    if (warp >= NCW) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegs) : "memory");
     // ---------------- producer warp: tap-table chunks ----------------
     if (warp == NCW) {
         if (t == 0) {
@@ -310,7 +331,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     // n % NSET owns.  It sums the 8 slots into its reduced buffer, hands the set
     // back, and adds the half chunk to the image's sums (rows 8q+4h..8q+4h+3 of
     // each of the 4 [s][j] planes) by 4 bulk reduce-adds of 1 KB.
-    if (warp >= NCW + 1) {
+    if (warp >= NCW + 1 && warp < NCW + 1 + NSET) {
         // reducer rid takes the pieces of slot set rid (every NSET-th half chunk)
         const int rid = warp - (NCW + 1);
         const float4* const sets = reinterpret_cast<const float4*>(smem + DSTG);
@@ -362,8 +383,63 @@ __global__ void __launch_bounds__(THREADS, 1)
         return;
     }
 
+    // ---------------- data producers ----------------
+    // Lane 0 of producer p streams the data chunks of compute warps 2p and 2p+1:
+    // chunk kk of warp w (plane 8*group + w of group blockIdx.x + (kk/32)*gridDim.x)
+    // is x, lambda_A, lambda_B (sweep 2 only) and dout of the chunk's 8 columns
+    // (row pass: [row % 2][row / 2][8 columns] through the 4-D view) or rows
+    // (column pass: [8 rows][64 columns]), into stage kk % NST of the warp's
+    // ring once the warp has read what the stage held.  The compute warps
+    // issue no copies themselves: issuing them took a fifth of their time.
+    if (warp >= NCW + 1 + NSET) {
+        if (t == 0) {
+            const int pw = warp - (NCW + 1 + NSET);
+            if (pw == 0) {
+                tma::prefetch_map(&tm_xc);
+                tma::prefetch_map(&tm_lc);
+                tma::prefetch_map(&tm_gc);
+                tma::prefetch_map(&tm_xr);
+                tma::prefetch_map(&tm_lr);
+                tma::prefetch_map(&tm_gr);
+            }
+            bool ok = true;
+            for (int kk = 0; ok && kk < nchunks; ++kk) {
+                const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
+                int pass, sweep, q;
+                chunk_info(kk, pass, sweep, q);
+                const int st = kk % NST;
+                const int la = pass ? 0 : 2, lb = pass ? 1 : 3;  // lambda slots of A and B
+                for (int w = 2 * pw; w < 2 * pw + 2; ++w) {
+                    if (!tma::mbar_wait(xempty0 + 8 * (w * NST + st), ((kk / NST) & 1) ^ 1, a.limit)) {
+                        ok = false;
+                        break;
+                    }
+                    const int plane = 8 * group + w;
+                    const uint32_t dst = sbase + w * WARP_BYTES + st * STAGE;
+                    const uint32_t bar = sbase + BARS + 8 * (w * NST + st);
+                    tma::mbar_expect_tx(bar, sweep ? 4 * BOX : 3 * BOX);
+                    if (pass == 0) {
+                        tma::load_4d(dst + 0 * BOX, &tm_xc, 8 * q, 0, 0, plane, bar);
+                        tma::load_4d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 0, la * BC + plane, bar);
+                        if (sweep) tma::load_4d(dst + 2 * BOX, &tm_lc, 8 * q, 0, 0, lb * BC + plane, bar);
+                        tma::load_4d(dst + 3 * BOX, &tm_gc, 8 * q, 0, 0, plane, bar);
+                    } else {
+                        tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
+                        tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, la * BC + plane, bar);
+                        if (sweep) tma::load_3d(dst + 2 * BOX, &tm_lr, 0, 8 * q, lb * BC + plane, bar);
+                        tma::load_3d(dst + 3 * BOX, &tm_gr, 0, 8 * q, plane, bar);
+                    }
+                }
+            }
+            if (!ok) atomicExch(a.err, 1);
+        }
+        return;
+    }
+    return;
+    }  // helper warpgroups
+
     // ---------------- consumer warps ----------------
-    const uint32_t ring = sbase + warp * WARP_BYTES;
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kComputeRegs) : "memory");
     unsigned char* const ringp = smem + warp * WARP_BYTES;
     float* const dxslot = a.dxh + ((size_t)blockIdx.x * NCW + warp) * S * S;
     // sweep-1 states of this warp's plane: lane t of TMEM quarter warp % 4,
@@ -375,44 +451,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     const unsigned char* const wring = smem + WRING;
     const uint32_t bar0 = sbase + BARS + 8 * NST * warp;
 
-    if (t == 0) {
-        tma::prefetch_map(&tm_xc);
-        tma::prefetch_map(&tm_lc);
-        tma::prefetch_map(&tm_gc);
-        tma::prefetch_map(&tm_xr);
-        tma::prefetch_map(&tm_lr);
-        tma::prefetch_map(&tm_gr);
-        tma::prefetch_map(&tm_dl);
-    }
-
-    // Data of chunk kk (lane 0): x, lambda_A, lambda_B (sweep 2 only), dout of
-    // the chunk's 8 columns (row pass: [row % 2][row / 2][8 columns] through the
-    // 4-D view, conflict-free 16-byte reads) or rows (column pass: [8 rows][64
-    // columns]).
-    auto issue = [&](int kk) {
-        if (kk >= nchunks) return;
-        const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
-        const int plane = 8 * group + warp;
-        int pass, sweep, q;
-        chunk_info(kk, pass, sweep, q);
-        const int st = kk % NST;
-        const uint32_t dst = ring + st * STAGE, bar = bar0 + 8 * st;
-        tma::mbar_expect_tx(bar, sweep ? 4 * BOX : 3 * BOX);
-        const int la = pass ? 0 : 2, lb = pass ? 1 : 3;  // lambda slots of A and B
-        if (pass == 0) {
-            tma::load_4d(dst + 0 * BOX, &tm_xc, 8 * q, 0, 0, plane, bar);
-            tma::load_4d(dst + 1 * BOX, &tm_lc, 8 * q, 0, 0, la * BC + plane, bar);
-            if (sweep) tma::load_4d(dst + 2 * BOX, &tm_lc, 8 * q, 0, 0, lb * BC + plane, bar);
-            tma::load_4d(dst + 3 * BOX, &tm_gc, 8 * q, 0, 0, plane, bar);
-        } else {
-            tma::load_3d(dst + 0 * BOX, &tm_xr, 0, 8 * q, plane, bar);
-            tma::load_3d(dst + 1 * BOX, &tm_lr, 0, 8 * q, la * BC + plane, bar);
-            if (sweep) tma::load_3d(dst + 2 * BOX, &tm_lr, 0, 8 * q, lb * BC + plane, bar);
-            tma::load_3d(dst + 3 * BOX, &tm_gr, 0, 8 * q, plane, bar);
-        }
-    };
-    if (t == 0)
-        for (int kk = 0; kk < NST; ++kk) issue(kk);
+    if (t == 0) tma::prefetch_map(&tm_dl);
 
     int k = 0, stage = 0;
     uint32_t phase = 0;
@@ -429,12 +468,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         const bool ok2 = tma::mbar_wait(wfull0 + 8 * (k % NWS), (k / NWS) & 1, a.limit);
         return __all_sync(FULL, ok1 && ok2);
     };
-    // the data stage is in registers: refill it (every lane orders its reads of
-    // the stage before the async-proxy writes with a proxy fence of its own)
+    // the data stage is in registers: hand it back to its producer (every lane
+    // orders its reads of the stage before the async-proxy refill with a proxy
+    // fence of its own, then arrives)
     auto release_data = [&]() {
         tma::fence_proxy_async();
-        __syncwarp();
-        if (t == 0) issue(k + NST);
+        tma::mbar_arrive(xempty0 + 8 * (warp * NST + stage));
         phase ^= 1u << stage;
         stage = stage == NST - 1 ? 0 : stage + 1;
     };
