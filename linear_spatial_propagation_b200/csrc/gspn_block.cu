@@ -50,13 +50,9 @@ namespace {
 using namespace lane;
 
 // ---- tcgen05 operand descriptors ------------------------------------------------
-// Shared-memory matrix descriptor (sm_100): start address, leading and stride
-// byte offsets (all >> 4), the fixed version bit 46, and the layout type.
-constexpr uint32_t kLayoutNone = 0, kLayoutSw128 = 2;
-__device__ __forceinline__ uint64_t sdesc(uint32_t saddr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
-           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | ((uint64_t)layout << 61);
-}
+using tmem::sdesc;
+using tmem::kLayoutNone;
+using tmem::kLayoutSw128;
 // Instruction descriptor of kind::f16 with bf16 A and B and an fp32
 // accumulator: D format bits 4-5, A and B formats bits 7-9 and 10-12, the
 // major-ness of A (bit 15) and B (bit 16), N >> 3 at bit 17, M >> 4 at bit 24.
@@ -74,10 +70,7 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 // arrive on `bar` once every MMA this thread issued before has completed
-__device__ __forceinline__ void mma_commit(uint32_t bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
-                 : "memory");
-}
+__device__ __forceinline__ void mma_commit(uint32_t bar) { tmem::commit(bar); }
 
 // ==================================================================================
 // block_proj_kernel: xp = V x, per 128-pixel tile

@@ -19,11 +19,14 @@
 //   image, one plane per consumer warp, 32 lanes per 64-wide line and 2
 //   positions per lane.  The 8 warps step through the same sequence of
 //   8-step chunks, so each chunk's tap weights (8 table rows, 8 KB) arrive
-//   with a single bulk copy into a 4-stage ring that all 8 warps read; the
-//   four producer warps take the chunks in turn (producer p fills stage p),
-//   so the producer that also feeds two warps' data is not the only one
-//   streaming weights.  Each warp reads a step's weights one step ahead and
-//   releases the stage after its last step.
+//   once per CTA by one bulk copy into shared memory.  Four weight warps,
+//   one per lane quarter of the tensor memory (TMEM), each read the chunk
+//   once and write it into their quarter (lane t: the taps of positions 2t,
+//   2t+1, 8 columns per step); the two consumer warps of a quarter read two
+//   steps' columns with one tcgen05.ld, a pair ahead.  Shared memory thus
+//   serves each chunk four times instead of eight, and the consumers issue
+//   no weight loads from it.  Chunks rotate over 4 stages (64 TMEM columns
+//   each); a quarter's stage is refilled once both its consumers loaded it.
 // * The two directions of a pair (left->right with right->left, top->bottom
 //   with bottom->top) advance together: lane values are float2 (one
 //   direction per half) and the update is the packed fp32x2 FMA of sm_100;
@@ -70,7 +73,7 @@ constexpr int S = 64;          // H = W
 constexpr int LPL = 32;        // lanes per line (2 positions per lane)
 constexpr int NCW = 8;         // consumer warps per CTA (one plane each), one CTA per SM
 constexpr int NST = 2;         // x/lambda ring stages per consumer warp
-constexpr int NWS = 4;         // tap-weight ring stages per CTA
+constexpr int NWS = 4;         // tap-weight stages, in shared memory (bulk copy) and in TMEM (64 columns)
 constexpr int BOX = 1024;      // bytes per TMA box (one plane)
 constexpr int SLICE = 512;     // the even or odd rows of a column chunk
 constexpr int STAGE = 4 * BOX;
@@ -79,12 +82,16 @@ constexpr int WCHUNK = 8 * S * 16;  // tap weights of 8 scan steps (8 table rows
 constexpr int WARP_BYTES = NST * STAGE + HACC;
 constexpr int WRING = NCW * WARP_BYTES;              // offset of the weight ring
 constexpr int BARS = WRING + NWS * WCHUNK;           // offset of the barriers
-constexpr int NBAR = 2 * NCW * NST + 2 * NWS + 1;
+constexpr int NBAR = 2 * NCW * NST + 2 * NWS + 8 * NWS + 1;
 constexpr int SMEM_BYTES = 1024 + BARS + 8 * NBAR + 16;  // + the TMEM address
 constexpr int CHUNKS_PER_GROUP = 16;  // 8 column chunks + 8 row chunks
-constexpr int NPW = NCW / 2;  // producer warps, each feeding two consumer warps
-constexpr int THREADS = (NCW + NPW) * 32;
-static_assert(NWS == NPW, "producer p fills weight stage p");
+constexpr int NPW = NCW / 2;  // data producer warps, each feeding two consumer warps
+constexpr int WW = NCW + NPW;  // the first of 4 tap-weight warps; warp WW + q writes lane quarter q
+static_assert(WW % 4 == 0, "weight warp WW + q sits on lane quarter q");
+constexpr int THREADS = (NCW + NPW + 4) * 32;
+constexpr uint32_t TMEM_COLS = 512;  // first arrivals: 256 columns, then the tap-weight stages
+constexpr uint32_t TW_COL = 256;     // first tap-weight column
+static_assert(TW_COL + NWS * 64 <= TMEM_COLS, "tensor memory budget");
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(WARP_BYTES % 1024 == 0 && WCHUNK % 1024 == 0, "TMA destinations stay 1024-byte aligned");
 
@@ -156,9 +163,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
     const uint32_t xfull0 = sbase + BARS;                  // [warp][stage] "data landed"
     const uint32_t xempty0 = xfull0 + 8 * NCW * NST;       // [warp][stage] "data read"
-    const uint32_t wfull0 = xempty0 + 8 * NCW * NST;       // NWS "weights landed" barriers
-    const uint32_t wempty0 = wfull0 + 8 * NWS;             // NWS "weights consumed" barriers
-    const uint32_t done0 = wempty0 + 8 * NWS;              // every consumer is done with the tensor memory
+    const uint32_t wfull0 = xempty0 + 8 * NCW * NST;       // [stage] weight chunk in shared memory
+    const uint32_t wempty0 = wfull0 + 8 * NWS;             // [stage] the 4 weight warps have read it
+    const uint32_t tfull0 = wempty0 + 8 * NWS;             // [stage][quarter] weight chunk in TMEM
+    const uint32_t tempty0 = tfull0 + 8 * 4 * NWS;         // [stage][quarter] both consumers have loaded it
+    const uint32_t done0 = tempty0 + 8 * 4 * NWS;          // every warp is done with the tensor memory
     uint32_t* const tslot = reinterpret_cast<uint32_t*>(smem + BARS + 8 * NBAR);
     if ((int)blockIdx.x >= a.groups) return;
 
@@ -169,13 +178,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
         for (int s = 0; s < NWS; ++s) {
             tma::mbar_init(wfull0 + 8 * s, 1);
-            tma::mbar_init(wempty0 + 8 * s, NCW);
+            tma::mbar_init(wempty0 + 8 * s, 4);
         }
-        tma::mbar_init(done0, NCW);
+        for (int s = 0; s < 4 * NWS; ++s) {
+            tma::mbar_init(tfull0 + 8 * s, 1);
+            tma::mbar_init(tempty0 + 8 * s, 2);
+        }
+        tma::mbar_init(done0, NCW + 4);
         tma::fence_barrier_init();
     }
-    if (warp == 0) {  // consumer warp 0 owns 256 TMEM columns: 128 per consumer warp
-        tmem::alloc(tma::smem_u32(tslot), 256);
+    if (warp == 0) {  // consumer warp 0 owns the CTA's 512 TMEM columns
+        tmem::alloc(tma::smem_u32(tslot), TMEM_COLS);
         tmem::relinquish();
     }
     tmem::fence_before();
@@ -188,14 +201,90 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     const int BC = a.B * a.C;
 
-    // ---------------- producer warps ----------------
+    // ---------------- tap-weight warps ----------------
+    // Lane 0 of weight warp 0 keeps NWS chunks of the tap-weight table in
+    // flight into shared memory: chunk c (table rows 8*(c%16) .. +7 of the
+    // group's image) into stage c % NWS, refilled with chunk c + NWS once all
+    // four weight warps have read it.  Weight warp q writes chunk c into TMEM
+    // stage c % NWS of lane quarter q once both consumers of the quarter have
+    // loaded what it held: lane t takes the 16 bytes of positions p = 0, 1 of
+    // each step e (table entry p*32 + t of row e) into columns 8e + 4p .. +3.
+    if (warp >= WW) {
+        const int qw = warp - WW;
+        const uint32_t tq = taddr + ((uint32_t)(32 * qw) << 16) + TW_COL;
+        auto fetch = [&](int c) {
+            const int group = (int)blockIdx.x + (c / CHUNKS_PER_GROUP) * (int)gridDim.x;
+            const int b = (8 * group) / a.C, ws = c % NWS;
+            const float4* src = a.wtab + ((size_t)b * 2 * S + 8 * (c % CHUNKS_PER_GROUP)) * S;
+            tma::mbar_expect_tx(wfull0 + 8 * ws, WCHUNK);
+            tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
+        };
+        const bool feeder = qw == 0 && t == 0;
+        int issued = 0;
+        if (feeder)
+            for (; issued < NWS && issued < nchunks; ++issued) fetch(issued);
+        bool ok = true;
+        for (int c = 0; c < nchunks; ++c) {
+            const int ws = c % NWS;
+            const uint32_t par = (uint32_t)(c / NWS) & 1u;
+            const bool okw = tma::mbar_wait(wfull0 + 8 * ws, par, a.limit) &&
+                             tma::mbar_wait(tempty0 + 8 * (ws * 4 + qw), par ^ 1u, a.limit);
+            if (!__all_sync(FULL, okw)) {
+                ok = false;
+                break;
+            }
+            const unsigned char* src = smem + WRING + ws * WCHUNK + t * 16;
+            tmem::fence_after();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                uint32_t v[32];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+#pragma unroll
+                    for (int p = 0; p < 2; ++p) {
+                        const uint4 w = lds128(src + (4 * hh + e) * 1024 + p * 512);
+                        v[e * 8 + p * 4 + 0] = w.x;
+                        v[e * 8 + p * 4 + 1] = w.y;
+                        v[e * 8 + p * 4 + 2] = w.z;
+                        v[e * 8 + p * 4 + 3] = w.w;
+                    }
+                tmem::st_x32(tq + 64u * (uint32_t)ws + 32u * (uint32_t)hh, v);
+            }
+            // the shared stage is read: hand it back to the feeder
+            tma::fence_proxy_async();
+            __syncwarp();
+            if (t == 0) tma::mbar_arrive(wempty0 + 8 * ws);
+            tmem::wait_st();
+            tmem::fence_before();
+            __syncwarp();
+            if (t == 0) tma::mbar_arrive(tfull0 + 8 * (ws * 4 + qw));
+            if (feeder && issued < nchunks) {
+                if (!tma::mbar_wait(wempty0 + 8 * ws, par, a.limit)) {
+                    ok = false;
+                } else {
+                    fetch(issued++);
+                }
+            }
+            if (!__all_sync(FULL, ok)) break;
+        }
+        // no bulk copy of the feeder is in flight when the CTA exits
+        if (feeder)
+            for (int c = 0; c < issued; ++c)
+                if (c + NWS >= issued) tma::mbar_wait(wfull0 + 8 * (c % NWS), (c / NWS) & 1, 100000000ull);
+        if (!ok && t == 0) atomicExch(a.err, 1);
+        tmem::wait_st();
+        tmem::fence_before();
+        __syncwarp();
+        if (t == 0) tma::mbar_arrive(done0);
+        return;
+    }
+
+    // ---------------- data producer warps ----------------
     // Lane 0 of producer warp p streams the x / lambda chunks of consumer warps
     // 2p and 2p+1: chunk kk of warp w (plane 8*group + w of group blockIdx.x +
     // (kk/16)*gridDim.x; chunk kk%16: 0..7 column chunks, 8..15 row chunks;
     // lambda plane (slot, b, c) at slot*B*C + plane) goes to stage kk % NST of the
-    // warp's ring once the warp has read what the stage held.  It also streams
-    // the tap-weight chunks kk with kk % 4 == p, into stage p of the ring
-    // shared by the CTA.
+    // warp's ring once the warp has read what the stage held.
     if (warp >= NCW) {
         if (t == 0) {
             const int pw = warp - NCW;
@@ -209,19 +298,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int kk = 0; ok && kk < nchunks; ++kk) {
                 const int group = (int)blockIdx.x + (kk / CHUNKS_PER_GROUP) * (int)gridDim.x;
                 const int local = kk % CHUNKS_PER_GROUP, st = kk % NST;
-                // the tap-weight chunks are spread over the producers: chunk kk goes
-                // to producer kk % NPW, which (NWS == NPW) always fills ring stage pw
-                if (kk % NPW == pw) {
-                    const int ws = kk % NWS;
-                    if (!tma::mbar_wait(wempty0 + 8 * ws, ((kk / NWS) & 1) ^ 1, a.limit)) {
-                        ok = false;
-                        break;
-                    }
-                    const int b = (8 * group) / a.C;
-                    const float4* src = a.wtab + ((size_t)b * 2 * S + 8 * local) * S;
-                    tma::mbar_expect_tx(wfull0 + 8 * ws, WCHUNK);
-                    tma::load_1d(sbase + WRING + ws * WCHUNK, src, WCHUNK, wfull0 + 8 * ws);
-                }
                 for (int w = 2 * pw; w < 2 * pw + 2; ++w) {
                     if (!tma::mbar_wait(xempty0 + 8 * (w * NST + st), ((kk / NST) & 1) ^ 1, a.limit)) {
                         ok = false;
@@ -257,7 +333,6 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------- consumer warps: one plane each ----------------
     unsigned char* const ringp = smem + warp * WARP_BYTES;
     unsigned char* const haccp = ringp + NST * STAGE;
-    const unsigned char* const wring = smem + WRING;
     const uint32_t bar0 = xfull0 + 8 * NST * warp, ebar0 = xempty0 + 8 * NST * warp;
     const int segmask = a.seg - 1;  // seg divides 64, so it is a power of two
 
@@ -271,36 +346,51 @@ __global__ void __launch_bounds__(THREADS, 1)
         // drain every data copy that may still be in flight, with a short bound
         for (int kk = k; kk < k + NST && kk < nchunks; ++kk)
             tma::mbar_wait(bar0 + 8 * (kk % NST), (kk / NST) & 1, 100000000ull);
-        // and the weight chunks this warp has not consumed (the producer issues at
-        // most NWS ahead of the slowest consumer)
-        for (int kk = k; kk < k + NWS && kk < nchunks; ++kk)
-            tma::mbar_wait(wfull0 + 8 * (kk % NWS), (kk / NWS) & 1, 100000000ull);
     };
 
-    // Tap weights are read one step ahead: during step e of chunk c a warp loads
-    // the 2 x 16 bytes of step e+1 into registers.  At the chunk's last step it
-    // hands the weight stage back (every lane fences its reads of the stage
-    // before the async-proxy refill; one arrival per warp) and takes step 0 of
-    // chunk c+1.  Data stages are copied to registers whole at the chunk's start.
-    float4 wc[2];  // tap weights of the current step
-    auto wstep = [&](int c, int e, float4 (&wn)[2]) -> bool {
-        if (e < 7) {
-            const unsigned char* wsrc = wring + (c % NWS) * WCHUNK + t * 16 + (e + 1) * 1024;
-            wn[0] = lds128f(wsrc);
-            wn[1] = lds128f(wsrc + 512);
-            return true;
-        }
-        tma::fence_proxy_async();
-        __syncwarp();
-        if (t == 0) tma::mbar_arrive(wempty0 + 8 * (c % NWS));
-        if (c + 1 < nchunks) {
-            const bool okw = tma::mbar_wait(wfull0 + 8 * ((c + 1) % NWS), ((c + 1) / NWS) & 1, a.limit);
-            if (!__all_sync(FULL, okw)) return false;
-            const unsigned char* wsrc = wring + ((c + 1) % NWS) * WCHUNK + t * 16;
-            wn[0] = lds128f(wsrc);
-            wn[1] = lds128f(wsrc + 512);
+    // Tap weights are read two steps at a time, one pair ahead: at the even
+    // step e of chunk c a warp issues the TMEM load of steps e+2, e+3 (16
+    // columns) and waits for it after step e+1's arithmetic.  At step 6 every
+    // load of the chunk has completed, so the warp hands the stage back (one
+    // arrival per warp) and loads steps 0, 1 of chunk c+1 once that chunk's
+    // copies are committed.  Data stages are copied to registers whole at the
+    // chunk's start.
+    const uint32_t twq = taddr + ((uint32_t)(32 * (warp & 3)) << 16) + TW_COL;
+    uint32_t wcur[16], wnxt[16];  // taps of steps (e, e+1) and of the next pair, 8 columns per step
+    auto wissue = [&](int c, int e) -> bool {
+        if ((e & 1) == 0) {
+            if (e < 6) {
+                tmem::ld_x16(twq + 64u * (uint32_t)(c % NWS) + 8u * (uint32_t)(e + 2), wnxt);
+                return true;
+            }
+            tmem::fence_before();
+            __syncwarp();
+            if (t == 0) tma::mbar_arrive(tempty0 + 8 * ((c % NWS) * 4 + (warp & 3)));
+            if (c + 1 < nchunks) {
+                const bool okw =
+                    tma::mbar_wait(tfull0 + 8 * (((c + 1) % NWS) * 4 + (warp & 3)), ((c + 1) / NWS) & 1, a.limit);
+                if (!__all_sync(FULL, okw)) return false;
+                tmem::fence_after();
+                tmem::ld_x16(twq + 64u * (uint32_t)((c + 1) % NWS), wnxt);
+            }
         }
         return true;
+    };
+    // the taps of step e as the (-w0_A, -w0_B, w2_A, w2_B) of positions 2t, 2t+1
+    auto wget = [&](int e, float4 (&w)[2]) {
+        const int o = (e & 1) * 8;
+        w[0] = make_float4(__uint_as_float(wcur[o]), __uint_as_float(wcur[o + 1]), __uint_as_float(wcur[o + 2]),
+                           __uint_as_float(wcur[o + 3]));
+        w[1] = make_float4(__uint_as_float(wcur[o + 4]), __uint_as_float(wcur[o + 5]), __uint_as_float(wcur[o + 6]),
+                           __uint_as_float(wcur[o + 7]));
+    };
+    // after the odd step: the next pair has arrived
+    auto wturn = [&](int e) {
+        if (e & 1) {
+            tmem::wait_ld16(wnxt);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) wcur[i] = wnxt[i];
+        }
     };
     auto acquire = [&]() -> bool {
         const bool ok = tma::mbar_wait(bar0 + 8 * stage, (phase >> stage) & 1u, a.limit);
@@ -370,11 +460,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                         base[p].y = fma_bf((7 - e) & 1, word_of(LB[p], (7 - e) >> 1), word_of(XB[p], (7 - e) >> 1),
                                            h[p].y);
                     }
-                    float4 wn[2];
-                    if (!wstep(c, e, wn)) return false;
-                    scan_core(h, base, wc);
-                    wc[0] = wn[0];
-                    wc[1] = wn[1];
+                    if (!wissue(c, e)) return false;
+                    {
+                        float4 wc[2];
+                        wget(e, wc);
+                        scan_core(h, base, wc);
+                    }
+                    wturn(e);
                     if constexpr (!SECOND) {
 #pragma unroll
                         for (int p = 0; p < 2; ++p) {
@@ -453,11 +545,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     base[1].x = fma_bf_hi(LA[e], XA[e], h[1].x);
                     base[0].y = fma_bf_lo(LB[e], XB[e], h[0].y);
                     base[1].y = fma_bf_hi(LB[e], XB[e], h[1].y);
-                    float4 wn[2];
-                    if (!wstep(c, e, wn)) return false;
-                    scan_core(h, base, wc);
-                    wc[0] = wn[0];
-                    wc[1] = wn[1];
+                    if (!wissue(c, e)) return false;
+                    {
+                        float4 wc[2];
+                        wget(e, wc);
+                        scan_core(h, base, wc);
+                    }
+                    wturn(e);
                     if (!SECOND) {
                         // first arrival of this pass: the row sum of the pixel plus this
                         // direction's value, parked in TMEM
@@ -494,10 +588,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         ok = __all_sync(FULL, tma::mbar_wait(done0, 0, a.limit));
     }
     if (ok && nchunks > 0) {
-        const bool okw = tma::mbar_wait(wfull0, 0, a.limit);
+        const bool okw = tma::mbar_wait(tfull0 + 8 * (warp & 3), 0, a.limit);
         ok = __all_sync(FULL, okw);
-        wc[0] = lds128f(wring + t * 16);
-        wc[1] = lds128f(wring + t * 16 + 512);
+        if (ok) {
+            tmem::fence_after();
+            tmem::ld_x16(twq, wcur);
+            tmem::wait_ld16(wcur);
+        }
     }
     for (int group = blockIdx.x; ok && group < a.groups; group += gridDim.x) {
         outp = a.out + (size_t)(8 * group + warp) * S * S + 2 * t;
@@ -514,7 +611,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (!ok) fail();
     // this warp no longer touches the tensor memory; warp 0 frees it after all
+    // consumers and the weight warps
     tmem::wait_st();
+    tmem::wait_ld_all();
     tmem::fence_before();
     __syncwarp();
     if (t == 0) tma::mbar_arrive(done0);
@@ -522,7 +621,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!tma::mbar_wait(done0, 0, 10 * tma::kTimeoutNs) && t == 0) atomicExch(a.err, 1);
         __syncwarp();
         tmem::fence_after();
-        tmem::dealloc(taddr, 256);
+        tmem::dealloc(taddr, TMEM_COLS);
     }
 }
 
