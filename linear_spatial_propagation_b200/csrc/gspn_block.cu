@@ -23,12 +23,17 @@
 //   proxy rows beyond C_proxy are the TMA's zero fill.  The fp32 accumulator
 //   lives in tensor memory (two buffers, so the epilogue of one tile overlaps
 //   the MMAs of the next) and is written out as xp in fp32.
+// * block_taps_kernel: the normalised taps (w0, w2) of every (direction,
+//   image, line, position), in scan order.  They are channel-shared, so they
+//   are formed once here, one thread each, instead of by every proxy plane's
+//   scan (where, one warp per direction, the sigmoids were the scan's
+//   critical path).
 // * block_scan_kernel: one CTA per proxy plane, one warp per direction; each
-//   warp walks its lines, lane t holding P adjacent positions, the taps
-//   normalised from the logits where they are used.  It writes h_d in fp32.
-//   The proxy workload is a few planes per image, so this kernel is short and
-//   latency bound: each warp stages its inputs in shared memory 8 lines at a
-//   time with cp.async, two chunks in flight, so no line waits on memory.
+//   warp walks its lines, lane t holding P adjacent positions.  It writes h_d
+//   in fp32.  The proxy workload is a few planes per image, so this kernel is
+//   short and latency bound: each warp stages its inputs (x_proxy, lambda and
+//   the taps) in shared memory 8 lines at a time with cp.async, two chunks in
+//   flight, so no line waits on memory.
 // * block_out_kernel: per 128-pixel tile its prologue merges the four h_d with
 //   alpha, normalises over k and writes the bf16 operand n^T (K-major, K =
 //   C_proxy padded to 16 or 32) to shared memory; then one tcgen05 MMA per
@@ -254,23 +259,47 @@ __global__ void __launch_bounds__(PJ_THREADS, 1)
 struct ScanArgs {
     const float* xp;                 // [B][Cp][HW]
     const __nv_bfloat16* lam;        // [4][B][Cp][HW]
-    const __nv_bfloat16* logits;     // [4][B][1][3][HW]
+    const float2* taps;              // [4][B][line][position]: (w0, w2)
     float* h;                        // [4][B][Cp][HW]
     int B, Cp, H, W, groups;
 };
 
 __device__ __forceinline__ float sigm(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
 
+// taps[((d*B + b)*L + i)*N + j] = (w0, w2) of position j of line i of
+// direction d in image b: the sigmoids of the pixel's three tap logits,
+// normalised over the taps that exist (w0 = 0 at j = 0, w2 = 0 at j = N-1).
+__global__ void __launch_bounds__(256) block_taps_kernel(const __nv_bfloat16* __restrict__ logits,
+                                                          float2* __restrict__ taps, int B, int H, int W) {
+    const int HW = H * W;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)4 * B * HW) return;
+    const int d = (int)(idx / ((int64_t)B * HW));
+    const int b = (int)(idx / HW % B);
+    const int r = (int)(idx % HW);
+    const int N = d < 2 ? W : H;  // positions per line
+    const int i = r / N, j = r % N;
+    const Walk wk = walk_of(d, H, W);
+    const int pix = wk.o + i * wk.si + j * wk.sj;
+    const unsigned short* lg = reinterpret_cast<const unsigned short*>(logits) + ((size_t)d * B + b) * 3 * HW;
+    const float s0 = j > 0 ? sigm(bf16_bits_to_float(lg[pix])) : 0.f;
+    const float s1 = sigm(bf16_bits_to_float(lg[HW + pix]));
+    const float s2 = j < N - 1 ? sigm(bf16_bits_to_float(lg[2 * HW + pix])) : 0.f;
+    const float rs = __fdividef(1.f, s0 + s1 + s2);
+    taps[idx] = make_float2(s0 * rs, s2 * rs);
+}
+
 // Inputs of the proxy scans are staged in shared memory a chunk of SC_CH lines
 // at a time with cp.async, two chunks per warp in flight, so a line never
-// waits for global memory.  Row scans (top->bottom, bottom->top) stage each
-// line as a contiguous row [line][position]; column scans (left->right,
-// right->left) stage, for every row, the chunk's SC_CH adjacent columns
-// [position][column].
+// waits for global memory.  Row scans (top->bottom, bottom->top) stage x_proxy
+// and lambda of each line as a contiguous row [line][position]; column scans
+// (left->right, right->left) stage, for every row, the chunk's SC_CH adjacent
+// columns [position][column].  The taps are in scan order already:
+// [line][position] in every direction.
 constexpr int SC_CH = 8;
 constexpr int SC_NMAX = 128;
-// per warp and buffer: xp (fp32), lambda and three logit taps (bf16)
-constexpr int SC_BUF = SC_CH * SC_NMAX * (4 + 2 + 3 * 2);
+// per warp and buffer: xp (fp32), lambda (bf16), taps (2 x fp32)
+constexpr int SC_BUF = SC_CH * SC_NMAX * (4 + 2 + 8);
 constexpr int SC_SMEM = 4 * 2 * SC_BUF;
 
 __device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
@@ -294,54 +323,51 @@ __global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
     const float* const xp = a.xp + (size_t)plane * HW;
     const unsigned short* const lam =
         reinterpret_cast<const unsigned short*>(a.lam) + ((size_t)d * a.B * a.Cp + plane) * HW;
-    const unsigned short* const lg = reinterpret_cast<const unsigned short*>(a.logits) + ((size_t)d * a.B + b) * 3 * HW;
+    const float2* const tp = a.taps + ((size_t)d * a.B + b) * HW;
     float* const out = a.h + ((size_t)d * a.B * a.Cp + plane) * HW;
     unsigned char* const wbuf = sc_smem + d * 2 * SC_BUF;
-    // buffer layout: xp [SC_CH * N] fp32, then lambda, logit 0, 1, 2 [SC_CH * N] bf16 each
+    // buffer layout: xp [SC_CH * N] fp32, taps [SC_CH][N] float2, lambda [SC_CH * N] bf16
     const int nch = SC_CH * N;
 
     // stage chunk c (lines c*SC_CH ..) into buffer c & 1
     auto stage = [&](int c) {
         unsigned char* const bx = wbuf + (c & 1) * SC_BUF;
-        unsigned char* const bl = bx + nch * 4;
+        unsigned char* const bt = bx + nch * 4;
+        unsigned char* const bl = bt + nch * 8;
         const int i0 = c * SC_CH;
+        const int nl = L - i0 < SC_CH ? L - i0 : SC_CH;  // lines in this chunk
+        // taps: the chunk's lines are contiguous in scan order, 2 per 16-byte piece
+        for (int u = t; u < nl * N / 2; u += 32) cp_async16(bt + u * 16, tp + (size_t)i0 * N + 2 * u);
         if (rows) {
-            // line i0 + e is row r: xp N*4 bytes, each bf16 tensor N*2 bytes, in 16-byte pieces
-            const int fx = N / 4, fb = N / 8, per_line = fx + 4 * fb;
-            for (int u = t; u < SC_CH * per_line; u += 32) {
+            // line i0 + e is row r: xp N*4 bytes, lambda N*2 bytes, in 16-byte pieces
+            const int fx = N / 4, fb = N / 8, per_line = fx + fb;
+            for (int u = t; u < nl * per_line; u += 32) {
                 const int e = u / per_line, v = u % per_line;
-                if (i0 + e >= L) continue;
                 const int row0 = wk.o + (i0 + e) * wk.si;  // pixel of position 0 of the line
-                if (v < fx) {
+                if (v < fx)
                     cp_async16(bx + (e * N + 4 * v) * 4, xp + row0 + 4 * v);
-                } else {
-                    const int g = (v - fx) / fb, q = (v - fx) % fb;
-                    const unsigned short* src = g == 0 ? lam : lg + (g - 1) * HW;
-                    cp_async16(bl + ((size_t)g * nch + e * N + 8 * q) * 2, src + row0 + 8 * q);
-                }
+                else
+                    cp_async16(bl + (e * N + 8 * (v - fx)) * 2, lam + row0 + 8 * (v - fx));
             }
         } else {
             // for every row j: the chunk's SC_CH adjacent columns, ascending in the image
             const int c0 = wk.si > 0 ? i0 : a.W - SC_CH - i0;
-            for (int u = t; u < N * 6; u += 32) {
-                const int j = u / 6, v = u % 6;
+            for (int u = t; u < N * 3; u += 32) {
+                const int j = u / 3, v = u % 3;
                 const int pix = j * a.W + c0;
-                if (v < 2) {
+                if (v < 2)
                     cp_async16(bx + (j * SC_CH + 4 * v) * 4, xp + pix + 4 * v);
-                } else {
-                    const int g = v - 2;
-                    const unsigned short* src = g == 0 ? lam : lg + (g - 1) * HW;
-                    cp_async16(bl + ((size_t)g * nch + j * SC_CH) * 2, src + pix);
-                }
+                else
+                    cp_async16(bl + j * SC_CH * 2, lam + pix);
             }
         }
         cp_async_commit();
     };
-    // value of tensor g (0: xp, 1: lambda, 2..4: logit taps) at line e of the chunk, position j
+    // x_proxy (g = 0) or lambda (g = 1) at line e of the chunk, position j
     auto val = [&](const unsigned char* bx, int g, int e, int j) -> float {
         const int idx = rows ? e * N + j : j * SC_CH + (wk.si > 0 ? e : SC_CH - 1 - e);
         if (g == 0) return reinterpret_cast<const float*>(bx)[idx];
-        const unsigned short* bl = reinterpret_cast<const unsigned short*>(bx + nch * 4) + (size_t)(g - 1) * nch;
+        const unsigned short* bl = reinterpret_cast<const unsigned short*>(bx + nch * 12);
         return bf16_bits_to_float(bl[idx]);
     };
 
@@ -371,12 +397,9 @@ __global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
                 w0c[e][p] = w2c[e][p] = uc[e][p] = 0.f;
                 if (j < N) {
                     uc[e][p] = val(bx, 1, e, j) * val(bx, 0, e, j);
-                    const float s0 = j > 0 ? sigm(val(bx, 2, e, j)) : 0.f;
-                    const float s1 = sigm(val(bx, 3, e, j));
-                    const float s2 = j < N - 1 ? sigm(val(bx, 4, e, j)) : 0.f;
-                    const float r = __fdividef(1.f, s0 + s1 + s2);
-                    w0c[e][p] = s0 * r;
-                    w2c[e][p] = s2 * r;
+                    const float2 w = reinterpret_cast<const float2*>(bx + nch * 4)[e * N + j];
+                    w0c[e][p] = w.x;
+                    w2c[e][p] = w.y;
                 }
             }
         __syncwarp();  // every lane is done with buffer c & 1 before it is refilled
@@ -655,14 +678,15 @@ bool encode_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* d
 }
 
 struct BlockLayout {
-    size_t xp, h, total;
+    size_t xp, h, taps, total;
 };
 BlockLayout block_layout(const gspn_block_desc& d) {
     BlockLayout l;
     const size_t planes = (size_t)d.B * d.Cp * d.H * d.W;
     l.xp = kWsAlign;
     l.h = l.xp + align_up(planes * 4, kWsAlign);
-    l.total = l.h + align_up(4 * planes * 4, kWsAlign);
+    l.taps = l.h + align_up(4 * planes * 4, kWsAlign);
+    l.total = l.taps + align_up((size_t)4 * d.B * d.H * d.W * 8, kWsAlign);
     return l;
 }
 
@@ -777,10 +801,17 @@ gspn_status block_fwd(const gspn_block_desc* d, const void* x, const void* v, co
     if (cudaMemsetAsync(err, 0, sizeof(int), s) != cudaSuccess) return GSPN_ERR_CUDA;
     st = d->Cp <= 16 ? launch_proj<16>(dev, *d, x, v, xp, err, s) : launch_proj<32>(dev, *d, x, v, xp, err, s);
     if (st != GSPN_OK) return st;
+    float2* taps = reinterpret_cast<float2*>(w + l.taps);
+    {
+        const int64_t n = (int64_t)4 * d->B * d->H * d->W;
+        block_taps_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(logits), taps,
+                                                                        (int)d->B, (int)d->H, (int)d->W);
+        if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
+    }
     ScanArgs sa;
     sa.xp = xp;
     sa.lam = static_cast<const __nv_bfloat16*>(lam);
-    sa.logits = static_cast<const __nv_bfloat16*>(logits);
+    sa.taps = taps;
     sa.h = h;
     sa.B = (int)d->B;
     sa.Cp = d->Cp;

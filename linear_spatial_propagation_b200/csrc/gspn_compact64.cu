@@ -352,11 +352,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     // step e of chunk c a warp issues the TMEM load of steps e+2, e+3 (16
     // columns) and waits for it after step e+1's arithmetic.  At step 6 every
     // load of the chunk has completed, so the warp hands the stage back (one
-    // arrival per warp) and loads steps 0, 1 of chunk c+1 once that chunk's
-    // copies are committed.  Data stages are copied to registers whole at the
+    // arrival per warp) and loads steps 0, 1 of chunk c+1 once the quarter's
+    // weight warp has written it.  Data stages are copied to registers whole at the
     // chunk's start.
     const uint32_t twq = taddr + ((uint32_t)(32 * (warp & 3)) << 16) + TW_COL;
-    uint32_t wcur[16], wnxt[16];  // taps of steps (e, e+1) and of the next pair, 8 columns per step
+    uint32_t wcur[16] = {}, wnxt[16];  // taps of steps (e, e+1) and of the next pair, 8 columns per step
     auto wissue = [&](int c, int e) -> bool {
         if ((e & 1) == 0) {
             if (e < 6) {
