@@ -83,7 +83,7 @@ def measured_peaks():
 
 # sources of the kernel each pass's traffic figure was taken on
 KERNEL_SOURCES = {
-    "fwd": ("gspn_compact64.cu", "gspn_tma.cuh", "gspn_lane.cuh", "gspn_common.cuh", "gspn_internal.h"),
+    "fwd": ("gspn_compact64.cu", "gspn_tma.cuh", "gspn_lane.cuh", "gspn_tmem.cuh", "gspn_common.cuh", "gspn_internal.h"),
     "bwd": ("gspn_compact64_bwd.cu", "gspn_tma.cuh", "gspn_lane.cuh", "gspn_tmem.cuh", "gspn_common.cuh", "gspn_internal.h"),
 }
 

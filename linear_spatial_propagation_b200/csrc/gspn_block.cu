@@ -39,7 +39,7 @@
 //   C_proxy padded to 16 or 32) to shared memory; then one tcgen05 MMA per
 //   128-channel chunk forms D[c, pixel] = sum_k U[c,k] n[k,pixel] in tensor
 //   memory (two buffers), and the epilogue converts it to bf16 and stores it
-//   with TMA.
+//   with TMA, each warp its own 32 channel rows.
 //
 // Every mbarrier wait is bounded; on expiry a warp records the error word at
 // offset 0 of the workspace and leaves through its error path.
@@ -567,10 +567,11 @@ __global__ void __launch_bounds__(OB_THREADS, 2)
         const int et = threadIdx.x - 32;  // 0..127
         bool ok = true;
         int lt = 0, ch = 0;
-        for (int tile = blockIdx.x; ok && tile < a.ntiles; tile += gridDim.x, ++lt) {
+        for (int tile = blockIdx.x; tile < a.ntiles; tile += gridDim.x, ++lt) {
             const int b = tile / a.tiles_per_img, pix0 = (tile % a.tiles_per_img) * OB_N;
-            // n^T of the previous tile may still be read by its MMAs
-            ok = bar_and_128(lt == 0 || tma::mbar_wait(ndone, (lt - 1) & 1, a.limit));
+            // n^T of the previous tile may still be read by its MMAs; every warp
+            // reaches this barrier once per tile, and all leave if one has failed
+            ok = bar_and_128(ok && (lt == 0 || tma::mbar_wait(ndone, (lt - 1) & 1, a.limit)));
             if (!ok) break;
             {
                 const int pix = pix0 + et;
@@ -612,51 +613,62 @@ __global__ void __launch_bounds__(OB_THREADS, 2)
                 __syncwarp();
                 if (t == 0) tma::mbar_arrive(nready);
             }
-            // epilogue of every 128-channel chunk of this tile
+            // epilogue of every 128-channel chunk of this tile: each warp converts
+            // and stores its own 32 channel rows (its TMEM lane quarter), so the
+            // warps of the CTA do not wait for one another within a tile.  A warp
+            // whose wait runs out skips the rest of the tile and all leave
+            // together at the next tile's collective barrier.
             for (int cb = 0; cb < a.nchunks; ++cb, ++ch) {
+                if (!ok) continue;
                 const int buf = ch & 1;
                 const bool got = tma::mbar_wait(accf0 + 8 * buf, (ch >> 1) & 1, a.limit);
-                // the staged chunk of two chunks ago has been read by its TMA stores
-                if (et == 0) tma::bulk_wait_read_n<1>();
-                ok = bar_and_128(got);
-                if (!ok) break;
+                // this warp's rows of the chunk staged two chunks ago have been read
+                // by its TMA stores
+                if (t == 0) tma::bulk_wait_read_n<1>();
+                ok = __all_sync(FULL, got);
+                if (!ok) continue;
                 tmem::fence_after();
                 unsigned char* const ys = smem + buf * OB_YBUF;
                 const int row = 32 * q + t;  // channel row of the chunk = TMEM lane
+                const uint32_t tq = taddr + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * OB_N);
 #pragma unroll
-                for (int c32 = 0; c32 < OB_N / 32; ++c32) {
-                    uint32_t v[32];
-                    tmem::ld_x32(taddr + ((uint32_t)(32 * q) << 16) + (uint32_t)(buf * OB_N + 32 * c32), v);
-                    tmem::wait_ld(v);
-                    // pixels 32 c32 .. +31 of this channel: 4 chunks of 16 B in box c32 / 2,
-                    // 16-byte chunk j of a 128-byte row stored at j ^ (row % 8)
-                    unsigned char* const box = ys + (c32 >> 1) * (OB_M * 128) + row * 128;
+                for (int c64 = 0; c64 < OB_N / 64; ++c64) {
+                    // pixels 64 c64 .. +63 of this channel (box c64): two 32-column loads
+                    // in flight together; 16-byte chunk j of the 128-byte row at j ^ (row % 8)
+                    uint32_t va[32], vb[32];
+                    tmem::ld_x32(tq + 64u * c64, va);
+                    tmem::ld_x32(tq + 64u * c64 + 32u, vb);
+                    tmem::wait_ld(va);
+                    tmem::wait_ld(vb);
+                    unsigned char* const box = ys + c64 * (OB_M * 128) + row * 128;
 #pragma unroll
-                    for (int j4 = 0; j4 < 4; ++j4) {
-                        const int j = (c32 & 1) * 4 + j4;
+                    for (int j = 0; j < 8; ++j) {
+                        const uint32_t* v = j < 4 ? va + 8 * j : vb + 8 * (j - 4);
                         uint4 w;
-                        w.x = pack_bf2(__uint_as_float(v[8 * j4 + 0]), __uint_as_float(v[8 * j4 + 1]));
-                        w.y = pack_bf2(__uint_as_float(v[8 * j4 + 2]), __uint_as_float(v[8 * j4 + 3]));
-                        w.z = pack_bf2(__uint_as_float(v[8 * j4 + 4]), __uint_as_float(v[8 * j4 + 5]));
-                        w.w = pack_bf2(__uint_as_float(v[8 * j4 + 6]), __uint_as_float(v[8 * j4 + 7]));
+                        w.x = pack_bf2(__uint_as_float(v[0]), __uint_as_float(v[1]));
+                        w.y = pack_bf2(__uint_as_float(v[2]), __uint_as_float(v[3]));
+                        w.z = pack_bf2(__uint_as_float(v[4]), __uint_as_float(v[5]));
+                        w.w = pack_bf2(__uint_as_float(v[6]), __uint_as_float(v[7]));
                         *reinterpret_cast<uint4*>(box + ((j ^ (row & 7)) << 4)) = w;
                     }
                 }
                 tmem::fence_before();
+                tma::fence_proxy_async();  // the staged rows are read by TMA stores
                 __syncwarp();
-                if (t == 0) tma::mbar_arrive(acce0 + 8 * buf);
-                tma::fence_proxy_async();  // the staged chunk is read by TMA stores
-                asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (et == 0) {
-                    const uint32_t ysa = sbase + buf * OB_YBUF;
-                    tma::store_3d(&tm_y, ysa, pix0, cb * OB_M, b);
-                    tma::store_3d(&tm_y, ysa + OB_M * 128, pix0 + 64, cb * OB_M, b);
+                if (t == 0) {
+                    tma::mbar_arrive(acce0 + 8 * buf);
+                    const int c0 = cb * OB_M + 32 * q;  // first channel of this warp's rows
+                    if (c0 < a.C) {
+                        const uint32_t ysa = sbase + buf * OB_YBUF + q * 32 * 128;
+                        tma::store_3d(&tm_y, ysa, pix0, c0, b);
+                        if (pix0 + 64 < a.HW) tma::store_3d(&tm_y, ysa + OB_M * 128, pix0 + 64, c0, b);
+                    }
                     tma::bulk_commit();
                 }
             }
         }
         if (!ok && t == 0) atomicExch(a.err, 1);
-        if (et == 0) tma::bulk_wait_all();
+        if (t == 0) tma::bulk_wait_all();  // this warp's stores have read shared memory
     }
     tmem::fence_before();
     __syncthreads();
@@ -744,7 +756,7 @@ gspn_status launch_out(const DeviceInfo& dev, const gspn_block_desc& d, const fl
     CUtensorMap my;
     const cuuint64_t yd[3] = {(cuuint64_t)HW, (cuuint64_t)d.C, (cuuint64_t)d.B};
     const cuuint64_t ys[2] = {(cuuint64_t)HW * 2, (cuuint64_t)HW * d.C * 2};
-    const cuuint32_t yb[3] = {64, OB_M, 1};
+    const cuuint32_t yb[3] = {64, 32, 1};  // one warp's 32 channel rows of a 64-pixel box
     if (!encode_bf16(&my, y, 3, yd, ys, yb, CU_TENSOR_MAP_SWIZZLE_128B)) return GSPN_ERR_UNSUPPORTED;
     OutArgs a;
     a.h = h;
