@@ -297,10 +297,10 @@ __global__ void __launch_bounds__(256) block_taps_kernel(const __nv_bfloat16* __
 // columns [position][column].  The taps are in scan order already:
 // [line][position] in every direction.
 constexpr int SC_CH = 8;
-constexpr int SC_NMAX = 128;
-// per warp and buffer: xp (fp32), lambda (bf16), taps (2 x fp32)
-constexpr int SC_BUF = SC_CH * SC_NMAX * (4 + 2 + 8);
-constexpr int SC_SMEM = 4 * 2 * SC_BUF;
+// per warp and buffer, for lines of up to nmax positions: xp (fp32), lambda
+// (bf16), taps (2 x fp32); sized by the plane so small planes fit more CTAs
+__host__ __device__ constexpr int sc_buf_bytes(int nmax) { return SC_CH * nmax * (4 + 2 + 8); }
+__host__ __device__ constexpr int sc_smem_bytes(int nmax) { return 4 * 2 * sc_buf_bytes(nmax); }
 
 __device__ __forceinline__ void cp_async16(void* sdst, const void* gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(tma::smem_u32(sdst)), "l"(gsrc) : "memory");
@@ -310,7 +310,7 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int P>
-__global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
+__global__ void __launch_bounds__(128, P <= 2 ? 4 : 1) block_scan_kernel(const ScanArgs a) {
     extern __shared__ __align__(16) unsigned char sc_smem[];
     const int d = threadIdx.x >> 5, t = threadIdx.x & 31;
     const int plane = blockIdx.x;  // b * Cp + k
@@ -325,13 +325,14 @@ __global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
         reinterpret_cast<const unsigned short*>(a.lam) + ((size_t)d * a.B * a.Cp + plane) * HW;
     const float2* const tp = a.taps + ((size_t)d * a.B + b) * HW;
     float* const out = a.h + ((size_t)d * a.B * a.Cp + plane) * HW;
-    unsigned char* const wbuf = sc_smem + d * 2 * SC_BUF;
+    const int sbuf = sc_buf_bytes(a.H > a.W ? a.H : a.W);  // a multiple of 16: H, W are multiples of 8
+    unsigned char* const wbuf = sc_smem + d * 2 * sbuf;
     // buffer layout: xp [SC_CH * N] fp32, taps [SC_CH][N] float2, lambda [SC_CH * N] bf16
     const int nch = SC_CH * N;
 
     // stage chunk c (lines c*SC_CH ..) into buffer c & 1
     auto stage = [&](int c) {
-        unsigned char* const bx = wbuf + (c & 1) * SC_BUF;
+        unsigned char* const bx = wbuf + (c & 1) * sbuf;
         unsigned char* const bt = bx + nch * 4;
         unsigned char* const bl = bt + nch * 8;
         const int i0 = c * SC_CH;
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(128) block_scan_kernel(const ScanArgs a) {
         else
             cp_async_wait<0>();
         __syncwarp();  // every lane's pieces of chunk c are in shared memory
-        const unsigned char* const bx = wbuf + (c & 1) * SC_BUF;
+        const unsigned char* const bx = wbuf + (c & 1) * sbuf;
         // the chunk's taps and lambda * x first (they do not depend on the
         // state): the sigmoids of all its lines overlap, and the buffer is free
         // to refill before the lines are walked
@@ -835,9 +836,10 @@ gspn_status block_fwd(const gspn_block_desc* d, const void* x, const void* v, co
     const void* sfn = nmax <= 32   ? (const void*)block_scan_kernel<1>
                       : nmax <= 64 ? (const void*)block_scan_kernel<2>
                                    : (const void*)block_scan_kernel<4>;
-    if (ensure_smem_attr(sfn, SC_SMEM, nmax <= 32 ? 36 : nmax <= 64 ? 37 : 38) != cudaSuccess) return GSPN_ERR_CUDA;
+    const int ssmem = sc_smem_bytes(nmax);
+    if (ensure_smem_attr(sfn, ssmem, nmax <= 32 ? 36 : nmax <= 64 ? 37 : 38) != cudaSuccess) return GSPN_ERR_CUDA;
     void* sargs[] = {&sa};
-    if (cudaLaunchKernel(sfn, dim3(grid), dim3(128), sargs, SC_SMEM, s) != cudaSuccess) return GSPN_ERR_CUDA;
+    if (cudaLaunchKernel(sfn, dim3(grid), dim3(128), sargs, ssmem, s) != cudaSuccess) return GSPN_ERR_CUDA;
     if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
     return d->Cp <= 16 ? launch_out<16>(dev, *d, h, alpha, gamma, u, y, err, s)
                        : launch_out<32>(dev, *d, h, alpha, gamma, u, y, err, s);
