@@ -20,8 +20,10 @@
 // ones add, the last one adds and writes the output in the I/O dtype), so the
 // sum is taken in direction order and does not depend on timing.  Tap weights
 // are normalised from the logits (Key design 1) for a whole chunk before its
-// lines are walked, so the sigmoids overlap and the line loop carries only
-// the dependent update.
+// lines are walked, so the line loop carries only the dependent update.  With
+// channel-shared taps they are formed once per (direction, image, pixel) by a
+// pre-kernel, in scan order, and every channel's CTA loads them with its
+// chunk instead of recomputing three sigmoids per position and line.
 #include "gspn_internal.h"
 
 namespace gspn {
@@ -37,11 +39,38 @@ struct LargeArgs {
     const void* logits;
     const void* lam;
     void* out;
-    float* acc;  // [planes][HW]
-    int nw;      // warps per CTA = ceil(max line length / 64)
+    float* acc;          // [planes][HW]
+    const float2* taps;  // channel-shared taps: [slot][B][line][position] (w0, w2); else unused
+    int nw;              // warps per CTA = ceil(max line length / 64)
 };
 
 __device__ __forceinline__ float lg_sigmoid(float z) { return __fdividef(1.f, 1.f + __expf(-z)); }
+
+// Channel-shared taps in scan order: taps[((slot*B + b)*L + i)*N + j] = (w0, w2)
+// of position j of line i of the slot's direction in image b: the sigmoids of
+// the pixel's three tap logits normalised over the taps that exist (w0 = 0 at
+// j = 0, w2 = 0 at j = N-1), with the same operations as the in-kernel path.
+template <typename T>
+__global__ void __launch_bounds__(256) large_taps_kernel(const T* __restrict__ logits, float2* __restrict__ taps,
+                                                          const Launch g) {
+    const int H = g.H, W = g.W, HW = H * W, B = g.B;
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx >= (int64_t)g.D * B * HW) return;
+    const int slot = (int)(idx / ((int64_t)B * HW));
+    const int b = (int)(idx / HW % B);
+    const int r = (int)(idx % HW);
+    const int d = dir_of(g, slot);
+    const int N = line_len(d, H, W);
+    const int i = r / N, j = r % N;
+    const Walk wk = walk_of(d, H, W);
+    const int pix = wk.o + i * wk.si + j * wk.sj;
+    const T* const lg = logits + ((int64_t)slot * B + b) * 3 * HW;
+    const float s0 = j > 0 ? lg_sigmoid(load_elt(lg, pix)) : 0.f;
+    const float s1 = lg_sigmoid(load_elt(lg, HW + pix));
+    const float s2 = j < N - 1 ? lg_sigmoid(load_elt(lg, 2 * HW + pix)) : 0.f;
+    const float rs = __fdividef(1.f, s0 + s1 + s2);
+    taps[idx] = make_float2(s0 * rs, s2 * rs);
+}
 
 // element access for both dtypes: a chunk is CH elements of one tensor, kept
 // as raw 32-bit words (two bf16 or one fp32 per word)
@@ -62,24 +91,35 @@ struct Elt<__nv_bfloat16> {
 };
 
 // The inputs of one chunk for this lane's two positions: for each of the five
-// tensors (x, lambda, logit taps 0..2) and each position p, CH values (one
-// per line) packed in WPP words.
-template <typename T>
+// tensors (x, lambda, logit taps 0..2; with a taps table only x and lambda)
+// and each position p, CH values (one per line) packed in WPP words.
+template <typename T, bool TAB>
 struct Chunk {
     static constexpr int CH = Elt<T>::CH;
     static constexpr int WPP = CH * (int)sizeof(T) / 4;  // words per position and tensor
-    uint32_t v[5][2][WPP];
+    static constexpr int NT = TAB ? 2 : 5;
+    uint32_t v[NT][2][WPP];
+    float4 tw[TAB ? CH : 1];  // with a taps table: (w0, w2) of positions j0, j0 + 1 per line
     float acc[2][CH];  // the accumulator at the chunk's pixels (not the first direction)
 };
 
 // The chunk of lines i0 .. i0 + CH - 1 at positions j0, j0 + 1, and, when
 // `with_acc`, the accumulator values there.  The accumulator was written by
 // this CTA's previous direction, so it is read through the coherent path.
-template <typename T>
-__device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5], const float* acc, bool with_acc,
-                                           bool rowscan, const Walk& wk, int W, int i0, int j0, int N) {
+template <typename T, bool TAB>
+__device__ __forceinline__ void load_chunk(Chunk<T, TAB>& ck, const T* const (&src)[5], const float2* tap,
+                                           const float* acc, bool with_acc, bool rowscan, const Walk& wk, int W,
+                                           int i0, int j0, int N) {
     constexpr int CH = Elt<T>::CH;
-    constexpr int WPP = Chunk<T>::WPP;
+    constexpr int WPP = Chunk<T, TAB>::WPP;
+    constexpr int NT = Chunk<T, TAB>::NT;
+    if constexpr (TAB) {
+        // the taps of lines i0 .. i0 + CH - 1 at positions j0, j0 + 1: 16 bytes per line
+#pragma unroll
+        for (int e = 0; e < CH; ++e)
+            ck.tw[e] = j0 < N ? __ldg(reinterpret_cast<const float4*>(tap + (size_t)(i0 + e) * N + j0))
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
     if (rowscan) {
         // line i0 + e: a row; positions j0, j0 + 1 are adjacent elements
 #pragma unroll
@@ -90,7 +130,7 @@ __device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5
             ck.acc[0][e] = av.x;
             ck.acc[1][e] = av.y;
 #pragma unroll
-            for (int s = 0; s < 5; ++s) {
+            for (int s = 0; s < NT; ++s) {
                 const uint16_t* b16 = reinterpret_cast<const uint16_t*>(src[s] + pix);
                 if constexpr (sizeof(T) == 4) {
                     const float* f = reinterpret_cast<const float*>(src[s]) + pix;
@@ -137,7 +177,7 @@ __device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5
                 for (int m = 0; m < CH; ++m) ck.acc[p][m] = av[CH - 1 - m];
             }
 #pragma unroll
-            for (int s = 0; s < 5; ++s) {
+            for (int s = 0; s < NT; ++s) {
                 uint4 q = make_uint4(0u, 0u, 0u, 0u);
                 if (j < N) q = __ldg(reinterpret_cast<const uint4*>(src[s] + first));
                 uint32_t w[4] = {q.x, q.y, q.z, q.w};
@@ -157,9 +197,10 @@ __device__ __forceinline__ void load_chunk(Chunk<T>& ck, const T* const (&src)[5
     }
 }
 
-template <typename T>
+template <typename T, bool TAB>
 __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const LargeArgs a) {
     constexpr int CH = Elt<T>::CH;
+    constexpr int NTAP0 = TAB ? 0 : 2;  // first logit tensor of a chunk (the in-kernel taps)
     __shared__ float edge[2][kLargeMaxWarps][2];  // [line parity][warp][first, last]
     const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
     const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C;
@@ -179,14 +220,15 @@ __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const La
         const T* const src[5] = {static_cast<const T*>(a.x) + plane * HW,
                                  static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW, lg,
                                  lg + HW, lg + 2 * HW};
+        const float2* const tap = TAB ? a.taps + (slot * (int64_t)B + b) * HW : nullptr;
         const bool first_dir = slot == 0, last_dir = slot == a.g.D - 1;
         float h0 = 0.f, h1 = 0.f;
         int gpos = 0;
-        Chunk<T> cur, nxt;
-        load_chunk<T>(cur, src, acc, !first_dir, rowscan, wk, W, 0, j0, N);
+        Chunk<T, TAB> cur, nxt;
+        load_chunk<T, TAB>(cur, src, tap, acc, !first_dir, rowscan, wk, W, 0, j0, N);
         float colbuf[2][CH];  // column scans: a chunk of outputs per row, stored at the chunk's end
         for (int i0 = 0; i0 < L; i0 += CH) {
-            if (i0 + CH < L) load_chunk<T>(nxt, src, acc, !first_dir, rowscan, wk, W, i0 + CH, j0, N);
+            if (i0 + CH < L) load_chunk<T, TAB>(nxt, src, tap, acc, !first_dir, rowscan, wk, W, i0 + CH, j0, N);
             // the chunk's taps and lambda * x first: they do not depend on the
             // state, so the sigmoids of all its lines and positions overlap, and
             // the line loop below is only the dependent update
@@ -197,12 +239,17 @@ __global__ void __launch_bounds__(kLargeMaxWarps * 32) large_fwd_kernel(const La
                 for (int p = 0; p < 2; ++p) {
                     const int j = j0 + p;
                     uc[e][p] = Elt<T>::get(cur.v[1][p], e) * Elt<T>::get(cur.v[0][p], e);
-                    const float s0 = j > 0 ? lg_sigmoid(Elt<T>::get(cur.v[2][p], e)) : 0.f;
-                    const float s1 = lg_sigmoid(Elt<T>::get(cur.v[3][p], e));
-                    const float s2 = j < N - 1 ? lg_sigmoid(Elt<T>::get(cur.v[4][p], e)) : 0.f;
-                    const float r = __fdividef(1.f, s0 + s1 + s2);
-                    w0c[e][p] = s0 * r;
-                    w2c[e][p] = s2 * r;
+                    if constexpr (TAB) {
+                        w0c[e][p] = p ? cur.tw[e].z : cur.tw[e].x;
+                        w2c[e][p] = p ? cur.tw[e].w : cur.tw[e].y;
+                    } else {
+                        const float s0 = j > 0 ? lg_sigmoid(Elt<T>::get(cur.v[NTAP0][p], e)) : 0.f;
+                        const float s1 = lg_sigmoid(Elt<T>::get(cur.v[NTAP0 + 1][p], e));
+                        const float s2 = j < N - 1 ? lg_sigmoid(Elt<T>::get(cur.v[NTAP0 + 2][p], e)) : 0.f;
+                        const float r = __fdividef(1.f, s0 + s1 + s2);
+                        w0c[e][p] = s0 * r;
+                        w2c[e][p] = s2 * r;
+                    }
                 }
 #pragma unroll
             for (int e = 0; e < CH; ++e) {
@@ -295,7 +342,11 @@ bool large_eligible(const Problem& p) {
     return nmax > 64 && nmax <= 64 * kLargeMaxWarps && H % 8 == 0 && W % 8 == 0 && p.HW <= (1 << 24);
 }
 
-size_t large_fwd_workspace(const Problem& p) { return align_up((size_t)p.planes * p.HW * sizeof(float), kWsAlign); }
+// the accumulator planes, then (channel-shared taps) the taps table
+size_t large_fwd_workspace(const Problem& p) {
+    const size_t acc = align_up((size_t)p.planes * p.HW * sizeof(float), kWsAlign);
+    return acc + (p.g.shared ? align_up((size_t)p.g.D * p.g.B * p.HW * sizeof(float2), kWsAlign) : 0);
+}
 
 gspn_status large_fwd(const Problem& p, const void* x, const void* logits, const void* lam, void* out, void* ws,
                       cudaStream_t s) {
@@ -306,14 +357,33 @@ gspn_status large_fwd(const Problem& p, const void* x, const void* logits, const
     a.lam = lam;
     a.out = out;
     a.acc = static_cast<float*>(ws);
+    a.taps = nullptr;
     const int nmax = p.g.H > p.g.W ? p.g.H : p.g.W;
     a.nw = (nmax + 63) / 64;
     if (p.planes > 0x7fffffff) return GSPN_ERR_UNSUPPORTED;
     const unsigned grid = (unsigned)p.planes;
-    if (p.d.dtype == GSPN_F32)
-        large_fwd_kernel<float><<<grid, a.nw * 32, 0, s>>>(a);
-    else
-        large_fwd_kernel<__nv_bfloat16><<<grid, a.nw * 32, 0, s>>>(a);
+    const bool f32 = p.d.dtype == GSPN_F32;
+    if (p.g.shared) {
+        float2* taps = reinterpret_cast<float2*>(static_cast<char*>(ws) +
+                                                 align_up((size_t)p.planes * p.HW * sizeof(float), kWsAlign));
+        const int64_t n = (int64_t)p.g.D * p.g.B * p.HW;
+        const unsigned tg = (unsigned)((n + 255) / 256);
+        if (f32)
+            large_taps_kernel<float><<<tg, 256, 0, s>>>(static_cast<const float*>(logits), taps, p.g);
+        else
+            large_taps_kernel<__nv_bfloat16><<<tg, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(logits), taps, p.g);
+        if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
+        a.taps = taps;
+        if (f32)
+            large_fwd_kernel<float, true><<<grid, a.nw * 32, 0, s>>>(a);
+        else
+            large_fwd_kernel<__nv_bfloat16, true><<<grid, a.nw * 32, 0, s>>>(a);
+    } else {
+        if (f32)
+            large_fwd_kernel<float, false><<<grid, a.nw * 32, 0, s>>>(a);
+        else
+            large_fwd_kernel<__nv_bfloat16, false><<<grid, a.nw * 32, 0, s>>>(a);
+    }
     return cudaGetLastError() == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
 }
 
