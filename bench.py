@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--pass", dest="passes", default="both", choices=["both", "fwd", "bwd"],
                     help="profiling aid: time only one pass (the JSON line then covers that pass)")
     ap.add_argument("--batch", type=int, default=0, help="profiling aid: override B (0 = the workload's)")
+    ap.add_argument("--graph", action="store_true",
+                    help="replay each pass from a CUDA graph captured once (no per-call host work in the timed loop)")
     return ap.parse_args()
 
 
@@ -288,11 +290,12 @@ def job_gbs(bytes_per_rank: int, n_ranks: int, ms: float) -> float:
     return bytes_per_rank * n_ranks / (ms * 1e-3) / 1e9
 
 
-def config_of(w, n, passes="both"):
+def config_of(w, n, passes="both", graph=False):
     return {"workload": w.name, "B": w.B, "C": w.C, "H": w.H, "W": w.W,
             "directions": "+".join(n_ for b, n_ in ((1, "T2B"), (2, "B2T"), (4, "L2R"), (8, "R2L")) if w.dir_mask & b),
             "groups": w.groups, "shared_taps": w.shared, "io_dtype": w.dtype,
             "pass": {"both": "fwd+bwd", "fwd": "fwd", "bwd": "bwd"}[passes],
+            "launch": "cuda_graph" if graph else "direct",
             "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"}
 
 
@@ -338,18 +341,20 @@ def run_gpu(args, w):
     stream = torch.cuda.current_stream(dev)
     sp = stream.cuda_stream
 
-    def fwd(din=d, o=None):
+    def fwd(din=d, o=None, strm=None):
         o = out if o is None else o
         st = lsp.gspn_fwd(desc, din["x"].data_ptr(), din["logits"].data_ptr(), din["lam"].data_ptr(), o.data_ptr(),
-                          wsf.data_ptr() if wsf is not None else 0, wsf.numel() if wsf is not None else 0, sp)
+                          wsf.data_ptr() if wsf is not None else 0, wsf.numel() if wsf is not None else 0,
+                          sp if strm is None else strm)
         if st:
             raise lsp.GspnError(st, "gspn_fwd")
 
-    def bwd(din=d, g=None):
+    def bwd(din=d, g=None, strm=None):
         g = grads if g is None else g
         st = lsp.gspn_bwd(desc, din["x"].data_ptr(), din["logits"].data_ptr(), din["lam"].data_ptr(),
                           din["dout"].data_ptr(), g[0].data_ptr(), g[1].data_ptr(), g[2].data_ptr(),
-                          wsb.data_ptr() if wsb is not None else 0, wsb.numel() if wsb is not None else 0, sp)
+                          wsb.data_ptr() if wsb is not None else 0, wsb.numel() if wsb is not None else 0,
+                          sp if strm is None else strm)
         if st:
             raise lsp.GspnError(st, "gspn_bwd")
 
@@ -370,6 +375,27 @@ def run_gpu(args, w):
         if do_b:
             bwd()
     barrier()
+    # --graph: each pass is captured once into a CUDA graph (the library's calls
+    # only enqueue work on the given stream) and the timed loop replays them
+    fwd_t, bwd_t = fwd, bwd
+    graphs = []
+    if args.graph:
+        gs = torch.cuda.Stream(dev)
+        gs.wait_stream(stream)
+        with torch.cuda.stream(gs):
+            for fn in (fwd, bwd):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g, stream=gs):
+                    fn(strm=gs.cuda_stream)
+                graphs.append(g)
+        stream.wait_stream(gs)
+        fwd_t, bwd_t = graphs[0].replay, graphs[1].replay
+        for _ in range(max(3, args.warmup)):
+            if do_f:
+                fwd_t()
+            if do_b:
+                bwd_t()
+        barrier()
     K = args.steps
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -380,10 +406,10 @@ def run_gpu(args, w):
     for k in range(K):
         ev[k][0].record(stream)
         if do_f:
-            fwd()
+            fwd_t()
         ev[k][1].record(stream)
         if do_b:
-            bwd()
+            bwd_t()
         ev[k][2].record(stream)
     e_end.record(stream)
     barrier()
@@ -477,7 +503,7 @@ def run_gpu(args, w):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_gpu, "steps": K,
             "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded numpy PCG64, per-rank seed)",
-            "config": config_of(w, n_gpu, args.passes),
+            "config": config_of(w, n_gpu, args.passes, args.graph),
             "pct_of_peak": 100.0 * value / n_gpu / peak,
             "gpix_ch_per_s": pixch * n_gpu / (ms * 1e-3) / 1e9,
             "fwd": {"ms": fwd_ms, "GB/s": fwd_gbs, "pct_of_peak": 100.0 * fwd_gbs / peak,
