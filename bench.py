@@ -51,7 +51,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="libgspn", choices=["libgspn", "reference"])
     ap.add_argument("--workload", default=synth.HEADLINE,
-                    choices=list(synth.WORKLOADS) + list(synth.BLOCK_WORKLOADS))
+                    choices=list(synth.WORKLOADS) + list(synth.EXTRA_WORKLOADS) + list(synth.BLOCK_WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target length of the oracle sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -688,7 +688,7 @@ def main():
         if args.impl == "reference":
             return run_block_reference(args, bw)
         return run_block(args, bw)
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS.get(args.workload) or synth.EXTRA_WORKLOADS[args.workload]
     if not w.backward:
         w = w.replace(backward=True)
     if args.batch:

@@ -326,6 +326,10 @@ Plan plan_for(const Problem& p, const DeviceInfo& dev, int line_bufs) {
         pl.wpc = (int)(budget / lines);
     }
     if (pl.wpc > kMaxWarps) pl.wpc = kMaxWarps;
+    // spread the planes over the SMs before stacking them in a CTA: with fewer
+    // planes than 8 per SM, CTAs of fewer warps (one warp is one plane)
+    const int64_t per_sm = (p.planes + dev.sm_count - 1) / (dev.sm_count > 0 ? dev.sm_count : 1);
+    if ((int64_t)pl.wpc > per_sm) pl.wpc = (int)per_sm;
     if (pl.wpc < 1) pl.wpc = 1;
     if ((int64_t)pl.wpc > p.planes) pl.wpc = (int)p.planes;
     pl.smem = (size_t)pl.wpc * (lines + (pl.acc_in_smem ? acc : 0));
@@ -365,7 +369,7 @@ gspn_status generic_fwd(const Problem& p, const DeviceInfo& dev, const void* x, 
     if (grid > 0x7fffffff) return GSPN_ERR_UNSUPPORTED;
     const int nmax = p.g.H > p.g.W ? p.g.H : p.g.W;
     const bool f32 = p.d.dtype == GSPN_F32;
-    // lines of up to 128 positions: the pipelined kernel with 1, 2 or 4 positions per lane
+    // lines of up to 256 positions: the pipelined kernel with 1, 2, 4 or 8 positions per lane
     const void* fn;
     int slot;
     if (nmax <= 32) {
@@ -380,6 +384,10 @@ gspn_status generic_fwd(const Problem& p, const DeviceInfo& dev, const void* x, 
         fn = f32 ? (const void*)generic_fwd_pipelined_kernel<float, 4>
                  : (const void*)generic_fwd_pipelined_kernel<__nv_bfloat16, 4>;
         slot = f32 ? 15 : 16;
+    } else if (nmax <= 256) {
+        fn = f32 ? (const void*)generic_fwd_pipelined_kernel<float, 8>
+                 : (const void*)generic_fwd_pipelined_kernel<__nv_bfloat16, 8>;
+        slot = f32 ? 39 : 40;
     } else {
         fn = f32 ? (const void*)generic_fwd_kernel<float> : (const void*)generic_fwd_kernel<__nv_bfloat16>;
         slot = f32 ? 0 : 1;

@@ -91,6 +91,16 @@ WORKLOADS: Dict[str, Workload] = {
 
 HEADLINE = "compact_4dir_bf16_b32c1152_64x64"
 
+# Shapes outside the five, timed by the bench only: planes whose sides are not
+# multiples of 8 and longer than 64 take the generic kernels (one warp per
+# plane, directions in turn).
+EXTRA_WORKLOADS: Dict[str, Workload] = {
+    w.name: w
+    for w in (
+        Workload("generic_4dir_f32_b2c64_130x70", 2, 64, 130, 70, ALL_DIRS, 1, False, "f32", 1.0, 30),
+    )
+}
+
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
     """Round float32 values to the nearest-even bf16; return the uint16 bits."""

@@ -152,6 +152,7 @@ SHAPES = [
     (3, 24, 64, 64, 15, 64, True, "bf16"),
     (5, 8, 64, 64, 15, 2, True, "bf16"),
     (1, 2, 130, 70, 15, 1, True, "bf16"),
+    (1, 2, 150, 90, 15, 3, False, "f32"),  # lines of 129..256 positions: 8 positions per lane
     # 128x128 compact bf16 with C % 4 == 0: the TMA-fed 128x128 forward
     (1, 4, 128, 128, 15, 1, True, "bf16"),
     (2, 12, 128, 128, 15, 1, True, "bf16"),
