@@ -259,9 +259,16 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) smal
     const int64_t plane = blockIdx.x;
     const int64_t b = plane / C, c = plane % C, cw = a.g.shared ? 0 : c;
     const int Cw = a.g.shared ? 1 : C;
-    float* const hst = smem + (size_t)warp * HW;                 // this direction's lines, scan coordinates
-    float* const dxacc = smem + (size_t)(D + warp) * HW;         // this direction's share of dx
-    float* const lb = smem + (size_t)2 * D * HW + (size_t)warp * 6 * kLS;  // line buffers
+    // this direction's lines in scan coordinates (line i at i * N).  With two
+    // positions per lane (lines of 33..64) its share of dx then takes the place
+    // of the lines the adjoint has left (line i's h is last read as the
+    // predecessor of line i+1), so a plane needs half the shared memory and
+    // more CTAs fit; with one per lane (where registers, not shared memory,
+    // bound the CTAs per SM) dx has planes of its own, in image coordinates.
+    constexpr bool kDxInPlace = P == 2;
+    float* const hst = smem + (size_t)warp * HW;
+    float* const dxacc = smem + (size_t)(D + warp) * HW;  // one position per lane only
+    float* const lb = smem + (size_t)(kDxInPlace ? 1 : 2) * D * HW + (size_t)warp * 6 * kLS;  // line buffers
 
     const int slot = warp, d = dir_of(a.g, slot);
     const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
@@ -359,7 +366,7 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) smal
                     const int p = pi + j * wk.sj;
                     float av = vg[r][e];
                     if (carry_in) av += qn[j + 2] + qn[kLS + j + 1] + qn[2 * kLS + j];
-                    dxacc[p] = vl[r][e] * av;
+                    const float dxv = vl[r][e] * av;
                     if (kPieces && col)
                         put_bf16<CH>(cl[r], e, vx[r][e] * av);
                     else
@@ -385,6 +392,10 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) smal
                     qc[j + 1] = q0;
                     qc[kLS + j + 1] = q1;
                     qc[2 * kLS + j + 1] = q2;
+                    if constexpr (kDxInPlace)
+                        hst[i * N + j] = dxv;  // h of line i is dead: line i+1 has been processed
+                    else
+                        dxacc[p] = dxv;
                     if (a.g.shared) {
                         if (carry_out) {
                             unsigned long long* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
@@ -430,10 +441,28 @@ __global__ void __launch_bounds__(128, P == 2 ? 3 : sizeof(T) == 2 ? 5 : 6) smal
     __syncthreads();
     // dx: the directions' shares summed in direction order
     T* dx = static_cast<T*>(a.dx) + plane * HW;
-    for (int q = threadIdx.x; q < HW; q += blockDim.x) {
-        float s = smem[(size_t)D * HW + q];
-        for (int k = 1; k < D; ++k) s += smem[(size_t)(D + k) * HW + q];
-        store_elt(dx, q, s);
+    if constexpr (kDxInPlace) {
+        // share k sits in scan coordinates of its direction: pixel (row, col) at
+        // line i, position j
+        for (int q = threadIdx.x; q < HW; q += blockDim.x) {
+            const int row = q / W, col = q - row * W;
+            float s = 0.f;
+            for (int k = 0; k < D; ++k) {
+                const int dk = dir_of(a.g, k);
+                const int idx = dk == T2B   ? row * W + col
+                                : dk == B2T ? (H - 1 - row) * W + col
+                                : dk == L2R ? col * H + row
+                                            : (W - 1 - col) * H + row;
+                s = k == 0 ? smem[(size_t)k * HW + idx] : s + smem[(size_t)k * HW + idx];
+            }
+            store_elt(dx, q, s);
+        }
+    } else {
+        for (int q = threadIdx.x; q < HW; q += blockDim.x) {
+            float s = smem[(size_t)D * HW + q];
+            for (int k = 1; k < D; ++k) s += smem[(size_t)(D + k) * HW + q];
+            store_elt(dx, q, s);
+        }
     }
 }
 
@@ -449,7 +478,12 @@ __global__ void small_convert_kernel(const unsigned long long* src, T* dst, int6
 }
 
 size_t fwd_smem(const Problem& p) { return ((size_t)p.g.D * p.HW + (size_t)p.g.D * 2 * kLS) * sizeof(float); }
-size_t bwd_smem(const Problem& p) { return ((size_t)2 * p.g.D * p.HW + (size_t)p.g.D * 6 * kLS) * sizeof(float); }
+// one plane per direction with two positions per lane (dx in place of the dead
+// lines), two with one per lane (lines of at most 32 positions)
+size_t bwd_smem(const Problem& p) {
+    const bool one = (p.g.H > p.g.W ? p.g.H : p.g.W) <= 32;
+    return ((size_t)(one ? 2 : 1) * p.g.D * p.HW + (size_t)p.g.D * 6 * kLS) * sizeof(float);
+}
 unsigned grid_1d(int64_t n) {
     const int64_t g = (n + 255) / 256;
     return (unsigned)(g < 4096 ? (g > 0 ? g : 1) : 4096);
