@@ -293,6 +293,195 @@ __global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_kernel(BwdArgs a) 
     for (int q = lane; q < HW; q += 32) store_elt(dx, q, dxacc[q]);
 }
 
+// The backward with the inputs of the next line in flight: lane l holds
+// positions l + 32r (r < P) of a line in registers, as in the pipelined
+// forward.  The recompute loads line i+1's lambda*x and tap logits before it
+// computes line i; the adjoint loads line i-1's dout, lambda, x, tap logits and
+// the three recomputed states it reads before it computes line i (with 8
+// positions per lane the states are read where they are used, which keeps the
+// kernel within its registers).  Same arithmetic in the same order as
+// generic_bwd_kernel, so the same results.
+template <typename T, int P>
+__global__ void __launch_bounds__(kMaxWarps * 32) generic_bwd_pipelined_kernel(BwdArgs a) {
+    extern __shared__ float smem[];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int H = a.g.H, W = a.g.W, HW = H * W, B = a.g.B, C = a.g.C;
+    const int64_t plane = (int64_t)blockIdx.x * a.warps_per_cta + warp;
+    if (plane >= (int64_t)B * C) return;
+    constexpr bool kPrefH = P <= 4;  // the states of the next line in flight too
+    const int ls = a.lstride;
+    float* wsm = smem + (size_t)warp * (6 * ls + (a.acc_in_smem ? HW : 0));
+    float* dxacc = a.acc_in_smem ? wsm + 6 * ls : a.dx_ws + plane * HW;
+    float* hst = a.hstore + plane * HW;
+    const int64_t b = plane / C, c = plane % C, cw = a.g.shared ? 0 : c;
+    const int Cw = a.g.shared ? 1 : C;
+    const T* x = static_cast<const T*>(a.x) + plane * HW;
+    const T* g = static_cast<const T*>(a.dout) + plane * HW;
+
+    for (int slot = 0; slot < a.g.D; ++slot) {
+        const int d = dir_of(a.g, slot);
+        const int L = scan_len(d, H, W), N = line_len(d, H, W), seg = L / a.g.groups;
+        const T* lam = static_cast<const T*>(a.lam) + ((slot * (int64_t)B + b) * C + c) * HW;
+        const T* lg = static_cast<const T*>(a.logits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+        T* dlam = static_cast<T*>(a.dlam) + ((slot * (int64_t)B + b) * C + c) * HW;
+        const Walk wk = walk_of(d, H, W);
+
+        // 1. recompute this direction's lines into hst (scan coordinates)
+        {
+            float* hp = wsm;
+            float* hc = wsm + ls;
+            if (lane == 0) hp[0] = hp[N + 1] = hc[0] = hc[N + 1] = 0.f;
+            __syncwarp();
+            float lx[P], g0[P], g1[P], g2[P];
+            auto fetch = [&](int i, float (&flx)[P], float (&f0)[P], float (&f1)[P], float (&f2)[P]) {
+#pragma unroll
+                for (int r = 0; r < P; ++r) {
+                    const int j = lane + 32 * r;
+                    const int pp = j < N ? wk.o + i * wk.si + j * wk.sj : 0;  // in bounds for idle lanes
+                    flx[r] = load_elt(lam, pp) * load_elt(x, pp);
+                    f0[r] = load_elt(lg, pp);
+                    f1[r] = load_elt(lg, HW + pp);
+                    f2[r] = load_elt(lg, 2 * HW + pp);
+                }
+            };
+            fetch(0, lx, g0, g1, g2);
+            for (int i = 0, gi = 0; i < L; ++i, gi = gi + 1 == seg ? 0 : gi + 1) {  // gi = i % seg
+                float nlx[P], n0[P], n1[P], n2[P];
+                if (i + 1 < L) fetch(i + 1, nlx, n0, n1, n2);
+                const bool carry = gi != 0;
+#pragma unroll
+                for (int r = 0; r < P; ++r) {
+                    const int j = lane + 32 * r;
+                    if (j < N) {
+                        float v = lx[r];
+                        if (carry) {
+                            const float s0 = j > 0 ? sigmoidf(g0[r]) : 0.f;
+                            const float s1 = sigmoidf(g1[r]);
+                            const float s2 = j < N - 1 ? sigmoidf(g2[r]) : 0.f;
+                            v += (s0 * hp[j] + s1 * hp[j + 1] + s2 * hp[j + 2]) / (s0 + s1 + s2);
+                        }
+                        hc[j + 1] = v;
+                        hst[i * N + j] = v;
+                    }
+                }
+                __syncwarp();
+                float* t = hp; hp = hc; hc = t;
+#pragma unroll
+                for (int r = 0; r < P; ++r) {
+                    lx[r] = nlx[r];
+                    g0[r] = n0[r];
+                    g1[r] = n1[r];
+                    g2[r] = n2[r];
+                }
+            }
+        }
+        // 2. reverse scan of the adjoint
+        float* qn = wsm;           // 3 buffers: products of line i+1
+        float* qc = wsm + 3 * ls;  // 3 buffers: products of line i
+        for (int q = lane; q < 6 * ls; q += 32) wsm[q] = 0.f;
+        __syncwarp();
+        // line i's inputs: dout, lambda, x, the three tap logits, and the states
+        // h_{i-1}[j-1], h_{i-1}[j], h_{i-1}[j+1] its tap gradients read
+        float vg[P], vl[P], vx[P], t0[P], t1[P], t2[P], hm[P], hz[P], hq[P];
+        auto fetch2 = [&](int i, float (&fg)[P], float (&fl)[P], float (&fx)[P], float (&f0)[P], float (&f1)[P],
+                          float (&f2)[P], float (&fm)[P], float (&fz)[P], float (&fq)[P]) {
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                const int j = lane + 32 * r;
+                const int pp = j < N ? wk.o + i * wk.si + j * wk.sj : 0;  // in bounds for idle lanes
+                fg[r] = load_elt(g, pp);
+                fl[r] = load_elt(lam, pp);
+                fx[r] = load_elt(x, pp);
+                f0[r] = load_elt(lg, pp);
+                f1[r] = load_elt(lg, HW + pp);
+                f2[r] = load_elt(lg, 2 * HW + pp);
+                if constexpr (kPrefH) {
+                    const float* hprev = hst + (i > 0 ? i - 1 : 0) * N;
+                    const bool in = i > 0 && j < N;
+                    fm[r] = in && j > 0 ? hprev[j - 1] : 0.f;
+                    fz[r] = in ? hprev[j] : 0.f;
+                    fq[r] = in && j < N - 1 ? hprev[j + 1] : 0.f;
+                }
+            }
+        };
+        fetch2(L - 1, vg, vl, vx, t0, t1, t2, hm, hz, hq);
+        // gi = i % seg, counted down from L-1 (seg divides L)
+        for (int i = L - 1, gi = seg - 1; i >= 0; --i, gi = gi == 0 ? seg - 1 : gi - 1) {
+            float ng[P], nl[P], nx[P], n0[P], n1[P], n2[P], nm[P], nz[P], nq[P];
+            if (i > 0) fetch2(i - 1, ng, nl, nx, n0, n1, n2, nm, nz, nq);
+            const bool carry_out = gi != 0;                      // line i reads line i-1
+            const bool carry_in = (i + 1 < L) && gi != seg - 1;  // line i+1 read line i
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                const int j = lane + 32 * r;
+                if (j < N) {
+                    const int p = wk.o + i * wk.si + j * wk.sj;
+                    float av = vg[r];
+                    if (carry_in) av += qn[j + 2] + qn[ls + j + 1] + qn[2 * ls + j];
+                    dxacc[p] = slot == 0 ? vl[r] * av : dxacc[p] + vl[r] * av;
+                    store_elt(dlam, p, vx[r] * av);
+                    float dl0 = 0.f, dl1 = 0.f, dl2 = 0.f, q0 = 0.f, q1 = 0.f, q2 = 0.f;
+                    if (carry_out) {
+                        const float s0 = j > 0 ? sigmoidf(t0[r]) : 0.f;
+                        const float s1 = sigmoidf(t1[r]);
+                        const float s2 = j < N - 1 ? sigmoidf(t2[r]) : 0.f;
+                        const float rr = 1.f / (s0 + s1 + s2);
+                        const float w0 = s0 * rr, w1 = s1 * rr, w2 = s2 * rr;
+                        float hl, hm0, hr;
+                        if constexpr (kPrefH) {
+                            hl = hm[r];
+                            hm0 = hz[r];
+                            hr = hq[r];
+                        } else {
+                            const float* hprev = hst + (i - 1) * N;
+                            hl = j > 0 ? hprev[j - 1] : 0.f;
+                            hm0 = hprev[j];
+                            hr = j < N - 1 ? hprev[j + 1] : 0.f;
+                        }
+                        const float dw0 = j > 0 ? av * hl : 0.f;
+                        const float dw1 = av * hm0;
+                        const float dw2 = j < N - 1 ? av * hr : 0.f;
+                        const float r2 = rr * rr;
+                        dl0 = s0 * (1.f - s0) * r2 * (s1 * (dw0 - dw1) + s2 * (dw0 - dw2));
+                        dl1 = s1 * (1.f - s1) * r2 * (s0 * (dw1 - dw0) + s2 * (dw1 - dw2));
+                        dl2 = s2 * (1.f - s2) * r2 * (s0 * (dw2 - dw0) + s1 * (dw2 - dw1));
+                        q0 = w0 * av; q1 = w1 * av; q2 = w2 * av;
+                    }
+                    qc[j + 1] = q0;
+                    qc[ls + j + 1] = q1;
+                    qc[2 * ls + j + 1] = q2;
+                    if (a.g.shared) {
+                        if (carry_out) {
+                            unsigned long long* dw = a.dlog_ws + ((int64_t)slot * B + b) * 3 * HW;
+                            if (j > 0) fix_add(dw + p, dl0);
+                            fix_add(dw + HW + p, dl1);
+                            if (j < N - 1) fix_add(dw + 2 * HW + p, dl2);
+                        }
+                    } else {
+                        T* dlg = static_cast<T*>(a.dlogits) + ((slot * (int64_t)B + b) * Cw + cw) * 3 * HW;
+                        store_elt(dlg, p, dl0);
+                        store_elt(dlg, HW + p, dl1);
+                        store_elt(dlg, 2 * HW + p, dl2);
+                    }
+                }
+            }
+            __syncwarp();
+            float* t = qn; qn = qc; qc = t;
+#pragma unroll
+            for (int r = 0; r < P; ++r) {
+                vg[r] = ng[r]; vl[r] = nl[r]; vx[r] = nx[r];
+                t0[r] = n0[r]; t1[r] = n1[r]; t2[r] = n2[r];
+                if constexpr (kPrefH) {
+                    hm[r] = nm[r]; hz[r] = nz[r]; hq[r] = nq[r];
+                }
+            }
+        }
+        __syncwarp();
+    }
+    T* dx = static_cast<T*>(a.dx) + plane * HW;
+    for (int q = lane; q < HW; q += 32) store_elt(dx, q, dxacc[q]);
+}
+
 __global__ void zero_fix_kernel(unsigned long long* p, int64_t n) {
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
         p[i] = 0ull;
@@ -444,14 +633,36 @@ gspn_status generic_bwd(const Problem& p, const DeviceInfo& dev, const void* x, 
     }
     const int64_t grid = (p.planes + pl.wpc - 1) / pl.wpc;
     if (grid > 0x7fffffff) return GSPN_ERR_UNSUPPORTED;
-    const void* fn = p.d.dtype == GSPN_F32 ? (const void*)generic_bwd_kernel<float>
-                                           : (const void*)generic_bwd_kernel<__nv_bfloat16>;
-    cudaError_t e = ensure_smem_attr(fn, (int)pl.smem, p.d.dtype == GSPN_F32 ? 2 : 3);
+    // lines of up to 256 positions: the pipelined kernel with 1, 2, 4 or 8 positions per lane
+    const int nmax = p.g.H > p.g.W ? p.g.H : p.g.W;
+    const bool f32 = p.d.dtype == GSPN_F32;
+    const void* fn;
+    int slot;
+    if (nmax <= 32) {
+        fn = f32 ? (const void*)generic_bwd_pipelined_kernel<float, 1>
+                 : (const void*)generic_bwd_pipelined_kernel<__nv_bfloat16, 1>;
+        slot = f32 ? 4 : 5;
+    } else if (nmax <= 64) {
+        fn = f32 ? (const void*)generic_bwd_pipelined_kernel<float, 2>
+                 : (const void*)generic_bwd_pipelined_kernel<__nv_bfloat16, 2>;
+        slot = f32 ? 6 : 7;
+    } else if (nmax <= 128) {
+        fn = f32 ? (const void*)generic_bwd_pipelined_kernel<float, 4>
+                 : (const void*)generic_bwd_pipelined_kernel<__nv_bfloat16, 4>;
+        slot = f32 ? 30 : 31;
+    } else if (nmax <= 256) {
+        fn = f32 ? (const void*)generic_bwd_pipelined_kernel<float, 8>
+                 : (const void*)generic_bwd_pipelined_kernel<__nv_bfloat16, 8>;
+        slot = f32 ? 41 : 42;
+    } else {
+        fn = f32 ? (const void*)generic_bwd_kernel<float> : (const void*)generic_bwd_kernel<__nv_bfloat16>;
+        slot = f32 ? 2 : 3;
+    }
+    cudaError_t e = ensure_smem_attr(fn, (int)pl.smem, slot);
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
-    if (p.d.dtype == GSPN_F32)
-        generic_bwd_kernel<float><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
-    else
-        generic_bwd_kernel<__nv_bfloat16><<<(unsigned)grid, pl.wpc * 32, pl.smem, s>>>(a);
+    void* kargs[] = {&a};
+    e = cudaLaunchKernel(fn, dim3((unsigned)grid), dim3(pl.wpc * 32), kargs, pl.smem, s);
+    if (e != cudaSuccess) return GSPN_ERR_CUDA;
     e = cudaGetLastError();
     if (e != cudaSuccess) return GSPN_ERR_CUDA;
     if (p.g.shared) {
