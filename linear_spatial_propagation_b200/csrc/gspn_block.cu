@@ -450,8 +450,9 @@ __device__ __forceinline__ bool bar_and_128(bool p) {
 // ==================================================================================
 constexpr int OB_M = 128;       // channels per chunk (MMA M)
 constexpr int OB_N = 128;       // pixels per tile (MMA N)
+static_assert(OB_N % 64 == 0 && OB_N <= 128, "whole 64-pixel output boxes; the prologue has 128 threads");
 constexpr int OB_THREADS = 160;  // warp 0 MMA, warps 1..4 prologue / epilogue
-constexpr int OB_YBUF = OB_M * OB_N * 2;  // one staged output chunk: two 64-pixel SW128 boxes
+constexpr int OB_YBUF = OB_M * OB_N * 2;  // one staged output chunk: OB_N / 64 SW128 boxes of 64 pixels
 
 struct OutArgs {
     const float* h;          // [4][B][Cp][HW]
@@ -517,7 +518,7 @@ __global__ void __launch_bounds__(OB_THREADS, 2)
     }
     tma::fence_proxy_async();  // the generic writes of U are read by the tensor cores
     if (warp == 0) {
-        tmem::alloc(tma::smem_u32(tslot), 256);  // two 128-column accumulators
+        tmem::alloc(tma::smem_u32(tslot), 2 * OB_N);  // two accumulators of OB_N columns
         tmem::relinquish();
     }
     tmem::fence_before();
@@ -574,7 +575,7 @@ __global__ void __launch_bounds__(OB_THREADS, 2)
             // reaches this barrier once per tile, and all leave if one has failed
             ok = bar_and_128(ok && (lt == 0 || tma::mbar_wait(ndone, (lt - 1) & 1, a.limit)));
             if (!ok) break;
-            {
+            if (et < OB_N) {
                 const int pix = pix0 + et;
                 float m[KPAD];
 #pragma unroll
@@ -610,10 +611,11 @@ __global__ void __launch_bounds__(OB_THREADS, 2)
                     v.w = pack_bf2(m[k + 6], m[k + 7]);
                     *reinterpret_cast<uint4*>(nopp + core_off<KPAD>(et, k)) = v;
                 }
-                tma::fence_proxy_async();
-                __syncwarp();
-                if (t == 0) tma::mbar_arrive(nready);
             }
+            // every prologue warp arrives (its lanes wrote their rows of n^T, or none)
+            tma::fence_proxy_async();
+            __syncwarp();
+            if (t == 0) tma::mbar_arrive(nready);
             // epilogue of every 128-channel chunk of this tile: each warp converts
             // and stores its own 32 channel rows (its TMEM lane quarter), so the
             // warps of the CTA do not wait for one another within a tile.  A warp
@@ -661,8 +663,10 @@ __global__ void __launch_bounds__(OB_THREADS, 2)
                     const int c0 = cb * OB_M + 32 * q;  // first channel of this warp's rows
                     if (c0 < a.C) {
                         const uint32_t ysa = sbase + buf * OB_YBUF + q * 32 * 128;
-                        tma::store_3d(&tm_y, ysa, pix0, c0, b);
-                        if (pix0 + 64 < a.HW) tma::store_3d(&tm_y, ysa + OB_M * 128, pix0 + 64, c0, b);
+#pragma unroll
+                        for (int c64 = 0; c64 < OB_N / 64; ++c64)
+                            if (pix0 + 64 * c64 < a.HW)
+                                tma::store_3d(&tm_y, ysa + c64 * OB_M * 128, pix0 + 64 * c64, c0, b);
                     }
                     tma::bulk_commit();
                 }
@@ -675,7 +679,7 @@ __global__ void __launch_bounds__(OB_THREADS, 2)
     __syncthreads();
     if (warp == 0) {
         tmem::fence_after();
-        tmem::dealloc(taddr, 256);
+        tmem::dealloc(taddr, 2 * OB_N);
     }
 }
 
