@@ -290,13 +290,18 @@ def job_gbs(bytes_per_rank: int, n_ranks: int, ms: float) -> float:
     return bytes_per_rank * n_ranks / (ms * 1e-3) / 1e9
 
 
-def config_of(w, n, passes="both", graph=False):
+L2_BYTES = 126 * 2**20  # B200 L2
+
+
+def config_of(w, n, passes="both", graph=False, flushed=False):
     return {"workload": w.name, "B": w.B, "C": w.C, "H": w.H, "W": w.W,
             "directions": "+".join(n_ for b, n_ in ((1, "T2B"), (2, "B2T"), (4, "L2R"), (8, "R2L")) if w.dir_mask & b),
             "groups": w.groups, "shared_taps": w.shared, "io_dtype": w.dtype,
             "pass": {"both": "fwd+bwd", "fwd": "fwd", "bwd": "bwd"}[passes],
             "launch": "cuda_graph" if graph else "direct",
-            "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"}
+            "l2": "flushed before every timed pass (a pass's bytes fit in L2)" if flushed
+            else "inputs larger than L2 (no flush needed)",
+            "parallelism": f"replicas x{n}" if n > 1 else "1 GPU"}
 
 
 # ------------------------------------------------------------------------------
@@ -396,28 +401,40 @@ def run_gpu(args, w):
             if do_b:
                 bwd_t()
         barrier()
+    # A pass whose compulsory bytes fit in L2 (126 MB) could find its
+    # inputs there from the step before: then every timed pass starts after a
+    # write of a buffer twice the size of L2, outside the pass's own events,
+    # and the step time is the sum of the passes.
+    fb0, bb0 = pass_bytes(w)
+    flush = (do_f and fb0 < L2_BYTES) or (do_b and bb0 < L2_BYTES)
+    flush_buf = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev) if flush else None
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
     e_start.record(stream)
     for k in range(K):
+        if flush:
+            flush_buf.zero_()
         ev[k][0].record(stream)
         if do_f:
             fwd_t()
         ev[k][1].record(stream)
+        if flush:
+            flush_buf.zero_()
+        ev[k][2].record(stream)
         if do_b:
             bwd_t()
-        ev[k][2].record(stream)
+        ev[k][3].record(stream)
     e_end.record(stream)
     barrier()
     clk = clocks.stop()
     total_ms = rank_max(e_start.elapsed_time(e_end))
     fwd_ms = rank_max(sum(e[0].elapsed_time(e[1]) for e in ev) / K)
-    bwd_ms = rank_max(sum(e[1].elapsed_time(e[2]) for e in ev) / K)
-    ms = total_ms / K
+    bwd_ms = rank_max(sum(e[2].elapsed_time(e[3]) for e in ev) / K)
+    ms = fwd_ms + bwd_ms if flush else total_ms / K
 
     # end to end: pinned host inputs -> device -> fwd + bwd -> results back to pinned
     # host, every step.  The copies run on their own streams so that step k+1's
@@ -503,7 +520,7 @@ def run_gpu(args, w):
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": n_gpu, "steps": K,
             "warmup": max(3, args.warmup), "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded numpy PCG64, per-rank seed)",
-            "config": config_of(w, n_gpu, args.passes, args.graph),
+            "config": config_of(w, n_gpu, args.passes, args.graph, flush),
             "pct_of_peak": 100.0 * value / n_gpu / peak,
             "gpix_ch_per_s": pixch * n_gpu / (ms * 1e-3) / 1e9,
             "fwd": {"ms": fwd_ms, "GB/s": fwd_gbs, "pct_of_peak": 100.0 * fwd_gbs / peak,
