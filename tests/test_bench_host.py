@@ -128,3 +128,35 @@ def test_roofline_traffic_only_for_the_sources_it_was_captured_on(monkeypatch):
         assert bench.ncu_traffic(kernel_pass, w) is None
     # a workload without a capture has no traffic either
     assert bench.ncu_traffic("bwd", synth.WORKLOADS["t2b_f32_b1c4_16x16"]) is None
+
+
+def test_l2_flush_only_where_a_pass_fits_in_l2():
+    """The timing rule: inputs larger than L2, or L2 flushed between timed
+    passes.  Passes of at least the L2's 126 MB are timed back to back; a
+    smaller pass (the 16x16 problem, the generic 130x70 forward) gets a flush."""
+    import bench
+    import synth
+    fits = {}
+    for name, w in list(synth.WORKLOADS.items()) + list(synth.EXTRA_WORKLOADS.items()):
+        fb, bb = bench.pass_bytes(w)
+        fits[name] = fb < bench.L2_BYTES or bb < bench.L2_BYTES
+    assert fits == {
+        "t2b_f32_b1c4_16x16": True,
+        "4dir_f32_b8c96_56x56": False,
+        "4dir_local4_bf16_b32c192_28x28": False,
+        "compact_4dir_bf16_b32c1152_64x64": False,
+        "compact_4dir_bf16_b2c1152_128x128_fwdbwd": False,
+        "generic_4dir_f32_b2c64_130x70": True,
+    }
+    assert bench.L2_BYTES == 126 * 2**20
+
+
+def test_config_names_the_launch_form_and_the_l2_rule():
+    import bench
+    import synth
+    w = synth.WORKLOADS["compact_4dir_bf16_b32c1152_64x64"]
+    c = bench.config_of(w, 1)
+    assert c["workload"] == w.name and c["launch"] == "direct" and c["l2"].startswith("inputs larger than L2")
+    c = bench.config_of(w, 1, graph=True, flushed=True)
+    assert c["launch"] == "cuda_graph" and c["l2"].startswith("flushed")
+    assert "model" not in c
