@@ -1,5 +1,6 @@
 """GPU parity of the large-plane forward (lines of 65..512 positions, one CTA
-streaming a plane line by line) against the oracle.
+streaming a plane line by line) against the oracle, and of the backward of
+such planes (the generic kernels, pipelined up to 256 positions per line).
 
 Shapes: 256x256 and 512x512 compact bf16 (the planes beyond the on-chip
 kernels), rectangular planes whose two scan directions use different warp
@@ -55,3 +56,29 @@ def test_large_plane_forward_is_deterministic():
     o2 = gu.run_fwd(w, dinp)
     t.cuda.synchronize()
     assert bool(t.equal(o1, o2))
+
+
+BWD_CASES = [
+    # B, C, H, W, dir_mask, groups, shared, dtype, backward variant
+    (1, 2, 256, 256, 15, 1, True, "bf16", "generic_bwd"),    # lines of 256: the pipelined kernel, 8 per lane
+    (1, 2, 200, 136, 15, 2, False, "f32", "generic_bwd"),    # per-channel, local groups, two line lengths
+    (1, 1, 512, 512, 15, 1, True, "bf16", "generic_bwd"),    # lines of 512: the kernel without prefetch
+]
+
+
+@pytest.mark.parametrize("case", BWD_CASES, ids=lambda c: "x".join(map(str, c[:8])))
+def test_large_plane_backward_matches_oracle(case):
+    """Backward of planes above 64x64 (other than the compact 64x64 / 128x128
+    ones): dx, dlambda and dlogits against the oracle's adjoint."""
+    import linear_spatial_propagation_b200 as lsp
+    B, C, H, W, mask, g, shared, dtype, variant = case
+    w = synth.Workload(f"large_bwd_{'x'.join(map(str, case[:8]))}", B, C, H, W, mask, g, shared, dtype, 1.0,
+                       4200 + H + W + C, backward=True)
+    assert lsp.gspn_variant_name(lsp.make_desc(B, C, H, W, mask, g, shared, dtype), 1) == variant
+    inp = synth.make_inputs(w, with_dout=True)
+    dinp = gu.dev_inputs(w, inp)
+    dx, dlg, dlam = (gu.from_dev(t) for t in gu.run_bwd(w, dinp))
+    rdx, rdlg, rdlam = oracle.bwd_workload(w, inp, nthreads=8)
+    gu.assert_close(dx, rdx, dtype, f"{w.name} dx")
+    gu.assert_close(dlam, rdlam, dtype, f"{w.name} dlam")
+    gu.assert_close(dlg, rdlg, dtype, f"{w.name} dlogits")
