@@ -683,11 +683,11 @@ def run_block(args, w):
             "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded numpy PCG64, per-rank seed)",
             "config": block_config(w, world), "bytes_per_step": nb,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                         "peak_source": f"{peak_src} copy bandwidth", "kernel": "gspn_block_fwd (3 launches)",
+                         "peak_source": f"{peak_src} copy bandwidth", "kernel": "gspn_block_fwd (4 launches)",
                          "traffic": None},
             "e2e": ({"value": job_gbs(nb, world, e2e_ms), "unit": "GB/s", "h2d_bytes_per_step": h2d,
                      "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms} if e2e_ms else None),
-            "gpu_launches": 3 * K, "clocks": clk, "cpu_baseline": cpu,
+            "gpu_launches": 4 * K, "clocks": clk, "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:

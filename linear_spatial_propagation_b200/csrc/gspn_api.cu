@@ -203,7 +203,7 @@ int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     case Path::kC64:
     case Path::kC128: return backward ? 3 : 2;
     case Path::kSmall: return backward ? small_bwd_launches(p) : 1;
-    case Path::kLarge: return 1;
+    case Path::kLarge: return p.g.shared ? 2 : 1;  // channel-shared taps: the taps pre-kernel first
     default: return backward ? generic_bwd_launches(p) : 1;
     }
 }

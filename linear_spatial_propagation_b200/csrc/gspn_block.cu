@@ -15,7 +15,7 @@
 //   n[b,k]   = gamma[k] m[b,k] / sqrt(mean_k m[b,k]^2 + eps) (RMS norm over k)
 //   y[b,c]   = sum_k U[c,k] n[b,k]                          (back-projection)
 //
-// Three launches:
+// Four launches:
 // * block_proj_kernel: the projection as a tcgen05 GEMM per 128-pixel tile,
 //   D[pixel, k] = sum_c X^T[pixel, c] V^T[c, k], K = C in blocks of 64 channels.
 //   X tiles arrive by TMA with the 128-byte swizzle, pixels contiguous (the

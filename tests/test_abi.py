@@ -131,8 +131,8 @@ def test_python_helpers_raise_on_error():
     ((3, 9, 64, 64, 15, 1, True, "bf16"), ("small_plane_fwd", 1), ("small_plane_bwd", 3)),  # C % 8 != 0
     ((1, 1, 16, 16, 1, 1, False, "f32"), ("small_plane_fwd", 1), ("small_plane_bwd", 1)),
     # longer lines with H, W multiples of 8 (up to 512): the large-plane forward
-    ((2, 6, 128, 128, 15, 1, True, "bf16"), ("large_plane_fwd", 1), ("generic_bwd", 3)),  # C % 4 != 0
-    ((1, 4, 512, 256, 15, 1, True, "bf16"), ("large_plane_fwd", 1), ("generic_bwd", 3)),
+    ((2, 6, 128, 128, 15, 1, True, "bf16"), ("large_plane_fwd", 2), ("generic_bwd", 3)),  # C % 4 != 0; taps kernel
+    ((1, 4, 512, 256, 15, 1, True, "bf16"), ("large_plane_fwd", 2), ("generic_bwd", 3)),
     ((1, 2, 72, 320, 5, 1, False, "f32"), ("large_plane_fwd", 1), ("generic_bwd", 1)),
     # anything else: the generic kernels
     ((1, 2, 65, 64, 15, 1, False, "f32"), ("generic_fwd", 1), ("generic_bwd", 1)),
