@@ -165,3 +165,42 @@ def test_compact_shapes_take_the_tma_kernels_when_the_encoder_is_there(args, fas
         else:
             fallback = "small_plane" if small else ("generic" if bwd else "large_plane")
             assert name == fallback + suffix
+
+
+# ---- the compressed propagation block ---------------------------------------------
+
+def _block_fwd(desc, ptr=A):
+    return lsp.gspn_block_fwd(desc, ptr, ptr, ptr, ptr, ptr, ptr, ptr, ptr, 0, 0, 0)
+
+
+@pytest.mark.parametrize("args, status", [
+    ((0, 64, 16, 16, 2), 1),        # B < 1
+    ((1, 0, 16, 16, 2), 1),         # C < 1
+    ((1, 64, 16, 16, 0), 1),        # C_proxy < 1
+    ((1, 64, 18, 16, 2, 4), 1),     # groups not dividing H
+    ((1, 64, 16, 16, 33), 2),       # C_proxy above 32
+    ((1, 64, 136, 16, 2), 2),       # lines above 128
+    ((1, 60, 16, 16, 2), 2),        # C not a multiple of 8
+    ((1, 64, 12, 16, 2), 2),        # H not a multiple of 8
+    ((1, 3072 + 8, 16, 16, 2), 2),  # U beyond shared memory at C_proxy <= 16
+    ((1, 1536 + 8, 16, 16, 32), 2),  # and at C_proxy 32
+])
+def test_block_rejects_descriptors_on_the_host(args, status):
+    """Dimension and limit checks come before any device query, so the same
+    status holds with or without a GPU; a rejected descriptor also has no
+    workspace size."""
+    d = lsp.make_block_desc(*args)
+    assert _block_fwd(d) == status
+    assert lsp.gspn_block_workspace_size(d) == 0
+
+
+def test_block_rejects_a_bad_eps():
+    for eps in (-1.0, 2.0, float("nan")):
+        assert _block_fwd(lsp.make_block_desc(1, 64, 16, 16, 2, eps=eps)) == 1
+
+
+def test_block_null_descriptor_and_status():
+    lib = lsp.load()
+    assert lib.gspn_block_fwd(None, *([None] * 8), None, 0, None) == 1
+    assert lib.gspn_block_workspace_size(None) == 0
+    assert lib.gspn_block_device_status(None, None, None) == 1
