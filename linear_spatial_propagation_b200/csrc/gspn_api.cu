@@ -76,11 +76,12 @@ gspn_status check_ws(void* ws, size_t have, size_t need) {
 // The kernel family a descriptor runs on: the TMA-fed compact kernels for their
 // shapes, the one-CTA-per-plane kernels for planes of at most 64x64, the generic
 // kernels for everything else.
-enum class Path { kC64, kC128, kSmall, kLarge, kGeneric };
+enum class Path { kC64, kC128, kSmall, kLargeCompact, kLarge, kGeneric };
 Path pick(const Problem& p, int backward) {
     if (backward ? c64_bwd_eligible(p) : c64_eligible(p)) return Path::kC64;
     if (backward ? c128_bwd_eligible(p) : c128_eligible(p)) return Path::kC128;
     if (small_eligible(p, backward)) return Path::kSmall;
+    if (!backward && lc_eligible(p)) return Path::kLargeCompact;
     if (!backward && large_eligible(p)) return Path::kLarge;
     return Path::kGeneric;
 }
@@ -91,7 +92,9 @@ std::atomic<int> g_sync_check{0};
 
 // The error word a TMA-fed kernel family sets when a bounded wait expires sits
 // at offset 0 of its workspace; the other families have no device-side waits.
-bool has_status_word(Path path) { return path == Path::kC64 || path == Path::kC128; }
+bool has_status_word(Path path) {
+    return path == Path::kC64 || path == Path::kC128 || path == Path::kLargeCompact;
+}
 
 // Synchronises `s` and maps the call's outcome to a status: a CUDA error, an
 // expired wait recorded in the error word at `word` (null: none), or OK.
@@ -191,6 +194,7 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     case Path::kC64: return backward ? c64_bwd_workspace(p, dev) : c64_fwd_workspace(p);
     case Path::kC128: return backward ? c128_bwd_workspace(p, dev) : c128_fwd_workspace(p, dev);
     case Path::kSmall: return backward ? small_bwd_workspace(p) : 0;
+    case Path::kLargeCompact: return lc_fwd_workspace(p);
     case Path::kLarge: return large_fwd_workspace(p);
     default: return backward ? generic_bwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
     }
@@ -203,6 +207,7 @@ int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     case Path::kC64:
     case Path::kC128: return backward ? 3 : 2;
     case Path::kSmall: return backward ? small_bwd_launches(p) : 1;
+    case Path::kLargeCompact: return 2;  // the taps table, then the scan
     case Path::kLarge: return p.g.shared ? 2 : 1;  // channel-shared taps: the taps pre-kernel first
     default: return backward ? generic_bwd_launches(p) : 1;
     }
@@ -215,6 +220,7 @@ const char* gspn_variant_name(const gspn_desc* desc, int backward) {
     case Path::kC64: return backward ? "compact64_tma_bwd" : "compact64_tma_fwd";
     case Path::kC128: return backward ? "compact128_tma_bwd" : "compact128_tma_fwd";
     case Path::kSmall: return backward ? "small_plane_bwd" : "small_plane_fwd";
+    case Path::kLargeCompact: return "large_compact_fwd";
     case Path::kLarge: return "large_plane_fwd";
     default: return backward ? "generic_bwd" : "generic_fwd";
     }
@@ -234,6 +240,7 @@ gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, c
                   path == Path::kC64    ? c64_fwd_workspace(p)
                   : path == Path::kC128 ? c128_fwd_workspace(p, dev)
                   : path == Path::kSmall ? 0
+                  : path == Path::kLargeCompact ? lc_fwd_workspace(p)
                   : path == Path::kLarge ? large_fwd_workspace(p)
                                          : generic_fwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
@@ -241,6 +248,7 @@ gspn_status gspn_fwd(const gspn_desc* desc, const void* x, const void* logits, c
     st = path == Path::kC64    ? c64_fwd(p, dev, x, logits, lambda, out, workspace, cs)
          : path == Path::kC128 ? c128_fwd(p, dev, x, logits, lambda, out, workspace, cs)
          : path == Path::kSmall ? small_fwd(p, dev, x, logits, lambda, out, cs)
+         : path == Path::kLargeCompact ? lc_fwd(p, dev, x, logits, lambda, out, workspace, cs)
          : path == Path::kLarge ? large_fwd(p, x, logits, lambda, out, workspace, cs)
                                 : generic_fwd(p, dev, x, logits, lambda, out, workspace, cs);
     if (st != GSPN_OK || !g_sync_check.load(std::memory_order_relaxed)) return st;

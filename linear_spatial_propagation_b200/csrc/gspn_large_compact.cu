@@ -1,0 +1,596 @@
+// gspn_large_compact.cu -- GSPN forward of channel-shared (compact) bf16 planes
+// whose lines are 129..256 positions long: 256x256 latents and the like, the
+// planes "Parallel Sequence Modeling via Generalized Spatial Propagation
+// Network" scales to (one-line summary: 16K generation) with the compact
+// weights of "GSPN-2: Efficient Parallel Sequence Modeling" (Justification for
+// Channel-Agnostic Propagation).
+//
+// One warp owns one plane and walks its lines; lane t holds positions 8t..8t+7
+// of a line in registers, so the three-tap mix needs two shuffles per line and
+// no exchange between warps.  A CTA runs 8 warps = 8 consecutive channels of
+// one batch image; they share the image's tap weights, which stream through a
+// shared ring (one bulk copy per chunk of lines, issued by the last warp to
+// finish with a stage) from a table a pre-kernel forms once per image (Key
+// design 1: sigmoids of the tap logits, normalised over the taps that exist).
+// Two warps per scheduler leave each warp up to 255 registers.
+//
+// The four directions of a plane run one after another and merge by summing
+// through fp32 planes in the workspace (the planes do not fit on chip):
+// * column scans (left->right, right->left) first; their running sum is kept
+//   column-major (acct[plane][col][row]), so the sum of a column line is 8
+//   contiguous floats per lane;
+// * the first row scan reads that sum transposed by a 4-D tensor copy into
+//   shared memory, the others row-major (acc[plane][row][col]);
+// * the last direction writes the bf16 output.
+// x and lambda arrive by tensor copies into a 3-stage ring per warp: rows as
+// 256 x 4 boxes, columns as 8-column boxes through a (column, row / 8,
+// row % 8, plane) view, so that lane t's 16-byte reads of rows 8t..8t+7 are
+// free of bank conflicts.  The warp issues its own copies, three chunks ahead.
+// Every wait is bounded; an expired one sets the error word (workspace offset
+// 0), drains the copies in flight and leaves.
+#include <cstring>
+#include <type_traits>
+
+#include "gspn_internal.h"
+#include "gspn_lane.cuh"
+#include "gspn_tma.cuh"
+
+namespace gspn {
+
+namespace {
+
+using lane::FULL;
+
+constexpr int NCW = 8;                    // consumer warps (planes in flight per CTA)
+constexpr int THREADS = NCW * 32;
+constexpr int P = 8;                      // positions per lane
+constexpr int LMAX = 256;                 // longest line
+constexpr int NST = 3;                    // data stages per consumer warp
+constexpr int STAGE = 8192;               // rows: x 2 KB, lambda 2 KB, column sums 4 KB; columns: x, lambda 4 KB
+constexpr int NTS = 4;                    // tap stages (4 lines each)
+constexpr int TLINE = 2048;               // taps of one line: 256 positions x (w0, w2)
+constexpr int TSTAGE = 4 * TLINE;
+constexpr int OFF_T = NCW * NST * STAGE;
+constexpr int OFF_BAR = OFF_T + NTS * TSTAGE;
+constexpr int NBAR = NCW * NST + NTS + 1;
+constexpr int OFF_CNT = OFF_BAR + NBAR * 8;          // per tap stage: warps done with it
+constexpr int SMEM_BYTES = OFF_CNT + NTS * 4 + 128;  // + alignment slack
+
+// k-th direction in processing order (columns first): dir | slot << 2 | in << 4 | out << 6
+// in:  0 nothing (first direction), 1 column sums row by row (acct, direct loads),
+//      2 column sums transposed (acct, tensor copy), 3 row sums (acc, direct loads)
+// out: 0 column sums (acct), 1 row sums (acc), 2 the bf16 output
+struct LcArgs {
+    const float4* taps;   // [slot][b][LMAX lines][4][32]: (-w0, -w0', w2, w2') of positions 8t+2q, 8t+2q+1
+    float* acc;           // [plane][H][W]
+    float* acct;          // [plane][W][H]
+    __nv_bfloat16* out;
+    int* err;
+    int B, C, H, W, D;
+    int kinfo[4];
+    int groups;           // B * C / 8
+    int segr, segc;       // local group lengths of row and column scans
+    uint64_t limit;       // bound of every wait on data, a stage or another warp (ns)
+    int stall;            // test hook: consumer warp 0 of CTA 0 first waits on a barrier nothing completes
+};
+
+__device__ __forceinline__ int kinfo_of(const LcArgs& a, int k) {
+    return k == 0 ? a.kinfo[0] : k == 1 ? a.kinfo[1] : k == 2 ? a.kinfo[2] : a.kinfo[3];
+}
+
+// The taps table: one thread per (slot, image, line, quad q, lane t) writes the
+// normalised (w0, w2) of positions 8t+2q and 8t+2q+1 of that line in scan
+// order, w0 negated; positions beyond the line are zero.  Also clears the
+// error word.
+__global__ void __launch_bounds__(256) lc_taps_kernel(const __nv_bfloat16* __restrict__ logits,
+                                                      float4* __restrict__ taps, int* err, const Launch g) {
+    const int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (idx == 0) *err = 0;
+    if (idx >= (int64_t)g.D * g.B * LMAX * 128) return;
+    const int t = (int)(idx & 31), q = (int)((idx >> 5) & 3);
+    const int i = (int)((idx >> 7) % LMAX);
+    const int sb = (int)(idx / (128 * LMAX));  // slot * B + b
+    const int slot = sb / g.B;
+    const int d = dir_of(g, slot);
+    const int L = scan_len(d, g.H, g.W), N = line_len(d, g.H, g.W);
+    if (i >= L) return;
+    const Walk wk = walk_of(d, g.H, g.W);
+    const int HW = g.H * g.W;
+    const __nv_bfloat16* const lg = logits + (size_t)sb * 3 * HW;
+    float w[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+        const int j = 8 * t + 2 * q + u;
+        if (j >= N) continue;
+        const int pix = wk.o + i * wk.si + j * wk.sj;
+        const float s0 = j > 0 ? sigmoidf(load_elt(lg, pix)) : 0.f;
+        const float s1 = sigmoidf(load_elt(lg, HW + pix));
+        const float s2 = j < N - 1 ? sigmoidf(load_elt(lg, 2 * HW + pix)) : 0.f;
+        const float r = 1.f / (s0 + s1 + s2);
+        w[u] = -s0 * r;
+        w[2 + u] = s2 * r;
+    }
+    taps[idx] = make_float4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ float comp(const float4& v, int i) { return i == 0 ? v.x : i == 1 ? v.y : i == 2 ? v.z : v.w; }
+
+__global__ void __launch_bounds__(THREADS, 1)
+    lc_fwd_kernel(const __grid_constant__ CUtensorMap tm_xr, const __grid_constant__ CUtensorMap tm_lr,
+                  const __grid_constant__ CUtensorMap tm_xc, const __grid_constant__ CUtensorMap tm_lc,
+                  const __grid_constant__ CUtensorMap tm_at, const LcArgs a) {
+    extern __shared__ __align__(128) unsigned char smem_raw[];
+    unsigned char* const smem = smem_raw + ((128u - (tma::smem_u32(smem_raw) & 127u)) & 127u);
+    const uint32_t sbase = tma::smem_u32(smem);
+    const int warp = threadIdx.x >> 5, t = threadIdx.x & 31;
+    const uint32_t full0 = sbase + OFF_BAR;            // full[w][s]: a warp's data stage has landed
+    const uint32_t tfull0 = full0 + 8 * NCW * NST;      // tfull[s]: a tap stage has landed
+    const uint32_t never = tfull0 + 8 * NTS;            // stall-test barrier: nothing completes it
+    int* const tcount = reinterpret_cast<int*>(smem + OFF_CNT);
+    // The taps stream in quads of 4 lines; every warp walks the same sequence
+    // (group, direction index, quad).
+    struct Cursor {
+        int g, k, qd;
+    };
+    auto advance = [&](Cursor& c) {
+        if (++c.qd == ((kinfo_of(a, c.k) & 3) < 2 ? a.H : a.W) / 4) {
+            c.qd = 0;
+            if (++c.k == a.D) {
+                c.k = 0;
+                c.g += gridDim.x;
+            }
+        }
+    };
+    // one bulk copy of the taps of quad c into tap stage ts
+    auto issue_taps = [&](const Cursor& c, int ts) {
+        const int info = kinfo_of(a, c.k);
+        const int slot = (info >> 2) & 3;
+        const int b = (8 * c.g) / a.C;
+        const unsigned char* src = reinterpret_cast<const unsigned char*>(a.taps) +
+                                   ((size_t)(slot * a.B + b) * LMAX + (size_t)c.qd * 4) * TLINE;
+        tma::mbar_expect_tx(tfull0 + 8 * ts, TSTAGE);
+        tma::load_1d(sbase + OFF_T + ts * TSTAGE, src, TSTAGE, tfull0 + 8 * ts);
+    };
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < NCW * NST; ++i) tma::mbar_init(full0 + 8 * i, 1);
+        for (int s = 0; s < NTS; ++s) {
+            tma::mbar_init(tfull0 + 8 * s, 1);
+            tcount[s] = 0;
+        }
+        tma::mbar_init(never, 1);
+        tma::fence_barrier_init();
+    }
+    if (threadIdx.x == 32) {
+        tma::prefetch_map(&tm_xr);
+        tma::prefetch_map(&tm_lr);
+        if ((a.kinfo[0] & 3) >= 2) {  // the column maps exist only with a column direction (processed first)
+            tma::prefetch_map(&tm_xc);
+            tma::prefetch_map(&tm_lc);
+            tma::prefetch_map(&tm_at);
+        }
+    }
+    __syncthreads();
+    // lane 0: the taps quad NTS ahead of this warp (a stage's refill), and per
+    // tap stage the last quad this warp issued into it (-1: none)
+    Cursor tnext{(int)blockIdx.x, 0, 0};
+    int tlast[NTS];
+#pragma unroll
+    for (int s = 0; s < NTS; ++s) tlast[s] = -1;
+    if (threadIdx.x == 0) {
+#pragma unroll
+        for (int s = 0; s < NTS; ++s) {
+            if (tnext.g < a.groups) {
+                issue_taps(tnext, s);
+                tlast[s] = s;
+                advance(tnext);
+            }
+        }
+    } else {
+        for (int s = 0; s < NTS && tnext.g < a.groups; ++s) advance(tnext);
+    }
+
+    // ---------------- consumer warps: one plane each ----------------
+    unsigned char* const ring = smem + warp * NST * STAGE;
+    const uint32_t ringa = sbase + warp * NST * STAGE;
+    const uint32_t fullw = full0 + 8 * warp * NST;
+    int n = 0;  // data chunks consumed
+    int m = 0;  // taps quads consumed
+    // lane 0: the next data chunk to issue
+    int issued = 0, ig = blockIdx.x, ik = 0, ich = 0;
+    auto nch_of = [&](int k) { return (kinfo_of(a, k) & 3) < 2 ? a.H / 4 : a.W / 8; };
+    auto issue_one = [&]() {
+        const int info = kinfo_of(a, ik);
+        const int d = info & 3, slot = (info >> 2) & 3, in = (info >> 4) & 3;
+        const int s = issued % NST;
+        const uint32_t bar = fullw + 8 * s, dst = ringa + s * STAGE;
+        const int pl = 8 * ig + warp;
+        const int b = (8 * ig) / a.C, c = pl - b * a.C;
+        const int lpl = (slot * a.B + b) * a.C + c;
+        if (d < 2) {
+            const int y0 = d == B2T ? a.H - 4 - 4 * ich : 4 * ich;
+            tma::mbar_expect_tx(bar, in == 2 ? 8192u : 4096u);
+            tma::load_3d(dst, &tm_xr, 0, y0, pl, bar);
+            tma::load_3d(dst + 2048, &tm_lr, 0, y0, lpl, bar);
+            if (in == 2) tma::load_4d(dst + 4096, &tm_at, y0, 0, 0, pl, bar);
+        } else {
+            const int x0 = d == R2L ? a.W - 8 - 8 * ich : 8 * ich;
+            tma::mbar_expect_tx(bar, 8192u);
+            tma::load_4d(dst, &tm_xc, x0, 0, 0, pl, bar);
+            tma::load_4d(dst + 4096, &tm_lc, x0, 0, 0, lpl, bar);
+        }
+        ++issued;
+        if (++ich == nch_of(ik)) {
+            ich = 0;
+            if (++ik == a.D) {
+                ik = 0;
+                ig += gridDim.x;
+            }
+        }
+    };
+    // Keep NST chunks in flight.  A chunk of a direction that reads the column
+    // sums by tensor copy waits until this warp has finished writing them.
+    auto issue_more = [&](int g, int k) {
+        if (t == 0) {
+            while (issued < n + NST && ig < a.groups) {
+                if (((kinfo_of(a, ik) >> 4) & 3) == 2 && (ig != g || ik != k)) break;
+                issue_one();
+            }
+        }
+        __syncwarp();
+    };
+    auto fail = [&]() {
+        if (t == 0) {
+            atomicExch(a.err, 1);
+            // the copies this warp issued land before the CTA can leave
+            for (int m = n; m < issued; ++m) tma::mbar_wait(fullw + 8 * (m % NST), (m / NST) & 1, 100000000ull);
+#pragma unroll
+            for (int s = 0; s < NTS; ++s)
+                if (tlast[s] >= 0) tma::mbar_wait(tfull0 + 8 * s, (tlast[s] / NTS) & 1, 100000000ull);
+        }
+        __syncwarp();
+    };
+
+    // One direction of plane 8g + warp: lines i = 0 .. L-1 in scan order.
+    auto run_dir = [&](auto rows_c, auto in_c, auto out_c, int g, int k) -> bool {
+        constexpr bool ROWS = decltype(rows_c)::value;
+        constexpr int IN = decltype(in_c)::value, OUT = decltype(out_c)::value;
+        const int d = kinfo_of(a, k) & 3;
+        const bool rev = d == B2T || d == R2L;
+        const int L = ROWS ? a.H : a.W, N = ROWS ? a.W : a.H;
+        const int seg = ROWS ? a.segr : a.segc;
+        const size_t pl = (size_t)(8 * g + warp);
+        const bool act = 8 * t < N;  // this lane's positions lie on the line
+        float* const accp = a.acc + pl * a.H * a.W;
+        float* const actp = a.acct + pl * a.W * a.H;
+        __nv_bfloat16* const outp = a.out + pl * a.H * a.W;
+        // element offset of position 8t of line i: row-major for row lines, column-major for column lines
+        auto line_off = [&](int i) -> size_t { return (size_t)(rev ? L - 1 - i : i) * N + 8 * t; };
+        const float* const sump = IN == 1 ? actp : accp;
+        float4 ar[4][2];  // IN 1, 3: the sums of lines i .. i+3, by i % 4
+        if constexpr (IN == 1 || IN == 3) {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                ar[r][0] = ar[r][1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (act && r < L) {
+                    const float4* src = reinterpret_cast<const float4*>(sump + line_off(r));
+                    ar[r][0] = src[0];
+                    ar[r][1] = src[1];
+                }
+            }
+        }
+        float h[P];
+#pragma unroll
+        for (int p = 0; p < P; ++p) h[p] = 0.f;
+        int gpos = 0;
+        int nt = 0;                      // the data chunk being read
+        const unsigned char* st = ring;  // its stage
+        uint4 X[ROWS ? 4 : 1], Lm[ROWS ? 4 : 1];  // rows: line e, lane positions 8t..8t+7
+        uint2 Xh[ROWS ? 1 : P], Lh[ROWS ? 1 : P];  // columns: row 8t+p, the quad's 4 lines
+        float4 A[IN == 2 ? P : 1];
+        // the stage's reads are done: hand it back to this warp's next copies
+        auto release = [&]() {
+            tma::fence_proxy_async();  // these reads come before the stage's refill
+            __syncwarp();
+            ++n;
+            issue_more(g, k);
+        };
+        // columns: the quad's lines 4hh .. 4hh+3 of the chunk are columns 4hh.. of
+        // the box (left->right), or the 8-byte piece at the other end, reversed
+        // (right->left)
+        auto read_half = [&](int hh) {
+#pragma unroll
+            for (int p = 0; p < P; ++p) {
+                const int o = (p * 32 + t) * 16 + 8 * (rev ? 1 - hh : hh);
+                const uint2 xv = *reinterpret_cast<const uint2*>(st + o);
+                const uint2 lv = *reinterpret_cast<const uint2*>(st + 4096 + o);
+                Xh[p] = rev ? make_uint2(__byte_perm(xv.y, 0, 0x1032), __byte_perm(xv.x, 0, 0x1032)) : xv;
+                Lh[p] = rev ? make_uint2(__byte_perm(lv.y, 0, 0x1032), __byte_perm(lv.x, 0, 0x1032)) : lv;
+            }
+        };
+        const int nq = L / 4;
+        for (int qd = 0; qd < nq; ++qd) {
+            // data: one row chunk per quad, one column chunk per two quads
+            if (ROWS || (qd & 1) == 0) {
+                nt = n;
+                const int s = nt % NST;
+                if (!__all_sync(FULL, tma::mbar_wait(fullw + 8 * s, (nt / NST) & 1, a.limit))) return false;
+                st = ring + s * STAGE;
+                if constexpr (ROWS) {
+                    // line e is stage row e (top->bottom) or 3-e (bottom->top)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int r = rev ? 3 - e : e;
+                        X[e] = lane::lds128(st + r * 512 + t * 16);
+                        Lm[e] = lane::lds128(st + 2048 + r * 512 + t * 16);
+                    }
+                    if constexpr (IN == 2) {
+                        // column 8t+p of the chunk's 4 rows
+#pragma unroll
+                        for (int p = 0; p < P; ++p) {
+                            const float4 v = lane::lds128f(st + 4096 + (p * 32 + t) * 16);
+                            A[p] = rev ? make_float4(v.w, v.z, v.y, v.x) : v;
+                        }
+                    }
+                    release();
+                } else {
+                    read_half(0);
+                }
+            } else {
+                read_half(1);
+                release();
+            }
+            const int mt = m++;
+            const int ts = mt % NTS;
+            if (!__all_sync(FULL, tma::mbar_wait(tfull0 + 8 * ts, (mt / NTS) & 1, a.limit))) return false;
+            const unsigned char* tp = smem + OFF_T + ts * TSTAGE + t * 16;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int i = 4 * qd + e;
+                if (gpos == 0) {
+#pragma unroll
+                    for (int p = 0; p < P; ++p) h[p] = 0.f;  // a scan or local group starts: h_{-1} = 0
+                }
+                gpos = gpos + 1 == seg ? 0 : gpos + 1;
+                float4 T[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) T[q] = lane::lds128f(tp + e * TLINE + q * 512);
+                float base[P];
+#pragma unroll
+                for (int p = 0; p < P; ++p) {
+                    if constexpr (ROWS)
+                        base[p] = lane::fma_bf(p & 1, lane::word_of(Lm[e], p >> 1), lane::word_of(X[e], p >> 1), h[p]);
+                    else
+                        base[p] = lane::fma_bf(e & 1, (e & 2) ? Lh[p].y : Lh[p].x, (e & 2) ? Xh[p].y : Xh[p].x, h[p]);
+                }
+                // neighbours of the previous line; the rotation brings lane 31's last
+                // position to lane 0 and lane 0's first to lane 31, where w0 = 0 and w2 = 0
+                const float hl = __shfl_sync(FULL, h[P - 1], (t + 31) & 31);
+                const float hr = __shfl_sync(FULL, h[0], (t + 1) & 31);
+                float dd[P + 1];  // dd[p] = h[p] - h[p-1]
+                dd[0] = h[0] - hl;
+#pragma unroll
+                for (int p = 1; p < P; ++p) dd[p] = h[p] - h[p - 1];
+                dd[P] = hr - h[P - 1];
+                // h' = lambda x + h + w0 (h[j-1] - h) + w2 (h[j+1] - h)
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    h[2 * q] = fmaf(T[q].x, dd[2 * q], fmaf(T[q].z, dd[2 * q + 1], base[2 * q]));
+                    h[2 * q + 1] = fmaf(T[q].y, dd[2 * q + 1], fmaf(T[q].w, dd[2 * q + 2], base[2 * q + 1]));
+                }
+                float v[P];
+#pragma unroll
+                for (int p = 0; p < P; ++p) {
+                    float sprev = 0.f;
+                    if constexpr (IN == 1 || IN == 3) sprev = comp(ar[e][p >> 2], p & 3);
+                    if constexpr (IN == 2) sprev = comp(A[p], e);
+                    v[p] = h[p] + sprev;
+                }
+                if (act) {
+                    const size_t o = line_off(i);
+                    if constexpr (OUT == 2) {
+                        const uint4 w = make_uint4(lane::pack_bf2(v[0], v[1]), lane::pack_bf2(v[2], v[3]),
+                                                   lane::pack_bf2(v[4], v[5]), lane::pack_bf2(v[6], v[7]));
+                        *reinterpret_cast<uint4*>(outp + o) = w;
+                    } else {
+                        float4* dst = reinterpret_cast<float4*>((OUT == 0 ? actp : accp) + o);
+                        dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+                        dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+                    }
+                }
+                if constexpr (IN == 1 || IN == 3) {
+                    if (act && i + 4 < L) {
+                        const float4* src = reinterpret_cast<const float4*>(sump + line_off(i + 4));
+                        ar[e][0] = src[0];
+                        ar[e][1] = src[1];
+                    }
+                }
+            }
+            // This warp is done with the tap stage; the last of the 8 warps refills
+            // it with the quad NTS ahead.  Each lane orders its reads before the
+            // copy (proxy fence); the fences around the counter order the warps.
+            tma::fence_proxy_async();
+            __syncwarp();
+            if (t == 0) {
+                __threadfence_block();
+                if (atomicAdd(tcount + ts, 1) == NCW - 1) {
+                    __threadfence_block();
+                    tcount[ts] = 0;
+                    if (tnext.g < a.groups) {
+                        issue_taps(tnext, ts);
+#pragma unroll
+                        for (int s = 0; s < NTS; ++s)
+                            if (s == ts) tlast[s] = mt + NTS;
+                    }
+                }
+                advance(tnext);
+            }
+            __syncwarp();
+        }
+        return true;
+    };
+
+    using tru = std::true_type;
+    using fal = std::false_type;
+    using i0 = std::integral_constant<int, 0>;
+    using i1 = std::integral_constant<int, 1>;
+    using i2 = std::integral_constant<int, 2>;
+    using i3 = std::integral_constant<int, 3>;
+    bool ok = true;
+    if (a.stall && blockIdx.x == 0 && warp == 0) {
+        // test hook: nothing completes `never`, so this wait can only run out
+        ok = __all_sync(FULL, tma::mbar_wait(never, 0, a.limit));
+    }
+    if (ok) issue_more(blockIdx.x, 0);
+    for (int g = blockIdx.x; ok && g < a.groups; g += gridDim.x) {
+        for (int k = 0; ok && k < a.D; ++k) {
+            const int info = kinfo_of(a, k);
+            const int d = info & 3, in = (info >> 4) & 3, out = (info >> 6) & 3;
+            if (in == 2) {
+                // the column sums this warp stored (generic proxy) are read next by tensor copies
+                tma::fence_proxy_async_global();
+                __syncwarp();
+                issue_more(g, k);
+            }
+            if (d >= 2)
+                ok = in == 0 ? run_dir(fal{}, i0{}, i0{}, g, k) : run_dir(fal{}, i1{}, i0{}, g, k);
+            else if (in == 0)
+                ok = out == 1 ? run_dir(tru{}, i0{}, i1{}, g, k) : run_dir(tru{}, i0{}, i2{}, g, k);
+            else if (in == 2)
+                ok = out == 1 ? run_dir(tru{}, i2{}, i1{}, g, k) : run_dir(tru{}, i2{}, i2{}, g, k);
+            else
+                ok = run_dir(tru{}, i3{}, i2{}, g, k);
+        }
+    }
+    if (!ok) fail();
+}
+
+// ---- host side ----------------------------------------------------------------
+// (column, row, plane) view of bf16 planes; boxes of 256 columns x 4 rows
+bool map_rows(CUtensorMap* m, const void* base, int H, int W, uint64_t planes) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)W, (cuuint64_t)H, planes};
+    const cuuint64_t strides[2] = {(cuuint64_t)W * 2, (cuuint64_t)H * W * 2};
+    const cuuint32_t box[3] = {LMAX, 4, 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// (column, row / 8, row % 8, plane) view of bf16 planes; boxes of 8 columns x
+// all rows, laid out [row % 8][row / 8][8 columns]
+bool map_cols(CUtensorMap* m, const void* base, int H, int W, uint64_t planes) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)W, (cuuint64_t)H / 8, 8, planes};
+    const cuuint64_t strides[3] = {(cuuint64_t)W * 2 * 8, (cuuint64_t)W * 2, (cuuint64_t)H * W * 2};
+    const cuuint32_t box[4] = {8, LMAX / 8, 8, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// (row, column / 8, column % 8, plane) view of the column-major fp32 sums
+// acct[plane][col][row]; boxes of 4 rows x all columns, laid out
+// [column % 8][column / 8][4 rows]
+bool map_sums_t(CUtensorMap* m, const void* base, int H, int W, uint64_t planes) {
+    EncodeTiledFn fn = encode_tiled();
+    if (!fn) return false;
+    const cuuint64_t dims[4] = {(cuuint64_t)H, (cuuint64_t)W / 8, 8, planes};
+    const cuuint64_t strides[3] = {(cuuint64_t)H * 4 * 8, (cuuint64_t)H * 4, (cuuint64_t)H * W * 4};
+    const cuuint32_t box[4] = {4, LMAX / 8, 8, 1};
+    const cuuint32_t es[4] = {1, 1, 1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, const_cast<void*>(base), dims, strides, box, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int row_dirs(const Problem& p) { return __builtin_popcount(p.d.dir_mask & 3u); }
+int col_dirs(const Problem& p) { return __builtin_popcount(p.d.dir_mask & 12u); }
+
+size_t taps_bytes(const Problem& p) { return align_up((size_t)p.g.D * p.g.B * LMAX * TLINE, kWsAlign); }
+size_t sums_bytes(const Problem& p) { return align_up((size_t)p.planes * p.HW * sizeof(float), kWsAlign); }
+
+}  // namespace
+
+// Compact bf16 planes with lines of 129..256 positions (H, W multiples of 8, at
+// most 256, one of them above 128), whole groups of 8 channels, and at least
+// one row direction (the last direction processed writes the output row by row).
+bool lc_eligible(const Problem& p) {
+    const int H = p.g.H, W = p.g.W;
+    return p.d.dtype == GSPN_BF16 && p.g.shared && (p.d.dir_mask & 3u) && H <= LMAX && W <= LMAX &&
+           (H > 128 || W > 128) && H % 8 == 0 && W % 8 == 0 && p.g.C % 8 == 0 &&
+           p.planes * p.g.D <= ((int64_t)1 << 28) && encode_tiled() != nullptr;
+}
+
+// error word, taps table, row sums (two row directions), column sums (any column direction)
+size_t lc_fwd_workspace(const Problem& p) {
+    return kWsAlign + taps_bytes(p) + (row_dirs(p) == 2 ? sums_bytes(p) : 0) + (col_dirs(p) ? sums_bytes(p) : 0);
+}
+
+gspn_status lc_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
+                   void* out, void* ws, cudaStream_t s) {
+    const uint64_t BC = (uint64_t)p.planes;
+    const int H = p.g.H, W = p.g.W;
+    char* w = static_cast<char*>(ws);
+    LcArgs a;
+    a.err = reinterpret_cast<int*>(w);
+    a.taps = reinterpret_cast<const float4*>(w + kWsAlign);
+    char* sums = w + kWsAlign + taps_bytes(p);
+    a.acc = nullptr;
+    a.acct = nullptr;
+    if (row_dirs(p) == 2) {
+        a.acc = reinterpret_cast<float*>(sums);
+        sums += sums_bytes(p);
+    }
+    if (col_dirs(p)) a.acct = reinterpret_cast<float*>(sums);
+    a.out = static_cast<__nv_bfloat16*>(out);
+    a.B = p.g.B;
+    a.C = p.g.C;
+    a.H = H;
+    a.W = W;
+    a.D = p.g.D;
+    // processing order: left->right, right->left, top->bottom, bottom->top (those enabled)
+    const int order[4] = {L2R, R2L, T2B, B2T};
+    int k = 0, prev = -1;
+    for (int o = 0; o < 4; ++o) {
+        const int d = order[o];
+        if (!(p.d.dir_mask & (1u << d))) continue;
+        const int slot = __builtin_popcount(p.d.dir_mask & ((1u << d) - 1u));
+        const bool rows = d < 2;
+        const int in = prev < 0 ? 0 : !rows ? 1 : prev >= 2 ? 2 : 3;
+        const int outm = k == p.g.D - 1 ? 2 : rows ? 1 : 0;
+        a.kinfo[k++] = d | slot << 2 | in << 4 | outm << 6;
+        prev = d;
+    }
+    for (; k < 4; ++k) a.kinfo[k] = 0;
+    a.groups = (int)(BC / 8);
+    a.segr = H / p.g.groups;
+    a.segc = W / p.g.groups;
+    const WaitCfg wc = wait_cfg();
+    a.limit = wc.limit_ns;
+    a.stall = wc.stall;
+
+    CUtensorMap xr, lr, xc, lc, at;
+    std::memset(&xc, 0, sizeof(xc));
+    std::memset(&lc, 0, sizeof(lc));
+    std::memset(&at, 0, sizeof(at));
+    if (!map_rows(&xr, x, H, W, BC) || !map_rows(&lr, lam, H, W, (uint64_t)p.g.D * BC)) return GSPN_ERR_UNSUPPORTED;
+    if (col_dirs(p) && (!map_cols(&xc, x, H, W, BC) || !map_cols(&lc, lam, H, W, (uint64_t)p.g.D * BC) ||
+                        !map_sums_t(&at, a.acct, H, W, BC)))
+        return GSPN_ERR_UNSUPPORTED;
+
+    const int64_t nt = (int64_t)p.g.D * p.g.B * LMAX * 128;
+    lc_taps_kernel<<<(unsigned)((nt + 255) / 256), 256, 0, s>>>(static_cast<const __nv_bfloat16*>(logits),
+                                                                const_cast<float4*>(a.taps), a.err, p.g);
+    if (cudaGetLastError() != cudaSuccess) return GSPN_ERR_CUDA;
+    const void* fn = (const void*)lc_fwd_kernel;
+    if (ensure_smem_attr(fn, SMEM_BYTES, 43) != cudaSuccess) return GSPN_ERR_CUDA;
+    const int grid = a.groups < dev.sm_count ? a.groups : dev.sm_count;
+    lc_fwd_kernel<<<grid, THREADS, SMEM_BYTES, s>>>(xr, lr, xc, lc, at, a);
+    return cudaGetLastError() == cudaSuccess ? GSPN_OK : GSPN_ERR_CUDA;
+}
+
+}  // namespace gspn

@@ -36,9 +36,9 @@ def dev_inputs(w, inp):
     return {k: to_dev(v, w.dtype) for k, v in inp.items()}
 
 
-def run_fwd(w, dinp, out=None):
+def run_fwd(w, dinp, out=None, ws=None):
     return lsp.forward(dinp["x"], dinp["logits"], dinp["lam"], dir_mask=w.dir_mask, groups=w.groups,
-                       shared=w.shared, out=out)
+                       shared=w.shared, out=out, ws=ws)
 
 
 def run_bwd(w, dinp):

@@ -167,6 +167,35 @@ def test_compact_shapes_take_the_tma_kernels_when_the_encoder_is_there(args, fas
             assert name == fallback + suffix
 
 
+@pytest.mark.parametrize("args", [
+    (2, 1152, 256, 256, 15, 1, True, "bf16"),
+    (1, 16, 136, 200, 15, 2, True, "bf16"),
+    (1, 8, 256, 168, 10, 4, True, "bf16"),
+    (1, 8, 144, 256, 1, 1, True, "bf16"),
+])
+def test_compact_large_planes_take_the_warp_per_plane_kernel_when_the_encoder_is_there(args):
+    """Compact bf16 planes with lines of 129..256 positions, whole groups of 8
+    channels and a row direction run on the compact large-plane forward (two
+    launches: the taps table, then the scan) where the tensor-map encoder is
+    available, else on the general large-plane forward."""
+    d = lsp.make_desc(*args)
+    name = lsp.gspn_variant_name(d, 0)
+    assert name in ("large_compact_fwd", "large_plane_fwd")
+    assert lsp.gspn_launches_per_call(d, 0) == 2
+
+
+@pytest.mark.parametrize("args", [
+    (1, 4, 256, 256, 15, 1, True, "bf16"),     # C % 8 != 0
+    (1, 8, 256, 256, 15, 1, False, "bf16"),    # per-channel taps
+    (1, 8, 256, 256, 15, 1, True, "f32"),      # fp32
+    (1, 8, 256, 256, 12, 1, True, "bf16"),     # column scans only: the output would be written by columns
+    (1, 8, 512, 256, 15, 1, True, "bf16"),     # lines above 256
+    (1, 8, 128, 96, 15, 1, True, "bf16"),      # no line above 128
+])
+def test_other_large_planes_stay_off_the_compact_kernel(args):
+    assert lsp.gspn_variant_name(lsp.make_desc(*args), 0) != "large_compact_fwd"
+
+
 # ---- the compressed propagation block ---------------------------------------------
 
 def _block_fwd(desc, ptr=A):

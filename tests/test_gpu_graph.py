@@ -6,7 +6,8 @@ replay must give the direct results: the forward, dx and dlambda bit for bit
 (every path sums in a fixed order), dlogits within 1e-5 of max|dlogits| (the
 channel-shared TMA paths add their per-CTA tap sums with fp32 reductions
 whose order may vary).  One case per kernel family: small plane, compact
-64x64 and 128x128, large plane (its backward on the generic kernel), generic,
+64x64 and 128x128, both large-plane forwards (their backward on the generic
+kernel), generic,
 and the compressed propagation block.
 """
 import numpy as np
@@ -24,6 +25,7 @@ CASES = [
     (2, 16, 64, 64, 15, 1, True, "bf16", "compact64_tma_fwd"),
     (1, 8, 128, 128, 15, 1, True, "bf16", "compact128_tma_fwd"),
     (1, 2, 256, 256, 15, 1, True, "bf16", "large_plane_fwd"),
+    (1, 8, 136, 136, 15, 1, True, "bf16", "large_compact_fwd"),
     (1, 2, 97, 41, 15, 1, False, "f32", None),
 ]
 

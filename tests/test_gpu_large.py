@@ -1,6 +1,8 @@
-"""GPU parity of the large-plane forward (lines of 65..512 positions, one CTA
-streaming a plane line by line) against the oracle, and of the backward of
-such planes (the generic kernels, pipelined up to 256 positions per line).
+"""GPU parity of the large-plane forwards against the oracle: the compact
+kernel for channel-shared bf16 planes with lines of 129..256 positions (one
+warp per plane, groups of 8 channels), the general one (lines of 65..512
+positions, one CTA streaming a plane line by line), and the backward of such
+planes (the generic kernels, pipelined up to 256 positions per line).
 
 Shapes: 256x256 and 512x512 compact bf16 (the planes beyond the on-chip
 kernels), rectangular planes whose two scan directions use different warp
@@ -82,3 +84,68 @@ def test_large_plane_backward_matches_oracle(case):
     gu.assert_close(dx, rdx, dtype, f"{w.name} dx")
     gu.assert_close(dlam, rdlam, dtype, f"{w.name} dlam")
     gu.assert_close(dlg, rdlg, dtype, f"{w.name} dlogits")
+
+
+LC_CASES = [
+    # B, C, H, W, dir_mask, groups: compact bf16, whole groups of 8 channels
+    (1, 8, 256, 256, 15, 1),
+    (2, 16, 136, 200, 15, 2),   # H != W, local groups of 68 / 100 lines, 2 images
+    (1, 8, 200, 256, 5, 1),     # top->bottom + left->right
+    (1, 8, 256, 168, 10, 4),    # bottom->top + right->left (the transposed read in reverse), groups
+    (1, 8, 256, 256, 3, 1),     # row scans only (no column sums)
+    (1, 8, 144, 256, 1, 1),     # top->bottom only: straight to the output
+    (1, 8, 256, 248, 2, 1),     # bottom->top only
+    (1, 16, 248, 136, 11, 2),   # top->bottom + bottom->top + right->left
+    (1, 8, 64, 144, 12 | 1, 1), # short columns (lanes beyond the line idle), all but bottom->top
+]
+
+
+@pytest.mark.parametrize("case", LC_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_large_compact_forward_matches_oracle(case):
+    import linear_spatial_propagation_b200 as lsp
+    t = gu.torch()
+    B, C, H, W, mask, g = case
+    w = synth.Workload(f"lc_{'x'.join(map(str, case))}", B, C, H, W, mask, g, True, "bf16", 1.0, 4400 + H + W + mask)
+    d = lsp.make_desc(B, C, H, W, mask, g, True, "bf16")
+    assert lsp.gspn_variant_name(d, 0) == "large_compact_fwd"
+    assert lsp.gspn_launches_per_call(d, 0) == 2
+    inp = synth.make_inputs(w, with_dout=False)
+    dinp = gu.dev_inputs(w, inp)
+    guard = 4096
+    buf = t.full((dinp["x"].numel() + 2 * guard,), -3.0, dtype=dinp["x"].dtype, device="cuda")
+    out = buf[guard:guard + dinp["x"].numel()].view(dinp["x"].shape)
+    ws = t.empty(lsp.gspn_workspace_size(d, 0), dtype=t.uint8, device="cuda")
+    gu.run_fwd(w, dinp, out=out, ws=ws)
+    stream = t.cuda.current_stream().cuda_stream
+    assert lsp.gspn_device_status(d, 0, ws.data_ptr(), stream) == 0
+    assert bool((buf[:guard] == -3.0).all()) and bool((buf[guard + out.numel():] == -3.0).all())
+    gu.assert_close(gu.from_dev(out), oracle.fwd_workload(w, inp, nthreads=8), "bf16", w.name)
+
+
+def test_large_compact_forward_is_deterministic():
+    t = gu.torch()
+    w = synth.Workload("lc_det", 1, 16, 256, 256, 15, 1, True, "bf16", 1.0, 4500)
+    dinp = gu.dev_inputs(w, synth.make_inputs(w, with_dout=False))
+    o1 = gu.run_fwd(w, dinp)
+    o2 = gu.run_fwd(w, dinp)
+    t.cuda.synchronize()
+    assert bool(t.equal(o1, o2))
+
+
+def test_large_compact_forward_full_size_sampled_planes():
+    """2 x 1152 x 256 x 256 (the 256-square latent at the 1K channel count) in
+    the launch configuration the bench times; the oracle checks sampled planes."""
+    import numpy as np
+    import linear_spatial_propagation_b200 as lsp
+    w = synth.Workload("lc_full", 2, 1152, 256, 256, 15, 1, True, "bf16", 1.0, 4600)
+    assert lsp.gspn_variant_name(lsp.make_desc(2, 1152, 256, 256, 15, 1, True, "bf16"), 0) == "large_compact_fwd"
+    inp = synth.make_inputs(w, with_dout=False)
+    out = gu.run_fwd(w, gu.dev_inputs(w, inp))
+    rng = np.random.default_rng(5)
+    picks = {(0, 0), (1, 1151), (0, 577)}
+    while len(picks) < 6:
+        picks.add((int(rng.integers(2)), int(rng.integers(1152))))
+    one = w.replace(B=1, C=1)
+    for b, c in sorted(picks):
+        got = gu.from_dev(out[b:b + 1, c:c + 1])
+        gu.assert_close(got, oracle.fwd_workload(one, synth.plane_slice(w, inp, b, c)), "bf16", f"plane ({b},{c})")

@@ -1,6 +1,7 @@
 """Device-side timeouts reach the caller.
 
-The TMA-fed kernels (compact 64x64 and 128x128, forward and backward) hand
+The TMA-fed kernels (compact 64x64 and 128x128, forward and backward, and
+the compact large-plane forward) hand
 data between warps through shared-memory barriers, and every wait is bounded.
 These tests make one wait run out without any fault: gspn_set_stall_test(1)
 makes one warp wait on a barrier that only its own final arrival can complete,
@@ -75,7 +76,8 @@ def _gpu_answers():
     assert float((a * 2).sum().item()) == float(2 * (1 << 20) * ((1 << 20) - 1) / 2)
 
 
-@pytest.mark.parametrize("S,variant", [(64, "compact64_tma_fwd"), (128, "compact128_tma_fwd")])
+@pytest.mark.parametrize("S,variant", [(64, "compact64_tma_fwd"), (128, "compact128_tma_fwd"),
+                                       (136, "large_compact_fwd")])
 def test_forward_timeout_is_reported_and_the_next_call_is_clean(lsp, S, variant):
     t = gu.torch()
     w = _case(2, 16 if S == 64 else 8, S, 900 + S)
