@@ -93,11 +93,13 @@ HEADLINE = "compact_4dir_bf16_b32c1152_64x64"
 
 # Shapes outside the five, timed by the bench only: planes whose sides are not
 # multiples of 8 and longer than 64 take the generic kernels (one warp per
-# plane, directions in turn).
+# plane, directions in turn); the 256-square compact latent at the 1K channel
+# count takes the compact large-plane forward (its backward: the generic kernel).
 EXTRA_WORKLOADS: Dict[str, Workload] = {
     w.name: w
     for w in (
         Workload("generic_4dir_f32_b2c64_130x70", 2, 64, 130, 70, ALL_DIRS, 1, False, "f32", 1.0, 30),
+        Workload("large_compact_4dir_bf16_b2c1152_256x256", 2, 1152, 256, 256, ALL_DIRS, 1, True, "bf16", 1.0, 31),
     )
 }
 

@@ -147,6 +147,7 @@ def test_l2_flush_only_where_a_pass_fits_in_l2():
         "compact_4dir_bf16_b32c1152_64x64": False,
         "compact_4dir_bf16_b2c1152_128x128_fwdbwd": False,
         "generic_4dir_f32_b2c64_130x70": True,
+        "large_compact_4dir_bf16_b2c1152_256x256": False,
     }
     assert bench.L2_BYTES == 126 * 2**20
 
