@@ -97,6 +97,9 @@ LC_CASES = [
     (1, 8, 256, 248, 2, 1),     # bottom->top only
     (1, 16, 248, 136, 11, 2),   # top->bottom + bottom->top + right->left
     (1, 8, 64, 144, 12 | 1, 1), # short columns (lanes beyond the line idle), all but bottom->top
+    (1, 8, 8, 256, 15, 1),      # 8-row planes: row chunks of 4 lines, one lane per column line
+    (1, 8, 256, 8, 15, 2),      # 8-column planes: one column chunk per direction, local groups
+    (1, 8, 16, 144, 13, 1),     # top->bottom + left->right + right->left on a flat plane
 ]
 
 
