@@ -6,6 +6,7 @@
 #include <cstring>
 
 #include "gspn_internal.h"
+#include "gspn_large_compact.h"
 
 namespace gspn {
 

@@ -75,12 +75,6 @@ size_t large_fwd_workspace(const Problem& p);
 gspn_status large_fwd(const Problem& p, const void* x, const void* logits, const void* lam, void* out, void* ws,
                       cudaStream_t s);
 
-// ---- compact bf16 planes with lines of 129..256 positions: one warp per plane (forward) ----
-bool lc_eligible(const Problem& p);
-size_t lc_fwd_workspace(const Problem& p);
-gspn_status lc_fwd(const Problem& p, const DeviceInfo& dev, const void* x, const void* logits, const void* lam,
-                   void* out, void* ws, cudaStream_t s);
-
 // ---- compact 64x64 bf16 forward (TMA-fed, packed fp32x2) ------------------------
 bool c64_eligible(const Problem& p);
 size_t c64_fwd_workspace(const Problem& p);

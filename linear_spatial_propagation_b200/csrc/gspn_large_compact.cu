@@ -31,7 +31,7 @@
 #include <cstring>
 #include <type_traits>
 
-#include "gspn_internal.h"
+#include "gspn_large_compact.h"
 #include "gspn_lane.cuh"
 #include "gspn_tma.cuh"
 
@@ -40,6 +40,10 @@ namespace gspn {
 namespace {
 
 using lane::FULL;
+
+// order this thread's generic-proxy global-memory writes before later
+// async-proxy (tensor copy) reads of the same memory
+__device__ __forceinline__ void fence_proxy_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
 
 constexpr int NCW = 8;                    // consumer warps (planes in flight per CTA)
 constexpr int THREADS = NCW * 32;
@@ -447,7 +451,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int d = info & 3, in = (info >> 4) & 3, out = (info >> 6) & 3;
             if (in == 2) {
                 // the column sums this warp stored (generic proxy) are read next by tensor copies
-                tma::fence_proxy_async_global();
+                fence_proxy_async_global();
                 __syncwarp();
                 issue_more(g, k);
             }
