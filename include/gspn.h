@@ -72,11 +72,12 @@
  *   GSPN_ERR_SCRATCH_LIMIT  (gspn_fwd_noalloc only) the problem does not fit
  *                         the library's fixed scratch.
  * Device-side timeouts.  The TMA-fed kernels (the compact 64x64 and 128x128
- * paths; gspn_variant_name names them "compact*_tma_*") hand data between
- * warps through shared-memory barriers.  Every such wait is bounded (2 s by
- * default, gspn_set_wait_limit_ns); when one runs out, the kernel records an
- * error word in its workspace, waits for its own copies in flight, frees its
- * tensor memory and returns, so the GPU stays usable but the outputs are not
+ * paths, which gspn_variant_name names "compact*_tma_*", and the compact
+ * large-plane forward, "large_compact_fwd") hand data between warps through
+ * shared-memory barriers.  Every such wait is bounded (2 s by default,
+ * gspn_set_wait_limit_ns); when one runs out, the kernel records an error
+ * word in its workspace, waits for its own copies in flight, frees its tensor
+ * memory and returns, so the GPU stays usable but the outputs are not
  * valid.  The launching call has already returned GSPN_OK by then; the caller
  * learns of the timeout with gspn_device_status (or gspn_noalloc_status),
  * which synchronises the stream and returns
