@@ -82,7 +82,7 @@ Path pick(const Problem& p, int backward) {
     if (backward ? c64_bwd_eligible(p) : c64_eligible(p)) return Path::kC64;
     if (backward ? c128_bwd_eligible(p) : c128_eligible(p)) return Path::kC128;
     if (small_eligible(p, backward)) return Path::kSmall;
-    if (!backward && lc_eligible(p)) return Path::kLargeCompact;
+    if (lc_eligible(p)) return Path::kLargeCompact;
     if (!backward && large_eligible(p)) return Path::kLarge;
     return Path::kGeneric;
 }
@@ -195,7 +195,7 @@ size_t gspn_workspace_size(const gspn_desc* desc, int backward) {
     case Path::kC64: return backward ? c64_bwd_workspace(p, dev) : c64_fwd_workspace(p);
     case Path::kC128: return backward ? c128_bwd_workspace(p, dev) : c128_fwd_workspace(p, dev);
     case Path::kSmall: return backward ? small_bwd_workspace(p) : 0;
-    case Path::kLargeCompact: return lc_fwd_workspace(p);
+    case Path::kLargeCompact: return backward ? lc_bwd_workspace(p) : lc_fwd_workspace(p);
     case Path::kLarge: return large_fwd_workspace(p);
     default: return backward ? generic_bwd_workspace(p, dev) : generic_fwd_workspace(p, dev);
     }
@@ -208,7 +208,7 @@ int gspn_launches_per_call(const gspn_desc* desc, int backward) {
     case Path::kC64:
     case Path::kC128: return backward ? 3 : 2;
     case Path::kSmall: return backward ? small_bwd_launches(p) : 1;
-    case Path::kLargeCompact: return 2;  // the taps table, then the scan
+    case Path::kLargeCompact: return backward ? 4 : 2;  // the taps table, then the scan (backward: states, adjoint, dlogits)
     case Path::kLarge: return p.g.shared ? 2 : 1;  // channel-shared taps: the taps pre-kernel first
     default: return backward ? generic_bwd_launches(p) : 1;
     }
@@ -221,7 +221,7 @@ const char* gspn_variant_name(const gspn_desc* desc, int backward) {
     case Path::kC64: return backward ? "compact64_tma_bwd" : "compact64_tma_fwd";
     case Path::kC128: return backward ? "compact128_tma_bwd" : "compact128_tma_fwd";
     case Path::kSmall: return backward ? "small_plane_bwd" : "small_plane_fwd";
-    case Path::kLargeCompact: return "large_compact_fwd";
+    case Path::kLargeCompact: return backward ? "large_compact_bwd" : "large_compact_fwd";
     case Path::kLarge: return "large_plane_fwd";
     default: return backward ? "generic_bwd" : "generic_fwd";
     }
@@ -322,12 +322,14 @@ gspn_status gspn_bwd(const gspn_desc* desc, const void* x, const void* logits, c
                   path == Path::kC64     ? c64_bwd_workspace(p, dev)
                   : path == Path::kC128  ? c128_bwd_workspace(p, dev)
                   : path == Path::kSmall ? small_bwd_workspace(p)
+                  : path == Path::kLargeCompact ? lc_bwd_workspace(p)
                                          : generic_bwd_workspace(p, dev));
     if (st != GSPN_OK) return st;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
     st = path == Path::kC64     ? c64_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs)
          : path == Path::kC128  ? c128_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs)
          : path == Path::kSmall ? small_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs)
+         : path == Path::kLargeCompact ? lc_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs)
                                 : generic_bwd(p, dev, x, logits, lambda, dout, dx, dlogits, dlambda, workspace, cs);
     if (st != GSPN_OK || !g_sync_check.load(std::memory_order_relaxed)) return st;
     return sync_status(has_status_word(path) ? workspace : nullptr, cs);

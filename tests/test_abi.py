@@ -175,13 +175,17 @@ def test_compact_shapes_take_the_tma_kernels_when_the_encoder_is_there(args, fas
 ])
 def test_compact_large_planes_take_the_warp_per_plane_kernel_when_the_encoder_is_there(args):
     """Compact bf16 planes with lines of 129..256 positions, whole groups of 8
-    channels and a row direction run on the compact large-plane forward (two
-    launches: the taps table, then the scan) where the tensor-map encoder is
-    available, else on the general large-plane forward."""
+    channels and a row direction run on the compact large-plane kernels (the
+    forward in two launches: the taps table, then the scan) where the
+    tensor-map encoder is available, else on the general large-plane forward."""
     d = lsp.make_desc(*args)
     name = lsp.gspn_variant_name(d, 0)
     assert name in ("large_compact_fwd", "large_plane_fwd")
     assert lsp.gspn_launches_per_call(d, 0) == 2
+    if name == "large_compact_fwd":
+        # and its backward: states pass, adjoint pass, dlogits, after the taps table
+        assert lsp.gspn_variant_name(d, 1) == "large_compact_bwd"
+        assert lsp.gspn_launches_per_call(d, 1) == 4
 
 
 @pytest.mark.parametrize("args", [
@@ -193,7 +197,9 @@ def test_compact_large_planes_take_the_warp_per_plane_kernel_when_the_encoder_is
     (1, 8, 128, 96, 15, 1, True, "bf16"),      # no line above 128
 ])
 def test_other_large_planes_stay_off_the_compact_kernel(args):
-    assert lsp.gspn_variant_name(lsp.make_desc(*args), 0) != "large_compact_fwd"
+    d = lsp.make_desc(*args)
+    assert lsp.gspn_variant_name(d, 0) != "large_compact_fwd"
+    assert lsp.gspn_variant_name(d, 1) != "large_compact_bwd"
 
 
 # ---- the compressed propagation block ---------------------------------------------

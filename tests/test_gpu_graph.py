@@ -5,9 +5,10 @@ then captures them with the same buffers and replays the graph twice; the
 replay must give the direct results: the forward, dx and dlambda bit for bit
 (every path sums in a fixed order), dlogits within 1e-5 of max|dlogits| (the
 channel-shared TMA paths add their per-CTA tap sums with fp32 reductions
-whose order may vary).  One case per kernel family: small plane, compact
-64x64 and 128x128, both large-plane forwards (their backward on the generic
-kernel), generic,
+whose order may vary; the compact large-plane backward adds every warp's tap
+values that way, so there one bf16 step, within 1e-2).  One case per kernel family: small plane, compact
+64x64 and 128x128, both large-plane forwards (the compact one with its own
+backward, the general one with the generic backward), generic,
 and the compressed propagation block.
 """
 import numpy as np
@@ -68,7 +69,10 @@ def test_captured_step_replays_the_direct_results(case):
     assert bool(t.equal(grads_g[2], grads_d[2])), "dlambda"
     a, b = gu.from_dev(grads_g[1]), gu.from_dev(grads_d[1])
     scale = max(float(np.max(np.abs(b))), 1e-30)
-    assert float(np.max(np.abs(a - b))) <= 1e-5 * scale, "dlogits"
+    # the compact large-plane backward adds every warp's tap values into fp32
+    # sums in arrival order, so a sum can round to the neighbouring bf16 value
+    tol = 1e-2 if lsp.gspn_variant_name(desc, 1) == "large_compact_bwd" else 1e-5
+    assert float(np.max(np.abs(a - b))) <= tol * scale, "dlogits"
     del graph
 
 

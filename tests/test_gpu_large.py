@@ -1,8 +1,9 @@
-"""GPU parity of the large-plane forwards against the oracle: the compact
-kernel for channel-shared bf16 planes with lines of 129..256 positions (one
-warp per plane, groups of 8 channels), the general one (lines of 65..512
-positions, one CTA streaming a plane line by line), and the backward of such
-planes (the generic kernels, pipelined up to 256 positions per line).
+"""GPU parity of the large-plane kernels against the oracle: the compact
+forward and backward for channel-shared bf16 planes with lines of 129..256
+positions (one warp per plane, groups of 8 channels), the general forward
+(lines of 65..512 positions, one CTA streaming a plane line by line), and the
+backward of the other large planes (the generic kernels, pipelined up to 256
+positions per line).
 
 Shapes: 256x256 and 512x512 compact bf16 (the planes beyond the on-chip
 kernels), rectangular planes whose two scan directions use different warp
@@ -152,3 +153,68 @@ def test_large_compact_forward_full_size_sampled_planes():
     for b, c in sorted(picks):
         got = gu.from_dev(out[b:b + 1, c:c + 1])
         gu.assert_close(got, oracle.fwd_workload(one, synth.plane_slice(w, inp, b, c)), "bf16", f"plane ({b},{c})")
+
+
+LCB_CASES = [
+    # B, C, H, W, dir_mask, groups: compact bf16 backward, whole groups of 8 channels
+    (1, 8, 256, 256, 15, 1),
+    (2, 16, 136, 200, 15, 2),   # H != W, local groups, 2 images (2 CTAs per image)
+    (1, 8, 200, 256, 5, 1),     # top->bottom + left->right
+    (1, 8, 256, 168, 10, 4),    # bottom->top + right->left, groups
+    (1, 8, 256, 256, 3, 1),     # row scans only
+    (1, 8, 144, 256, 1, 1),     # top->bottom only
+    (1, 16, 248, 136, 11, 2),   # three directions
+    (1, 8, 8, 256, 15, 1),      # 8-row planes
+    (1, 8, 256, 8, 15, 2),      # 8-column planes, groups
+]
+
+
+@pytest.mark.parametrize("case", LCB_CASES, ids=lambda c: "x".join(map(str, c)))
+def test_large_compact_backward_matches_oracle(case):
+    """The compact large-plane backward (a states pass, the adjoint pass, the
+    dlogits kernel): dx, dlambda and the channel-summed dlogits against the
+    oracle's adjoint."""
+    import linear_spatial_propagation_b200 as lsp
+    t = gu.torch()
+    B, C, H, W, mask, g = case
+    w = synth.Workload(f"lcb_{'x'.join(map(str, case))}", B, C, H, W, mask, g, True, "bf16", 1.0, 4700 + H + W + mask,
+                       backward=True)
+    d = lsp.make_desc(B, C, H, W, mask, g, True, "bf16")
+    assert lsp.gspn_variant_name(d, 1) == "large_compact_bwd"
+    assert lsp.gspn_launches_per_call(d, 1) == 4
+    inp = synth.make_inputs(w, with_dout=True)
+    dinp = gu.dev_inputs(w, inp)
+    ws = t.empty(lsp.gspn_workspace_size(d, 1), dtype=t.uint8, device="cuda")
+    dx, dlg, dlam = lsp.backward(dinp["x"], dinp["logits"], dinp["lam"], dinp["dout"], dir_mask=mask, groups=g,
+                                 shared=True, ws=ws)
+    assert lsp.gspn_device_status(d, 1, ws.data_ptr(), t.cuda.current_stream().cuda_stream) == 0
+    rdx, rdlg, rdlam = oracle.bwd_workload(w, inp, nthreads=8)
+    gu.assert_close(gu.from_dev(dx), rdx, "bf16", f"{w.name} dx")
+    gu.assert_close(gu.from_dev(dlam), rdlam, "bf16", f"{w.name} dlam")
+    gu.assert_close(gu.from_dev(dlg), rdlg, "bf16", f"{w.name} dlogits")
+
+
+def test_large_compact_backward_2x64_256_square():
+    """256-square planes, 2 images of 64 channels (8 CTAs per image add their
+    tap values into the same sums), checked whole against the oracle."""
+    w = synth.Workload("lcb_2x64_256", 2, 64, 256, 256, 15, 1, True, "bf16", 1.0, 4800, backward=True)
+    inp = synth.make_inputs(w, with_dout=True)
+    dx, dlg, dlam = (gu.from_dev(x) for x in gu.run_bwd(w, gu.dev_inputs(w, inp)))
+    rdx, rdlg, rdlam = oracle.bwd_workload(w, inp, nthreads=8)
+    gu.assert_close(dx, rdx, "bf16", "dx")
+    gu.assert_close(dlam, rdlam, "bf16", "dlam")
+    gu.assert_close(dlg, rdlg, "bf16", "dlogits")
+
+
+def test_large_compact_backward_repeats():
+    """dx and dlambda repeat bit for bit; dlogits are fp32 sums of the warps'
+    tap values in arrival order, so they repeat to within rounding."""
+    t = gu.torch()
+    w = synth.Workload("lcb_det", 1, 16, 136, 144, 15, 1, True, "bf16", 1.0, 4900, backward=True)
+    d = gu.dev_inputs(w, synth.make_inputs(w, with_dout=True))
+    r1 = tuple(x.clone() for x in gu.run_bwd(w, d))
+    r2 = gu.run_bwd(w, d)
+    t.cuda.synchronize()
+    assert bool(t.equal(r1[0], r2[0])) and bool(t.equal(r1[2], r2[2]))
+    a, b = r1[1].float(), r2[1].float()
+    assert float((a - b).abs().max()) <= 1e-2 * float(a.abs().max())

@@ -1,7 +1,7 @@
 """Device-side timeouts reach the caller.
 
-The TMA-fed kernels (compact 64x64 and 128x128, forward and backward, and
-the compact large-plane forward) hand
+The TMA-fed kernels (compact 64x64 and 128x128, and the compact large-plane
+kernels, forward and backward) hand
 data between warps through shared-memory barriers, and every wait is bounded.
 These tests make one wait run out without any fault: gspn_set_stall_test(1)
 makes one warp wait on a barrier that only its own final arrival can complete,
@@ -99,7 +99,8 @@ def test_forward_timeout_is_reported_and_the_next_call_is_clean(lsp, S, variant)
     gu.assert_close(gu.from_dev(out), oracle.fwd_workload(w, inp), w.dtype, f"{variant} after a timeout")
 
 
-@pytest.mark.parametrize("S,variant", [(64, "compact64_tma_bwd"), (128, "compact128_tma_bwd")])
+@pytest.mark.parametrize("S,variant", [(64, "compact64_tma_bwd"), (128, "compact128_tma_bwd"),
+                                       (136, "large_compact_bwd")])
 def test_backward_timeout_is_reported_and_the_next_call_is_clean(lsp, S, variant):
     t = gu.torch()
     w = _case(1, 16 if S == 64 else 8, S, 910 + S)
