@@ -94,7 +94,7 @@ HEADLINE = "compact_4dir_bf16_b32c1152_64x64"
 # Shapes outside the five, timed by the bench only: planes whose sides are not
 # multiples of 8 and longer than 64 take the generic kernels (one warp per
 # plane, directions in turn); the 256-square compact latent at the 1K channel
-# count takes the compact large-plane forward (its backward: the generic kernel).
+# count takes the compact large-plane forward and backward.
 EXTRA_WORKLOADS: Dict[str, Workload] = {
     w.name: w
     for w in (
