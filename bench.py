@@ -58,6 +58,7 @@ def parse():
     ap.add_argument("--pass", dest="passes", default="both", choices=["both", "fwd", "bwd"],
                     help="profiling aid: time only one pass (the JSON line then covers that pass)")
     ap.add_argument("--batch", type=int, default=0, help="profiling aid: override B (0 = the workload's)")
+    ap.add_argument("--channels", type=int, default=0, help="profiling aid: override C (0 = the workload's)")
     ap.add_argument("--graph", action="store_true",
                     help="replay each pass from a CUDA graph captured once (no per-call host work in the timed loop)")
     return ap.parse_args()
@@ -710,6 +711,8 @@ def main():
         w = w.replace(backward=True)
     if args.batch:
         w = w.replace(B=args.batch, name=f"{w.name}@B{args.batch}")
+    if args.channels:
+        w = w.replace(C=args.channels, name=f"{w.name}@C{args.channels}")
     if args.impl == "reference":
         return run_reference(args, w)
     return run_gpu(args, w)
