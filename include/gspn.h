@@ -73,7 +73,7 @@
  *                         the library's fixed scratch.
  * Device-side timeouts.  The TMA-fed kernels (the compact 64x64 and 128x128
  * paths, which gspn_variant_name names "compact*_tma_*", and the compact
- * large-plane forward, "large_compact_fwd") hand data between warps through
+ * large-plane kernels, "large_compact_*") hand data between warps through
  * shared-memory barriers.  Every such wait is bounded (2 s by default,
  * gspn_set_wait_limit_ns); when one runs out, the kernel records an error
  * word in its workspace, waits for its own copies in flight, frees its tensor
