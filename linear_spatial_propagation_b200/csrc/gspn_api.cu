@@ -75,8 +75,10 @@ gspn_status check_ws(void* ws, size_t have, size_t need) {
 }
 
 // The kernel family a descriptor runs on: the TMA-fed compact kernels for their
-// shapes, the one-CTA-per-plane kernels for planes of at most 64x64, the generic
-// kernels for everything else.
+// shapes (64x64, 128x128, and compact planes with lines of 129..256), the
+// one-CTA-per-plane kernels for planes of at most 64x64, the large-plane
+// forward for the other lines of 65..512, the generic kernels for everything
+// else.
 enum class Path { kC64, kC128, kSmall, kLargeCompact, kLarge, kGeneric };
 Path pick(const Problem& p, int backward) {
     if (backward ? c64_bwd_eligible(p) : c64_eligible(p)) return Path::kC64;
