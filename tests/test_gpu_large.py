@@ -218,3 +218,23 @@ def test_large_compact_backward_repeats():
     assert bool(t.equal(r1[0], r2[0])) and bool(t.equal(r1[2], r2[2]))
     a, b = r1[1].float(), r2[1].float()
     assert float((a - b).abs().max()) <= 1e-2 * float(a.abs().max())
+
+
+def test_large_compact_backward_writes_only_its_outputs():
+    """Guard bands around dx, dlogits and dlambda stay untouched (column
+    directions write dlambda as 4-column pieces per row)."""
+    import linear_spatial_propagation_b200 as lsp
+    t = gu.torch()
+    w = synth.Workload("lcb_guard", 1, 8, 144, 136, 15, 2, True, "bf16", 1.0, 4950, backward=True)
+    d = gu.dev_inputs(w, synth.make_inputs(w, with_dout=True))
+    guard = 4096
+
+    def framed(like):
+        buf = t.full((like.numel() + 2 * guard,), -5.0, dtype=like.dtype, device="cuda")
+        return buf, buf[guard:guard + like.numel()].view(like.shape)
+
+    (bx, dx), (bg, dlg), (bl, dlam) = framed(d["x"]), framed(d["logits"]), framed(d["lam"])
+    lsp.backward(d["x"], d["logits"], d["lam"], d["dout"], dir_mask=15, groups=2, shared=True, grads=(dx, dlg, dlam))
+    t.cuda.synchronize()
+    for name, buf, inner in (("dx", bx, dx), ("dlogits", bg, dlg), ("dlambda", bl, dlam)):
+        assert bool((buf[:guard] == -5.0).all()) and bool((buf[guard + inner.numel():] == -5.0).all()), name
